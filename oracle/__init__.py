@@ -1,0 +1,193 @@
+"""fp64 CPU oracle for block-causal linear attention (ctypes binding of oracle.c).
+
+TEST INFRASTRUCTURE ONLY.  The tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg are the only callers.  The CUDA library never
+imports this package and this package never imports the CUDA library; the two
+share nothing but the seeded input generator's tensors.
+
+Every function takes CPU torch tensors laid out ``[B, N, H, d]`` (fp64, fp32 or
+bf16 -- bf16 is passed as its bit pattern and widened exactly in C) and returns
+fp64 numpy arrays.  What each function computes, with the passages it follows,
+is written next to it in ``oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+ORC_F64, ORC_F32, ORC_BF16 = 0, 1, 2
+
+
+class Rope(ctypes.Structure):
+    """3D RoPE description: grid rows Hg, columns Wg, first frame t_offset,
+    section dims (dt, dh, dw) for the frame/row/column axes, frequency base."""
+
+    _fields_ = [
+        ("enabled", ctypes.c_int),
+        ("Hg", ctypes.c_int),
+        ("Wg", ctypes.c_int),
+        ("t_offset", ctypes.c_int),
+        ("dt", ctypes.c_int),
+        ("dh", ctypes.c_int),
+        ("dw", ctypes.c_int),
+        ("base", ctypes.c_double),
+    ]
+
+
+def make_rope(Hg, Wg, t_offset=0, dims=(8, 12, 12), base=10000.0):
+    return Rope(1, int(Hg), int(Wg), int(t_offset), int(dims[0]), int(dims[1]), int(dims[2]), float(base))
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so with gcc (-O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        vp, ip, lp, dp = ctypes.c_void_p, ctypes.c_int, ctypes.c_long, ctypes.c_double
+        rp = ctypes.POINTER(Rope)
+        L.orc_brute.argtypes = [vp, vp, vp, ip, vp, ip, lp, ip, ip, lp, rp, lp, dp]
+        L.orc_block_kv.argtypes = [vp, vp, ip, ip, lp, ip, ip, lp, lp, rp, lp, vp, vp]
+        L.orc_apply.argtypes = [vp, ip, ip, lp, ip, ip, vp, vp, vp, lp, rp, lp, dp, vp]
+        L.orc_block_forward.argtypes = [vp, vp, vp, ip, vp, ip, lp, ip, ip, vp, vp, ip, rp, lp, dp]
+        L.orc_full_forward.argtypes = [vp, vp, vp, ip, vp, ip, lp, ip, ip, lp, rp, dp]
+        L.orc_set_threads.argtypes = [ip]
+        L.orc_get_threads.restype = ip
+        for f in ("orc_brute", "orc_block_kv", "orc_apply", "orc_block_forward", "orc_full_forward"):
+            getattr(L, f).restype = ip
+        _lib = L
+    return _lib
+
+
+def set_threads(n: int) -> None:
+    lib().orc_set_threads(int(n))
+
+
+def get_threads() -> int:
+    return int(lib().orc_get_threads())
+
+
+def _prep(x: torch.Tensor):
+    """Contiguous CPU tensor and its dtype code; bf16 travels as raw bits."""
+    x = x.detach()
+    if x.device.type != "cpu":
+        raise ValueError("the oracle takes CPU tensors only")
+    x = x.contiguous()
+    if x.dtype == torch.float64:
+        return x, ORC_F64
+    if x.dtype == torch.float32:
+        return x, ORC_F32
+    if x.dtype == torch.bfloat16:
+        return x.view(torch.int16), ORC_BF16
+    raise TypeError(f"unsupported dtype {x.dtype}")
+
+
+def _shape(q):
+    if q.dim() != 4:
+        raise ValueError("expected [B, N, H, d]")
+    return tuple(int(s) for s in q.shape)
+
+
+def _rope_ptr(rope):
+    return ctypes.byref(rope) if rope is not None else None
+
+
+def _check(rc, name):
+    if rc != 0:
+        raise ValueError(f"oracle {name} rejected its arguments")
+
+
+def brute(q, k, v, tokens_per_block=0, rope=None, eps=1e-6, tok_base=0):
+    """Definition form, O(N^2 d): out_i over all j in blocks <= blk(i)."""
+    B, N, H, d = _shape(q)
+    (qc, dt), (kc, dt2), (vc, dt3) = _prep(q), _prep(k), _prep(v)
+    assert dt == dt2 == dt3
+    out = np.zeros((B, N, H, d), dtype=np.float64)
+    rc = lib().orc_brute(qc.data_ptr(), kc.data_ptr(), vc.data_ptr(), dt, out.ctypes.data,
+                         B, N, H, d, int(tokens_per_block), _rope_ptr(rope), int(tok_base), float(eps))
+    _check(rc, "brute")
+    return out
+
+
+def block_kv(k, v, t0=0, t1=None, rope=None, tok_base=0):
+    """KV_n [B,H,d,d] and z_n [B,H,d] over tokens [t0, t1) of k, v."""
+    B, N, H, d = _shape(k)
+    t1 = N if t1 is None else t1
+    (kc, dt), (vc, dt2) = _prep(k), _prep(v)
+    assert dt == dt2
+    KV = np.zeros((B, H, d, d), dtype=np.float64)
+    z = np.zeros((B, H, d), dtype=np.float64)
+    rc = lib().orc_block_kv(kc.data_ptr(), vc.data_ptr(), dt, B, N, H, d, int(t0), int(t1),
+                            _rope_ptr(rope), int(tok_base), KV.ctypes.data, z.ctypes.data)
+    _check(rc, "block_kv")
+    return KV, z
+
+
+def apply(q, S_eff, Z_eff, toks=None, rope=None, eps=1e-6, tok_base=0):
+    """out [B, len(toks), H, d] = psi(q) S_eff / (phi(q).Z_eff + eps) for the listed tokens."""
+    B, N, H, d = _shape(q)
+    qc, dt = _prep(q)
+    toks = np.arange(N, dtype=np.int64) if toks is None else np.ascontiguousarray(toks, dtype=np.int64)
+    S = np.ascontiguousarray(S_eff, dtype=np.float64)
+    Z = np.ascontiguousarray(Z_eff, dtype=np.float64)
+    assert S.shape == (B, H, d, d) and Z.shape == (B, H, d)
+    out = np.zeros((B, len(toks), H, d), dtype=np.float64)
+    rc = lib().orc_apply(qc.data_ptr(), dt, B, N, H, d, S.ctypes.data, Z.ctypes.data,
+                         toks.ctypes.data, len(toks), _rope_ptr(rope), int(tok_base), float(eps),
+                         out.ctypes.data)
+    _check(rc, "apply")
+    return out
+
+
+class State:
+    """The oracle's own fp64 constant-size state: S [B,H,d,d], Z [B,H,d]."""
+
+    def __init__(self, B, H, d):
+        self.S = np.zeros((B, H, d, d), dtype=np.float64)
+        self.Z = np.zeros((B, H, d), dtype=np.float64)
+
+    def nbytes(self):
+        return self.S.nbytes + self.Z.nbytes
+
+
+def block_forward(q, k, v, state: State, commit=True, rope=None, eps=1e-6, tok_base=0):
+    """One streaming block: KV_n, z_n, out with S+KV_n, Z+z_n, commit if asked."""
+    B, N, H, d = _shape(q)
+    (qc, dt), (kc, _), (vc, _) = _prep(q), _prep(k), _prep(v)
+    out = np.zeros((B, N, H, d), dtype=np.float64)
+    rc = lib().orc_block_forward(qc.data_ptr(), kc.data_ptr(), vc.data_ptr(), dt, out.ctypes.data,
+                                 B, N, H, d, state.S.ctypes.data, state.Z.ctypes.data, int(bool(commit)),
+                                 _rope_ptr(rope), int(tok_base), float(eps))
+    _check(rc, "block_forward")
+    return out
+
+
+def full_forward(q, k, v, tokens_per_block=0, rope=None, eps=1e-6):
+    """Whole sequence from a zero state, block after block (recurrence form)."""
+    B, N, H, d = _shape(q)
+    (qc, dt), (kc, _), (vc, _) = _prep(q), _prep(k), _prep(v)
+    out = np.zeros((B, N, H, d), dtype=np.float64)
+    rc = lib().orc_full_forward(qc.data_ptr(), kc.data_ptr(), vc.data_ptr(), dt, out.ctypes.data,
+                                B, N, H, d, int(tokens_per_block), _rope_ptr(rope), float(eps))
+    _check(rc, "full_forward")
+    return out
