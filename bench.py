@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Throughput of block-causal linear attention on B200, through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
+
+One step is one of the workloads (default: configuration 2, the 5 s 480p
+latent as a single bidirectional block, 8190 tokens x 64 heads x d 32, bf16)
+run once through the library from a zero state, with every input already
+resident in HBM.  L2 is flushed (a 256 MiB device write) before every timed
+step; the step time is the device time between CUDA events recorded before
+its first and after its last kernel, so the flush is not in it.  The metric
+is token*heads per second (every pass counts), whole job over all ranks.
+
+Multi-GPU: one process per GPU (torchrun), each rank an independent problem
+of the same shape (its own seed), no data-path collective: weak scaling.  The
+timed totals are reduced with MAX over ranks.
+
+--impl reference times the fp64 CPU oracle (the test oracle, unchanged) on
+the host cores on a bounded sample of the same workload; only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from datetime import timedelta
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_causal_linear_b200 import synth  # noqa: E402
+
+METRIC = "block linear-attn tokens·heads/s and achieved HBM GB/s vs B200 peak (1 GPU)"
+UNIT = "token·heads/s"
+FLUSH_BYTES = 256 << 20          # > 2x the 126 MB L2 of a B200
+FALLBACK_HBM_GBS = 6650.0
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def workload_config(w: synth.Workload, extra=None):
+    c = {"workload": w.name, "B": w.B, "N_per_call": w.n_blk if w.mode == "stream" else w.n_total,
+         "H": w.H, "d": w.d, "blocks": w.n_blocks, "passes_per_block": w.passes,
+         "calls_per_step": w.calls, "api": "la_full_forward" if w.mode == "full" else "la_block_forward",
+         "rope": "3d 8/12/12 base 1e4" if w.rope else None, "input_dtype": w.dtype,
+         "accumulate": "f32", "state": "f32",
+         "l2": "flushed before every timed step (256 MiB device write, outside the step's events)"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_sources_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_causal_linear_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, units_per_launch: int):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, scaled
+    to this launch by token-heads, or None when the kernels changed since."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    e = j.get(kernel)
+    if not e or e.get("sources_sha") != kernel_sources_sha():
+        return None
+    return e["dram_bytes_per_token_head"] * units_per_launch
+
+
+class ClockSampler:
+    def __init__(self):
+        self.proc = None
+        self.path = None
+
+    def start(self, device):
+        """Sample the GPU behind `device` (selected by UUID, since nvidia-smi
+        numbers the machine's GPUs regardless of CUDA_VISIBLE_DEVICES)."""
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = []
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", *sel, f"--query-gpu={CLOCK_FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+            self.filtered = bool(sel)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self, device_index: int):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9 or not parts[0].isdigit():
+                    continue
+                if not self.filtered and int(parts[0]) != device_index:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                    power.append(float(parts[3]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names[1:], parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- oracle timing
+
+def oracle_sample(w: synth.Workload, budget_s: float, orc):
+    """Time the oracle on the first call's inputs of the workload: all tokens of
+    that call, a head subset sized to take about budget_s.  Returns
+    (token_heads, seconds, description)."""
+    import numpy as np  # noqa: F401
+
+    _, _, q, k, v = next(iter(synth.stream(w, "cpu", blocks=1)))
+    rope = (orc.make_rope(Hg=w.Hg, Wg=w.Wg, t_offset=0, dims=w.rope_dims, base=w.rope_base)
+            if w.rope else None)
+
+    def run(nh):
+        qs, ks, vs = (t[:, :, :nh].contiguous() for t in (q, k, v))
+        st = orc.State(w.B, nh, w.d)
+        t0 = time.perf_counter()
+        orc.block_forward(qs, ks, vs, st, commit=True, rope=rope, eps=w.eps)
+        return time.perf_counter() - t0
+
+    t1 = run(1)
+    nh = int(max(1, min(w.H, budget_s / max(t1, 1e-6))))
+    dt = run(nh)
+    th = w.B * q.shape[1] * nh
+    desc = (f"first call of the workload ({w.B}x{q.shape[1]} tokens) on {nh} of {w.H} heads, "
+            f"one recurrence pass (block KV, state combine, apply, commit) in fp64")
+    return th, dt, desc
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    import oracle as orc
+
+    orc.build()
+    w = synth.WORKLOADS[args.config]
+    total_steps = args.steps if args.steps is not None else 10
+    per_step = min(10.0, 150.0 / max(1, total_steps + args.warmup))
+    _, _, q, k, v = next(iter(synth.stream(w, "cpu", blocks=1)))
+    rope = (orc.make_rope(Hg=w.Hg, Wg=w.Wg, t_offset=0, dims=w.rope_dims, base=w.rope_base)
+            if w.rope else None)
+    # calibrate tokens per step on one head
+    ntok = q.shape[1]
+    t0 = time.perf_counter()
+    orc.block_forward(q[:, :, :1].contiguous(), k[:, :, :1].contiguous(), v[:, :, :1].contiguous(),
+                      orc.State(w.B, 1, w.d), rope=rope, eps=w.eps)
+    per_th = (time.perf_counter() - t0) / (w.B * ntok)
+    want = max(1, int(per_step / per_th))            # token-heads per step
+    nh = max(1, min(w.H, want // (w.B * ntok)))
+    nt = ntok if nh > 1 else max(1, min(ntok, want // w.B))
+    qs, ks, vs = (t[:, :nt, :nh].contiguous() for t in (q, k, v))
+
+    def step():
+        orc.block_forward(qs, ks, vs, orc.State(w.B, nh, w.d), rope=rope, eps=w.eps)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(total_steps):
+        step()
+    dt = time.perf_counter() - t0
+    th = w.B * nt * nh * total_steps
+    value = th / dt
+    sample = (f"each step: {w.B}x{nt} tokens of the workload's first call on {nh} of {w.H} heads, "
+              f"fp64 recurrence (block KV, state combine, apply, commit)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": total_steps, "warmup": args.warmup, "ms_per_step": 1000 * dt / total_steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w, {"l2": "n/a (CPU)"}),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": orc.get_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our arm
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+
+    from block_causal_linear_b200 import build as la_build
+
+    la_build.build()
+    from block_causal_linear_b200 import la
+    from block_causal_linear_b200.runner import Runner
+
+    base = synth.WORKLOADS[args.config]
+    w = base.shrink(seed=base.seed + 1000 * rank) if rank else base
+    dev = torch.device("cuda", local_rank)
+    runner = Runner(w, dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    n_calls = len(runner.calls)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    # warm-up (untimed)
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        runner.step()
+    torch.cuda.synchronize()
+    # steps: about 2 s of timed region unless given
+    if args.steps is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.fill_(2.0)
+        e0.record()
+        runner.step()
+        e1.record()
+        torch.cuda.synchronize()
+        est = e0.elapsed_time(e1) / 1e3 + 1e-4
+        args.steps = int(min(20000, max(20, 2.0 / est)))
+        if dist is not None:
+            t = torch.tensor([args.steps], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MIN)
+            args.steps = int(t.item())
+    K = args.steps
+
+    def ev():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()          # creates the underlying event now
+        return e
+
+    step_ev = [(ev(), ev()) for _ in range(K)]
+    stage_ev = [[tuple(ev() for _ in range(4)) for _ in range(n_calls)] for _ in range(K)]
+    torch.cuda.synchronize()
+
+    def set_stage(k, i):
+        e = stage_ev[k][i]
+        la.la_set_stage_events(*(x.cuda_event for x in e))
+
+    sampler = ClockSampler()
+    barrier()
+    torch.cuda.synchronize()
+    if rank == 0:
+        sampler.start(dev)
+        time.sleep(0.3)
+    launches = 0
+    for kk in range(K):
+        flush.fill_(float(kk))
+        step_ev[kk][0].record(stream)
+        set_stage(kk, 0)
+
+        def after(i, kk=kk):
+            if i + 1 < n_calls:
+                set_stage(kk, i + 1)
+
+        runner.step(after_call=after)
+        step_ev[kk][1].record(stream)
+        launches += runner.launches_per_step
+    la.la_set_stage_events(None, None, None, None)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop(local_rank) if rank == 0 else None
+    la.device_status()
+
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    stage_ms = [0.0, 0.0, 0.0]
+    for k in range(K):
+        for i in range(n_calls):
+            e = stage_ev[k][i]
+            for j in range(3):
+                stage_ms[j] += e[j].elapsed_time(e[j + 1])
+    total_ms = sum(step_ms)
+    tot = torch.tensor([total_ms] + stage_ms, dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
+    total_ms, red_ms, fin_ms, app_ms = (float(x) for x in tot.tolist())
+
+    th_step = w.token_heads                          # per rank per step
+    value = th_step * world * K / (total_ms / 1e3)
+    ms_per_step = total_ms / K
+    peak, peak_kind = measured_peaks()
+    step_gbs = w.alg_bytes / (ms_per_step / 1e3) / 1e9
+
+    launches_per_kernel = K * n_calls
+    # dominant kernel: the larger of reduce (reads k, v) and apply (reads q, writes out)
+    per_call_th = w.B * runner.tokens_per_call(0) * w.H
+    kern_bytes = per_call_th * 2 * w.d * w.elem_bytes
+    dom, dom_ms = ("reduce", red_ms) if red_ms >= app_ms else ("apply", app_ms)
+    avg_launch_s = dom_ms / launches_per_kernel / 1e3
+    achieved = kern_bytes / avg_launch_s / 1e9
+    path = la.la_last_path()
+    kname = f"{dom}_{path}"
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(runner, w, dev, world, dist, steps=max(3, min(20, K)))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle as orc
+
+        orc.build()
+        th, dt, desc = oracle_sample(w, 12.0, orc)
+        cpu = {"value": th / dt, "unit": UNIT, "cores": orc.get_threads(), "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+            "data": "synthetic", "config": workload_config(w, {"parallelism": f"independent problem per rank x{world}"}),
+            "achieved_hbm_gbs": step_gbs, "hbm_frac_of_" + peak_kind: step_gbs / peak,
+            "stage_ms_per_step": {"reduce": red_ms / K, "finish": fin_ms / K, "apply": app_ms / K},
+            "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": ncu_traffic(kname, per_call_th)},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "path": path, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def measure_e2e(runner, w, dev, world, dist, steps):
+    """Same metric through the public API with host buffers: every step copies
+    its inputs from pinned host memory to the device, runs the workload, and
+    copies every output back."""
+    from block_causal_linear_b200 import la  # noqa: F401
+
+    host_in = [tuple(t.cpu().pin_memory() for t in c[2:]) for c in runner.calls]
+    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in runner.outs]
+    h2d = sum(t.numel() * t.element_size() for c in host_in for t in c)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def one():
+        for (q, k, v), c in zip(host_in, runner.calls):
+            c[2].copy_(q, non_blocking=True)
+            c[3].copy_(k, non_blocking=True)
+            c[4].copy_(v, non_blocking=True)
+        runner.step()
+        for ho, o in zip(host_out, runner.outs):
+            ho.copy_(o, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    return {"value": w.token_heads * world * steps / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,241 @@
+// la_api.cu -- the C ABI of libla_b200.so (declared in include/la.h).
+//
+// Host side only: argument validation, the launch plan (split counts), the
+// workspace layout, RoPE frequency tables, and the sequence of kernel
+// launches of one call.  Every step of the computation runs in the kernels of
+// k_ffma.cu, k_finish.cu and k_tc.cu.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+
+#include "../../include/la.h"
+#include "la_internal.cuh"
+
+namespace {
+
+int g_last_launches = 0;
+const char *g_last_path = "none";
+cudaEvent_t g_ev[4] = {nullptr, nullptr, nullptr, nullptr};
+
+inline bool mark(int i, cudaStream_t s) {
+    return !g_ev[i] || cudaEventRecord(g_ev[i], s) == cudaSuccess;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
+
+// Deterministic split plan: a function of the shapes only (never of the GPU),
+// so that results are reproducible bit for bit.
+void make_splits(la::Plan &p) {
+    const long long groups = (long long)p.B * ceil_div(p.H, 4) * p.nb;
+    long long want = ceil_div(la::kTargetCtas, groups);
+    if (want < 1) want = 1;
+    long long chunk = ceil_div(ceil_div(p.L, want), la::kReduceRows) * la::kReduceRows;
+    if (chunk < la::kReduceRows) chunk = la::kReduceRows;
+    p.chunk = (int)chunk;
+    p.P = (int)ceil_div(p.L, chunk);
+
+    const long long pairs = (long long)p.B * ceil_div(p.H, 2) * p.nb;
+    long long wanta = ceil_div(la::kTargetCtas, pairs);
+    if (wanta < 1) wanta = 1;
+    long long chunka = ceil_div(ceil_div(p.L, wanta), la::kApplyRows) * la::kApplyRows;
+    if (chunka < la::kApplyRows) chunka = la::kApplyRows;
+    p.chunka = (int)chunka;
+    p.Pa = (int)ceil_div(p.L, chunka);
+}
+
+bool sizes_ok(int B, int N, int H, int d) {
+    return B > 0 && N > 0 && H > 0 && d > 0 &&
+           (long long)B * N * H * d < (1LL << 40);
+}
+
+la_status check_rope(const la_rope *r, int d, bool allow_state_offset) {
+    if (!r) return LA_OK;
+    if (r->Hg <= 0 || r->Wg <= 0 || r->T < 0) return LA_EINVAL;
+    if (r->dt < 0 || r->dh < 0 || r->dw < 0) return LA_EINVAL;
+    if ((r->dt | r->dh | r->dw) & 1) return LA_EINVAL;
+    if (r->dt + r->dh + r->dw != d) return LA_EINVAL;
+    if (!(r->base > 0.0f) || !std::isfinite(r->base)) return LA_EINVAL;
+    if (r->t_offset < 0 && !allow_state_offset) return LA_EINVAL;
+    return LA_OK;
+}
+
+// Frequencies of the 16 feature pairs, computed in double and rounded once.
+void fill_rope(la::Plan &p, const la_rope *r, int t_offset) {
+    p.rope = r != nullptr;
+    p.Hg = r ? r->Hg : 1;
+    p.Wg = r ? r->Wg : 1;
+    p.t_offset = t_offset;
+    for (int pr = 0; pr < la::kD / 2; ++pr) {
+        p.theta[pr] = 0.0f;
+        p.axis[pr] = 0;
+        if (!r) continue;
+        int f = 2 * pr, lo, D, ax;
+        if (f < r->dt) { lo = 0; D = r->dt; ax = 0; }
+        else if (f < r->dt + r->dh) { lo = r->dt; D = r->dh; ax = 1; }
+        else { lo = r->dt + r->dh; D = r->dw; ax = 2; }
+        int i = (f - lo) / 2;
+        p.theta[pr] = (float)std::pow((double)r->base, -2.0 * (double)i / (double)D);
+        p.axis[pr] = ax;
+    }
+}
+
+la_status common_checks(const void *q, const void *k, const void *v, void *out, la_dtype dt,
+                        int B, int N, int H, int d, float eps) {
+    if (!q || !k || !v || !out) return LA_EINVAL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LA_EINVAL;
+    if (dt != LA_F32 && dt != LA_BF16) return LA_EINVAL;
+    if (!sizes_ok(B, N, H, d)) return LA_EINVAL;
+    if (d != la::kD) return LA_EUNSUPPORTED;
+    if (!(eps >= 0.0f) || !std::isfinite(eps)) return LA_EINVAL;
+    return LA_OK;
+}
+
+bool use_tc(la_dtype dt, int H) {
+    return dt == LA_BF16 && (H % 4) == 0 && la::tc_available();
+}
+
+// Enqueue reduce -> finish -> apply for a prepared plan.
+la_status run(const void *q, const void *k, const void *v, void *out, la_dtype dt,
+              la::Plan &p, float *S, float *Z, void *ws, cudaStream_t s) {
+    la::WsLayout w = la::ws_layout(p.B, p.H, p.nb, p.P);
+    char *base = static_cast<char *>(ws);
+    float *partials = reinterpret_cast<float *>(base + w.partials);
+    float *seff = reinterpret_cast<float *>(base + w.seff);
+    void *bop = base + w.bop;
+    const bool tc = use_tc(dt, p.H);
+    int n = 0, r;
+
+    if (!mark(0, s)) return LA_ECUDA;
+    r = tc ? la::launch_reduce_tc(k, v, partials, p, s)
+           : la::launch_reduce_ffma(dt == LA_BF16, k, v, partials, p, s);
+    if (r < 0 || !mark(1, s)) return LA_ECUDA;
+    n += r;
+    r = la::launch_finish(partials, seff, bop, S, Z, p, tc ? 1 : 0, s);
+    if (r < 0 || !mark(2, s)) return LA_ECUDA;
+    n += r;
+    r = tc ? la::launch_apply_tc(q, out, bop, p, s)
+           : la::launch_apply_ffma(dt == LA_BF16, q, out, seff, p, s);
+    if (r < 0 || !mark(3, s)) return LA_ECUDA;
+    n += r;
+    g_last_launches = n;
+    g_last_path = tc ? "tc" : "ffma";
+    return LA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t la_workspace_size(int B, int N, int H, int d, int tokens_per_block) {
+    if (!sizes_ok(B, N, H, d) || tokens_per_block < 0) return 0;
+    la::Plan p{};
+    p.B = B; p.N = N; p.H = H;
+    p.L = tokens_per_block > 0 && tokens_per_block < N ? tokens_per_block : N;
+    p.nb = (int)ceil_div(N, p.L);
+    make_splits(p);
+    return la::ws_layout(B, H, p.nb, p.P).total;
+}
+
+la_status la_state_init(la_state *st, float *S, float *Z, int B, int H, int d, void *stream) {
+    if (!st || !S || !Z) return LA_EINVAL;
+    if (B <= 0 || H <= 0 || d <= 0) return LA_EINVAL;
+    if (d != la::kD) return LA_EUNSUPPORTED;
+    if (!aligned16(S) || !aligned16(Z)) return LA_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t nS = size_t(B) * H * d * d, nZ = size_t(B) * H * d;
+    if (cudaMemsetAsync(S, 0, nS * sizeof(float), s) != cudaSuccess) return LA_ECUDA;
+    if (cudaMemsetAsync(Z, 0, nZ * sizeof(float), s) != cudaSuccess) return LA_ECUDA;
+    st->S = S; st->Z = Z; st->B = B; st->H = H; st->d = d;
+    st->blocks_committed = 0;
+    st->t_next = 0;
+    return LA_OK;
+}
+
+la_status la_block_forward(const void *q, const void *k, const void *v, void *out, la_dtype dt,
+                           int B, int N_blk, int H, int d, la_state *st, int commit,
+                           const la_rope *rope, float eps, void *ws, size_t ws_bytes,
+                           void *stream) {
+    la_status e = common_checks(q, k, v, out, dt, B, N_blk, H, d, eps);
+    if (e != LA_OK) return e;
+    if (!st || !st->S || !st->Z) return LA_EINVAL;
+    if (st->B != B || st->H != H || st->d != d) return LA_EINVAL;
+    if ((e = check_rope(rope, d, true)) != LA_OK) return e;
+    const size_t need = la_workspace_size(B, N_blk, H, d, N_blk);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return LA_EWORKSPACE;
+
+    la::Plan p{};
+    p.B = B; p.N = N_blk; p.H = H; p.L = N_blk; p.nb = 1;
+    p.commit = commit != 0;
+    p.has_state = 1;
+    p.eps = eps;
+    make_splits(p);
+    fill_rope(p, rope, rope ? (rope->t_offset < 0 ? st->t_next : rope->t_offset) : 0);
+    e = run(q, k, v, out, dt, p, st->S, st->Z, ws, static_cast<cudaStream_t>(stream));
+    if (e != LA_OK) return e;
+    if (commit) {
+        st->blocks_committed += 1;
+        if (rope) st->t_next += rope->T;
+    }
+    return LA_OK;
+}
+
+la_status la_full_forward(const void *q, const void *k, const void *v, void *out, la_dtype dt,
+                          int B, int N, int H, int d, int tokens_per_block,
+                          const la_rope *rope, float eps, void *ws, size_t ws_bytes,
+                          void *stream) {
+    la_status e = common_checks(q, k, v, out, dt, B, N, H, d, eps);
+    if (e != LA_OK) return e;
+    if (tokens_per_block < 0) return LA_EINVAL;
+    if ((e = check_rope(rope, d, false)) != LA_OK) return e;
+    const size_t need = la_workspace_size(B, N, H, d, tokens_per_block);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return LA_EWORKSPACE;
+
+    la::Plan p{};
+    p.B = B; p.N = N; p.H = H;
+    p.L = tokens_per_block > 0 && tokens_per_block < N ? tokens_per_block : N;
+    p.nb = (int)ceil_div(N, p.L);
+    p.commit = 0;
+    p.has_state = 0;
+    p.eps = eps;
+    make_splits(p);
+    fill_rope(p, rope, rope ? rope->t_offset : 0);
+    return run(q, k, v, out, dt, p, nullptr, nullptr, ws, static_cast<cudaStream_t>(stream));
+}
+
+la_status la_device_status(void *stream) {
+    unsigned flag = 0;
+    if (la::read_and_clear_device_flag(static_cast<cudaStream_t>(stream), &flag) != 0)
+        return LA_ECUDA;
+    return flag ? LA_ETIMEOUT : LA_OK;
+}
+
+const char *la_status_string(la_status s) {
+    switch (s) {
+        case LA_OK: return "LA_OK";
+        case LA_EINVAL: return "LA_EINVAL: invalid argument";
+        case LA_EUNSUPPORTED: return "LA_EUNSUPPORTED: unsupported shape (d must be 32)";
+        case LA_ECUDA: return "LA_ECUDA: CUDA call or kernel launch failed";
+        case LA_ETIMEOUT: return "LA_ETIMEOUT: a device-side bounded wait gave up";
+        case LA_EWORKSPACE: return "LA_EWORKSPACE: workspace missing, misaligned or too small";
+    }
+    return "LA_?: unknown status";
+}
+
+void la_set_stage_events(void *before_reduce, void *after_reduce, void *after_finish,
+                         void *after_apply) {
+    g_ev[0] = static_cast<cudaEvent_t>(before_reduce);
+    g_ev[1] = static_cast<cudaEvent_t>(after_reduce);
+    g_ev[2] = static_cast<cudaEvent_t>(after_finish);
+    g_ev[3] = static_cast<cudaEvent_t>(after_apply);
+}
+
+int la_last_launch_count(void) { return g_last_launches; }
+
+int la_tc_enabled(void) { return la::tc_available() ? 1 : 0; }
+
+const char *la_last_path(void) { return g_last_path; }
+
+}  // extern "C"

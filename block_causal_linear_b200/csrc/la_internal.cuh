@@ -1,0 +1,84 @@
+// la_internal.cuh -- shared host/device declarations of libla_b200.so.
+//
+// The launch plan, the workspace layout and the kernel launchers that
+// la_api.cu calls.  Nothing here is part of the public ABI (include/la.h).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace la {
+
+constexpr int kD = 32;                 // head dim supported by this build
+constexpr int kKVZ = kD * kD + kD;     // floats per (b, h) of [KV | z]: KV[dk][dv] then z[dk]
+constexpr int kTargetCtas = 296;       // 2 resident CTAs on each of the 148 SMs of a B200
+constexpr int kReduceRows = 64;        // token rows per reduce pipeline stage
+constexpr int kApplyRows = 128;        // token rows per apply tile (= MMA M)
+constexpr int kOpRows = 48;            // N of the apply MMA: 32 S columns, Z, 15 zero rows
+constexpr int kOpBytes = kOpRows * kD * 2;   // one bf16 operand (hi or lo) = 3072 B
+
+// Everything a kernel needs to know about one call, passed by value.
+struct Plan {
+    int B, N, H;          // batch, tokens in the call, heads
+    int L;                // tokens per block (the last block may be shorter)
+    int nb;               // number of blocks in the call
+    int P;                // reduce splits per (b, h, block)
+    int chunk;            // tokens per reduce split (multiple of kReduceRows)
+    int Pa;               // apply splits per (b, head pair, block)
+    int chunka;           // tokens per apply split (multiple of kApplyRows)
+    int commit;           // write S_eff of the last block back to the state
+    int has_state;        // S, Z hold a prior state (block_forward) or not (full_forward)
+    int rope;             // numerator RoPE on phi(q), phi(k)
+    int Hg, Wg;           // latent grid of one frame
+    int t_offset;         // frame of token 0 of the call
+    float eps;
+    float theta[kD / 2];  // RoPE frequency of feature pair p
+    int axis[kD / 2];     // 0: frame, 1: row, 2: column
+};
+
+// Workspace layout (byte offsets from the 256-byte aligned base).
+struct WsLayout {
+    size_t partials;      // float [B][H][nb][P][kKVZ]
+    size_t seff;          // float [B][H][nb][kKVZ]  effective state S + sum of KV, Z + sum of z
+    size_t bop;           // bf16  [B][H][nb][2][kOpRows][kD] packed MMA operand (hi, lo)
+    size_t total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline WsLayout ws_layout(int B, int H, int nb, int P) {
+    WsLayout w;
+    size_t bhn = size_t(B) * H * nb;
+    w.partials = 0;
+    w.seff = align256(w.partials + bhn * P * kKVZ * sizeof(float));
+    w.bop = align256(w.seff + bhn * kKVZ * sizeof(float));
+    w.total = align256(w.bop + bhn * 2 * size_t(kOpBytes));
+    return w;
+}
+
+// ---------------------------------------------------------------- launchers
+// Each returns the number of kernels enqueued (>= 0) or -1 on a launch error.
+
+// fp32/bf16 CUDA-core path (any H).  T is float or __nv_bfloat16.
+int launch_reduce_ffma(int is_bf16, const void *k, const void *v, float *partials,
+                       const Plan &p, cudaStream_t s);
+int launch_apply_ffma(int is_bf16, const void *q, void *out, const float *seff,
+                      const Plan &p, cudaStream_t s);
+
+// Fixed-order sum of the split partials, prefix over blocks, + prior state;
+// writes S_eff (fp32), the packed bf16 hi/lo tensor-core operand, and on
+// commit the state.
+int launch_finish(const float *partials, float *seff, void *bop, float *S, float *Z,
+                  const Plan &p, int write_bop, cudaStream_t s);
+
+// Tensor-core path (bf16, H % 4 == 0): tcgen05 MMAs, TMA tiles.
+int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &p,
+                     cudaStream_t s);
+int launch_apply_tc(const void *q, void *out, const void *bop, const Plan &p, cudaStream_t s);
+bool tc_available();
+
+// Device flag raised by a bounded wait that gave up; read-and-clear.
+int read_and_clear_device_flag(cudaStream_t s, unsigned *flag_out);
+
+}  // namespace la

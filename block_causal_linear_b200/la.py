@@ -1,0 +1,233 @@
+"""ctypes binding of libla_b200.so (the C ABI in include/la.h).
+
+Argument marshalling only: every step of the computation runs in the
+library's CUDA kernels.  The raw entry points keep their C names
+(``la_workspace_size``, ``la_state_init``, ``la_block_forward``,
+``la_full_forward``, ``la_device_status``, ``la_status_string``); the
+lower-case wrappers below take torch CUDA tensors, pass their device pointers
+and the current CUDA stream, and raise ``LAError`` on a non-zero status.
+
+There is no fallback: if the library is missing or a call fails, this module
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libla_b200.so")
+
+LA_OK, LA_EINVAL, LA_EUNSUPPORTED, LA_ECUDA, LA_ETIMEOUT, LA_EWORKSPACE = range(6)
+LA_F32, LA_BF16 = 0, 1
+
+
+class LAError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {la_status_string(status)}" if what else la_status_string(status))
+
+
+class la_rope(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int), ("Hg", ctypes.c_int), ("Wg", ctypes.c_int),
+                ("t_offset", ctypes.c_int), ("dt", ctypes.c_int), ("dh", ctypes.c_int),
+                ("dw", ctypes.c_int), ("base", ctypes.c_float)]
+
+
+class la_state(ctypes.Structure):
+    _fields_ = [("S", ctypes.c_void_p), ("Z", ctypes.c_void_p), ("B", ctypes.c_int),
+                ("H", ctypes.c_int), ("d", ctypes.c_int), ("blocks_committed", ctypes.c_longlong),
+                ("t_next", ctypes.c_int)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libla_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m block_causal_linear_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, ip, fp, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.la_workspace_size.argtypes = [ip, ip, ip, ip, ip]
+        L.la_workspace_size.restype = sz
+        L.la_state_init.argtypes = [ctypes.POINTER(la_state), vp, vp, ip, ip, ip, vp]
+        L.la_state_init.restype = ip
+        L.la_block_forward.argtypes = [vp, vp, vp, vp, ip, ip, ip, ip, ip, ctypes.POINTER(la_state), ip,
+                                       ctypes.POINTER(la_rope), fp, vp, sz, vp]
+        L.la_block_forward.restype = ip
+        L.la_full_forward.argtypes = [vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, ctypes.POINTER(la_rope),
+                                      fp, vp, sz, vp]
+        L.la_full_forward.restype = ip
+        L.la_device_status.argtypes = [vp]
+        L.la_device_status.restype = ip
+        L.la_status_string.argtypes = [ip]
+        L.la_status_string.restype = ctypes.c_char_p
+        L.la_set_stage_events.argtypes = [vp, vp, vp, vp]
+        L.la_set_stage_events.restype = None
+        L.la_last_launch_count.argtypes = []
+        L.la_last_launch_count.restype = ip
+        L.la_tc_enabled.argtypes = []
+        L.la_tc_enabled.restype = ip
+        L.la_last_path.argtypes = []
+        L.la_last_path.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------- raw C names
+
+def la_workspace_size(B, N, H, d, tokens_per_block) -> int:
+    return int(lib().la_workspace_size(B, N, H, d, tokens_per_block))
+
+
+def la_state_init(st, S, Z, B, H, d, stream) -> int:
+    return int(lib().la_state_init(ctypes.byref(st), S, Z, B, H, d, stream))
+
+
+def la_block_forward(q, k, v, out, dt, B, N_blk, H, d, st, commit, rope, eps, ws, ws_bytes, stream) -> int:
+    return int(lib().la_block_forward(q, k, v, out, dt, B, N_blk, H, d, ctypes.byref(st), commit,
+                                      ctypes.byref(rope) if rope is not None else None, eps, ws,
+                                      ws_bytes, stream))
+
+
+def la_full_forward(q, k, v, out, dt, B, N, H, d, tokens_per_block, rope, eps, ws, ws_bytes, stream) -> int:
+    return int(lib().la_full_forward(q, k, v, out, dt, B, N, H, d, tokens_per_block,
+                                     ctypes.byref(rope) if rope is not None else None, eps, ws,
+                                     ws_bytes, stream))
+
+
+def la_device_status(stream) -> int:
+    return int(lib().la_device_status(stream))
+
+
+def la_status_string(status: int) -> str:
+    return lib().la_status_string(int(status)).decode()
+
+
+def la_set_stage_events(before_reduce, after_reduce, after_finish, after_apply) -> None:
+    lib().la_set_stage_events(before_reduce, after_reduce, after_finish, after_apply)
+
+
+def la_last_launch_count() -> int:
+    return int(lib().la_last_launch_count())
+
+
+def la_last_path() -> str:
+    return lib().la_last_path().decode()
+
+
+def tc_enabled() -> bool:
+    """Whether this build routes bf16 (H % 4 == 0) through the tensor-core kernels."""
+    return bool(lib().la_tc_enabled())
+
+
+# ---------------------------------------------------------------- torch wrappers
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return LA_F32
+    if t.dtype == torch.bfloat16:
+        return LA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _check_qkv(q, k, v):
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("q, k, v must be contiguous CUDA tensors [B, N, H, d]")
+    if not (q.shape == k.shape == v.shape and q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must agree in shape and dtype")
+
+
+def make_rope(Hg, Wg, T=0, t_offset=0, dims=(8, 12, 12), base=10000.0) -> la_rope:
+    return la_rope(int(T), int(Hg), int(Wg), int(t_offset), int(dims[0]), int(dims[1]), int(dims[2]),
+                   float(base))
+
+
+def workspace_bytes(B, N, H, d=32, tokens_per_block=0) -> int:
+    n = la_workspace_size(B, N, H, d, tokens_per_block)
+    if n == 0:
+        raise LAError(LA_EINVAL, "la_workspace_size")
+    return n
+
+
+def alloc_workspace(B, N, H, d=32, tokens_per_block=0, device=None) -> torch.Tensor:
+    """A uint8 CUDA tensor of la_workspace_size bytes (torch allocations are
+    256-byte aligned)."""
+    return torch.empty(workspace_bytes(B, N, H, d, tokens_per_block), dtype=torch.uint8,
+                       device=device or "cuda")
+
+
+class State:
+    """The constant-memory state: S [B,H,d,d] and Z [B,H,d] fp32 CUDA tensors
+    bound to a C ``la_state``."""
+
+    def __init__(self, B, H, d=32, device=None, stream=None):
+        dev = device or "cuda"
+        self.S = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
+        self.Z = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+        self.c = la_state()
+        rc = la_state_init(self.c, self.S.data_ptr(), self.Z.data_ptr(), B, H, d, _stream_ptr(stream))
+        if rc != LA_OK:
+            raise LAError(rc, "la_state_init")
+
+    @property
+    def blocks_committed(self) -> int:
+        return int(self.c.blocks_committed)
+
+    @property
+    def t_next(self) -> int:
+        return int(self.c.t_next)
+
+    def nbytes(self) -> int:
+        return self.S.numel() * 4 + self.Z.numel() * 4
+
+
+def block_forward(q, k, v, state: State, commit=True, rope: Optional[la_rope] = None, eps=1e-6,
+                  ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None, stream=None):
+    _check_qkv(q, k, v)
+    B, N, H, d = q.shape
+    if ws is None:
+        ws = alloc_workspace(B, N, H, d, N, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    rc = la_block_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _dtype_code(q),
+                          B, N, H, d, state.c, int(bool(commit)), rope, float(eps), ws.data_ptr(),
+                          ws.numel() * ws.element_size(), _stream_ptr(stream))
+    if rc != LA_OK:
+        raise LAError(rc, "la_block_forward")
+    return out
+
+
+def full_forward(q, k, v, tokens_per_block=0, rope: Optional[la_rope] = None, eps=1e-6,
+                 ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None, stream=None):
+    _check_qkv(q, k, v)
+    B, N, H, d = q.shape
+    if ws is None:
+        ws = alloc_workspace(B, N, H, d, tokens_per_block, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    rc = la_full_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _dtype_code(q),
+                         B, N, H, d, int(tokens_per_block), rope, float(eps), ws.data_ptr(),
+                         ws.numel() * ws.element_size(), _stream_ptr(stream))
+    if rc != LA_OK:
+        raise LAError(rc, "la_full_forward")
+    return out
+
+
+def device_status(stream=None) -> None:
+    rc = la_device_status(_stream_ptr(stream))
+    if rc != LA_OK:
+        raise LAError(rc, "la_device_status")

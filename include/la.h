@@ -1,0 +1,189 @@
+/*
+ * la.h -- C ABI of libla_b200.so: block-causal linear attention with a
+ * constant-memory fp32 state, on NVIDIA B200 (sm_100a).
+ *
+ * The operation (sources cited by page title and section):
+ *   - "Nvidia, MIT ve diğerleri video yapay zeka devrimini başlattı"
+ *     (aihaber.org), section "Sabit Bellekli KV önbelleğe alma mekanizması":
+ *     a video is cut into blocks; later blocks see earlier ones through linear
+ *     attention, never the reverse; the KV products of the blocks are summed
+ *     (KV_{1-2} = KV_1 + KV_2, ...) into a cache of fixed size; each block
+ *     needs only that sum plus its own KV.
+ *   - sd114.wiki SANA-Video summary, section "两大核心技术突破": item 1, linear
+ *     attention as a kernel feature map plus global aggregation, with RoPE for
+ *     spatio-temporal position; item 2, chunk-wise linear attention whose only
+ *     context is one cumulative state, constant in memory.
+ *   - "SANA-Video: Efficient Video Generation with Block Linear Diffusion
+ *     Transformer" (chatpaper.ai abstract), design (2): the constant-memory
+ *     state replaces a growing KV cache.
+ *
+ * Per batch element b and head h, with phi = ReLU applied elementwise:
+ *   KV_n = sum_{t in block n} psi(k_t)^T v_t      (d x d, fp32)
+ *   z_n  = sum_{t in block n} phi(k_t)            (d, fp32)
+ *   out_t = psi(q_t) (S + KV_n) / ( phi(q_t) . (Z + z_n) + eps )   for t in block n
+ * where S, Z are the sums over earlier blocks.  psi = phi, or with RoPE
+ * psi = R(position) o phi in the numerator only.
+ *
+ * Conventions for every entry point
+ *   - Tensors q, k, v, out are DEVICE pointers, row-major [B][N][H][d] with d
+ *     fastest, element type given by la_dtype (out has the input type; bf16 out
+ *     is rounded to nearest even from fp32).  Base addresses must be 16-byte
+ *     aligned.  d must be 32.
+ *   - The caller owns every buffer (q, k, v, out, S, Z, workspace) and keeps it
+ *     alive until the enqueued work has finished.  The library allocates no
+ *     device memory and never synchronises; all work is enqueued on `stream`
+ *     (a cudaStream_t passed as void*, NULL = legacy default stream).
+ *   - Validation is synchronous and happens before anything is enqueued; an
+ *     error status means nothing was enqueued.  No C++ exception crosses the ABI.
+ *   - Results are deterministic: identical inputs and shapes on the same GPU
+ *     model give bitwise-identical out, S and Z (fixed reduction order, no
+ *     floating-point atomics).
+ *   - Inputs must be finite.
+ */
+#ifndef LA_B200_LA_H
+#define LA_B200_LA_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define LA_API __attribute__((visibility("default")))
+#else
+#define LA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LA_OK = 0,
+    LA_EINVAL = 1,        /* null pointer, bad size, misaligned pointer, bad RoPE */
+    LA_EUNSUPPORTED = 2,  /* d != 32, or a shape this build does not handle */
+    LA_ECUDA = 3,         /* a CUDA call or kernel launch failed */
+    LA_ETIMEOUT = 4,      /* a device-side bounded wait gave up (la_device_status) */
+    LA_EWORKSPACE = 5     /* workspace null or smaller than la_workspace_size() */
+} la_status;
+
+typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
+
+/*
+ * 3D rotary position embedding (RoPE) on phi(q), phi(k) in the numerator.
+ * The d features are cut into sections of dt, dh, dw dims (each even, sum d)
+ * for the latent frame, row and column.  Inside a section of D dims, features
+ * (2i, 2i+1) rotate by angle pos * base^(-2i/D):
+ *   x'_{2i} = x_{2i} cos - x_{2i+1} sin,   x'_{2i+1} = x_{2i} sin + x_{2i+1} cos.
+ * Token j of a call (0-based, in token order) sits at frame t_offset + j/(Hg*Wg),
+ * row (j % (Hg*Wg)) / Wg, column j % Wg.  The pages name RoPE but fix neither
+ * pairing, sections nor frequencies; this is the library's stated reading.
+ */
+typedef struct {
+    int T;          /* latent frames per block: la_block_forward with commit advances
+                       state->t_next by T */
+    int Hg, Wg;     /* latent rows and columns per frame, > 0 */
+    int t_offset;   /* frame of token 0 of the call; < 0 in la_block_forward means
+                       "use state->t_next" */
+    int dt, dh, dw; /* section dims, even, dt + dh + dw == d */
+    float base;     /* frequency base, > 0 (10000 in SANA-style 3D RoPE) */
+} la_rope;
+
+/*
+ * The constant-memory state of the streaming method: per (b, h) the running
+ * S = sum KV_i (d x d) and Z = sum z_i (d) over committed blocks, fp32.
+ * S and Z are caller-owned DEVICE buffers of B*H*d*d and B*H*d floats,
+ * layout S[b][h][row = key feature][column = value feature], Z[b][h][feature].
+ * Their size never depends on how many blocks have been committed.
+ * blocks_committed and t_next are host-side counters kept by the library.
+ * Saving and restoring S, Z and the two counters checkpoints the stream.
+ */
+typedef struct {
+    float *S;
+    float *Z;
+    int B, H, d;
+    long long blocks_committed;
+    int t_next;
+} la_state;
+
+/*
+ * Bytes of caller-provided device workspace that la_full_forward needs for
+ * these sizes (tokens_per_block 0 = one block of N tokens), and that
+ * la_block_forward needs with N = tokens_per_block = N_blk.  Pure host
+ * function, no CUDA call.  Returns 0 for invalid sizes.  The workspace holds
+ * the split partial sums, the per-block effective state and the packed
+ * tensor-core operand; its size never depends on how many blocks were
+ * streamed before.  Its base must be 256-byte aligned.
+ */
+LA_API size_t la_workspace_size(int B, int N, int H, int d, int tokens_per_block);
+
+/*
+ * Bind the caller's S, Z buffers to *st, zero them (cudaMemsetAsync on
+ * `stream`) and reset blocks_committed and t_next to 0.
+ */
+LA_API la_status la_state_init(la_state *st, float *S, float *Z, int B, int H, int d, void *stream);
+
+/*
+ * One block of the streaming method ("each block computes only KVsum plus its
+ * own KV"): for the N_blk tokens of this block,
+ *   S_eff = S + KV_n,  Z_eff = Z + z_n,  out = psi(q) S_eff / (phi(q).Z_eff + eps),
+ * every token of the block attending to every other token of it
+ * (bidirectional inside the block) and to all committed blocks.
+ * commit != 0: S <- S_eff, Z <- Z_eff on the device, blocks_committed += 1,
+ *   t_next += rope ? rope->T : 0.
+ * commit == 0: a read-only pass (e.g. a denoising step before the last); S, Z
+ *   stay bitwise unchanged.
+ * rope may be NULL.  st must have been set up by la_state_init with the same
+ * B, H, d.  ws must hold la_workspace_size(B, N_blk, H, d, N_blk) bytes.
+ */
+LA_API la_status la_block_forward(const void *q, const void *k, const void *v, void *out, la_dtype dt,
+                           int B, int N_blk, int H, int d, la_state *st, int commit,
+                           const la_rope *rope, float eps, void *ws, size_t ws_bytes,
+                           void *stream);
+
+/*
+ * The whole sequence from a zero state in one call: blocks of tokens_per_block
+ * tokens (0 = a single bidirectional block of all N tokens; the last block may
+ * be shorter), block n seeing blocks 0..n.  Equal to la_state_init followed by
+ * la_block_forward(commit=1) on each block, up to the order of fp32 sums.
+ * rope may be NULL; positions run over the whole sequence (t_offset >= 0).
+ * ws must hold la_workspace_size(B, N, H, d, tokens_per_block) bytes.
+ */
+LA_API la_status la_full_forward(const void *q, const void *k, const void *v, void *out, la_dtype dt,
+                          int B, int N, int H, int d, int tokens_per_block,
+                          const la_rope *rope, float eps, void *ws, size_t ws_bytes,
+                          void *stream);
+
+/*
+ * Device-side status of the kernels enqueued so far on this device: every
+ * wait inside a kernel is bounded; one that gives up records the fact in a
+ * device flag and the kernel returns early.  This call synchronises `stream`,
+ * reads and clears the flag, and returns LA_ETIMEOUT if it was set, LA_ECUDA
+ * on a CUDA error, else LA_OK.
+ */
+LA_API la_status la_device_status(void *stream);
+
+/* Static, human-readable name of a status. */
+LA_API const char *la_status_string(la_status s);
+
+/*
+ * Measurement hook.  When set (non-NULL cudaEvent_t handles passed as void*,
+ * created on the current device), every following forward call records
+ * before_reduce before its first kernel, after_reduce after the state
+ * reduction, after_finish after the state combine and after_apply after its
+ * last kernel, all on its stream.  Pass four NULLs to stop.  Process-global;
+ * not thread-safe.  Changes no result.
+ */
+LA_API void la_set_stage_events(void *before_reduce, void *after_reduce, void *after_finish,
+                                void *after_apply);
+
+/* Number of kernels the last successful forward call enqueued (for launch
+ * accounting), and a short name of the path it took ("tc" or "ffma"). */
+LA_API int la_last_launch_count(void);
+/* 1 if this build routes bf16 inputs with H % 4 == 0 through the tensor-core
+ * (tcgen05) kernels, 0 if every shape takes the CUDA-core kernels. */
+LA_API int la_tc_enabled(void);
+LA_API const char *la_last_path(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA_B200_LA_H */

@@ -1,0 +1,116 @@
+"""The C ABI without a GPU: the library loads, exports every entry point that
+include/la.h declares, sizes its workspace on the host, and rejects bad
+arguments before enqueuing anything (so no call here reaches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_causal_linear_b200 import build as la_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def la():
+    la_build.build()
+    from block_causal_linear_b200 import la as _la
+
+    return _la
+
+
+def declared_symbols():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"LA_API\s+[\w\s\*]+?\b(la_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for n in ("la_state_init", "la_block_forward", "la_full_forward", "la_workspace_size",
+              "la_status_string", "la_device_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(la):
+    lib = la.lib()
+    for n in declared_symbols():
+        assert hasattr(lib, n), n
+        assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
+
+
+def test_status_strings(la):
+    for s in range(6):
+        assert la.la_status_string(s).startswith("LA_")
+    assert "unknown" in la.la_status_string(99)
+
+
+def test_workspace_size_host_only(la):
+    a = la.la_workspace_size(1, 8190, 64, 32, 0)
+    assert a > 0 and a % 256 == 0
+    # invalid sizes
+    assert la.la_workspace_size(0, 10, 1, 32, 0) == 0
+    assert la.la_workspace_size(1, 0, 1, 32, 0) == 0
+    assert la.la_workspace_size(1, 10, 1, 32, -1) == 0
+    # the workspace of a streaming block does not grow with the number of blocks
+    # already streamed (it only depends on this block's shape)
+    blk = la.la_workspace_size(1, 15600, 64, 32, 15600)
+    assert blk == la.la_workspace_size(1, 15600, 64, 32, 0)
+    # many blocks in one call need one effective state per block
+    assert la.la_workspace_size(1, 24 * 15600, 64, 32, 15600) > blk
+
+
+FAKE = 1 << 20    # never dereferenced: every call below fails validation first
+
+
+def _full(la, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, dt=la.LA_BF16, B=1, N=256, H=4, d=32, tpb=0,
+             rope=None, eps=1e-6, ws=FAKE, ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return la.la_full_forward(a["q"], a["k"], a["v"], a["out"], a["dt"], a["B"], a["N"], a["H"], a["d"],
+                              a["tpb"], a["rope"], a["eps"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+def test_full_forward_validation(la):
+    assert _full(la, q=None) == la.LA_EINVAL
+    assert _full(la, out=FAKE + 8) == la.LA_EINVAL              # misaligned
+    assert _full(la, d=16) == la.LA_EUNSUPPORTED
+    assert _full(la, d=64) == la.LA_EUNSUPPORTED
+    assert _full(la, N=0) == la.LA_EINVAL
+    assert _full(la, B=-1) == la.LA_EINVAL
+    assert _full(la, dt=7) == la.LA_EINVAL
+    assert _full(la, eps=float("nan")) == la.LA_EINVAL
+    assert _full(la, eps=-1.0) == la.LA_EINVAL
+    assert _full(la, tpb=-3) == la.LA_EINVAL
+    assert _full(la, ws=None) == la.LA_EWORKSPACE
+    assert _full(la, ws_bytes=16) == la.LA_EWORKSPACE
+    assert _full(la, ws=FAKE + 16) == la.LA_EWORKSPACE        # not 256-byte aligned
+    bad = la.make_rope(Hg=2, Wg=2, dims=(8, 12, 10))            # sections do not sum to d
+    assert _full(la, rope=bad) == la.LA_EINVAL
+    odd = la.make_rope(Hg=2, Wg=2, dims=(7, 13, 12))
+    assert _full(la, rope=odd) == la.LA_EINVAL
+    neg = la.make_rope(Hg=2, Wg=2, t_offset=-1)                 # only block_forward may defer t
+    assert _full(la, rope=neg) == la.LA_EINVAL
+    zero = la.make_rope(Hg=0, Wg=2)
+    assert _full(la, rope=zero) == la.LA_EINVAL
+
+
+def test_block_forward_and_state_validation(la):
+    st = la.la_state()
+    assert la.la_state_init(st, None, FAKE, 1, 4, 32, None) == la.LA_EINVAL
+    assert la.la_state_init(st, FAKE, FAKE, 1, 4, 16, None) == la.LA_EUNSUPPORTED
+    # a state that was never bound
+    assert la.la_block_forward(FAKE, FAKE, FAKE, FAKE, la.LA_BF16, 1, 64, 4, 32, st, 1, None, 1e-6,
+                               FAKE, 1 << 30, None) == la.LA_EINVAL
+    # a state bound to other sizes
+    st.S, st.Z, st.B, st.H, st.d = FAKE, FAKE, 1, 8, 32
+    assert la.la_block_forward(FAKE, FAKE, FAKE, FAKE, la.LA_BF16, 1, 64, 4, 32, st, 1, None, 1e-6,
+                               FAKE, 1 << 30, None) == la.LA_EINVAL
+    st.H = 4
+    assert la.la_block_forward(FAKE, FAKE, FAKE, FAKE, la.LA_BF16, 1, 64, 4, 32, st, 1, None, 1e-6,
+                               FAKE, 8, None) == la.LA_EWORKSPACE
+    assert st.blocks_committed == 0

@@ -1,0 +1,50 @@
+"""Error metrics and tolerances of the parity tests (the oracle is fp64).
+
+fp32 path:  max_i |g_i - o_i| / max(|o_i|, 1e-2 * RMS(o)) <= 1e-4
+            (relative error per element; the floor keeps outputs near zero
+            from dividing by almost nothing)
+bf16 path:  max_i |g_i - o_i| / RMS(o) <= 2e-2
+state:      max |S_gpu - S_oracle| / max |S_oracle| <= 1e-5
+"""
+import numpy as np
+import torch
+
+TOL_F32 = 1e-4
+TOL_BF16 = 2e-2
+TOL_STATE = 1e-5
+
+
+def as_np(x):
+    if isinstance(x, torch.Tensor):
+        return x.detach().to("cpu", torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def err_f32(g, o):
+    g, o = as_np(g), as_np(o)
+    rms = float(np.sqrt(np.mean(o * o))) if o.size else 0.0
+    den = np.maximum(np.abs(o), 1e-2 * rms)
+    den = np.where(den > 0, den, 1.0)
+    return float(np.max(np.abs(g - o) / den)) if o.size else 0.0
+
+
+def err_bf16(g, o):
+    g, o = as_np(g), as_np(o)
+    rms = float(np.sqrt(np.mean(o * o))) if o.size else 0.0
+    if rms == 0.0:
+        return float(np.max(np.abs(g - o))) if o.size else 0.0
+    return float(np.max(np.abs(g - o)) / rms)
+
+
+def err_out(g, o, dtype):
+    return err_f32(g, o) if dtype == torch.float32 else err_bf16(g, o)
+
+
+def tol_out(dtype):
+    return TOL_F32 if dtype == torch.float32 else TOL_BF16
+
+
+def err_state(g, o):
+    g, o = as_np(g), as_np(o)
+    m = float(np.max(np.abs(o)))
+    return float(np.max(np.abs(g - o))) / (m if m > 0 else 1.0)
