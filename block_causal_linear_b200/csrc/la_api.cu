@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "../../include/la.h"
@@ -239,3 +240,45 @@ int la_tc_enabled(void) { return la::tc_available() ? 1 : 0; }
 const char *la_last_path(void) { return g_last_path; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- static scratch
+// la_full_forward_static_ws: la_full_forward with its workspace in a file-scope
+// device array, for callers that cannot allocate.  In host code the array's
+// name only stands for the symbol; its device address comes from
+// cudaGetSymbolAddress, once per device, with that device current.
+static __device__ __align__(256) unsigned char g_la_static_ws[LA_STATIC_WS_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 128;
+void *g_static_ws_ptr[kMaxDevices] = {};
+std::mutex g_static_ws_mutex;
+
+la_status static_ws_for_current_device(void **out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LA_ECUDA;
+    std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+    if (!g_static_ws_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_la_static_ws) != cudaSuccess || !p) return LA_ECUDA;
+        g_static_ws_ptr[dev] = p;
+    }
+    *out = g_static_ws_ptr[dev];
+    return LA_OK;
+}
+}  // namespace
+
+extern "C" la_status la_full_forward_static_ws(const void *q, const void *k, const void *v, void *out,
+                                               la_dtype dt, int B, int N, int H, int d,
+                                               int tokens_per_block, const la_rope *rope, float eps,
+                                               void *stream) {
+    la_status e = common_checks(q, k, v, out, dt, B, N, H, d, eps);
+    if (e != LA_OK) return e;
+    if (tokens_per_block < 0) return LA_EINVAL;
+    if ((e = check_rope(rope, d, false)) != LA_OK) return e;
+    const size_t need = la_workspace_size(B, N, H, d, tokens_per_block);
+    if (need == 0 || need > LA_STATIC_WS_BYTES) return LA_EWORKSPACE;
+    void *ws = nullptr;
+    if ((e = static_ws_for_current_device(&ws)) != LA_OK) return e;
+    return la_full_forward(q, k, v, out, dt, B, N, H, d, tokens_per_block, rope, eps, ws,
+                           LA_STATIC_WS_BYTES, stream);
+}

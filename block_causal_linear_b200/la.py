@@ -65,6 +65,9 @@ def lib() -> ctypes.CDLL:
         L.la_full_forward.argtypes = [vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, ctypes.POINTER(la_rope),
                                       fp, vp, sz, vp]
         L.la_full_forward.restype = ip
+        L.la_full_forward_static_ws.argtypes = [vp, vp, vp, vp, ip, ip, ip, ip, ip, ip,
+                                                ctypes.POINTER(la_rope), fp, vp]
+        L.la_full_forward_static_ws.restype = ip
         L.la_device_status.argtypes = [vp]
         L.la_device_status.restype = ip
         L.la_status_string.argtypes = [ip]
@@ -101,6 +104,17 @@ def la_full_forward(q, k, v, out, dt, B, N, H, d, tokens_per_block, rope, eps, w
     return int(lib().la_full_forward(q, k, v, out, dt, B, N, H, d, tokens_per_block,
                                      ctypes.byref(rope) if rope is not None else None, eps, ws,
                                      ws_bytes, stream))
+
+
+def la_full_forward_static_ws(q, k, v, out, dt, B, N, H, d, tokens_per_block, rope, eps, stream) -> int:
+    """la_full_forward with the library's static device scratch (for callers
+    that cannot allocate; see include/la.h)."""
+    return int(lib().la_full_forward_static_ws(q, k, v, out, dt, B, N, H, d, tokens_per_block,
+                                               ctypes.byref(rope) if rope is not None else None,
+                                               eps, stream))
+
+
+LA_STATIC_WS_BYTES = 16 << 20
 
 
 def la_device_status(stream) -> int:

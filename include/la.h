@@ -152,6 +152,35 @@ LA_API la_status la_full_forward(const void *q, const void *k, const void *v, vo
                           void *stream);
 
 /*
+ * For callers that cannot allocate device memory at all.  Some code that
+ * calls this library runs inside a host framework that owns every device
+ * allocation and gives a plug-in no allocator and no way to size or keep a
+ * workspace between calls (a video pipeline or inference-server plug-in on a
+ * fixed memory budget, for example).  This variant of la_full_forward needs
+ * no workspace argument: its scratch (the split partial sums, the effective
+ * state and the packed tensor-core operand) lives in a static device array of
+ * LA_STATIC_WS_BYTES bytes that the library defines at file scope.  Every GPU
+ * that loads the library holds that array until the process exits.  The
+ * pages have no counterpart of this entry point.
+ *
+ * Arguments and results are those of la_full_forward without ws/ws_bytes.
+ * Shapes whose la_workspace_size() exceeds LA_STATIC_WS_BYTES are rejected
+ * with LA_EWORKSPACE before anything is enqueued.  The call allocates nothing
+ * (no cudaMalloc, no cudaFree, no allocating library routine).  The first call
+ * on each device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current); make that first call before any stream capture.
+ * All calls on a device share the one array and it keeps the last call's
+ * contents; each call writes every scratch byte it reads, so nothing needs to
+ * start at zero, but calls whose work overlaps on the GPU (different streams,
+ * no ordering between them) race on the array and give wrong results.
+ */
+#define LA_STATIC_WS_BYTES (16u << 20)
+LA_API la_status la_full_forward_static_ws(const void *q, const void *k, const void *v, void *out,
+                                           la_dtype dt, int B, int N, int H, int d,
+                                           int tokens_per_block, const la_rope *rope, float eps,
+                                           void *stream);
+
+/*
  * Device-side status of the kernels enqueued so far on this device: every
  * wait inside a kernel is bounded; one that gives up records the fact in a
  * device flag and the kernel returns early.  This call synchronises `stream`,
