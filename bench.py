@@ -294,51 +294,65 @@ def main():
             args.steps = int(t.item())
     K = args.steps
 
-    def ev():
-        e = torch.cuda.Event(enable_timing=True)
-        e.record()          # creates the underlying event now
-        return e
-
-    step_ev = [(ev(), ev()) for _ in range(K)]
-    stage_ev = [[tuple(ev() for _ in range(4)) for _ in range(n_calls)] for _ in range(K)]
+    # one step captured as a CUDA graph (the library is capture-safe: it never
+    # allocates or synchronises); kernels inside keep their programmatic
+    # dependent-launch edges
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        runner.step()
+    launches_per_step = runner.launches_per_step
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        flush.fill_(3.0)
+        graph.replay()
     torch.cuda.synchronize()
 
-    def set_stage(k, i):
-        e = stage_ev[k][i]
-        la.la_set_stage_events(*(x.cuda_event for x in e))
-
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     sampler = ClockSampler()
     barrier()
     torch.cuda.synchronize()
     if rank == 0:
         sampler.start(dev)
         time.sleep(0.3)
-    launches = 0
     for kk in range(K):
         flush.fill_(float(kk))
         step_ev[kk][0].record(stream)
-        set_stage(kk, 0)
-
-        def after(i, kk=kk):
-            if i + 1 < n_calls:
-                set_stage(kk, i + 1)
-
-        runner.step(after_call=after)
+        graph.replay()
         step_ev[kk][1].record(stream)
-        launches += runner.launches_per_step
-    la.la_set_stage_events(None, None, None, None)
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop(local_rank) if rank == 0 else None
+    launches = K * launches_per_step
     la.device_status()
-
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
+
+    # per-kernel durations: a second graph of the same step with the library's
+    # stage events between its kernels (they serialise the kernels, so this
+    # region is timed separately and only feeds the per-kernel roofline)
+    Ks = min(K, 200)
+    stage_ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(n_calls)]
+    for e in stage_ev:
+        for x in e:
+            x.record()
+    torch.cuda.synchronize()
+
+    def set_stage(i):
+        la.la_set_stage_events(*(x.cuda_event for x in stage_ev[i]))
+
+    graph2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph2):
+        set_stage(0)
+        runner.step(after_call=lambda i: set_stage(i + 1) if i + 1 < n_calls else None)
+    la.la_set_stage_events(None, None, None, None)
     stage_ms = [0.0, 0.0, 0.0]
-    for k in range(K):
-        for i in range(n_calls):
-            e = stage_ev[k][i]
+    for kk in range(Ks):
+        flush.fill_(float(kk))
+        graph2.replay()
+        torch.cuda.synchronize()
+        for e in stage_ev:
             for j in range(3):
                 stage_ms[j] += e[j].elapsed_time(e[j + 1])
+    stage_ms = [x * K / Ks for x in stage_ms]      # scaled to K steps like total_ms
     total_ms = sum(step_ms)
     tot = torch.tensor([total_ms] + stage_ms, dtype=torch.float64, device=dev)
     if dist is not None:
@@ -351,7 +365,7 @@ def main():
     peak, peak_kind = measured_peaks()
     step_gbs = w.alg_bytes / (ms_per_step / 1e3) / 1e9
 
-    launches_per_kernel = K * n_calls
+    launches_per_kernel = K * n_calls                # stage_ms is scaled to K steps
     # dominant kernel: the larger of reduce (reads k, v) and apply (reads q, writes out)
     per_call_th = w.B * runner.tokens_per_call(0) * w.H
     kern_bytes = per_call_th * 2 * w.d * w.elem_bytes
@@ -385,6 +399,7 @@ def main():
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": ncu_traffic(kname, per_call_th)},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "path": path, "clocks": clocks,
+            "launch": "one CUDA graph per step (programmatic dependent launch between kernels)",
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

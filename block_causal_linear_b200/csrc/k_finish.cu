@@ -1,8 +1,9 @@
 // k_finish.cu -- state combine: fixed-order split sum, prefix over blocks,
 // commit.
 //
-// Per (b, h), in a fixed order (so that results are reproducible bit for bit):
-//   run = S_prior (or 0)                                   [S | Z], 1056 floats
+// Per (b, h) and each of the 1056 numbers of [S | Z], in a fixed order (so
+// that results are reproducible bit for bit):
+//   run = S_prior (or 0)
 //   for block n = 0 .. nb-1:
 //       run += partial[n][0] + partial[n][1] + ... + partial[n][P-1]
 //       S_eff[n] = run
@@ -18,6 +19,9 @@
 // sees S_eff to about 16 mantissa bits.  Layout: K-major, no swizzle, core
 // matrices of 8 rows x 16 bytes; element (n, k) at byte
 //   (n / 8) * 512 + (k / 8) * 128 + (n % 8) * 16 + (k % 8) * 2.
+//
+// One thread per number: the P partial loads of a block are issued together
+// and then added in split order.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -27,6 +31,9 @@ namespace la {
 namespace {
 
 constexpr int kFinThreads = 256;
+constexpr int kBatch = 8;          // partial loads in flight per thread
+constexpr int kZeroRows = kOpRows - kD - 1;
+constexpr int kPerBH = kKVZ + kZeroRows * kD;   // numbers + zero-padding entries per (b, h)
 
 __device__ __forceinline__ int op_offset(int nrow, int kcol) {
     return (nrow >> 3) * 512 + (kcol >> 3) * 128 + (nrow & 7) * 16 + (kcol & 7) * 2;
@@ -36,40 +43,53 @@ __global__ void __launch_bounds__(kFinThreads)
 finish_kernel(const float *__restrict__ partials, float *__restrict__ seff,
               unsigned char *__restrict__ bop, float *__restrict__ S, float *__restrict__ Z,
               Plan p, int write_bop) {
-    const int bh = blockIdx.x;
-    for (int e = threadIdx.x; e < kKVZ; e += kFinThreads) {
-        float run = 0.f;
-        if (p.has_state) run = e < kD * kD ? S[(size_t)bh * kD * kD + e] : Z[(size_t)bh * kD + e - kD * kD];
-        const int nrow = e < kD * kD ? (e % kD) : kD;     // value column, or the Z column
-        const int kcol = e < kD * kD ? (e / kD) : (e - kD * kD);
+    // let the apply be scheduled now (it prefetches its q tiles), then wait
+    // for the reduce before reading its partials
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const long long w = (long long)blockIdx.x * kFinThreads + threadIdx.x;
+    const long long bh = w / kPerBH;
+    const int e = (int)(w % kPerBH);
+    if (bh >= (long long)p.B * p.H) return;
+
+    if (e >= kKVZ) {   // zero rows 33..47 of the packed operand (N padded to 48)
+        if (!write_bop) return;
+        const int z = e - kKVZ;
+        const int nrow = kD + 1 + z / kD, kcol = z % kD;
         for (int n = 0; n < p.nb; ++n) {
-            const float *src = partials + ((size_t)bh * p.nb + n) * p.P * kKVZ + e;
-            for (int sp = 0; sp < p.P; ++sp) run += src[(size_t)sp * kKVZ];
-            seff[((size_t)bh * p.nb + n) * kKVZ + e] = run;
-            if (write_bop) {
-                unsigned char *dst = bop + ((size_t)bh * p.nb + n) * 2 * kOpBytes + op_offset(nrow, kcol);
-                const __nv_bfloat16 hi = __float2bfloat16_rn(run);
-                const __nv_bfloat16 lo = __float2bfloat16_rn(run - __bfloat162float(hi));
-                *reinterpret_cast<__nv_bfloat16 *>(dst) = hi;
-                *reinterpret_cast<__nv_bfloat16 *>(dst + kOpBytes) = lo;
-            }
-        }
-        if (p.commit) {
-            if (e < kD * kD) S[(size_t)bh * kD * kD + e] = run;
-            else Z[(size_t)bh * kD + e - kD * kD] = run;
-        }
-    }
-    if (write_bop) {
-        // rows 33..47 of the operand are zero (N padded to a multiple of 16)
-        const int zrows = kOpRows - kD - 1;
-        for (int w = threadIdx.x; w < p.nb * zrows * kD; w += kFinThreads) {
-            const int n = w / (zrows * kD);
-            const int nrow = kD + 1 + (w / kD) % zrows;
-            const int kcol = w % kD;
             unsigned char *dst = bop + ((size_t)bh * p.nb + n) * 2 * kOpBytes + op_offset(nrow, kcol);
             *reinterpret_cast<unsigned short *>(dst) = 0;
             *reinterpret_cast<unsigned short *>(dst + kOpBytes) = 0;
         }
+        return;
+    }
+
+    float run = 0.f;
+    if (p.has_state) run = e < kD * kD ? S[(size_t)bh * kD * kD + e] : Z[(size_t)bh * kD + e - kD * kD];
+    const int nrow = e < kD * kD ? (e % kD) : kD;     // value column, or the Z column
+    const int kcol = e < kD * kD ? (e / kD) : (e - kD * kD);
+    for (int n = 0; n < p.nb; ++n) {
+        const float *src = partials + ((size_t)bh * p.nb + n) * p.P * kKVZ + e;
+        for (int s0 = 0; s0 < p.P; s0 += kBatch) {
+            float v[kBatch];
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) v[j] = s0 + j < p.P ? __ldg(src + (size_t)(s0 + j) * kKVZ) : 0.f;
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j)
+                if (s0 + j < p.P) run += v[j];
+        }
+        seff[((size_t)bh * p.nb + n) * kKVZ + e] = run;
+        if (write_bop) {
+            unsigned char *dst = bop + ((size_t)bh * p.nb + n) * 2 * kOpBytes + op_offset(nrow, kcol);
+            const __nv_bfloat16 hi = __float2bfloat16_rn(run);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(run - __bfloat162float(hi));
+            *reinterpret_cast<__nv_bfloat16 *>(dst) = hi;
+            *reinterpret_cast<__nv_bfloat16 *>(dst + kOpBytes) = lo;
+        }
+    }
+    if (p.commit) {
+        if (e < kD * kD) S[(size_t)bh * kD * kD + e] = run;
+        else Z[(size_t)bh * kD + e - kD * kD] = run;
     }
 }
 
@@ -77,11 +97,24 @@ finish_kernel(const float *__restrict__ partials, float *__restrict__ seff,
 
 int launch_finish(const float *partials, float *seff, void *bop, float *S, float *Z, const Plan &p,
                   int write_bop, cudaStream_t s) {
-    const long long grid = (long long)p.B * p.H;
+    const long long threads = (long long)p.B * p.H * kPerBH;
+    const long long grid = (threads + kFinThreads - 1) / kFinThreads;
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
-    finish_kernel<<<(unsigned)grid, kFinThreads, 0, s>>>(partials, seff, static_cast<unsigned char *>(bop),
-                                                       S, Z, p, write_bop);
-    return cudaGetLastError() == cudaSuccess ? 1 : -1;
+    // programmatic stream serialization: the kernel may start while the reduce
+    // drains; it waits for it (griddepcontrol.wait) before reading anything
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kFinThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, finish_kernel, partials, seff, static_cast<unsigned char *>(bop), S, Z, p,
+                              write_bop) == cudaSuccess
+               ? 1
+               : -1;
 }
 
 }  // namespace la

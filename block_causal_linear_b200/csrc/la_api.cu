@@ -19,8 +19,14 @@ int g_last_launches = 0;
 const char *g_last_path = "none";
 cudaEvent_t g_ev[4] = {nullptr, nullptr, nullptr, nullptr};
 
+// Record stage event i on s.  Under stream capture the record becomes an
+// event-record node of the graph (external), so that each replay records it.
 inline bool mark(int i, cudaStream_t s) {
-    return !g_ev[i] || cudaEventRecord(g_ev[i], s) == cudaSuccess;
+    if (!g_ev[i]) return true;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return false;
+    const unsigned flags = cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
+    return cudaEventRecordWithFlags(g_ev[i], s, flags) == cudaSuccess;
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -28,21 +34,23 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 
 // Deterministic split plan: a function of the shapes only (never of the GPU),
-// so that results are reproducible bit for bit.
+// so that results are reproducible bit for bit.  Each block is cut into P
+// reduce splits (16-token granularity) and Pa apply splits (128-token tiles)
+// so that one wave of at most kTargetCtas CTAs covers the call.
 void make_splits(la::Plan &p) {
     const long long groups = (long long)p.B * ceil_div(p.H, 4) * p.nb;
-    long long want = ceil_div(la::kTargetCtas, groups);
+    long long want = la::kTargetCtas / groups;
+    if (want > ceil_div(p.L, la::kReduceRows)) want = ceil_div(p.L, la::kReduceRows);
     if (want < 1) want = 1;
-    long long chunk = ceil_div(ceil_div(p.L, want), la::kReduceRows) * la::kReduceRows;
-    if (chunk < la::kReduceRows) chunk = la::kReduceRows;
+    const long long chunk = ceil_div(ceil_div(p.L, want), 16) * 16;
     p.chunk = (int)chunk;
     p.P = (int)ceil_div(p.L, chunk);
 
     const long long pairs = (long long)p.B * ceil_div(p.H, 2) * p.nb;
-    long long wanta = ceil_div(la::kTargetCtas, pairs);
+    long long wanta = la::kTargetCtas / pairs;
+    if (wanta > ceil_div(p.L, la::kApplyRows)) wanta = ceil_div(p.L, la::kApplyRows);
     if (wanta < 1) wanta = 1;
-    long long chunka = ceil_div(ceil_div(p.L, wanta), la::kApplyRows) * la::kApplyRows;
-    if (chunka < la::kApplyRows) chunka = la::kApplyRows;
+    const long long chunka = ceil_div(ceil_div(p.L, wanta), la::kApplyRows) * la::kApplyRows;
     p.chunka = (int)chunka;
     p.Pa = (int)ceil_div(p.L, chunka);
 }
@@ -94,8 +102,10 @@ la_status common_checks(const void *q, const void *k, const void *v, void *out, 
     return LA_OK;
 }
 
-bool use_tc(la_dtype dt, int H) {
-    return dt == LA_BF16 && (H % 4) == 0 && la::tc_available();
+// The tensor-core kernels take bf16 inputs with H a multiple of 4 (4-head
+// reduce groups, 2-head apply tiles) and no RoPE; the rest runs on CUDA cores.
+bool use_tc(la_dtype dt, const la::Plan &p) {
+    return dt == LA_BF16 && (p.H % 4) == 0 && !p.rope && la::tc_available();
 }
 
 // Enqueue reduce -> finish -> apply for a prepared plan.
@@ -106,7 +116,7 @@ la_status run(const void *q, const void *k, const void *v, void *out, la_dtype d
     float *partials = reinterpret_cast<float *>(base + w.partials);
     float *seff = reinterpret_cast<float *>(base + w.seff);
     void *bop = base + w.bop;
-    const bool tc = use_tc(dt, p.H);
+    const bool tc = use_tc(dt, p);
     int n = 0, r;
 
     if (!mark(0, s)) return LA_ECUDA;

@@ -24,7 +24,7 @@ struct Plan {
     int L;                // tokens per block (the last block may be shorter)
     int nb;               // number of blocks in the call
     int P;                // reduce splits per (b, h, block)
-    int chunk;            // tokens per reduce split (multiple of kReduceRows)
+    int chunk;            // tokens per reduce split (multiple of 16)
     int Pa;               // apply splits per (b, head pair, block)
     int chunka;           // tokens per apply split (multiple of kApplyRows)
     int commit;           // write S_eff of the last block back to the state

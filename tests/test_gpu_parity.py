@@ -31,9 +31,10 @@ def orc_rope(orc, r):
     return orc.make_rope(Hg=r.Hg, Wg=r.Wg, t_offset=r.t_offset, dims=(r.dt, r.dh, r.dw), base=r.base)
 
 
-def expect_path(la, dtype, H):
-    """bf16 with H % 4 == 0 runs the tensor-core kernels, the rest the FFMA ones."""
-    want = "tc" if (dtype == torch.bfloat16 and H % 4 == 0 and la.tc_enabled()) else "ffma"
+def expect_path(la, dtype, H, rope):
+    """bf16 with H % 4 == 0 and no RoPE runs the tensor-core kernels, the rest
+    the FFMA ones."""
+    want = "tc" if (dtype == torch.bfloat16 and H % 4 == 0 and not rope and la.tc_enabled()) else "ffma"
     assert la.la_last_path() == want
 
 
@@ -87,7 +88,7 @@ def test_full_forward_matches_oracle(la, orc, case):
     rope = la.make_rope(Hg=3, Wg=5, t_offset=2) if use_rope else None
     g = la.full_forward(q.cuda(), k.cuda(), v.cuda(), L, rope=rope, eps=EPS)
     torch.cuda.synchronize()
-    expect_path(la, dtype, H)
+    expect_path(la, dtype, H, use_rope)
     ref = orc.full_forward(q, k, v, L, rope=orc_rope(orc, rope), eps=EPS)
     assert err_out(g, ref, dtype) <= tol_out(dtype)
     la.device_status()
