@@ -1,24 +1,30 @@
 // k_tc.cu -- tensor-core (tcgen05 + TMA) reduce and apply kernels for bf16.
 //
-// reduce: KV_n = sum_t phi(k_t)^T v_t and z_n = sum_t phi(k_t) over one split
+// reduce: KV_n = sum_t psi(k_t)^T v_t and z_n = sum_t phi(k_t) over one split
 //   of a block, for 4 heads at a time ("KV product then accumulate",
 //   "Nvidia, MIT ve diğerleri video yapay zeka devrimini başlattı", section
 //   "Sabit Bellekli KV önbelleğe alma mekanizması").  The contraction over
-//   tokens is one M=128 x N=128 x K=16 MMA per 16 tokens: A = phi(K) of 4
+//   tokens is one M=128 x N=128 x K=16 MMA per 16 tokens: A = psi(K) of 4
 //   heads (M = 4 x 32 key features, stored MN-major as TMA lands it), B = V of
 //   the same 4 heads (N = 4 x 32 value features).  Only the 4 diagonal 32x32
-//   blocks of D are used.  z comes from a second MMA against a 16-column
-//   matrix of ones.  fp32 accumulation in TMEM across the whole split.
-// apply: out_t = phi(q_t) S_eff / (phi(q_t) . Z_eff + eps) for 128-token tiles
-//   of 2 heads: per head one M=128 x N=48 x K=32 contraction of phi(Q) against
-//   the packed [S | Z | 0] operand, as a hi and a lo bf16 part accumulated in
-//   the same TMEM columns (S_eff is carried to ~16 mantissa bits); the epilogue
-//   divides, rounds to bf16 and stores with TMA.
+//   blocks of D are used.  fp32 accumulation in TMEM across the whole split.
+//   Without RoPE, z comes from a second MMA against a 16-column matrix of
+//   ones.  With RoPE (sd114.wiki, "两大核心技术突破" item 1), the rotated
+//   features R phi(k) go to the MMA as a hi and a lo bf16 part (R phi(k) =
+//   hi + lo to ~16 bits), and z = sum phi(k) is summed on the CUDA cores while
+//   phi is applied.
+// apply: out_t = psi(q_t) S_eff / (phi(q_t) . Z_eff + eps) for 128-token tiles
+//   of 2 heads.  Without RoPE: per head one M=128 x N=48 x K=32 contraction of
+//   phi(Q) against the packed [S | Z | 0] operand, as a hi and a lo bf16 part
+//   accumulated in the same TMEM columns.  With RoPE: the numerator is
+//   (R phi(q))_hi.S_hi + (R phi(q))_hi.S_lo + (R phi(q))_lo.S_hi (N = 32) and the
+//   unrotated denominator phi(q).Z_eff is summed in fp32 on the CUDA cores.
+//   The epilogue divides, rounds to bf16 and stores with TMA.
 //
 // Both kernels: 6 warps; warp 0 issues TMA, warp 1 owns TMEM and issues the
-// MMAs, warps 2..5 apply phi = ReLU in shared memory and run the epilogue.
-// Every wait is bounded (la_sm100.cuh); a wait that gives up raises the device
-// flag read by la_device_status and the CTA drains and returns.
+// MMAs, warps 2..5 apply phi = ReLU (and RoPE) in shared memory and run the
+// epilogue.  Every wait is bounded (la_sm100.cuh); a wait that gives up raises
+// the device flag read by la_device_status and the CTA drains and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -43,7 +49,6 @@ constexpr int kThreads = 192;   // 6 warps
 constexpr int kWarpTma = 0;
 constexpr int kWarpMma = 1;
 constexpr int kWork = 128;      // threads of warps 2..5
-constexpr uint32_t kTmemCols = 256;
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     const uint32_t a = smem_u32(p);
@@ -56,6 +61,14 @@ __device__ __forceinline__ uint32_t relu2(uint32_t x) {
     return __vmaxs2(x, 0u);
 }
 
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
+    const __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&t);
+}
+
 // Drain at exit after an abort: wait (briefly, ignoring the abort word) for
 // anything still writing this CTA's shared memory or TMEM.
 __device__ __forceinline__ void final_wait(uint64_t *bar, uint32_t parity) {
@@ -66,25 +79,112 @@ __device__ __forceinline__ void final_wait(uint64_t *bar, uint32_t parity) {
     }
 }
 
+// ---------------------------------------------------------------- RoPE table
+// (cos, sin) of every feature pair at every position a CTA can meet: pair p of
+// the frame axis at frames [f_lo, f_lo + nf) of the call, of the row axis at
+// rows [0, Hg), of the column axis at columns [0, Wg).  The segment of pair p
+// starts at rope_seg(p).  The host only takes this path when the table fits.
+constexpr int kTabMax = 1024;
+
+__device__ __forceinline__ int rope_len(const Plan &p, int pr, int nf) {
+    return p.axis[pr] == 0 ? nf : (p.axis[pr] == 1 ? p.Hg : p.Wg);
+}
+
+__device__ __forceinline__ int rope_seg(const Plan &p, int pr, int nf) {
+    int off = 0;
+    for (int q = 0; q < pr; ++q) off += rope_len(p, q, nf);
+    return off;
+}
+
+__device__ void build_rope_table(float2 *tab, const Plan &p, int f_lo, int nf, int tid, int nthreads) {
+    int off = 0;
+    for (int pr = 0; pr < kD / 2; ++pr) {
+        const int len = rope_len(p, pr, nf);
+        for (int pos = tid; pos < len; pos += nthreads) {
+            const int apos = p.axis[pr] == 0 ? p.t_offset + f_lo + pos : pos;
+            float s, c;
+            sincosf((float)apos * p.theta[pr], &s, &c);
+            tab[off + pos] = make_float2(c, s);
+        }
+        off += len;
+    }
+}
+
+// Per-thread view of the 4 feature pairs of one 16-byte chunk (features
+// 8*(L%4) .. +7 of a head): table segment and axis of each pair.
+struct PairSet {
+    int seg[4];
+    int axis[4];
+};
+
+__device__ __forceinline__ PairSet pair_set(const Plan &p, int L, int nf) {
+    PairSet s;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int pr = (L & 3) * 4 + m;
+        s.seg[m] = rope_seg(p, pr, nf);
+        s.axis[m] = p.axis[pr];
+    }
+    return s;
+}
+
+// ReLU one chunk of 8 bf16, rotate its 4 pairs at token t (index in the
+// call), and split the rotated values into hi + lo bf16.  f receives phi(x).
+__device__ __forceinline__ void relu_rotate_chunk(uint4 x, const float2 *tab, const PairSet &ps, const Plan &p,
+                                                  long long t, int f_lo, uint4 &hi, uint4 &lo, float (&f)[8]) {
+    const long long hw = (long long)p.Hg * p.Wg;
+    const int fr = (int)(t / hw) - f_lo;
+    const int rem = (int)(t % hw);
+    const int row = rem / p.Wg, col = rem % p.Wg;
+    const uint32_t w[4] = {relu2(x.x), relu2(x.y), relu2(x.z), relu2(x.w)};
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const float x0 = bf_lo(w[m]), x1 = bf_hi(w[m]);
+        f[2 * m] = x0;
+        f[2 * m + 1] = x1;
+        const int pos = ps.axis[m] == 0 ? fr : (ps.axis[m] == 1 ? row : col);
+        const float2 cs = tab[ps.seg[m] + pos];
+        const float y0 = x0 * cs.x - x1 * cs.y;
+        const float y1 = x0 * cs.y + x1 * cs.x;
+        const __nv_bfloat162 yh = __floats2bfloat162_rn(y0, y1);
+        h[m] = *reinterpret_cast<const uint32_t *>(&yh);
+        l[m] = pack_bf2(y0 - __low2float(yh), y1 - __high2float(yh));
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
 // ================================================================ reduce
 
-constexpr int kRStages = 3;
-constexpr int kRBox = 64 * 128;             // [64 rows][64 bf16] = 8 KiB
-constexpr int kRStageBytes = 4 * kRBox;     // k: 2 boxes (4 heads), v: 2 boxes
-constexpr int kROnesOff = kRStages * kRStageBytes;
-constexpr int kRBarOff = kROnesOff + 512;
-constexpr int kRSmem = kRBarOff + (3 * kRStages + 1) * 8 + 16 + 1024;
+constexpr int kRBox = 64 * 128;   // [64 rows][64 bf16] = 8 KiB
 
+template <bool ROPE>
+struct RCfg {
+    static constexpr int kStages = ROPE ? 2 : 3;
+    // stage: k boxes (becoming R phi(k) hi with RoPE), [lo boxes], v boxes
+    static constexpr int kLoOff = 2 * kRBox;
+    static constexpr int kVOff = ROPE ? 4 * kRBox : 2 * kRBox;
+    static constexpr int kStageBytes = kVOff + 2 * kRBox;
+    static constexpr int kAuxOff = kStages * kStageBytes;          // ones (512 B) or RoPE table
+    static constexpr int kAuxBytes = ROPE ? kTabMax * 8 : 512;
+    static constexpr int kBarOff = kAuxOff + kAuxBytes;
+    static constexpr int kSmem = kBarOff + (3 * kStages + 1) * 8 + 16 + 1024;
+    static constexpr uint32_t kTmemCols = ROPE ? 128 : 256;
+};
+
+template <bool ROPE>
 __global__ void __launch_bounds__(kThreads, 2)
 reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  float *__restrict__ partials, const Plan p) {
+    using C = RCfg<ROPE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
-    uint8_t *ones = smem + kROnesOff;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kRBarOff);
-    uint64_t *relu_done = full + kRStages;
-    uint64_t *empty = relu_done + kRStages;
-    uint64_t *acc_ready = empty + kRStages;
+    uint8_t *aux = smem + C::kAuxOff;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+    uint64_t *relu_done = full + C::kStages;
+    uint64_t *empty = relu_done + C::kStages;
+    uint64_t *acc_ready = empty + C::kStages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_ready + 1);
     volatile int *abort_word = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -114,8 +214,12 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         return;
     }
 
+    const long long hw = (long long)p.Hg * p.Wg;
+    const int f_lo = ROPE ? (int)(t0 / hw) : 0;
+    const int nf = ROPE ? (int)((t1 - 1) / hw) - f_lo + 1 : 0;
+
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kRStages; ++s) {
+        for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&relu_done[s], kWork);
             mbar_init(&empty[s], 1);
@@ -124,10 +228,14 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         *abort_word = 0;
         fence_barrier_init();
     }
-    // B operand of the z contraction: 16 x 16 bf16 ones (any layout reads 1.0)
-    for (int i = threadIdx.x; i < 128; i += kThreads) reinterpret_cast<uint32_t *>(ones)[i] = 0x3F803F80u;
+    if constexpr (ROPE) {
+        build_rope_table(reinterpret_cast<float2 *>(aux), p, f_lo, nf, threadIdx.x, kThreads);
+    } else {
+        // B operand of the z contraction: 16 x 16 bf16 ones (any layout reads 1.0)
+        for (int i = threadIdx.x; i < 128; i += kThreads) reinterpret_cast<uint32_t *>(aux)[i] = 0x3F803F80u;
+    }
     if (warp == kWarpMma) {
-        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
     if (warp == kWarpTma && lane == 0) {
@@ -144,17 +252,17 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     if (warp == kWarpTma) {
         if (lane == 0) {
             for (int i = 0; i < nst; ++i) {
-                const int s = i % kRStages;
-                const uint32_t ph = (uint32_t)(i / kRStages) & 1u;
+                const int s = i % C::kStages;
+                const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
                 if (!mbar_wait(&empty[s], ph ^ 1u, abort_word, &g_wait_flag, 1)) break;
-                uint8_t *st = smem + s * kRStageBytes;
-                mbar_arrive_expect_tx(&full[s], kRStageBytes);
+                uint8_t *st = smem + s * C::kStageBytes;
+                mbar_arrive_expect_tx(&full[s], 4 * kRBox);
                 const int row = (int)(t0 + 64LL * i);
                 const int c0 = g * 128;
-                tma_load_3d(st + 0 * kRBox, &tm_k, &full[s], c0, row, b);
-                tma_load_3d(st + 1 * kRBox, &tm_k, &full[s], c0 + 64, row, b);
-                tma_load_3d(st + 2 * kRBox, &tm_v, &full[s], c0, row, b);
-                tma_load_3d(st + 3 * kRBox, &tm_v, &full[s], c0 + 64, row, b);
+                tma_load_3d(st, &tm_k, &full[s], c0, row, b);
+                tma_load_3d(st + kRBox, &tm_k, &full[s], c0 + 64, row, b);
+                tma_load_3d(st + C::kVOff, &tm_v, &full[s], c0, row, b);
+                tma_load_3d(st + C::kVOff + kRBox, &tm_v, &full[s], c0 + 64, row, b);
                 issued = i + 1;
             }
         }
@@ -162,14 +270,14 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         if (lane == 0) {
             const uint32_t id_kv = idesc_bf16(128, 128, 1, 1);
             const uint32_t id_z = idesc_bf16(128, 16, 1, 0);
-            const uint64_t d_ones = smem_desc(smem_u32(ones), 128, 256, kLayoutNone);
+            const uint64_t d_ones = smem_desc(smem_u32(aux), 128, 256, kLayoutNone);
             for (int i = 0; i < nst; ++i) {
-                const int s = i % kRStages;
-                const uint32_t ph = (uint32_t)(i / kRStages) & 1u;
+                const int s = i % C::kStages;
+                const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
                 if (!mbar_wait(&relu_done[s], ph, abort_word, &g_wait_flag, 2)) break;
                 tc_fence_after();
-                const uint32_t kaddr = smem_u32(smem + s * kRStageBytes);
-                const uint32_t vaddr = kaddr + 2 * kRBox;
+                const uint32_t kaddr = smem_u32(smem + s * C::kStageBytes);
+                const uint32_t vaddr = kaddr + C::kVOff;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     // MN-major, 128-byte swizzle: 64-wide MN atoms kRBox apart (LBO),
@@ -178,7 +286,12 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     const uint64_t db = smem_desc(vaddr + kk * 2048, kRBox, 1024, kLayoutSw128);
                     const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
                     mma_bf16(tmem, da, db, id_kv, acc);
-                    mma_bf16(tmem + 128, da, d_ones, id_z, acc);
+                    if constexpr (ROPE) {
+                        const uint64_t dl = smem_desc(kaddr + C::kLoOff + kk * 2048, kRBox, 1024, kLayoutSw128);
+                        mma_bf16(tmem, dl, db, id_kv, 1u);
+                    } else {
+                        mma_bf16(tmem + 128, da, d_ones, id_z, acc);
+                    }
                 }
                 mma_commit(&empty[s]);
             }
@@ -186,11 +299,23 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
     } else {
         const int wt = threadIdx.x - 64;   // 0..127
+        // with RoPE this thread always meets the same logical chunk L of a row
+        // (the swizzle phase (wt >> 3) & 7 is the same for all its chunks)
+        const int L = (wt & 7) ^ ((wt >> 3) & 7);
+        PairSet ps{};
+        if constexpr (ROPE) ps = pair_set(p, L, nf);
+        float zacc[2][8];
+#pragma unroll
+        for (int bx = 0; bx < 2; ++bx)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) zacc[bx][k] = 0.f;
+        const float2 *tab = reinterpret_cast<const float2 *>(aux);
+
         for (int i = 0; i < nst; ++i) {
-            const int s = i % kRStages;
-            const uint32_t ph = (uint32_t)(i / kRStages) & 1u;
+            const int s = i % C::kStages;
+            const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
             if (!mbar_wait(&full[s], ph, abort_word, &g_wait_flag, 3)) break;
-            uint8_t *kt = smem + s * kRStageBytes;
+            uint8_t *kt = smem + s * C::kStageBytes;
             const long long row0 = t0 + 64LL * i;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
@@ -198,26 +323,57 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 const int r = (c & 511) >> 3;         // token row inside its box
                 uint4 *ptr = reinterpret_cast<uint4 *>(kt + (size_t)c * 16);
                 uint4 x = *ptr;
-                if (row0 + r < t1) {
-                    x.x = relu2(x.x); x.y = relu2(x.y); x.z = relu2(x.z); x.w = relu2(x.w);
+                const bool valid = row0 + r < t1;     // rows past the split contribute nothing
+                if constexpr (ROPE) {
+                    uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
+                    if (valid) {
+                        float f[8];
+                        relu_rotate_chunk(x, tab, ps, p, row0 + r, f_lo, hi, lo, f);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) zacc[j >> 2][k] += f[k];
+                    }
+                    *ptr = hi;
+                    *reinterpret_cast<uint4 *>(kt + C::kLoOff + (size_t)c * 16) = lo;
                 } else {
-                    x = make_uint4(0u, 0u, 0u, 0u);   // rows past the split contribute nothing
+                    if (valid) {
+                        x.x = relu2(x.x); x.y = relu2(x.y); x.z = relu2(x.z); x.w = relu2(x.w);
+                    } else {
+                        x = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    *ptr = x;
                 }
-                *ptr = x;
             }
             fence_proxy_async_smem();
             mbar_arrive(&relu_done[s]);
         }
-        // epilogue: warp quarter q reads TMEM lanes 32q.. = key features of head 4g+q
-        if (mbar_wait(acc_ready, 0, abort_word, &g_wait_flag, 4)) {
-            __syncwarp();   // tcgen05.ld is warp-collective
+        // epilogue: warp quarter q reads TMEM lanes 32q.. = key features of head 4g+q.
+        // Every work thread reaches the named barrier, and the TMEM read is
+        // taken or skipped by whole warps, even after a wait gave up.
+        bool got = mbar_wait(acc_ready, 0, abort_word, &g_wait_flag, 4);
+        got = __all_sync(0xffffffffu, got);
+        const int qd = warp & 3;
+        const int h = g * 4 + qd;
+        float z = 0.f;
+        if constexpr (ROPE) {
+            // z: the 16 threads that met chunk L of a box each hold 8 sums;
+            // add them in thread order (stage 0 is free once every MMA is done)
+            float *zbuf = reinterpret_cast<float *>(smem);
+#pragma unroll
+            for (int bx = 0; bx < 2; ++bx)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) zbuf[wt * 16 + bx * 8 + k] = zacc[bx][k];
+            named_bar_sync(1, kWork);
+            const int bx = qd >> 1;
+            const int Lz = ((qd & 1) << 2) | (lane >> 3);
+            for (int u = 0; u < kWork; ++u)
+                if (((u & 7) ^ ((u >> 3) & 7)) == Lz) z += zbuf[u * 16 + bx * 8 + (lane & 7)];
+        }
+        if (got) {
             tc_fence_after();
-            const int qd = warp & 3;
-            const int h = g * 4 + qd;
             const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
             float kv[32];
             tmem_ld32(tmem + lane_off + 32 * qd, kv);
-            const float z = tmem_ld1(tmem + lane_off + 128);
+            if constexpr (!ROPE) z = tmem_ld1(tmem + lane_off + 128);
             tmem_wait_ld();
             float *dst = partials + ((((size_t)b * p.H + h) * p.nb + n) * p.P + sp) * kKVZ;
             float4 *drow = reinterpret_cast<float4 *>(dst + lane * kD);
@@ -229,42 +385,60 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 
     // teardown: nothing may still write this CTA's shared memory or TMEM
     if (warp == kWarpTma && lane == 0 && *abort_word) {
-        for (int i = issued - kRStages < 0 ? 0 : issued - kRStages; i < issued; ++i)
-            final_wait(&full[i % kRStages], (uint32_t)(i / kRStages) & 1u);
+        for (int i = issued - C::kStages < 0 ? 0 : issued - C::kStages; i < issued; ++i)
+            final_wait(&full[i % C::kStages], (uint32_t)(i / C::kStages) & 1u);
     }
     if (warp == kWarpMma && lane == 0) final_wait(acc_ready, 0);
     tc_fence_before();
     __syncthreads();
     if (warp == kWarpMma) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, C::kTmemCols);
     }
 }
 
 // ================================================================ apply
 
-constexpr int kAStages = 3;
 constexpr int kATile = 128 * 128;              // [128 rows][64 bf16] = 16 KiB: 2 heads
-constexpr int kAOutOff = kAStages * kATile;    // 2 staging buffers for the TMA store
-constexpr int kABopOff = kAOutOff + 2 * kATile;
 constexpr int kABopBytes = 2 * 2 * kOpBytes;   // 2 heads x (hi, lo)
-constexpr int kABarOff = kABopOff + kABopBytes;
-constexpr int kASmem = kABarOff + (3 * kAStages + 6) * 8 + 16 + 1024;
 
+template <bool ROPE>
+struct ACfg {
+    static constexpr int kStages = ROPE ? 2 : 3;
+    static constexpr int kStageBytes = ROPE ? 2 * kATile : kATile;   // [R phi(q) hi | lo] or phi(q)
+    static constexpr int kStgBufs = ROPE ? 1 : 2;                    // TMA store staging buffers
+    static constexpr int kOutOff = kStages * kStageBytes;
+    static constexpr int kBopOff = kOutOff + kStgBufs * kATile;
+    static constexpr int kDenOff = kBopOff + kABopBytes;             // RoPE: [2][128 rows][2 heads] fp32
+    static constexpr int kZOff = kDenOff + (ROPE ? 2 * 1024 : 0);     // RoPE: Z_eff of the 2 heads
+    static constexpr int kTabOff = kZOff + (ROPE ? 256 : 0);
+    static constexpr int kBarOff = kTabOff + (ROPE ? kTabMax * 8 : 0);
+    static constexpr int kSmem = kBarOff + (3 * kStages + 6) * 8 + 16 + 1024;
+    static constexpr int kAccCols = ROPE ? 64 : 96;                  // per TMEM buffer (2 heads)
+    static constexpr int kHeadCols = ROPE ? 32 : kOpRows;
+    static constexpr uint32_t kTmemCols = ROPE ? 128 : 256;
+};
+
+template <bool ROPE>
 __global__ void __launch_bounds__(kThreads, 2)
 apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_out,
-                __nv_bfloat16 *__restrict__ out, const uint8_t *__restrict__ bop, const Plan p) {
+                __nv_bfloat16 *__restrict__ out, const uint8_t *__restrict__ bop, const float *__restrict__ seff,
+                const Plan p) {
+    using C = ACfg<ROPE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
-    uint8_t *stg = smem + kAOutOff;
-    uint8_t *bops = smem + kABopOff;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kABarOff);
-    uint64_t *relu_done = full + kAStages;
-    uint64_t *empty = relu_done + kAStages;
-    uint64_t *acc_full = empty + kAStages;      // [2]
-    uint64_t *acc_empty = acc_full + 2;         // [2]
+    uint8_t *stg = smem + C::kOutOff;
+    uint8_t *bops = smem + C::kBopOff;
+    float *den_s = reinterpret_cast<float *>(smem + C::kDenOff);
+    float *zs = reinterpret_cast<float *>(smem + C::kZOff);
+    const float2 *tab = reinterpret_cast<const float2 *>(smem + C::kTabOff);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+    uint64_t *relu_done = full + C::kStages;
+    uint64_t *empty = relu_done + C::kStages;
+    uint64_t *acc_full = empty + C::kStages;   // [2]
+    uint64_t *acc_empty = acc_full + 2;        // [2]
     uint64_t *bop_full = acc_empty + 2;
-    uint64_t *drain = bop_full + 1;             // only used when a wait gave up
+    uint64_t *drain = bop_full + 1;            // only used when a wait gave up
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_word = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -284,9 +458,12 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (ta1 <= ta0) return;   // a split past the end of a short last block
     const int ntiles = (int)((ta1 - ta0 + 127) / 128);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long hw = (long long)p.Hg * p.Wg;
+    const int f_lo = ROPE ? (int)(ta0 / hw) : 0;
+    const int nf = ROPE ? (int)((ta1 - 1) / hw) - f_lo + 1 : 0;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kAStages; ++s) {
+        for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&relu_done[s], kWork);
             mbar_init(&empty[s], 1);
@@ -300,8 +477,10 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         *abort_word = 0;
         fence_barrier_init();
     }
+    if constexpr (ROPE)
+        build_rope_table(reinterpret_cast<float2 *>(smem + C::kTabOff), p, f_lo, nf, threadIdx.x, kThreads);
     if (warp == kWarpMma) {
-        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
     if (warp == kWarpTma && lane == 0) {
@@ -319,10 +498,10 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (lane == 0) {
             // q is an input of the call, complete before the reduce of this call
             // started: its first tiles are fetched while the state combine still runs
-            const int pre = ntiles < kAStages ? ntiles : kAStages;
+            const int pre = ntiles < C::kStages ? ntiles : C::kStages;
             for (int i = 0; i < pre; ++i) {
                 mbar_arrive_expect_tx(&full[i], kATile);
-                tma_load_3d(smem + i * kATile, &tm_q, &full[i], hp * 64, (int)(ta0 + 128LL * i), b);
+                tma_load_3d(smem + i * C::kStageBytes, &tm_q, &full[i], hp * 64, (int)(ta0 + 128LL * i), b);
                 issued = i + 1;
             }
             pdl_wait();   // the packed operand is written by the previous kernel
@@ -333,43 +512,47 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             bop_issued = true;
             for (int i = pre; i < ntiles; ++i) {
-                const int s = i % kAStages;
-                const uint32_t ph = (uint32_t)(i / kAStages) & 1u;
+                const int s = i % C::kStages;
+                const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
                 if (!mbar_wait(&empty[s], ph ^ 1u, abort_word, &g_wait_flag, 11)) break;
                 mbar_arrive_expect_tx(&full[s], kATile);
-                tma_load_3d(smem + s * kATile, &tm_q, &full[s], hp * 64, (int)(ta0 + 128LL * i), b);
+                tma_load_3d(smem + s * C::kStageBytes, &tm_q, &full[s], hp * 64, (int)(ta0 + 128LL * i), b);
                 issued = i + 1;
             }
         }
     } else if (warp == kWarpMma) {
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(128, kOpRows, 0, 0);
+            const uint32_t idesc = idesc_bf16(128, C::kHeadCols, 0, 0);
             const uint32_t baddr = smem_u32(bops);
             if (mbar_wait(bop_full, 0, abort_word, &g_wait_flag, 12)) {
                 for (int i = 0; i < ntiles; ++i) {
-                    const int s = i % kAStages;
-                    const uint32_t ph = (uint32_t)(i / kAStages) & 1u;
+                    const int s = i % C::kStages;
+                    const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
                     const int ab = i & 1;
                     const uint32_t aph = (uint32_t)(i >> 1) & 1u;
                     if (!mbar_wait(&relu_done[s], ph, abort_word, &g_wait_flag, 13)) break;
                     if (!mbar_wait(&acc_empty[ab], aph ^ 1u, abort_word, &g_wait_flag, 14)) break;
                     tc_fence_after();
-                    const uint32_t qaddr = smem_u32(smem + s * kATile);
+                    const uint32_t qaddr = smem_u32(smem + s * C::kStageBytes);
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
-                        const uint32_t d = tmem + ab * 96 + hh * 48;
+                        const uint32_t d = tmem + ab * C::kAccCols + hh * C::kHeadCols;
+                        // (A part, B part) products: hi.hi, hi.lo and, with RoPE, lo.hi
 #pragma unroll
-                        for (int part = 0; part < 2; ++part) {
+                        for (int prod = 0; prod < (ROPE ? 3 : 2); ++prod) {
+                            const int apart = prod == 2 ? 1 : 0;
+                            const int bpart = prod == 1 ? 1 : 0;
 #pragma unroll
                             for (int kk = 0; kk < 2; ++kk) {
                                 // A: K-major, 128-byte swizzle; head hh is the 64-byte half
                                 // of each 128-byte row, 16 features = 32 bytes per step
-                                const uint64_t da = smem_desc(qaddr + hh * 64 + kk * 32, 16, 1024, kLayoutSw128);
+                                const uint64_t da = smem_desc(qaddr + apart * kATile + hh * 64 + kk * 32, 16, 1024,
+                                                              kLayoutSw128);
                                 // B: K-major, no swizzle, core matrices 128 B apart along K,
                                 // 8-row groups 512 B apart; 16 features = 256 bytes per step
-                                const uint64_t db = smem_desc(baddr + hh * 2 * kOpBytes + part * kOpBytes + kk * 256,
+                                const uint64_t db = smem_desc(baddr + hh * 2 * kOpBytes + bpart * kOpBytes + kk * 256,
                                                               128, 512, kLayoutNone);
-                                mma_bf16(d, da, db, idesc, (part | kk) ? 1u : 0u);
+                                mma_bf16(d, da, db, idesc, (prod | kk) ? 1u : 0u);
                             }
                         }
                     }
@@ -384,45 +567,84 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int r = 32 * qd + lane;               // token row of this thread in a tile
         const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
         bool ok = true;
+        const int L = (wt & 7) ^ ((wt >> 3) & 7);   // logical chunk this thread meets (RoPE)
+        PairSet ps{};
+        if constexpr (ROPE) ps = pair_set(p, L, nf);
 
-        auto relu_tile = [&](int i) -> bool {
-            const int s = i % kAStages;
-            const uint32_t ph = (uint32_t)(i / kAStages) & 1u;
-            if (!mbar_wait(&full[s], ph, abort_word, &g_wait_flag, 15)) return false;
-            uint8_t *qt = smem + s * kATile;
+        pdl_wait();   // every write to `out` (and the read of Z_eff) comes after the previous kernel
+        if constexpr (ROPE) {
+            if (wt < 2 * kD)
+                zs[wt] = seff[(((size_t)b * p.H + 2 * hp + (wt >> 5)) * p.nb + n) * kKVZ + kD * kD + (wt & 31)];
+            named_bar_sync(1, kWork);
+        }
+
+        // A wait that gives up (abort) makes this thread skip work, never leave
+        // the loop: every work thread takes the same named barriers, and TMEM
+        // reads are taken or skipped by whole warps.
+        auto relu_tile = [&](int i) {
+            const int s = i % C::kStages;
+            const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
+            if (ok && !mbar_wait(&full[s], ph, abort_word, &g_wait_flag, 15)) ok = false;
+            uint8_t *qt = smem + s * C::kStageBytes;
+            const long long row0 = ta0 + 128LL * i;
+            if constexpr (ROPE) named_bar_sync(1, kWork);   // den_s[i & 1] was read by the epilogue of tile i-2
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                uint4 *ptr = reinterpret_cast<uint4 *>(qt + (size_t)(wt + 128 * j) * 16);
-                uint4 x = *ptr;
-                x.x = relu2(x.x); x.y = relu2(x.y); x.z = relu2(x.z); x.w = relu2(x.w);
-                *ptr = x;
+                const int c = wt + 128 * j;
+                uint4 *ptr = reinterpret_cast<uint4 *>(qt + (size_t)c * 16);
+                if constexpr (ROPE) {
+                    const int rr = c >> 3;                      // token row of this chunk
+                    const bool valid = ok && row0 + rr < ta1;
+                    uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
+                    float dp = 0.f;
+                    if (valid) {
+                        float f[8];
+                        relu_rotate_chunk(*ptr, tab, ps, p, row0 + rr, f_lo, hi, lo, f);
+                        const float *zh = zs + (L >> 2) * kD + (L & 3) * 8;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) dp = fmaf(f[k], zh[k], dp);
+                    }
+                    *ptr = hi;
+                    *reinterpret_cast<uint4 *>(qt + kATile + (size_t)c * 16) = lo;
+                    // the 4 chunks of one head in a row sit on lanes that differ in bits 0-1
+                    dp += __shfl_xor_sync(0xffffffffu, dp, 1);
+                    dp += __shfl_xor_sync(0xffffffffu, dp, 2);
+                    if ((lane & 3) == 0) den_s[(i & 1) * 256 + rr * 2 + (L >> 2)] = dp;
+                } else if (ok) {
+                    uint4 x = *ptr;
+                    x.x = relu2(x.x); x.y = relu2(x.y); x.z = relu2(x.z); x.w = relu2(x.w);
+                    *ptr = x;
+                }
             }
             fence_proxy_async_smem();
             mbar_arrive(&relu_done[s]);
-            return true;
         };
 
-        pdl_wait();   // every write to `out` comes after the previous kernel finished
-        if (ntiles > 0) ok = relu_tile(0);
-        for (int i = 0; i < ntiles && ok; ++i) {
-            if (i + 1 < ntiles && !relu_tile(i + 1)) { ok = false; break; }
+        if (ntiles > 0) relu_tile(0);
+        for (int i = 0; i < ntiles; ++i) {
+            if (i + 1 < ntiles) relu_tile(i + 1);
             const int ab = i & 1;
             const uint32_t aph = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait(&acc_full[ab], aph, abort_word, &g_wait_flag, 16)) { ok = false; break; }
-            __syncwarp();   // tcgen05.ld is warp-collective
-            tc_fence_after();
+            bool got = ok && mbar_wait(&acc_full[ab], aph, abort_word, &g_wait_flag, 16);
+            got = __all_sync(0xffffffffu, got);
+            if (!got) ok = false;
             uint32_t packed[2][16];
+            if (got) {
+                tc_fence_after();
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float num[32];
-                tmem_ld32(tmem + lane_off + ab * 96 + hh * 48, num);
-                const float den = tmem_ld1(tmem + lane_off + ab * 96 + hh * 48 + kD);
-                tmem_wait_ld();
-                const float inv = 1.0f / (den + p.eps);
+                for (int hh = 0; hh < 2; ++hh) {
+                    float num[32];
+                    tmem_ld32(tmem + lane_off + ab * C::kAccCols + hh * C::kHeadCols, num);
+                    float den;
+                    if constexpr (ROPE) {
+                        den = den_s[(i & 1) * 256 + r * 2 + hh];
+                    } else {
+                        den = tmem_ld1(tmem + lane_off + ab * C::kAccCols + hh * C::kHeadCols + kD);
+                    }
+                    tmem_wait_ld();
+                    const float inv = 1.0f / (den + p.eps);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const __nv_bfloat162 t = __floats2bfloat162_rn(num[2 * j] * inv, num[2 * j + 1] * inv);
-                    packed[hh][j] = *reinterpret_cast<const uint32_t *>(&t);
+                    for (int j = 0; j < 16; ++j) packed[hh][j] = pack_bf2(num[2 * j] * inv, num[2 * j + 1] * inv);
                 }
             }
             tc_fence_before();
@@ -431,23 +653,25 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const long long row0 = ta0 + 128LL * i;
             const bool whole = row0 + 128 <= ta1 || ta1 == p.N;   // TMA clips rows >= N
             if (whole) {
-                uint8_t *sb = stg + (i & 1) * kATile;
-                if (wt == 0) bulk_wait_read<1>();   // the store of tile i-2 has read this buffer
+                uint8_t *sb = stg + (i % C::kStgBufs) * kATile;
+                if (wt == 0) bulk_wait_read<C::kStgBufs - 1>();   // the last store from sb has read it
                 named_bar_sync(1, kWork);
+                if (got) {
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {       // logical 16-byte chunk c: head c/4
-                    const int pc = c ^ (r & 7);     // 128-byte swizzle
-                    *reinterpret_cast<uint4 *>(sb + r * 128 + pc * 16) =
-                        make_uint4(packed[c >> 2][4 * (c & 3)], packed[c >> 2][4 * (c & 3) + 1],
-                                   packed[c >> 2][4 * (c & 3) + 2], packed[c >> 2][4 * (c & 3) + 3]);
+                    for (int c = 0; c < 8; ++c) {       // logical 16-byte chunk c: head c/4
+                        const int pc = c ^ (r & 7);     // 128-byte swizzle
+                        *reinterpret_cast<uint4 *>(sb + r * 128 + pc * 16) =
+                            make_uint4(packed[c >> 2][4 * (c & 3)], packed[c >> 2][4 * (c & 3) + 1],
+                                       packed[c >> 2][4 * (c & 3) + 2], packed[c >> 2][4 * (c & 3) + 3]);
+                    }
                 }
                 fence_proxy_async_smem();
                 named_bar_sync(1, kWork);
-                if (wt == 0) {
+                if (wt == 0 && ok) {
                     tma_store_3d(&tm_out, sb, hp * 64, (int)row0, b);
                     bulk_commit();
                 }
-            } else if (row0 + r < ta1) {
+            } else if (got && row0 + r < ta1) {
                 // a short last tile inside the tensor: the rows after ta1 belong to another block
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
@@ -464,8 +688,8 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     if (warp == kWarpTma && lane == 0 && *abort_word) {
         if (bop_issued) final_wait(bop_full, 0);
-        for (int i = issued - kAStages < 0 ? 0 : issued - kAStages; i < issued; ++i)
-            final_wait(&full[i % kAStages], (uint32_t)(i / kAStages) & 1u);
+        for (int i = issued - C::kStages < 0 ? 0 : issued - C::kStages; i < issued; ++i)
+            final_wait(&full[i % C::kStages], (uint32_t)(i / C::kStages) & 1u);
     }
     if (warp == kWarpMma && lane == 0 && *abort_word) {
         // make every MMA issued so far finish before TMEM is released
@@ -476,7 +700,7 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
     if (warp == kWarpMma) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, C::kTmemCols);
     }
 }
 
@@ -532,6 +756,28 @@ bool set_smem(const void *kernel, int bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
 }
 
+bool smem_ready() {
+    static std::once_flag once;
+    static bool ok = false;
+    std::call_once(once, [] {
+        ok = set_smem((const void *)reduce_tc_kernel<false>, RCfg<false>::kSmem) &&
+             set_smem((const void *)reduce_tc_kernel<true>, RCfg<true>::kSmem) &&
+             set_smem((const void *)apply_tc_kernel<false>, ACfg<false>::kSmem) &&
+             set_smem((const void *)apply_tc_kernel<true>, ACfg<true>::kSmem);
+    });
+    return ok;
+}
+
+// Entries of the RoPE table of the widest CTA of a kernel whose CTAs cover
+// `span` consecutive tokens of a call.
+long long rope_table_entries(const Plan &p, long long span) {
+    const long long hw = (long long)p.Hg * p.Wg;
+    const long long nf = (span + hw - 1) / hw + 1;
+    long long e = 0;
+    for (int pr = 0; pr < kD / 2; ++pr) e += p.axis[pr] == 0 ? nf : (p.axis[pr] == 1 ? p.Hg : p.Wg);
+    return e;
+}
+
 }  // namespace
 
 bool tc_available() {
@@ -542,31 +788,32 @@ bool tc_available() {
     return major == 10 && minor == 0 && encode_fn() != nullptr;
 }
 
+bool tc_rope_fits(const Plan &p) {
+    return rope_table_entries(p, p.chunk) <= kTabMax && rope_table_entries(p, p.chunka) <= kTabMax;
+}
+
 int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &p, cudaStream_t s) {
-    static std::once_flag once;
-    static bool smem_ok = false;
-    std::call_once(once, [] { smem_ok = set_smem((const void *)reduce_tc_kernel, kRSmem); });
-    if (!smem_ok) return -1;
+    if (!smem_ready()) return -1;
     CUtensorMap mk, mv;
     if (!make_map(&mk, k, p.B, p.N, p.H, 64) || !make_map(&mv, v, p.B, p.N, p.H, 64)) return -1;
     const long long grid = (long long)p.B * (p.H / 4) * p.nb * p.P;
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
-    return launch_pdl(reduce_tc_kernel, (unsigned)grid, kRSmem, s, mk, mv, partials, p) ? 1 : -1;
+    const bool ok = p.rope ? launch_pdl(reduce_tc_kernel<true>, (unsigned)grid, RCfg<true>::kSmem, s, mk, mv, partials, p)
+                           : launch_pdl(reduce_tc_kernel<false>, (unsigned)grid, RCfg<false>::kSmem, s, mk, mv, partials, p);
+    return ok ? 1 : -1;
 }
 
-int launch_apply_tc(const void *q, void *out, const void *bop, const Plan &p, cudaStream_t s) {
-    static std::once_flag once;
-    static bool smem_ok = false;
-    std::call_once(once, [] { smem_ok = set_smem((const void *)apply_tc_kernel, kASmem); });
-    if (!smem_ok) return -1;
+int launch_apply_tc(const void *q, void *out, const void *bop, const float *seff, const Plan &p, cudaStream_t s) {
+    if (!smem_ready()) return -1;
     CUtensorMap mq, mo;
     if (!make_map(&mq, q, p.B, p.N, p.H, 128) || !make_map(&mo, out, p.B, p.N, p.H, 128)) return -1;
     const long long grid = (long long)p.B * p.nb * p.Pa * (p.H / 2);
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
-    return launch_pdl(apply_tc_kernel, (unsigned)grid, kASmem, s, mq, mo, static_cast<__nv_bfloat16 *>(out),
-                      static_cast<const uint8_t *>(bop), p)
-               ? 1
-               : -1;
+    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
+    const uint8_t *bb = static_cast<const uint8_t *>(bop);
+    const bool ok = p.rope ? launch_pdl(apply_tc_kernel<true>, (unsigned)grid, ACfg<true>::kSmem, s, mq, mo, o, bb, seff, p)
+                           : launch_pdl(apply_tc_kernel<false>, (unsigned)grid, ACfg<false>::kSmem, s, mq, mo, o, bb, seff, p);
+    return ok ? 1 : -1;
 }
 
 int read_and_clear_device_flag(cudaStream_t s, unsigned *flag_out) {

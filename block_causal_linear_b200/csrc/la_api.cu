@@ -103,9 +103,10 @@ la_status common_checks(const void *q, const void *k, const void *v, void *out, 
 }
 
 // The tensor-core kernels take bf16 inputs with H a multiple of 4 (4-head
-// reduce groups, 2-head apply tiles) and no RoPE; the rest runs on CUDA cores.
+// reduce groups, 2-head apply tiles) and, with RoPE, a cos/sin table that fits
+// their shared memory; the rest runs on the CUDA cores.
 bool use_tc(la_dtype dt, const la::Plan &p) {
-    return dt == LA_BF16 && (p.H % 4) == 0 && !p.rope && la::tc_available();
+    return dt == LA_BF16 && (p.H % 4) == 0 && (!p.rope || la::tc_rope_fits(p)) && la::tc_available();
 }
 
 // Enqueue reduce -> finish -> apply for a prepared plan.
@@ -127,7 +128,7 @@ la_status run(const void *q, const void *k, const void *v, void *out, la_dtype d
     r = la::launch_finish(partials, seff, bop, S, Z, p, tc ? 1 : 0, s);
     if (r < 0 || !mark(2, s)) return LA_ECUDA;
     n += r;
-    r = tc ? la::launch_apply_tc(q, out, bop, p, s)
+    r = tc ? la::launch_apply_tc(q, out, bop, seff, p, s)
            : la::launch_apply_ffma(dt == LA_BF16, q, out, seff, p, s);
     if (r < 0 || !mark(3, s)) return LA_ECUDA;
     n += r;

@@ -75,8 +75,12 @@ int launch_finish(const float *partials, float *seff, void *bop, float *S, float
 // Tensor-core path (bf16, H % 4 == 0): tcgen05 MMAs, TMA tiles.
 int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &p,
                      cudaStream_t s);
-int launch_apply_tc(const void *q, void *out, const void *bop, const Plan &p, cudaStream_t s);
+int launch_apply_tc(const void *q, void *out, const void *bop, const float *seff, const Plan &p,
+                    cudaStream_t s);
 bool tc_available();
+// The RoPE variants keep a per-CTA (cos, sin) table in shared memory; true if
+// it fits for this plan (else the call takes the CUDA-core kernels).
+bool tc_rope_fits(const Plan &p);
 
 // Device flag raised by a bounded wait that gave up; read-and-clear.
 int read_and_clear_device_flag(cudaStream_t s, unsigned *flag_out);

@@ -32,9 +32,9 @@ def orc_rope(orc, r):
 
 
 def expect_path(la, dtype, H, rope):
-    """bf16 with H % 4 == 0 and no RoPE runs the tensor-core kernels, the rest
-    the FFMA ones."""
-    want = "tc" if (dtype == torch.bfloat16 and H % 4 == 0 and not rope and la.tc_enabled()) else "ffma"
+    """bf16 with H % 4 == 0 runs the tensor-core kernels (with RoPE too: every
+    RoPE grid here fits their cos/sin table), the rest the FFMA ones."""
+    want = "tc" if (dtype == torch.bfloat16 and H % 4 == 0 and la.tc_enabled()) else "ffma"
     assert la.la_last_path() == want
 
 
