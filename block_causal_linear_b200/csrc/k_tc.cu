@@ -132,10 +132,12 @@ __device__ __forceinline__ PairSet pair_set(const Plan &p, int L, int nf) {
 // call), and split the rotated values into hi + lo bf16.  f receives phi(x).
 __device__ __forceinline__ void relu_rotate_chunk(uint4 x, const float2 *tab, const PairSet &ps, const Plan &p,
                                                   long long t, int f_lo, uint4 &hi, uint4 &lo, float (&f)[8]) {
-    const long long hw = (long long)p.Hg * p.Wg;
-    const int fr = (int)(t / hw) - f_lo;
-    const int rem = (int)(t % hw);
-    const int row = rem / p.Wg, col = rem % p.Wg;
+    const int ti = (int)t;                          // tokens of a call < 2^31
+    const int fq = fast_div(ti, p.hw_m, p.hw_s);
+    const int rem = ti - fq * p.Hg * p.Wg;
+    const int row = fast_div(rem, p.wg_m, p.wg_s);
+    const int col = rem - row * p.Wg;
+    const int fr = fq - f_lo;
     const uint32_t w[4] = {relu2(x.x), relu2(x.y), relu2(x.z), relu2(x.w)};
     uint32_t h[4], l[4];
 #pragma unroll

@@ -77,6 +77,8 @@ void fill_rope(la::Plan &p, const la_rope *r, int t_offset) {
     p.Hg = r ? r->Hg : 1;
     p.Wg = r ? r->Wg : 1;
     p.t_offset = t_offset;
+    la::magic_div((unsigned)((long long)p.Hg * p.Wg < (1LL << 31) ? p.Hg * p.Wg : 0x7fffffff), p.hw_m, p.hw_s);
+    la::magic_div((unsigned)p.Wg, p.wg_m, p.wg_s);
     for (int pr = 0; pr < la::kD / 2; ++pr) {
         p.theta[pr] = 0.0f;
         p.axis[pr] = 0;

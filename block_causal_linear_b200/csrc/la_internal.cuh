@@ -35,7 +35,26 @@ struct Plan {
     float eps;
     float theta[kD / 2];  // RoPE frequency of feature pair p
     int axis[kD / 2];     // 0: frame, 1: row, 2: column
+    // n / (Hg*Wg) and n / Wg for 0 <= n < 2^31 as (n * m) >> s (division by an
+    // invariant integer through a multiply, Granlund & Montgomery 1994)
+    unsigned long long hw_m, wg_m;
+    int hw_s, wg_s;
 };
+
+// m, s with floor(n / d) == (n * m) >> s for every 0 <= n < 2^31 (1 <= d < 2^31):
+// l = ceil(log2 d), s = 31 + l, m = ceil(2^s / d); then 2^s <= m d < 2^s + 2^l.
+inline void magic_div(unsigned d, unsigned long long &m, int &s) {
+    int l = 0;
+    while ((1ull << l) < d) ++l;
+    s = 31 + l;
+    m = ((1ull << s) + d - 1) / d;
+}
+
+#ifdef __CUDACC__
+__device__ __forceinline__ int fast_div(int n, unsigned long long m, int s) {
+    return (int)(((unsigned long long)(unsigned)n * m) >> s);
+}
+#endif
 
 // Workspace layout (byte offsets from the 256-byte aligned base).
 struct WsLayout {
