@@ -31,13 +31,9 @@ namespace la {
 namespace {
 
 constexpr int kFinThreads = 256;
-constexpr int kBatch = 8;          // partial loads in flight per thread
+constexpr int kBatch = 32;         // partial loads in flight per thread (one round for P <= 32)
 constexpr int kZeroRows = kOpRows - kD - 1;
 constexpr int kPerBH = kKVZ + kZeroRows * kD;   // numbers + zero-padding entries per (b, h)
-
-__device__ __forceinline__ int op_offset(int nrow, int kcol) {
-    return (nrow >> 3) * 512 + (kcol >> 3) * 128 + (nrow & 7) * 16 + (kcol & 7) * 2;
-}
 
 __global__ void __launch_bounds__(kFinThreads)
 finish_kernel(const float *__restrict__ partials, float *__restrict__ seff,

@@ -21,10 +21,12 @@
 //   unrotated denominator phi(q).Z_eff is summed in fp32 on the CUDA cores.
 //   The epilogue divides, rounds to bf16 and stores with TMA.
 //
-// Both kernels: 6 warps; warp 0 issues TMA, warp 1 owns TMEM and issues the
-// MMAs, warps 2..5 apply phi = ReLU (and RoPE) in shared memory and run the
-// epilogue.  Every wait is bounded (la_sm100.cuh); a wait that gives up raises
-// the device flag read by la_device_status and the CTA drains and returns.
+// Warp roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs.  In the
+// reduce, warps 2..5 apply phi = ReLU (and RoPE) in shared memory and run the
+// epilogue; in the apply, warps 6..9 transform the q tiles while warps 2..5 run
+// the epilogue of the previous tile.  Every wait is bounded (la_sm100.cuh); a
+// wait that gives up raises the device flag read by la_device_status and the
+// CTA drains and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -159,11 +161,13 @@ __device__ __forceinline__ void relu_rotate_chunk(uint4 x, const float2 *tab, co
 
 // ================================================================ reduce
 
-constexpr int kRBox = 64 * 128;   // [64 rows][64 bf16] = 8 KiB
+constexpr int kRRows = 32;                 // token rows per reduce pipeline stage
+constexpr int kRBox = kRRows * 128;        // [32 rows][64 bf16] = 4 KiB
+static_assert(kRRows == 32, "the ReLU pass below maps 128 threads x 4 chunks onto two 32-row boxes");
 
 template <bool ROPE>
 struct RCfg {
-    static constexpr int kStages = ROPE ? 2 : 3;
+    static constexpr int kStages = ROPE ? 4 : 6;
     // stage: k boxes (becoming R phi(k) hi with RoPE), [lo boxes], v boxes
     static constexpr int kLoOff = 2 * kRBox;
     static constexpr int kVOff = ROPE ? 4 * kRBox : 2 * kRBox;
@@ -200,7 +204,7 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     const long long blk1 = blk0 + p.L < p.N ? blk0 + p.L : (long long)p.N;
     const long long t0 = blk0 + (long long)sp * p.chunk;
     const long long t1 = t0 + p.chunk < blk1 ? t0 + p.chunk : blk1;
-    const int nst = t1 > t0 ? (int)((t1 - t0 + 63) / 64) : 0;
+    const int nst = t1 > t0 ? (int)((t1 - t0 + kRRows - 1) / kRRows) : 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     // k, v may come from the kernel just before this one: wait for it, then let
@@ -259,7 +263,7 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 if (!mbar_wait(&empty[s], ph ^ 1u, abort_word, &g_wait_flag, 1)) break;
                 uint8_t *st = smem + s * C::kStageBytes;
                 mbar_arrive_expect_tx(&full[s], 4 * kRBox);
-                const int row = (int)(t0 + 64LL * i);
+                const int row = (int)(t0 + (long long)kRRows * i);
                 const int c0 = g * 128;
                 tma_load_3d(st, &tm_k, &full[s], c0, row, b);
                 tma_load_3d(st + kRBox, &tm_k, &full[s], c0 + 64, row, b);
@@ -281,7 +285,7 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 const uint32_t kaddr = smem_u32(smem + s * C::kStageBytes);
                 const uint32_t vaddr = kaddr + C::kVOff;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
+                for (int kk = 0; kk < kRRows / 16; ++kk) {
                     // MN-major, 128-byte swizzle: 64-wide MN atoms kRBox apart (LBO),
                     // 8-token groups 1024 B apart (SBO); 16 tokens = 2048 B per step
                     const uint64_t da = smem_desc(kaddr + kk * 2048, kRBox, 1024, kLayoutSw128);
@@ -318,11 +322,12 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
             if (!mbar_wait(&full[s], ph, abort_word, &g_wait_flag, 3)) break;
             uint8_t *kt = smem + s * C::kStageBytes;
-            const long long row0 = t0 + 64LL * i;
+            const long long row0 = t0 + (long long)kRRows * i;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < 4; ++j) {             // 512 chunks of 16 bytes: 4 per thread
                 const int c = wt + 128 * j;           // 16-byte chunk of the two k boxes
-                const int r = (c & 511) >> 3;         // token row inside its box
+                const int bx = j >> 1;                // box (heads 0-1 or 2-3): c / 256, as wt < 128
+                const int r = (c % (8 * kRRows)) >> 3;   // token row inside its box
                 uint4 *ptr = reinterpret_cast<uint4 *>(kt + (size_t)c * 16);
                 uint4 x = *ptr;
                 const bool valid = row0 + r < t1;     // rows past the split contribute nothing
@@ -332,7 +337,7 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                         float f[8];
                         relu_rotate_chunk(x, tab, ps, p, row0 + r, f_lo, hi, lo, f);
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) zacc[j >> 2][k] += f[k];
+                        for (int k = 0; k < 8; ++k) zacc[bx][k] += f[k];
                     }
                     *ptr = hi;
                     *reinterpret_cast<uint4 *>(kt + C::kLoOff + (size_t)c * 16) = lo;
@@ -403,26 +408,34 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 
 constexpr int kATile = 128 * 128;              // [128 rows][64 bf16] = 16 KiB: 2 heads
 constexpr int kABopBytes = 2 * 2 * kOpBytes;   // 2 heads x (hi, lo)
+constexpr int kAThreads = 320;                 // 10 warps
+constexpr int kAXform0 = 192;                  // first thread of the transform warps 6..9
+constexpr int kAWarpStg = 32 * 128;            // one epilogue warp's staging box: [32 rows][64 bf16]
 
 template <bool ROPE>
 struct ACfg {
-    static constexpr int kStages = ROPE ? 2 : 3;
+    static constexpr int kStages = ROPE ? 2 : 4;
     static constexpr int kStageBytes = ROPE ? 2 * kATile : kATile;   // [R phi(q) hi | lo] or phi(q)
-    static constexpr int kStgBufs = ROPE ? 1 : 2;                    // TMA store staging buffers
+    static constexpr int kStgBufs = ROPE ? 1 : 2;                    // staging boxes per epilogue warp
     static constexpr int kOutOff = kStages * kStageBytes;
-    static constexpr int kBopOff = kOutOff + kStgBufs * kATile;
+    static constexpr int kBopOff = kOutOff + 4 * kStgBufs * kAWarpStg;
     static constexpr int kDenOff = kBopOff + kABopBytes;             // RoPE: [2][128 rows][2 heads] fp32
     static constexpr int kZOff = kDenOff + (ROPE ? 2 * 1024 : 0);     // RoPE: Z_eff of the 2 heads
     static constexpr int kTabOff = kZOff + (ROPE ? 256 : 0);
     static constexpr int kBarOff = kTabOff + (ROPE ? kTabMax * 8 : 0);
-    static constexpr int kSmem = kBarOff + (3 * kStages + 6) * 8 + 16 + 1024;
+    static constexpr int kNumBars = 3 * kStages + 2 + 2 + 2 + 2 + 3;  // + acc[2], acc_empty[2], den[2], den_free[2], bop, drain, dep
+    static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
     static constexpr int kAccCols = ROPE ? 64 : 96;                  // per TMEM buffer (2 heads)
     static constexpr int kHeadCols = ROPE ? 32 : kOpRows;
     static constexpr uint32_t kTmemCols = ROPE ? 128 : 256;
 };
 
+// Warp roles: 0 issues TMA, 1 owns TMEM and issues the MMAs, 2..5 run the
+// epilogue (warp w reads TMEM lanes 32*(w%4).. = token rows of the tile),
+// 6..9 apply phi (and RoPE) to the q tiles in shared memory.  The transform
+// of tile i+1 and the epilogue of tile i run at the same time.
 template <bool ROPE>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kAThreads, 2)
 apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_out,
                 __nv_bfloat16 *__restrict__ out, const uint8_t *__restrict__ bop, const float *__restrict__ seff,
                 const Plan p) {
@@ -435,13 +448,16 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float *zs = reinterpret_cast<float *>(smem + C::kZOff);
     const float2 *tab = reinterpret_cast<const float2 *>(smem + C::kTabOff);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
-    uint64_t *relu_done = full + C::kStages;
-    uint64_t *empty = relu_done + C::kStages;
+    uint64_t *xform_done = full + C::kStages;
+    uint64_t *empty = xform_done + C::kStages;
     uint64_t *acc_full = empty + C::kStages;   // [2]
     uint64_t *acc_empty = acc_full + 2;        // [2]
-    uint64_t *bop_full = acc_empty + 2;
+    uint64_t *den_ready = acc_empty + 2;       // [2] RoPE: den_s[i & 1] written
+    uint64_t *den_free = den_ready + 2;        // [2] RoPE: den_s[i & 1] read
+    uint64_t *bop_full = den_free + 2;
     uint64_t *drain = bop_full + 1;            // only used when a wait gave up
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *dep_ready = drain + 1;           // the previous kernel (state combine) has completed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(dep_ready + 1);
     volatile int *abort_word = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int Gp = p.H / 2;
@@ -467,20 +483,23 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&relu_done[s], kWork);
+            mbar_init(&xform_done[s], kWork);
             mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&acc_full[a], 1);
             mbar_init(&acc_empty[a], kWork);
+            mbar_init(&den_ready[a], kWork);
+            mbar_init(&den_free[a], kWork);
         }
         mbar_init(bop_full, 1);
         mbar_init(drain, 1);
+        mbar_init(dep_ready, 1);
         *abort_word = 0;
         fence_barrier_init();
     }
     if constexpr (ROPE)
-        build_rope_table(reinterpret_cast<float2 *>(smem + C::kTabOff), p, f_lo, nf, threadIdx.x, kThreads);
+        build_rope_table(reinterpret_cast<float2 *>(smem + C::kTabOff), p, f_lo, nf, threadIdx.x, kAThreads);
     if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
@@ -506,7 +525,8 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tma_load_3d(smem + i * C::kStageBytes, &tm_q, &full[i], hp * 64, (int)(ta0 + 128LL * i), b);
                 issued = i + 1;
             }
-            pdl_wait();   // the packed operand is written by the previous kernel
+            pdl_wait();   // the packed operand and Z_eff are written by the previous kernel
+            mbar_arrive(dep_ready);
             mbar_arrive_expect_tx(bop_full, kABopBytes);
             for (int hh = 0; hh < 2; ++hh) {
                 const size_t src = (((size_t)b * p.H + 2 * hp + hh) * p.nb + n) * 2 * kOpBytes;
@@ -532,7 +552,7 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
                     const int ab = i & 1;
                     const uint32_t aph = (uint32_t)(i >> 1) & 1u;
-                    if (!mbar_wait(&relu_done[s], ph, abort_word, &g_wait_flag, 13)) break;
+                    if (!mbar_wait(&xform_done[s], ph, abort_word, &g_wait_flag, 13)) break;
                     if (!mbar_wait(&acc_empty[ab], aph ^ 1u, abort_word, &g_wait_flag, 14)) break;
                     tc_fence_after();
                     const uint32_t qaddr = smem_u32(smem + s * C::kStageBytes);
@@ -563,129 +583,160 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
         }
-    } else {
-        const int wt = threadIdx.x - 64;
-        const int qd = warp & 3;
-        const int r = 32 * qd + lane;               // token row of this thread in a tile
-        const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
+    } else if (warp >= 6) {
+        // ------------------------------------------------ transform warps
+        const int tt = threadIdx.x - kAXform0;   // 0..127
         bool ok = true;
-        const int L = (wt & 7) ^ ((wt >> 3) & 7);   // logical chunk this thread meets (RoPE)
-        PairSet ps{};
-        if constexpr (ROPE) ps = pair_set(p, L, nf);
-
-        pdl_wait();   // every write to `out` (and the read of Z_eff) comes after the previous kernel
         if constexpr (ROPE) {
-            if (wt < 2 * kD)
-                zs[wt] = seff[(((size_t)b * p.H + 2 * hp + (wt >> 5)) * p.nb + n) * kKVZ + kD * kD + (wt & 31)];
-            named_bar_sync(1, kWork);
+            // Z_eff comes from the state combine (the previous kernel)
+            if (!mbar_wait(dep_ready, 0, abort_word, &g_wait_flag, 19)) ok = false;
+            if (tt < 2 * kD)
+                zs[tt] = __ldcg(seff + (((size_t)b * p.H + 2 * hp + (tt >> 5)) * p.nb + n) * kKVZ + kD * kD + (tt & 31));
+            named_bar_sync(2, kWork);
         }
-
-        // A wait that gives up (abort) makes this thread skip work, never leave
-        // the loop: every work thread takes the same named barriers, and TMEM
-        // reads are taken or skipped by whole warps.
-        auto relu_tile = [&](int i) {
+        // RoPE: this thread handles chunk pairs (pc, pc ^ 4) of one row: the same
+        // 8 features of both heads, so positions and cos/sin are shared.  Its
+        // swizzle phase, and so its logical chunk L0 (head 0 or 1), is fixed.
+        const int L0 = (tt & 3) ^ ((tt >> 2) & 7);
+        PairSet ps{};
+        if constexpr (ROPE) ps = pair_set(p, L0, nf);
+        for (int i = 0; i < ntiles; ++i) {
             const int s = i % C::kStages;
             const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
             if (ok && !mbar_wait(&full[s], ph, abort_word, &g_wait_flag, 15)) ok = false;
             uint8_t *qt = smem + s * C::kStageBytes;
             const long long row0 = ta0 + 128LL * i;
-            if constexpr (ROPE) named_bar_sync(1, kWork);   // den_s[i & 1] was read by the epilogue of tile i-2
+            if constexpr (ROPE) {
+                if (ok && !mbar_wait(&den_free[i & 1], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_word, &g_wait_flag, 17))
+                    ok = false;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int c = wt + 128 * j;
-                uint4 *ptr = reinterpret_cast<uint4 *>(qt + (size_t)c * 16);
-                if constexpr (ROPE) {
-                    const int rr = c >> 3;                      // token row of this chunk
+                for (int j = 0; j < 4; ++j) {
+                    const int u = tt + 128 * j;       // chunk pair index
+                    const int rr = u >> 2;            // token row
+                    const int pc0 = u & 3;            // physical chunk of the first of the pair
                     const bool valid = ok && row0 + rr < ta1;
-                    uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
-                    float dp = 0.f;
-                    if (valid) {
-                        float f[8];
-                        relu_rotate_chunk(*ptr, tab, ps, p, row0 + rr, f_lo, hi, lo, f);
-                        const float *zh = zs + (L >> 2) * kD + (L & 3) * 8;
+                    float dp[2] = {0.f, 0.f};
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) dp = fmaf(f[k], zh[k], dp);
+                    for (int e = 0; e < 2; ++e) {
+                        const int pc = pc0 + 4 * e;
+                        const int L = pc ^ (rr & 7);  // = L0 for e = 0, L0 ^ 4 for e = 1
+                        uint4 *ptr = reinterpret_cast<uint4 *>(qt + rr * 128 + pc * 16);
+                        uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
+                        if (valid) {
+                            float f[8];
+                            relu_rotate_chunk(*ptr, tab, ps, p, row0 + rr, f_lo, hi, lo, f);
+                            const float *zh = zs + (L >> 2) * kD + (L & 3) * 8;
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) dp[e] = fmaf(f[k], zh[k], dp[e]);
+                        }
+                        *ptr = hi;
+                        *reinterpret_cast<uint4 *>(qt + kATile + rr * 128 + pc * 16) = lo;
                     }
-                    *ptr = hi;
-                    *reinterpret_cast<uint4 *>(qt + kATile + (size_t)c * 16) = lo;
-                    // the 4 chunks of one head in a row sit on lanes that differ in bits 0-1
-                    dp += __shfl_xor_sync(0xffffffffu, dp, 1);
-                    dp += __shfl_xor_sync(0xffffffffu, dp, 2);
-                    if ((lane & 3) == 0) den_s[(i & 1) * 256 + rr * 2 + (L >> 2)] = dp;
-                } else if (ok) {
+                    // the 4 chunk pairs of a row sit on 4 consecutive lanes
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        dp[e] += __shfl_xor_sync(0xffffffffu, dp[e], 1);
+                        dp[e] += __shfl_xor_sync(0xffffffffu, dp[e], 2);
+                    }
+                    if ((lane & 3) == 0) {
+                        const int h0 = L0 >> 2;
+                        den_s[(i & 1) * 256 + rr * 2 + h0] = dp[0];
+                        den_s[(i & 1) * 256 + rr * 2 + (h0 ^ 1)] = dp[1];
+                    }
+                }
+            } else if (ok) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint4 *ptr = reinterpret_cast<uint4 *>(qt + (size_t)(tt + 128 * j) * 16);
                     uint4 x = *ptr;
                     x.x = relu2(x.x); x.y = relu2(x.y); x.z = relu2(x.z); x.w = relu2(x.w);
                     *ptr = x;
                 }
             }
             fence_proxy_async_smem();
-            mbar_arrive(&relu_done[s]);
-        };
-
-        if (ntiles > 0) relu_tile(0);
+            mbar_arrive(&xform_done[s]);
+            if constexpr (ROPE) mbar_arrive(&den_ready[i & 1]);
+        }
+    } else {
+        // ------------------------------------------------ epilogue warps 2..5
+        const int qd = warp & 3;
+        const int r = 32 * qd + lane;               // token row of this thread in a tile
+        const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
+        uint8_t *wstg = stg + qd * C::kStgBufs * kAWarpStg;   // this warp's staging boxes
+        bool ok = true;
         for (int i = 0; i < ntiles; ++i) {
-            if (i + 1 < ntiles) relu_tile(i + 1);
             const int ab = i & 1;
             const uint32_t aph = (uint32_t)(i >> 1) & 1u;
             bool got = ok && mbar_wait(&acc_full[ab], aph, abort_word, &g_wait_flag, 16);
+            if constexpr (ROPE) got = got && mbar_wait(&den_ready[i & 1], aph, abort_word, &g_wait_flag, 18);
             got = __all_sync(0xffffffffu, got);
             if (!got) ok = false;
-            uint32_t packed[2][16];
+            float num0[32], num1[32], den0 = 0.f, den1 = 0.f;
             if (got) {
                 tc_fence_after();
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float num[32];
-                    tmem_ld32(tmem + lane_off + ab * C::kAccCols + hh * C::kHeadCols, num);
-                    float den;
-                    if constexpr (ROPE) {
-                        den = den_s[(i & 1) * 256 + r * 2 + hh];
-                    } else {
-                        den = tmem_ld1(tmem + lane_off + ab * C::kAccCols + hh * C::kHeadCols + kD);
-                    }
-                    tmem_wait_ld();
-                    const float inv = 1.0f / (den + p.eps);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) packed[hh][j] = pack_bf2(num[2 * j] * inv, num[2 * j + 1] * inv);
+                const uint32_t base = tmem + lane_off + ab * C::kAccCols;
+                tmem_ld32(base, num0);
+                tmem_ld32(base + C::kHeadCols, num1);
+                if constexpr (!ROPE) {
+                    den0 = tmem_ld1(base + kD);
+                    den1 = tmem_ld1(base + C::kHeadCols + kD);
+                }
+                tmem_wait_ld();
+                if constexpr (ROPE) {
+                    den0 = den_s[(i & 1) * 256 + r * 2];
+                    den1 = den_s[(i & 1) * 256 + r * 2 + 1];
                 }
             }
             tc_fence_before();
             mbar_arrive(&acc_empty[ab]);
+            if constexpr (ROPE) mbar_arrive(&den_free[i & 1]);
 
             const long long row0 = ta0 + 128LL * i;
-            const bool whole = row0 + 128 <= ta1 || ta1 == p.N;   // TMA clips rows >= N
-            if (whole) {
-                uint8_t *sb = stg + (i % C::kStgBufs) * kATile;
-                if (wt == 0) bulk_wait_read<C::kStgBufs - 1>();   // the last store from sb has read it
-                named_bar_sync(1, kWork);
+            const long long wrow0 = row0 + 32 * qd;    // first row of this warp
+            // TMA store of the warp's 32 rows unless they run into another block
+            // (rows past the end of the tensor are clipped by TMA)
+            const bool boxed = wrow0 + 32 <= ta1 || ta1 == p.N;
+            if (boxed) {
+                uint8_t *sb = wstg + (i % C::kStgBufs) * kAWarpStg;
+                if (lane == 0) bulk_wait_read<C::kStgBufs - 1>();   // the last store from sb has read it
+                __syncwarp();
                 if (got) {
+                    const float inv0 = 1.0f / (den0 + p.eps), inv1 = 1.0f / (den1 + p.eps);
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {       // logical 16-byte chunk c: head c/4
-                        const int pc = c ^ (r & 7);     // 128-byte swizzle
-                        *reinterpret_cast<uint4 *>(sb + r * 128 + pc * 16) =
-                            make_uint4(packed[c >> 2][4 * (c & 3)], packed[c >> 2][4 * (c & 3) + 1],
-                                       packed[c >> 2][4 * (c & 3) + 2], packed[c >> 2][4 * (c & 3) + 3]);
+                        const float *v = c < 4 ? num0 : num1;
+                        const float inv = c < 4 ? inv0 : inv1;
+                        const int f0 = 8 * (c & 3);
+                        const int pc = c ^ (lane & 7);  // 128-byte swizzle (row % 8 == lane % 8)
+                        *reinterpret_cast<uint4 *>(sb + lane * 128 + pc * 16) =
+                            make_uint4(pack_bf2(v[f0] * inv, v[f0 + 1] * inv), pack_bf2(v[f0 + 2] * inv, v[f0 + 3] * inv),
+                                       pack_bf2(v[f0 + 4] * inv, v[f0 + 5] * inv), pack_bf2(v[f0 + 6] * inv, v[f0 + 7] * inv));
                     }
                 }
                 fence_proxy_async_smem();
-                named_bar_sync(1, kWork);
-                if (wt == 0 && ok) {
-                    tma_store_3d(&tm_out, sb, hp * 64, (int)row0, b);
+                __syncwarp();
+                if (lane == 0 && ok) {
+                    tma_store_3d(&tm_out, sb, hp * 64, (int)wrow0, b);
                     bulk_commit();
                 }
             } else if (got && row0 + r < ta1) {
                 // a short last tile inside the tensor: the rows after ta1 belong to another block
+                const float inv0 = 1.0f / (den0 + p.eps), inv1 = 1.0f / (den1 + p.eps);
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
+                    const float *v = hh ? num1 : num0;
+                    const float inv = hh ? inv1 : inv0;
                     uint4 *dst = reinterpret_cast<uint4 *>(out + (((size_t)b * p.N + row0 + r) * p.H + 2 * hp + hh) * kD);
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
-                        dst[c] = make_uint4(packed[hh][4 * c], packed[hh][4 * c + 1], packed[hh][4 * c + 2],
-                                            packed[hh][4 * c + 3]);
+                        dst[c] = make_uint4(pack_bf2(v[8 * c] * inv, v[8 * c + 1] * inv),
+                                            pack_bf2(v[8 * c + 2] * inv, v[8 * c + 3] * inv),
+                                            pack_bf2(v[8 * c + 4] * inv, v[8 * c + 5] * inv),
+                                            pack_bf2(v[8 * c + 6] * inv, v[8 * c + 7] * inv));
                 }
             }
         }
-        if (wt == 0) bulk_wait_all();
+        if (lane == 0) bulk_wait_all();
     }
 
     if (warp == kWarpTma && lane == 0 && *abort_word) {
@@ -740,10 +791,11 @@ bool make_map(CUtensorMap *m, const void *base, int B, int N, int H, int box_row
 // Launch with programmatic stream serialization (the kernel may start while
 // the previous kernel of the stream drains; it orders itself with pdl_wait).
 template <typename... KArgs, typename... Args>
-bool launch_pdl(void (*kernel)(KArgs...), unsigned grid, int smem, cudaStream_t s, Args &&...args) {
+bool launch_pdl(void (*kernel)(KArgs...), unsigned grid, int threads, int smem, cudaStream_t s,
+                Args &&...args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -797,24 +849,28 @@ bool tc_rope_fits(const Plan &p) {
 int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &p, cudaStream_t s) {
     if (!smem_ready()) return -1;
     CUtensorMap mk, mv;
-    if (!make_map(&mk, k, p.B, p.N, p.H, 64) || !make_map(&mv, v, p.B, p.N, p.H, 64)) return -1;
+    if (!make_map(&mk, k, p.B, p.N, p.H, kRRows) || !make_map(&mv, v, p.B, p.N, p.H, kRRows)) return -1;
     const long long grid = (long long)p.B * (p.H / 4) * p.nb * p.P;
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
-    const bool ok = p.rope ? launch_pdl(reduce_tc_kernel<true>, (unsigned)grid, RCfg<true>::kSmem, s, mk, mv, partials, p)
-                           : launch_pdl(reduce_tc_kernel<false>, (unsigned)grid, RCfg<false>::kSmem, s, mk, mv, partials, p);
+    const bool ok = p.rope ? launch_pdl(reduce_tc_kernel<true>, (unsigned)grid, kThreads, RCfg<true>::kSmem, s, mk,
+                                        mv, partials, p)
+                           : launch_pdl(reduce_tc_kernel<false>, (unsigned)grid, kThreads, RCfg<false>::kSmem, s, mk,
+                                        mv, partials, p);
     return ok ? 1 : -1;
 }
 
 int launch_apply_tc(const void *q, void *out, const void *bop, const float *seff, const Plan &p, cudaStream_t s) {
     if (!smem_ready()) return -1;
     CUtensorMap mq, mo;
-    if (!make_map(&mq, q, p.B, p.N, p.H, 128) || !make_map(&mo, out, p.B, p.N, p.H, 128)) return -1;
+    if (!make_map(&mq, q, p.B, p.N, p.H, 128) || !make_map(&mo, out, p.B, p.N, p.H, 32)) return -1;
     const long long grid = (long long)p.B * p.nb * p.Pa * (p.H / 2);
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
     const uint8_t *bb = static_cast<const uint8_t *>(bop);
-    const bool ok = p.rope ? launch_pdl(apply_tc_kernel<true>, (unsigned)grid, ACfg<true>::kSmem, s, mq, mo, o, bb, seff, p)
-                           : launch_pdl(apply_tc_kernel<false>, (unsigned)grid, ACfg<false>::kSmem, s, mq, mo, o, bb, seff, p);
+    const bool ok = p.rope ? launch_pdl(apply_tc_kernel<true>, (unsigned)grid, kAThreads, ACfg<true>::kSmem, s, mq,
+                                        mo, o, bb, seff, p)
+                           : launch_pdl(apply_tc_kernel<false>, (unsigned)grid, kAThreads, ACfg<false>::kSmem, s, mq,
+                                        mo, o, bb, seff, p);
     return ok ? 1 : -1;
 }
 

@@ -54,6 +54,13 @@ inline void magic_div(unsigned d, unsigned long long &m, int &s) {
 __device__ __forceinline__ int fast_div(int n, unsigned long long m, int s) {
     return (int)(((unsigned long long)(unsigned)n * m) >> s);
 }
+
+// Byte offset of element (n, k) of one packed bf16 MMA operand [S | Z | 0]
+// (K = 32 key features, N = 48 columns): K-major, no swizzle, core matrices
+// of 8 rows x 16 bytes, 128 B apart along K and 512 B apart along N.
+__device__ __forceinline__ int op_offset(int nrow, int kcol) {
+    return (nrow >> 3) * 512 + (kcol >> 3) * 128 + (nrow & 7) * 16 + (kcol & 7) * 2;
+}
 #endif
 
 // Workspace layout (byte offsets from the 256-byte aligned base).
@@ -92,8 +99,9 @@ int launch_finish(const float *partials, float *seff, void *bop, float *S, float
                   const Plan &p, int write_bop, cudaStream_t s);
 
 // Tensor-core path (bf16, H % 4 == 0): tcgen05 MMAs, TMA tiles.
-int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &p,
-                     cudaStream_t s);
+// The three kernels of a call (reduce, finish above, apply) order themselves
+// by grid through programmatic dependent launch.
+int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &p, cudaStream_t s);
 int launch_apply_tc(const void *q, void *out, const void *bop, const float *seff, const Plan &p,
                     cudaStream_t s);
 bool tc_available();

@@ -190,3 +190,18 @@ def test_runtime_errors_are_reported(la):
     with pytest.raises(la.LAError):
         la.full_forward(q, k, v, 0, eps=EPS, ws=torch.empty(16, dtype=torch.uint8, device="cuda"))
     la.device_status()
+
+
+
+def test_one_workspace_serves_calls_of_different_shapes(la, orc):
+    """A workspace sized for the largest call is reused, without clearing, by
+    calls of other shapes and block counts in turn."""
+    big = la.alloc_workspace(2, 3000, 8, 32, 0)
+    for (B, N, H, L) in [(1, 3000, 8, 0), (2, 1000, 8, 0), (1, 129, 4, 0), (2, 2000, 8, 700), (2, 3000, 8, 0)]:
+        q, k, v = synth.random_qkv(B, N, H, 32, seed=40 + N, dtype=torch.bfloat16)
+        assert la.la_workspace_size(B, N, H, 32, L) <= big.numel()
+        g = la.full_forward(q.cuda(), k.cuda(), v.cuda(), L, eps=EPS, ws=big)
+        torch.cuda.synchronize()
+        la.device_status()
+        ref = orc.full_forward(q, k, v, L, eps=EPS)
+        assert err_out(g, ref, torch.bfloat16) <= tol_out(torch.bfloat16)
