@@ -11,8 +11,10 @@ step; the step time is the device time between CUDA events recorded before
 its first and after its last kernel, so the flush is not in it.  The metric
 is token*heads per second (every pass counts), whole job over all ranks.
 
-Multi-GPU: one process per GPU (torchrun), each rank an independent problem
-of the same shape (its own seed), no data-path collective: weak scaling.  The
+Multi-GPU: one process per GPU (torchrun), no data-path collective.  By
+default each rank runs an independent problem of the same shape (its own
+seed): weak scaling.  With --shard heads the 64 heads of one problem are split
+over the ranks (each owns its heads' tensors and state): strong scaling.  The
 timed totals are reduced with MAX over ranks.
 
 --impl reference times the fp64 CPU oracle (the test oracle, unchanged) on
@@ -36,7 +38,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from block_causal_linear_b200 import synth  # noqa: E402
+from block_causal_linear_b200 import ranks, synth  # noqa: E402
 
 METRIC = "block linear-attn tokens·heads/s and achieved HBM GB/s vs B200 peak (1 GPU)"
 UNIT = "token·heads/s"
@@ -56,6 +58,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--shard", default="problem", choices=["problem", "heads"],
+                    help="problem: an independent problem per rank (weak scaling); "
+                         "heads: one problem's heads split over the ranks (strong scaling)")
     return ap.parse_args()
 
 
@@ -262,7 +267,13 @@ def main():
     from block_causal_linear_b200.runner import Runner
 
     base = synth.WORKLOADS[args.config]
-    w = base.shrink(seed=base.seed + 1000 * rank) if rank else base
+    if args.shard == "heads":
+        h0, h1 = ranks.head_slice(base.H, world, rank)
+        if h1 <= h0:
+            raise SystemExit(f"--shard heads: rank {rank} of {world} has no heads of {base.H}")
+        w = ranks.rank_workload(base, rank).shrink(H=h1 - h0)
+    else:
+        w = ranks.rank_workload(base, rank)
     dev = torch.device("cuda", local_rank)
     runner = Runner(w, dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -288,10 +299,7 @@ def main():
         torch.cuda.synchronize()
         est = e0.elapsed_time(e1) / 1e3 + 1e-4
         args.steps = int(min(20000, max(20, 2.0 / est)))
-        if dist is not None:
-            t = torch.tensor([args.steps], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MIN)
-            args.steps = int(t.item())
+        args.steps = ranks.agree_steps(args.steps, dist, dev)
     K = args.steps
 
     # one step captured as a CUDA graph (the library is capture-safe: it never
@@ -369,13 +377,11 @@ def main():
                 stage_ms[j] += e[j].elapsed_time(e[j + 1])
     stage_ms = [x * K / Ks for x in stage_ms]      # scaled to K steps like total_ms
     total_ms = sum(step_ms)
-    tot = torch.tensor([total_ms, sum(outer_ms)] + stage_ms, dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
-    total_ms, outer_total_ms, red_ms, fin_ms, app_ms = (float(x) for x in tot.tolist())
+    total_ms, outer_total_ms, red_ms, fin_ms, app_ms = ranks.max_over_ranks(
+        [total_ms, sum(outer_ms)] + stage_ms, dist, dev)
 
     th_step = w.token_heads                          # per rank per step
-    value = th_step * world * K / (total_ms / 1e3)
+    value = ranks.job_throughput(th_step, world, K, total_ms)
     ms_per_step = total_ms / K
     peak, peak_kind = measured_peaks()
     step_gbs = w.alg_bytes / (ms_per_step / 1e3) / 1e9
@@ -406,8 +412,11 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
-            "data": "synthetic", "config": workload_config(w, {"parallelism": f"independent problem per rank x{world}"}),
+            "scaling": "strong" if args.shard == "heads" else "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": workload_config(w, {"parallelism": (f"heads of one problem split over {world} ranks"
+                                                          if args.shard == "heads" else
+                                                          f"independent problem per rank x{world}")}),
             "achieved_hbm_gbs": step_gbs, "hbm_frac_of_" + peak_kind: step_gbs / peak,
             "stage_ms_per_step": {"reduce": red_ms / K, "finish": fin_ms / K, "apply": app_ms / K},
             "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
@@ -454,11 +463,8 @@ def measure_e2e(runner, w, dev, world, dist, steps):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
-    return {"value": w.token_heads * world * steps / (ms / 1e3), "unit": UNIT,
+    ms = ranks.max_over_ranks([ms], dist, dev)[0]
+    return {"value": ranks.job_throughput(w.token_heads, world, steps, ms), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
 
 

@@ -1,0 +1,130 @@
+"""Multi-rank host logic on CPU: world size 2 over gloo.
+
+A multi-GPU job runs one process per GPU with no data-path collective (every
+(batch, head) pair is independent); these tests run the same helpers bench.py
+uses (block_causal_linear_b200.ranks) in two gloo processes:
+
+- head sharding: each rank streams its slice of one problem's heads through
+  the oracle (three blocks, commit on each) and the gathered outputs and
+  states equal the unsharded run bit for bit;
+- weak scaling: the ranks' problems have the same shape and different inputs;
+- the collectives of the timing path: MIN over ranks for the step count, MAX
+  for the times, and the job throughput from the slowest rank.
+"""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, errfile):
+    try:
+        sys.path.insert(0, ROOT)
+        os.environ["MASTER_ADDR"] = "127.0.0.1"
+        os.environ["MASTER_PORT"] = str(port)
+        from datetime import timedelta
+
+        dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+        import oracle as orc
+        from block_causal_linear_b200 import ranks, synth
+
+        # ---- head sharding of one problem (configuration 1 shape, 6 heads)
+        w = synth.WORKLOADS[1].shrink(H=6)
+        calls = list(synth.stream(w, "cpu"))
+        h0, h1 = ranks.head_slice(w.H, world, rank)
+        st = orc.State(w.B, h1 - h0, w.d)
+        outs = []
+        for (_, _, q, k, v) in calls:
+            outs.append(orc.block_forward(q[:, :, h0:h1].contiguous(), k[:, :, h0:h1].contiguous(),
+                                          v[:, :, h0:h1].contiguous(), st, commit=True, eps=w.eps))
+        mine = {"h": (h0, h1), "out": np.concatenate(outs, 1), "S": st.S.copy(), "Z": st.Z.copy()}
+        got = [None] * world
+        dist.all_gather_object(got, mine)
+        if rank == 0:
+            got.sort(key=lambda x: x["h"][0])
+            assert got[0]["h"][0] == 0 and got[-1]["h"][1] == w.H
+            assert all(a["h"][1] == b["h"][0] for a, b in zip(got, got[1:]))
+            full = orc.State(w.B, w.H, w.d)
+            ref = np.concatenate([orc.block_forward(q, k, v, full, commit=True, eps=w.eps)
+                                  for (_, _, q, k, v) in calls], 1)
+            assert np.array_equal(np.concatenate([x["out"] for x in got], 2), ref)
+            assert np.array_equal(np.concatenate([x["S"] for x in got], 1), full.S)
+            assert np.array_equal(np.concatenate([x["Z"] for x in got], 1), full.Z)
+
+        # ---- weak scaling: same shape, own inputs
+        wr = ranks.rank_workload(synth.WORKLOADS[2], rank)
+        q = synth.random_qkv(1, 16, 4, 32, seed=wr.seed)[0]
+        shapes = [None] * world
+        dist.all_gather_object(shapes, ((wr.B, wr.n_total, wr.H, wr.d), wr.seed, q))
+        if rank == 0:
+            assert len({s[0] for s in shapes}) == 1
+            assert len({s[1] for s in shapes}) == world
+            assert not torch.equal(shapes[0][2], shapes[1][2])
+
+        # ---- timing collectives
+        assert ranks.agree_steps(20 + 7 * rank, dist) == 20
+        tmax = ranks.max_over_ranks([1.0 + rank, 10.0 - rank, 0.5], dist)
+        assert tmax == [float(world), 10.0, 0.5]
+        v = ranks.job_throughput(1000, world, 4, tmax[0])
+        assert v == pytest.approx(1000 * world * 4 / (world / 1e3))
+        dist.barrier()
+        dist.destroy_process_group()
+    except BaseException as e:  # report to the parent, which fails the test
+        import traceback
+
+        with open(errfile, "a") as f:
+            f.write(f"rank {rank}: {e!r}\n{traceback.format_exc()}\n")
+        raise
+
+
+def test_two_ranks_gloo(orc, tmp_path):
+    errfile = str(tmp_path / "errors.txt")
+    world = 2
+    ctx = mp.get_context("spawn")
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, errfile)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    alive = [p for p in procs if p.is_alive()]
+    for p in alive:
+        p.kill()
+        p.join()
+    err = open(errfile).read() if os.path.exists(errfile) else ""
+    assert not alive, "a rank did not finish"
+    assert all(p.exitcode == 0 for p in procs), err
+    assert not err, err
+
+
+def test_head_slice_partitions():
+    sys.path.insert(0, ROOT)
+    from block_causal_linear_b200 import ranks
+
+    for H in (1, 2, 4, 6, 8, 12, 64, 66):
+        for world in (1, 2, 3, 4, 8):
+            sl = [ranks.head_slice(H, world, r) for r in range(world)]
+            assert sl[0][0] == 0 and sl[-1][1] == H
+            assert all(a[1] == b[0] for a, b in zip(sl, sl[1:]))
+            sizes = [b - a for a, b in sl]
+            if H % 4 == 0:
+                assert all(s % 4 == 0 for s in sizes)
+                assert max(sizes) - min(sizes) <= 4
+            else:
+                assert max(sizes) - min(sizes) <= 1
+    assert ranks.head_slice(64, 8, 3) == (24, 32)
+    with pytest.raises(ValueError):
+        ranks.head_slice(64, 2, 2)
