@@ -6,8 +6,11 @@
 One step is one of the workloads (default: configuration 2, the 5 s 480p
 latent as a single bidirectional block, 8190 tokens x 64 heads x d 32, bf16)
 run once through the library from a zero state, with every input already
-resident in HBM.  L2 is flushed (a 256 MiB device write) before every timed
-step; the step time is the device time between CUDA events recorded before
+resident in HBM.  L2 is flushed before every timed step: a 256 MiB device
+write, then a read of another 256 MiB buffer, so that no input line is in L2
+and the flush's own dirty lines are written back before the step starts (a
+write alone leaves ~126 MB of them to be written back inside the step); the
+step time is the device time between CUDA events recorded before
 its first and after its last kernel, so the flush is not in it.  The metric
 is token*heads per second (every pass counts), whole job over all ranks.
 
@@ -70,7 +73,8 @@ def workload_config(w: synth.Workload, extra=None):
          "calls_per_step": w.calls, "api": "la_full_forward" if w.mode == "full" else "la_block_forward",
          "rope": "3d 8/12/12 base 1e4" if w.rope else None, "input_dtype": w.dtype,
          "accumulate": "f32", "state": "f32",
-         "l2": "flushed before every timed step (256 MiB device write, outside the step's events)"}
+         "l2": "flushed before every timed step (256 MiB device write, then a 256 MiB device read so that "
+               "the write's dirty lines leave L2 too; outside the step's events)"}
     if extra:
         c.update(extra)
     return c
@@ -276,7 +280,17 @@ def main():
         w = ranks.rank_workload(base, rank)
     dev = torch.device("cuda", local_rank)
     runner = Runner(w, dev)
-    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_w = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_acc = torch.empty(1, dtype=torch.float32, device=dev)
+
+    class _Flush:
+        @staticmethod
+        def fill_(x):
+            flush_w.fill_(x)
+            torch.sum(flush_r, dim=0, out=flush_acc)
+
+    flush = _Flush()
     stream = torch.cuda.current_stream()
     n_calls = len(runner.calls)
 

@@ -397,6 +397,9 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     }
     if (warp == kWarpMma && lane == 0) final_wait(acc_ready, 0);
     tc_fence_before();
+    // lanes that skipped the single-lane roles wait for their lane 0 here, so
+    // every warp reaches the block barrier whole
+    __syncwarp();
     __syncthreads();
     if (warp == kWarpMma) {
         tc_fence_after();
@@ -750,6 +753,9 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         final_wait(drain, 0);
     }
     tc_fence_before();
+    // lanes that skipped the single-lane roles wait for their lane 0 here, so
+    // every warp reaches the block barrier whole
+    __syncwarp();
     __syncthreads();
     if (warp == kWarpMma) {
         tc_fence_after();
