@@ -61,6 +61,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--blocks", type=int, default=None,
+                    help="streaming workloads: run only the first N blocks (small cases for profiling)")
     ap.add_argument("--shard", default="problem", choices=["problem", "heads"],
                     help="problem: an independent problem per rank (weak scaling); "
                          "heads: one problem's heads split over the ranks (strong scaling)")
@@ -279,6 +281,10 @@ def main():
     else:
         w = ranks.rank_workload(base, rank)
     dev = torch.device("cuda", local_rank)
+    if args.blocks is not None:
+        if w.mode != "stream" or not 1 <= args.blocks <= w.n_blocks:
+            raise SystemExit("--blocks needs a streaming workload and 1 <= N <= its block count")
+        w = w.shrink(n_blocks=args.blocks)
     runner = Runner(w, dev)
     flush_w = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -408,7 +414,7 @@ def main():
     avg_launch_s = dom_ms / launches_per_kernel / 1e3
     achieved = kern_bytes / avg_launch_s / 1e9
     path = la.la_last_path()
-    kname = f"{dom}_{path}"
+    kname = f"{dom}_{path}" + ("_rope" if w.rope and path == "tc" else "")
 
     e2e = None
     if not args.no_e2e:
