@@ -113,50 +113,66 @@ __device__ void build_rope_table(float2 *tab, const Plan &p, int f_lo, int nf, i
 }
 
 // Per-thread view of the 4 feature pairs of one 16-byte chunk (features
-// 8*(L%4) .. +7 of a head): table segment and axis of each pair.
+// 8*(L%4) .. +7 of a head): table segment and axis of each pair, as scalars
+// (so that they stay in registers).
 struct PairSet {
-    int seg[4];
-    int axis[4];
+    int seg0, seg1, seg2, seg3;
+    int ax0, ax1, ax2, ax3;
 };
 
 __device__ __forceinline__ PairSet pair_set(const Plan &p, int L, int nf) {
+    const int pr = (L & 3) * 4;
     PairSet s;
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const int pr = (L & 3) * 4 + m;
-        s.seg[m] = rope_seg(p, pr, nf);
-        s.axis[m] = p.axis[pr];
-    }
+    s.seg0 = rope_seg(p, pr, nf);
+    s.seg1 = s.seg0 + rope_len(p, pr, nf);
+    s.seg2 = s.seg1 + rope_len(p, pr + 1, nf);
+    s.seg3 = s.seg2 + rope_len(p, pr + 2, nf);
+    s.ax0 = p.axis[pr];
+    s.ax1 = p.axis[pr + 1];
+    s.ax2 = p.axis[pr + 2];
+    s.ax3 = p.axis[pr + 3];
     return s;
 }
 
-// ReLU one chunk of 8 bf16, rotate its 4 pairs at token t (index in the
-// call), and split the rotated values into hi + lo bf16.  f receives phi(x).
-__device__ __forceinline__ void relu_rotate_chunk(uint4 x, const float2 *tab, const PairSet &ps, const Plan &p,
-                                                  long long t, int f_lo, uint4 &hi, uint4 &lo, float (&f)[8]) {
-    const int ti = (int)t;                          // tokens of a call < 2^31
+// (cos, sin) of the thread's 4 pairs at token t of the call: one position
+// (frame, row, column) per token, shared by every chunk of that token that
+// holds the same features (the same features of other heads).
+struct RowCS {
+    float2 c0, c1, c2, c3;
+};
+
+__device__ __forceinline__ RowCS row_cs(const float2 *tab, const PairSet &ps, const Plan &p, int ti, int f_lo) {
     const int fq = fast_div(ti, p.hw_m, p.hw_s);
     const int rem = ti - fq * p.Hg * p.Wg;
     const int row = fast_div(rem, p.wg_m, p.wg_s);
     const int col = rem - row * p.Wg;
     const int fr = fq - f_lo;
-    const uint32_t w[4] = {relu2(x.x), relu2(x.y), relu2(x.z), relu2(x.w)};
-    uint32_t h[4], l[4];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const float x0 = bf_lo(w[m]), x1 = bf_hi(w[m]);
-        f[2 * m] = x0;
-        f[2 * m + 1] = x1;
-        const int pos = ps.axis[m] == 0 ? fr : (ps.axis[m] == 1 ? row : col);
-        const float2 cs = tab[ps.seg[m] + pos];
-        const float y0 = x0 * cs.x - x1 * cs.y;
-        const float y1 = x0 * cs.y + x1 * cs.x;
-        const __nv_bfloat162 yh = __floats2bfloat162_rn(y0, y1);
-        h[m] = *reinterpret_cast<const uint32_t *>(&yh);
-        l[m] = pack_bf2(y0 - __low2float(yh), y1 - __high2float(yh));
-    }
-    hi = make_uint4(h[0], h[1], h[2], h[3]);
-    lo = make_uint4(l[0], l[1], l[2], l[3]);
+    RowCS r;
+    r.c0 = tab[ps.seg0 + (ps.ax0 == 0 ? fr : (ps.ax0 == 1 ? row : col))];
+    r.c1 = tab[ps.seg1 + (ps.ax1 == 0 ? fr : (ps.ax1 == 1 ? row : col))];
+    r.c2 = tab[ps.seg2 + (ps.ax2 == 0 ? fr : (ps.ax2 == 1 ? row : col))];
+    r.c3 = tab[ps.seg3 + (ps.ax3 == 0 ? fr : (ps.ax3 == 1 ? row : col))];
+    return r;
+}
+
+// ReLU one bf16 pair (one word), rotate it by cs, split into hi + lo bf16.
+__device__ __forceinline__ void rotate_pair(uint32_t x, float2 cs, float &x0, float &x1, uint32_t &h, uint32_t &l) {
+    const uint32_t w = relu2(x);
+    x0 = bf_lo(w);
+    x1 = bf_hi(w);
+    const float y0 = x0 * cs.x - x1 * cs.y;
+    const float y1 = x0 * cs.y + x1 * cs.x;
+    const __nv_bfloat162 yh = __floats2bfloat162_rn(y0, y1);
+    h = *reinterpret_cast<const uint32_t *>(&yh);
+    l = pack_bf2(y0 - __low2float(yh), y1 - __high2float(yh));
+}
+
+// ReLU one chunk of 8 bf16 and rotate its 4 pairs; f receives phi(x).
+__device__ __forceinline__ void relu_rotate_chunk(uint4 x, const RowCS &cs, uint4 &hi, uint4 &lo, float (&f)[8]) {
+    rotate_pair(x.x, cs.c0, f[0], f[1], hi.x, lo.x);
+    rotate_pair(x.y, cs.c1, f[2], f[3], hi.y, lo.y);
+    rotate_pair(x.z, cs.c2, f[4], f[5], hi.z, lo.z);
+    rotate_pair(x.w, cs.c3, f[6], f[7], hi.w, lo.w);
 }
 
 // ================================================================ reduce
@@ -323,29 +339,42 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             if (!mbar_wait(&full[s], ph, abort_word, &g_wait_flag, 3)) break;
             uint8_t *kt = smem + s * C::kStageBytes;
             const long long row0 = t0 + (long long)kRRows * i;
+            if constexpr (ROPE) {
+                // the thread's 4 chunks: token rows r and r + 16, each in both
+                // boxes (heads 0-1 and 2-3), all with the same 8 features, so
+                // one position and one set of cos/sin per row
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {             // 512 chunks of 16 bytes: 4 per thread
-                const int c = wt + 128 * j;           // 16-byte chunk of the two k boxes
-                const int bx = j >> 1;                // box (heads 0-1 or 2-3): c / 256, as wt < 128
-                const int r = (c % (8 * kRRows)) >> 3;   // token row inside its box
-                uint4 *ptr = reinterpret_cast<uint4 *>(kt + (size_t)c * 16);
-                uint4 x = *ptr;
-                const bool valid = row0 + r < t1;     // rows past the split contribute nothing
-                if constexpr (ROPE) {
-                    uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
-                    if (valid) {
-                        float f[8];
-                        relu_rotate_chunk(x, tab, ps, p, row0 + r, f_lo, hi, lo, f);
+                for (int jr = 0; jr < 2; ++jr) {
+                    const int r = (wt >> 3) + 16 * jr;
+                    const bool valid = row0 + r < t1;   // rows past the split contribute nothing
+                    RowCS cs{};
+                    if (valid) cs = row_cs(tab, ps, p, (int)(row0 + r), f_lo);
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) zacc[bx][k] += f[k];
+                    for (int bx = 0; bx < 2; ++bx) {
+                        const int c = wt + 128 * jr + 256 * bx;   // 16-byte chunk of the two k boxes
+                        uint4 *ptr = reinterpret_cast<uint4 *>(kt + (size_t)c * 16);
+                        uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
+                        if (valid) {
+                            float f[8];
+                            relu_rotate_chunk(*ptr, cs, hi, lo, f);
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) zacc[bx][k] += f[k];
+                        }
+                        *ptr = hi;
+                        *reinterpret_cast<uint4 *>(kt + C::kLoOff + (size_t)c * 16) = lo;
                     }
-                    *ptr = hi;
-                    *reinterpret_cast<uint4 *>(kt + C::kLoOff + (size_t)c * 16) = lo;
-                } else {
-                    if (valid) {
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {             // 512 chunks of 16 bytes: 4 per thread
+                    const int c = wt + 128 * j;           // 16-byte chunk of the two k boxes
+                    const int r = (c % (8 * kRRows)) >> 3;   // token row inside its box
+                    uint4 *ptr = reinterpret_cast<uint4 *>(kt + (size_t)c * 16);
+                    uint4 x = *ptr;
+                    if (row0 + r < t1) {
                         x.x = relu2(x.x); x.y = relu2(x.y); x.z = relu2(x.z); x.w = relu2(x.w);
                     } else {
-                        x = make_uint4(0u, 0u, 0u, 0u);
+                        x = make_uint4(0u, 0u, 0u, 0u);   // rows past the split contribute nothing
                     }
                     *ptr = x;
                 }
@@ -602,7 +631,22 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // swizzle phase, and so its logical chunk L0 (head 0 or 1), is fixed.
         const int L0 = (tt & 3) ^ ((tt >> 2) & 7);
         PairSet ps{};
-        if constexpr (ROPE) ps = pair_set(p, L0, nf);
+        // Z_eff of this thread's 8 features of both heads (e = 0: logical chunk
+        // L0, e = 1: L0 ^ 4), for the unrotated denominator
+        float zf[2][8];
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) zf[e][k] = 0.f;
+        if constexpr (ROPE) {
+            ps = pair_set(p, L0, nf);
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int L = L0 ^ (4 * e);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) zf[e][k] = zs[(L >> 2) * kD + (L & 3) * 8 + k];
+            }
+        }
         for (int i = 0; i < ntiles; ++i) {
             const int s = i % C::kStages;
             const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
@@ -619,18 +663,18 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     const int pc0 = u & 3;            // physical chunk of the first of the pair
                     const bool valid = ok && row0 + rr < ta1;
                     float dp[2] = {0.f, 0.f};
+                    RowCS cs{};
+                    if (valid) cs = row_cs(tab, ps, p, (int)(row0 + rr), f_lo);
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int pc = pc0 + 4 * e;
-                        const int L = pc ^ (rr & 7);  // = L0 for e = 0, L0 ^ 4 for e = 1
+                        const int pc = pc0 + 4 * e;   // logical chunk pc ^ (rr & 7): L0, then L0 ^ 4
                         uint4 *ptr = reinterpret_cast<uint4 *>(qt + rr * 128 + pc * 16);
                         uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
                         if (valid) {
                             float f[8];
-                            relu_rotate_chunk(*ptr, tab, ps, p, row0 + rr, f_lo, hi, lo, f);
-                            const float *zh = zs + (L >> 2) * kD + (L & 3) * 8;
+                            relu_rotate_chunk(*ptr, cs, hi, lo, f);
 #pragma unroll
-                            for (int k = 0; k < 8; ++k) dp[e] = fmaf(f[k], zh[k], dp[e]);
+                            for (int k = 0; k < 8; ++k) dp[e] = fmaf(f[k], zf[e][k], dp[e]);
                         }
                         *ptr = hi;
                         *reinterpret_cast<uint4 *>(qt + kATile + rr * 128 + pc * 16) = lo;
