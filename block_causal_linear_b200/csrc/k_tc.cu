@@ -193,10 +193,15 @@ struct RCfg {
     static constexpr int kBarOff = kAuxOff + kAuxBytes;
     static constexpr int kSmem = kBarOff + (3 * kStages + 1) * 8 + 16 + 1024;
     static constexpr uint32_t kTmemCols = ROPE ? 128 : 256;
+    // threads that transform the k boxes (warps 2..): RoPE has 8 such warps,
+    // one token row per thread and stage, to hide the latency of its longer
+    // per-chunk work; without RoPE 4 warps, 4 chunks per thread
+    static constexpr int kXform = ROPE ? 256 : 128;
+    static constexpr int kThreadsR = 64 + kXform;
 };
 
 template <bool ROPE>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(RCfg<ROPE>::kThreadsR, 2)
 reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  float *__restrict__ partials, const Plan p) {
     using C = RCfg<ROPE>;
@@ -229,7 +234,7 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     pdl_trigger();
 
     if (nst == 0) {   // a split past the end of a short last block: its sums are zero
-        for (int e = threadIdx.x; e < 4 * kKVZ; e += kThreads) {
+        for (int e = threadIdx.x; e < 4 * kKVZ; e += C::kThreadsR) {
             const int h = g * 4 + e / kKVZ;
             partials[((((size_t)b * p.H + h) * p.nb + n) * p.P + sp) * kKVZ + e % kKVZ] = 0.f;
         }
@@ -243,7 +248,7 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&relu_done[s], kWork);
+            mbar_init(&relu_done[s], C::kXform);
             mbar_init(&empty[s], 1);
         }
         mbar_init(acc_ready, 1);
@@ -251,10 +256,10 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         fence_barrier_init();
     }
     if constexpr (ROPE) {
-        build_rope_table(reinterpret_cast<float2 *>(aux), p, f_lo, nf, threadIdx.x, kThreads);
+        build_rope_table(reinterpret_cast<float2 *>(aux), p, f_lo, nf, threadIdx.x, C::kThreadsR);
     } else {
         // B operand of the z contraction: 16 x 16 bf16 ones (any layout reads 1.0)
-        for (int i = threadIdx.x; i < 128; i += kThreads) reinterpret_cast<uint32_t *>(aux)[i] = 0x3F803F80u;
+        for (int i = threadIdx.x; i < 128; i += C::kThreadsR) reinterpret_cast<uint32_t *>(aux)[i] = 0x3F803F80u;
     }
     if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, C::kTmemCols);
@@ -320,7 +325,7 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             mma_commit(acc_ready);
         }
     } else {
-        const int wt = threadIdx.x - 64;   // 0..127
+        const int wt = threadIdx.x - 64;   // 0 .. C::kXform - 1
         // with RoPE this thread always meets the same logical chunk L of a row
         // (the swizzle phase (wt >> 3) & 7 is the same for all its chunks)
         const int L = (wt & 7) ^ ((wt >> 3) & 7);
@@ -340,18 +345,18 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             uint8_t *kt = smem + s * C::kStageBytes;
             const long long row0 = t0 + (long long)kRRows * i;
             if constexpr (ROPE) {
-                // the thread's 4 chunks: token rows r and r + 16, each in both
-                // boxes (heads 0-1 and 2-3), all with the same 8 features, so
-                // one position and one set of cos/sin per row
+                // the thread's chunks: token row r (and r + 16 with 4 warps), each
+                // in both boxes (heads 0-1 and 2-3), all with the same 8 features,
+                // so one position and one set of cos/sin per row
 #pragma unroll
-                for (int jr = 0; jr < 2; ++jr) {
-                    const int r = (wt >> 3) + 16 * jr;
+                for (int jr = 0; jr < 256 / C::kXform; ++jr) {
+                    const int r = (wt >> 3) + (C::kXform / 8) * jr;
                     const bool valid = row0 + r < t1;   // rows past the split contribute nothing
                     RowCS cs{};
                     if (valid) cs = row_cs(tab, ps, p, (int)(row0 + r), f_lo);
 #pragma unroll
                     for (int bx = 0; bx < 2; ++bx) {
-                        const int c = wt + 128 * jr + 256 * bx;   // 16-byte chunk of the two k boxes
+                        const int c = wt + C::kXform * jr + 256 * bx;   // 16-byte chunk of the two k boxes
                         uint4 *ptr = reinterpret_cast<uint4 *>(kt + (size_t)c * 16);
                         uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
                         if (valid) {
@@ -391,20 +396,24 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         const int h = g * 4 + qd;
         float z = 0.f;
         if constexpr (ROPE) {
-            // z: the 16 threads that met chunk L of a box each hold 8 sums;
-            // add them in thread order (stage 0 is free once every MMA is done)
+            // z: the threads that met chunk L of a box each hold 8 sums; add
+            // them in thread order (stage 0 is free once every MMA is done)
             float *zbuf = reinterpret_cast<float *>(smem);
+            static_assert(C::kXform * 16 * 4 <= C::kStageBytes, "z partials fit in stage 0");
 #pragma unroll
             for (int bx = 0; bx < 2; ++bx)
 #pragma unroll
                 for (int k = 0; k < 8; ++k) zbuf[wt * 16 + bx * 8 + k] = zacc[bx][k];
-            named_bar_sync(1, kWork);
-            const int bx = qd >> 1;
-            const int Lz = ((qd & 1) << 2) | (lane >> 3);
-            for (int u = 0; u < kWork; ++u)
-                if (((u & 7) ^ ((u >> 3) & 7)) == Lz) z += zbuf[u * 16 + bx * 8 + (lane & 7)];
+            named_bar_sync(1, C::kXform);
+            if (warp < 6) {
+                const int bx = qd >> 1;
+                const int Lz = ((qd & 1) << 2) | (lane >> 3);
+                for (int u = 0; u < C::kXform; ++u)
+                    if (((u & 7) ^ ((u >> 3) & 7)) == Lz) z += zbuf[u * 16 + bx * 8 + (lane & 7)];
+            }
         }
-        if (got) {
+        // warps 2..5 (one per TMEM lane quarter) write the split sums
+        if (got && warp < 6) {
             tc_fence_after();
             const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
             float kv[32];
@@ -902,9 +911,9 @@ int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &
     if (!make_map(&mk, k, p.B, p.N, p.H, kRRows) || !make_map(&mv, v, p.B, p.N, p.H, kRRows)) return -1;
     const long long grid = (long long)p.B * (p.H / 4) * p.nb * p.P;
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
-    const bool ok = p.rope ? launch_pdl(reduce_tc_kernel<true>, (unsigned)grid, kThreads, RCfg<true>::kSmem, s, mk,
+    const bool ok = p.rope ? launch_pdl(reduce_tc_kernel<true>, (unsigned)grid, RCfg<true>::kThreadsR, RCfg<true>::kSmem, s, mk,
                                         mv, partials, p)
-                           : launch_pdl(reduce_tc_kernel<false>, (unsigned)grid, kThreads, RCfg<false>::kSmem, s, mk,
+                           : launch_pdl(reduce_tc_kernel<false>, (unsigned)grid, RCfg<false>::kThreadsR, RCfg<false>::kSmem, s, mk,
                                         mv, partials, p);
     return ok ? 1 : -1;
 }
