@@ -71,9 +71,11 @@ def lib():
         L.orc_apply.argtypes = [vp, ip, ip, lp, ip, ip, vp, vp, vp, lp, rp, lp, dp, vp]
         L.orc_block_forward.argtypes = [vp, vp, vp, ip, vp, ip, lp, ip, ip, vp, vp, ip, rp, lp, dp]
         L.orc_full_forward.argtypes = [vp, vp, vp, ip, vp, ip, lp, ip, ip, lp, rp, dp]
+        L.orc_full_backward.argtypes = [vp, vp, vp, vp, ip, vp, vp, vp, ip, lp, ip, ip, lp, rp, dp]
         L.orc_set_threads.argtypes = [ip]
         L.orc_get_threads.restype = ip
-        for f in ("orc_brute", "orc_block_kv", "orc_apply", "orc_block_forward", "orc_full_forward"):
+        for f in ("orc_brute", "orc_block_kv", "orc_apply", "orc_block_forward", "orc_full_forward",
+                  "orc_full_backward"):
             getattr(L, f).restype = ip
         _lib = L
     return _lib
@@ -191,3 +193,19 @@ def full_forward(q, k, v, tokens_per_block=0, rope=None, eps=1e-6):
                                 B, N, H, d, int(tokens_per_block), _rope_ptr(rope), float(eps))
     _check(rc, "full_forward")
     return out
+
+
+def full_backward(q, k, v, dout, tokens_per_block=0, rope=None, eps=1e-6):
+    """Gradients (dq, dk, dv) of sum(full_forward(q, k, v) * dout), fp64 numpy
+    [B, N, H, d] each: the chain rule through the block recurrence (zero
+    initial state), ReLU derivative 1[x > 0]."""
+    B, N, H, d = _shape(q)
+    (qc, dt), (kc, _), (vc, _), (oc, dto) = _prep(q), _prep(k), _prep(v), _prep(dout)
+    if dto != dt:
+        raise TypeError("dout must have the dtype of q, k, v")
+    dq, dk, dv = (np.zeros((B, N, H, d), dtype=np.float64) for _ in range(3))
+    rc = lib().orc_full_backward(qc.data_ptr(), kc.data_ptr(), vc.data_ptr(), oc.data_ptr(), dt,
+                                 dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, B, N, H, d,
+                                 int(tokens_per_block), _rope_ptr(rope), float(eps))
+    _check(rc, "full_backward")
+    return dq, dk, dv

@@ -343,3 +343,145 @@ done:
     free(S); free(Z); free(qb); free(kb); free(vb); free(ob);
     return rc;
 }
+
+/* psi^T: the transpose of rope_apply (rotation by the negative angle). */
+static void rope_apply_t(double *f, const orc_rope *r, long j)
+{
+    if (!r || !r->enabled) return;
+    long per_frame = (long)r->Hg * (long)r->Wg;
+    long tpos = (long)r->t_offset + j / per_frame;
+    long rem = j % per_frame;
+    rotate_section(f, 0, r->dt, -tpos, r->base);
+    rotate_section(f, r->dt, r->dh, -(rem / r->Wg), r->base);
+    rotate_section(f, r->dt + r->dh, r->dw, -(rem % r->Wg), r->base);
+}
+
+/*
+ * Gradient of orc_full_forward (zero initial state, blocks of
+ * tokens_per_block tokens): with dout [B][N][H][d] given, dq, dk, dv
+ * [B][N][H][d] are the gradients of sum(out * dout) with respect to q, k, v.
+ * The chain rule through the recurrence of the method, per (b, h):
+ *   forward:  S_n = sum_{m<=n} KV_m, Z_n = sum_{m<=n} z_m (inclusive)
+ *   block n, token t:  num_t = psi(q_t) S_n,  den_t = phi(q_t) . Z_n + eps,
+ *     g_t = dout_t / den_t,  c_t = -(dout_t . num_t) / den_t^2,
+ *     d psi(q_t) = S_n g_t,  d phi(q_t) += c_t Z_n,
+ *     dS_n += psi(q_t) g_t^T,  dZ_n += c_t phi(q_t)
+ *   the state of block m enters every later block:
+ *     G_m = sum_{n>=m} dS_n,  g_m = sum_{n>=m} dZ_n
+ *   block m, token t:  d psi(k_t) = G_m v_t,  dv_t = G_m^T psi(k_t),
+ *     d phi(k_t) += g_m
+ *   then d phi = R^T d psi (+ the unrotated part) and the ReLU mask 1[x > 0].
+ * The pages state only the forward recurrence ([aihaber "Sabit Bellekli ..."]);
+ * the backward is its derivative, for block-autoregressive training.
+ */
+int orc_full_backward(const void *q, const void *k, const void *v, const void *dout, int dtype,
+                      double *dq, double *dk, double *dv, int B, long N, int H, int d,
+                      long tokens_per_block, const orc_rope *rope, double eps)
+{
+    if (B < 0 || N < 0 || H < 0 || d <= 0 || d > 256 || tokens_per_block < 0) return 1;
+    if (!rope_ok(rope, d)) return 1;
+    long L = tokens_per_block > 0 ? tokens_per_block : (N > 0 ? N : 1);
+    long nb = N > 0 ? (N + L - 1) / L : 0;
+    long total = (long)B * H;
+    int bad = 0;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1) ORC_THREADS reduction(| : bad)
+#endif
+    for (long w = 0; w < total; ++w) {
+        int b = (int)(w / H), h = (int)(w % H);
+        size_t dd = (size_t)d * d;
+        double *S = calloc((size_t)nb * dd + 1, sizeof(double));
+        double *Z = calloc((size_t)nb * d + 1, sizeof(double));
+        double *dS = calloc((size_t)nb * dd + 1, sizeof(double));
+        double *dZ = calloc((size_t)nb * d + 1, sizeof(double));
+        double *G = calloc(dd + 1, sizeof(double));
+        double *gz = calloc((size_t)d + 1, sizeof(double));
+        if (!S || !Z || !dS || !dZ || !G || !gz) {
+            bad = 1;
+            goto next;
+        }
+        double f[256], p[256], dp[256], df[256], num[256], g[256];
+        /* forward prefix: S_n, Z_n after block n */
+        for (long n = 0; n < nb; ++n) {
+            double *Sn = S + (size_t)n * dd, *Zn = Z + (size_t)n * d;
+            if (n > 0) {
+                memcpy(Sn, Sn - dd, sizeof(double) * dd);
+                memcpy(Zn, Zn - d, sizeof(double) * d);
+            }
+            long t1 = (n + 1) * L < N ? (n + 1) * L : N;
+            for (long t = n * L; t < t1; ++t) {
+                phi_row(k, dtype, b, t, h, N, H, d, f);
+                memcpy(p, f, sizeof(double) * d);
+                rope_apply(p, rope, t);
+                for (int a = 0; a < d; ++a) {
+                    Zn[a] += f[a];
+                    for (int c = 0; c < d; ++c) Sn[(size_t)a * d + c] += p[a] * elem(v, dtype, idx4(b, t, h, c, N, H, d));
+                }
+            }
+        }
+        /* query side: dq, dS_n, dZ_n */
+        for (long n = 0; n < nb; ++n) {
+            const double *Sn = S + (size_t)n * dd, *Zn = Z + (size_t)n * d;
+            double *dSn = dS + (size_t)n * dd, *dZn = dZ + (size_t)n * d;
+            long t1 = (n + 1) * L < N ? (n + 1) * L : N;
+            for (long t = n * L; t < t1; ++t) {
+                phi_row(q, dtype, b, t, h, N, H, d, f);
+                memcpy(p, f, sizeof(double) * d);
+                rope_apply(p, rope, t);
+                double den = eps, dn = 0.0;
+                for (int a = 0; a < d; ++a) den += f[a] * Zn[a];
+                for (int c = 0; c < d; ++c) {
+                    num[c] = 0.0;
+                    for (int a = 0; a < d; ++a) num[c] += p[a] * Sn[(size_t)a * d + c];
+                    double o = elem(dout, dtype, idx4(b, t, h, c, N, H, d));
+                    g[c] = o / den;
+                    dn += o * num[c];
+                }
+                double cc = -dn / (den * den);
+                for (int a = 0; a < d; ++a) {
+                    dp[a] = 0.0;
+                    for (int c = 0; c < d; ++c) dp[a] += Sn[(size_t)a * d + c] * g[c];
+                }
+                memcpy(df, dp, sizeof(double) * d);
+                rope_apply_t(df, rope, t);
+                for (int a = 0; a < d; ++a) {
+                    df[a] += cc * Zn[a];
+                    double x = elem(q, dtype, idx4(b, t, h, a, N, H, d));
+                    dq[idx4(b, t, h, a, N, H, d)] = x > 0.0 ? df[a] : 0.0;
+                    dZn[a] += cc * f[a];
+                    for (int c = 0; c < d; ++c) dSn[(size_t)a * d + c] += p[a] * g[c];
+                }
+            }
+        }
+        /* key side, last block first: G_m = sum_{n>=m} dS_n */
+        for (long m = nb - 1; m >= 0; --m) {
+            for (size_t a = 0; a < dd; ++a) G[a] += dS[(size_t)m * dd + a];
+            for (int a = 0; a < d; ++a) gz[a] += dZ[(size_t)m * d + a];
+            long t1 = (m + 1) * L < N ? (m + 1) * L : N;
+            for (long t = m * L; t < t1; ++t) {
+                phi_row(k, dtype, b, t, h, N, H, d, f);
+                memcpy(p, f, sizeof(double) * d);
+                rope_apply(p, rope, t);
+                for (int a = 0; a < d; ++a) {
+                    dp[a] = 0.0;
+                    for (int c = 0; c < d; ++c) dp[a] += G[(size_t)a * d + c] * elem(v, dtype, idx4(b, t, h, c, N, H, d));
+                }
+                for (int c = 0; c < d; ++c) {
+                    double s = 0.0;
+                    for (int a = 0; a < d; ++a) s += G[(size_t)a * d + c] * p[a];
+                    dv[idx4(b, t, h, c, N, H, d)] = s;
+                }
+                memcpy(df, dp, sizeof(double) * d);
+                rope_apply_t(df, rope, t);
+                for (int a = 0; a < d; ++a) {
+                    df[a] += gz[a];
+                    double x = elem(k, dtype, idx4(b, t, h, a, N, H, d));
+                    dk[idx4(b, t, h, a, N, H, d)] = x > 0.0 ? df[a] : 0.0;
+                }
+            }
+        }
+    next:
+        free(S); free(Z); free(dS); free(dZ); free(G); free(gz);
+    }
+    return bad;
+}
