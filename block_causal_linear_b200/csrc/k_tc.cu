@@ -47,7 +47,6 @@ __device__ unsigned int g_wait_flag = 0;
 
 namespace {
 
-constexpr int kThreads = 192;   // 6 warps
 constexpr int kWarpTma = 0;
 constexpr int kWarpMma = 1;
 constexpr int kWork = 128;      // threads of warps 2..5

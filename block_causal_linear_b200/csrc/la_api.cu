@@ -219,6 +219,65 @@ la_status la_full_forward(const void *q, const void *k, const void *v, void *out
     return run(q, k, v, out, dt, p, nullptr, nullptr, ws, static_cast<cudaStream_t>(stream));
 }
 
+size_t la_backward_workspace_size(int B, int N, int H, int d, int tokens_per_block) {
+    if (!sizes_ok(B, N, H, d) || tokens_per_block < 0) return 0;
+    la::Plan p{};
+    p.B = B; p.N = N; p.H = H;
+    p.L = tokens_per_block > 0 && tokens_per_block < N ? tokens_per_block : N;
+    p.nb = (int)ceil_div(N, p.L);
+    make_splits(p);
+    return la::bwd_layout(B, H, p.nb, p.P).total;
+}
+
+la_status la_full_backward(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk,
+                           void *dv, la_dtype dt, int B, int N, int H, int d, int tokens_per_block,
+                           const la_rope *rope, float eps, void *ws, size_t ws_bytes, void *stream) {
+    la_status e = common_checks(q, k, v, dq, dt, B, N, H, d, eps);
+    if (e != LA_OK) return e;
+    if (!dout || !dk || !dv || !aligned16(dout) || !aligned16(dk) || !aligned16(dv)) return LA_EINVAL;
+    if (tokens_per_block < 0) return LA_EINVAL;
+    if ((e = check_rope(rope, d, false)) != LA_OK) return e;
+    const size_t need = la_backward_workspace_size(B, N, H, d, tokens_per_block);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return LA_EWORKSPACE;
+
+    la::Plan p{};
+    p.B = B; p.N = N; p.H = H;
+    p.L = tokens_per_block > 0 && tokens_per_block < N ? tokens_per_block : N;
+    p.nb = (int)ceil_div(N, p.L);
+    p.commit = 0;
+    p.has_state = 0;
+    p.eps = eps;
+    make_splits(p);
+    fill_rope(p, rope, rope ? rope->t_offset : 0);
+
+    const la::BwdLayout w = la::bwd_layout(B, H, p.nb, p.P);
+    char *base = static_cast<char *>(ws);
+    float *partials = reinterpret_cast<float *>(base + w.fwd.partials);
+    float *seff = reinterpret_cast<float *>(base + w.fwd.seff);
+    float *bpart = reinterpret_cast<float *>(base + w.bpart);
+    float *G = reinterpret_cast<float *>(base + w.G);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool tc = use_tc(dt, p);
+    const int bf = dt == LA_BF16;
+    int n = 0, r;
+    // the forward prefix state S_n, Z_n of every block, as the forward computes it
+    r = tc ? la::launch_reduce_tc(k, v, partials, p, s) : la::launch_reduce_ffma(bf, k, v, partials, p, s);
+    if (r < 0) return LA_ECUDA;
+    n += r;
+    if ((r = la::launch_finish(partials, seff, base + w.fwd.bop, nullptr, nullptr, p, tc ? 1 : 0, s)) < 0)
+        return LA_ECUDA;
+    n += r;
+    if ((r = la::launch_bwd_q(bf, q, dout, seff, dq, bpart, p, s)) < 0) return LA_ECUDA;
+    n += r;
+    if ((r = la::launch_bwd_finish(bpart, G, p, s)) < 0) return LA_ECUDA;
+    n += r;
+    if ((r = la::launch_bwd_k(bf, k, v, G, dk, dv, p, s)) < 0) return LA_ECUDA;
+    n += r;
+    g_last_launches = n;
+    g_last_path = tc ? "bwd(tc state)" : "bwd";
+    return LA_OK;
+}
+
 la_status la_device_status(void *stream) {
     unsigned flag = 0;
     if (la::read_and_clear_device_flag(static_cast<cudaStream_t>(stream), &flag) != 0)

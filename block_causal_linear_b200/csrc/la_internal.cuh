@@ -109,6 +109,32 @@ bool tc_available();
 // it fits for this plan (else the call takes the CUDA-core kernels).
 bool tc_rope_fits(const Plan &p);
 
+// Backward pass (CUDA cores, fp32 or bf16 tensors): dq and the per-split
+// [dS | dZ] sums from q, dout and the forward prefix state; the suffix sums
+// over blocks; dk and dv from k, v and those sums.
+int launch_bwd_q(int is_bf16, const void *q, const void *dout, const float *seff, void *dq, float *bpart,
+                 const Plan &p, cudaStream_t s);
+int launch_bwd_finish(const float *bpart, float *G, const Plan &p, cudaStream_t s);
+int launch_bwd_k(int is_bf16, const void *k, const void *v, const float *G, void *dk, void *dv, const Plan &p,
+                 cudaStream_t s);
+
+// Backward workspace: the forward layout, then the split sums of [dS | dZ]
+// ([B][H][nb][P][kKVZ]) and their suffix sums G ([B][H][nb][kKVZ]), fp32.
+struct BwdLayout {
+    WsLayout fwd;
+    size_t bpart, G, total;
+};
+
+inline BwdLayout bwd_layout(int B, int H, int nb, int P) {
+    BwdLayout w;
+    w.fwd = ws_layout(B, H, nb, P);
+    const size_t bhn = size_t(B) * H * nb;
+    w.bpart = w.fwd.total;
+    w.G = align256(w.bpart + bhn * P * kKVZ * sizeof(float));
+    w.total = align256(w.G + bhn * kKVZ * sizeof(float));
+    return w;
+}
+
 // Device flag raised by a bounded wait that gave up; read-and-clear.
 int read_and_clear_device_flag(cudaStream_t s, unsigned *flag_out);
 

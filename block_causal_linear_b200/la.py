@@ -68,6 +68,11 @@ def lib() -> ctypes.CDLL:
         L.la_full_forward_static_ws.argtypes = [vp, vp, vp, vp, ip, ip, ip, ip, ip, ip,
                                                 ctypes.POINTER(la_rope), fp, vp]
         L.la_full_forward_static_ws.restype = ip
+        L.la_backward_workspace_size.argtypes = [ip, ip, ip, ip, ip]
+        L.la_backward_workspace_size.restype = sz
+        L.la_full_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip,
+                                       ctypes.POINTER(la_rope), fp, vp, sz, vp]
+        L.la_full_backward.restype = ip
         L.la_device_status.argtypes = [vp]
         L.la_device_status.restype = ip
         L.la_status_string.argtypes = [ip]
@@ -115,6 +120,17 @@ def la_full_forward_static_ws(q, k, v, out, dt, B, N, H, d, tokens_per_block, ro
 
 
 LA_STATIC_WS_BYTES = 16 << 20
+
+
+def la_backward_workspace_size(B, N, H, d, tokens_per_block) -> int:
+    return int(lib().la_backward_workspace_size(B, N, H, d, tokens_per_block))
+
+
+def la_full_backward(q, k, v, dout, dq, dk, dv, dt, B, N, H, d, tokens_per_block, rope, eps, ws, ws_bytes,
+                     stream) -> int:
+    return int(lib().la_full_backward(q, k, v, dout, dq, dk, dv, dt, B, N, H, d, tokens_per_block,
+                                      ctypes.byref(rope) if rope is not None else None, eps, ws,
+                                      ws_bytes, stream))
 
 
 def la_device_status(stream) -> int:
@@ -239,6 +255,30 @@ def full_forward(q, k, v, tokens_per_block=0, rope: Optional[la_rope] = None, ep
     if rc != LA_OK:
         raise LAError(rc, "la_full_forward")
     return out
+
+
+def alloc_backward_workspace(B, N, H, d=32, tokens_per_block=0, device=None) -> torch.Tensor:
+    n = la_backward_workspace_size(B, N, H, d, tokens_per_block)
+    if n == 0:
+        raise LAError(LA_EINVAL, "la_backward_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def full_backward(q, k, v, dout, tokens_per_block=0, rope: Optional[la_rope] = None, eps=1e-6,
+                  ws: Optional[torch.Tensor] = None, grads=None, stream=None):
+    """(dq, dk, dv) of sum(full_forward(q, k, v, ...) * dout)."""
+    _check_qkv(q, k, v)
+    _check_qkv(q, dout, dout)
+    B, N, H, d = q.shape
+    if ws is None:
+        ws = alloc_backward_workspace(B, N, H, d, tokens_per_block, device=q.device)
+    dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    rc = la_full_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                          dv.data_ptr(), _dtype_code(q), B, N, H, d, int(tokens_per_block), rope, float(eps),
+                          ws.data_ptr(), ws.numel() * ws.element_size(), _stream_ptr(stream))
+    if rc != LA_OK:
+        raise LAError(rc, "la_full_backward")
+    return dq, dk, dv
 
 
 def device_status(stream=None) -> None:

@@ -152,6 +152,32 @@ LA_API la_status la_full_forward(const void *q, const void *k, const void *v, vo
                           void *stream);
 
 /*
+ * Backward pass of la_full_forward, for block-autoregressive training.  The
+ * pages give the forward recurrence ("Nvidia, MIT ve diğerleri video yapay
+ * zeka devrimini başlattı", section "Sabit Bellekli KV önbelleğe alma
+ * mekanizması"); this is its derivative.  Given dout = d loss / d out for
+ * la_full_forward(q, k, v, tokens_per_block, rope, eps) (zero initial state),
+ * writes dq, dk, dv = d loss / d q, k, v:
+ *   per (b, h), token t of block n, S_n and Z_n the state after block n:
+ *   g_t = dout_t / den_t,  c_t = -(dout_t . num_t) / den_t^2,
+ *   dq_t = 1[q_t > 0] (R^T (S_n g_t) + c_t Z_n),
+ *   G_m = sum_{n >= m} sum_{t in n} [psi(q_t) g_t^T | c_t phi(q_t)],
+ *   dk_t = 1[k_t > 0] (R^T (G_m v_t) + Gz_m),  dv_t = G_m^T psi(k_t)
+ * (ReLU derivative 1[x > 0]; R the numerator rotation when rope is given).
+ * Tensors: q, k, v, dout, dq, dk, dv all [B][N][H][d] of type dt, device
+ * pointers, 16-byte aligned, caller-owned; dq, dk, dv may not overlap the
+ * inputs.  ws must hold la_backward_workspace_size(B, N, H, d,
+ * tokens_per_block) bytes (256-byte aligned), else LA_EWORKSPACE; argument
+ * errors return LA_EINVAL / LA_EUNSUPPORTED before anything is enqueued.
+ * fp32 sums in fixed orders: repeated calls give the same bits.
+ */
+LA_API size_t la_backward_workspace_size(int B, int N, int H, int d, int tokens_per_block);
+LA_API la_status la_full_backward(const void *q, const void *k, const void *v, const void *dout,
+                                  void *dq, void *dk, void *dv, la_dtype dt, int B, int N, int H,
+                                  int d, int tokens_per_block, const la_rope *rope, float eps,
+                                  void *ws, size_t ws_bytes, void *stream);
+
+/*
  * For callers that cannot allocate device memory at all.  Some code that
  * calls this library runs inside a host framework that owns every device
  * allocation and gives a plug-in no allocator and no way to size or keep a

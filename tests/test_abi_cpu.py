@@ -114,3 +114,33 @@ def test_block_forward_and_state_validation(la):
     assert la.la_block_forward(FAKE, FAKE, FAKE, FAKE, la.LA_BF16, 1, 64, 4, 32, st, 1, None, 1e-6,
                                FAKE, 8, None) == la.LA_EWORKSPACE
     assert st.blocks_committed == 0
+
+
+def _bwd(la, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, dt=la.LA_BF16, B=1, N=256, H=4,
+             d=32, tpb=0, rope=None, eps=1e-6, ws=FAKE, ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return la.la_full_backward(a["q"], a["k"], a["v"], a["dout"], a["dq"], a["dk"], a["dv"], a["dt"], a["B"],
+                               a["N"], a["H"], a["d"], a["tpb"], a["rope"], a["eps"], a["ws"], a["ws_bytes"],
+                               a["stream"])
+
+
+def test_full_backward_validation(la):
+    for name in ("q", "k", "v", "dout", "dq", "dk", "dv"):
+        assert _bwd(la, **{name: None}) == la.LA_EINVAL
+        assert _bwd(la, **{name: FAKE + 8}) == la.LA_EINVAL      # misaligned
+    assert _bwd(la, d=16) == la.LA_EUNSUPPORTED
+    assert _bwd(la, N=0) == la.LA_EINVAL
+    assert _bwd(la, dt=7) == la.LA_EINVAL
+    assert _bwd(la, tpb=-1) == la.LA_EINVAL
+    assert _bwd(la, eps=float("inf")) == la.LA_EINVAL
+    assert _bwd(la, ws=None) == la.LA_EWORKSPACE
+    assert _bwd(la, ws_bytes=la.la_backward_workspace_size(1, 256, 4, 32, 0) - 1) == la.LA_EWORKSPACE
+    assert _bwd(la, rope=la.make_rope(Hg=2, Wg=2, t_offset=-1)) == la.LA_EINVAL
+
+
+def test_backward_workspace_size(la):
+    fwd = la.la_workspace_size(1, 4 * 640, 8, 32, 640)
+    bwd = la.la_backward_workspace_size(1, 4 * 640, 8, 32, 640)
+    assert bwd > fwd and bwd % 256 == 0
+    assert la.la_backward_workspace_size(1, 0, 8, 32, 0) == 0
