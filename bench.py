@@ -44,6 +44,7 @@ sys.path.insert(0, ROOT)
 from block_causal_linear_b200 import ranks, synth  # noqa: E402
 
 METRIC = "block linear-attn tokens·heads/s and achieved HBM GB/s vs B200 peak (1 GPU)"
+METRIC_BWD = "block linear-attn backward tokens·heads/s and achieved HBM GB/s vs B200 peak (1 GPU)"
 UNIT = "token·heads/s"
 FLUSH_BYTES = 256 << 20          # > 2x the 126 MB L2 of a B200
 FALLBACK_HBM_GBS = 6650.0
@@ -61,6 +62,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "backward"],
+                    help="backward: la_full_backward over the workload's whole sequence (dq, dk, dv)")
     ap.add_argument("--blocks", type=int, default=None,
                     help="streaming workloads: run only the first N blocks (small cases for profiling)")
     ap.add_argument("--shard", default="problem", choices=["problem", "heads"],
@@ -174,10 +177,10 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- oracle timing
 
-def oracle_sample(w: synth.Workload, budget_s: float, orc):
+def oracle_sample(w: synth.Workload, budget_s: float, orc, backward=False):
     """Time the oracle on the first call's inputs of the workload: all tokens of
-    that call, a head subset sized to take about budget_s.  Returns
-    (token_heads, seconds, description)."""
+    that call, a head subset sized to take about budget_s (backward: the fp64
+    backward of that block).  Returns (token_heads, seconds, description)."""
     import numpy as np  # noqa: F401
 
     _, _, q, k, v = next(iter(synth.stream(w, "cpu", blocks=1)))
@@ -188,7 +191,10 @@ def oracle_sample(w: synth.Workload, budget_s: float, orc):
         qs, ks, vs = (t[:, :, :nh].contiguous() for t in (q, k, v))
         st = orc.State(w.B, nh, w.d)
         t0 = time.perf_counter()
-        orc.block_forward(qs, ks, vs, st, commit=True, rope=rope, eps=w.eps)
+        if backward:
+            orc.full_backward(qs, ks, vs, vs, 0, rope=rope, eps=w.eps)
+        else:
+            orc.block_forward(qs, ks, vs, st, commit=True, rope=rope, eps=w.eps)
         return time.perf_counter() - t0
 
     t1 = run(1)
@@ -196,7 +202,8 @@ def oracle_sample(w: synth.Workload, budget_s: float, orc):
     dt = run(nh)
     th = w.B * q.shape[1] * nh
     desc = (f"first call of the workload ({w.B}x{q.shape[1]} tokens) on {nh} of {w.H} heads, "
-            f"one recurrence pass (block KV, state combine, apply, commit) in fp64")
+            + ("the fp64 backward of that block (state, dq and state gradients, dk, dv)" if backward else
+               "one recurrence pass (block KV, state combine, apply, commit) in fp64"))
     return th, dt, desc
 
 
@@ -270,7 +277,7 @@ def main():
 
     la_build.build()
     from block_causal_linear_b200 import la
-    from block_causal_linear_b200.runner import Runner
+    from block_causal_linear_b200.runner import BackwardRunner, Runner
 
     base = synth.WORKLOADS[args.config]
     if args.shard == "heads":
@@ -285,7 +292,9 @@ def main():
         if w.mode != "stream" or not 1 <= args.blocks <= w.n_blocks:
             raise SystemExit("--blocks needs a streaming workload and 1 <= N <= its block count")
         w = w.shrink(n_blocks=args.blocks)
-    runner = Runner(w, dev)
+    bwd = args.pass_ == "backward"
+    runner = BackwardRunner(w, dev) if bwd else Runner(w, dev)
+    w = runner.w
     flush_w = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_acc = torch.empty(1, dtype=torch.float32, device=dev)
@@ -404,17 +413,28 @@ def main():
     value = ranks.job_throughput(th_step, world, K, total_ms)
     ms_per_step = total_ms / K
     peak, peak_kind = measured_peaks()
-    step_gbs = w.alg_bytes / (ms_per_step / 1e3) / 1e9
+    # algorithmic bytes: forward reads q, k, v and writes out (4 tensors);
+    # backward reads q, k, v, dout and writes dq, dk, dv (7 tensors)
+    alg_bytes = w.token_heads * (7 if bwd else 4) * w.d * w.elem_bytes if bwd else w.alg_bytes
+    step_gbs = alg_bytes / (ms_per_step / 1e3) / 1e9
 
     launches_per_kernel = K * n_calls                # stage_ms is scaled to K steps
-    # dominant kernel: the larger of reduce (reads k, v) and apply (reads q, writes out)
     per_call_th = w.B * runner.tokens_per_call(0) * w.H
-    kern_bytes = per_call_th * 2 * w.d * w.elem_bytes
-    dom, dom_ms = ("reduce", red_ms) if red_ms >= app_ms else ("apply", app_ms)
+    path = la.la_last_path()
+    if bwd:
+        # stages: forward state | query side (reads q, dout, writes dq) | key side
+        # (reads k, v, writes dk, dv); the dominant one of the two sides
+        side = [("bwd_q", fin_ms, 3), ("bwd_k", app_ms, 4)]
+        dom, dom_ms, ntens = max(side, key=lambda x: x[1])
+        kname = dom
+    else:
+        # dominant kernel: the larger of reduce (reads k, v) and apply (reads q, writes out)
+        dom, dom_ms = ("reduce", red_ms) if red_ms >= app_ms else ("apply", app_ms)
+        ntens = 2
+        kname = f"{dom}_{path}" + ("_rope" if w.rope and path == "tc" else "")
+    kern_bytes = per_call_th * ntens * w.d * w.elem_bytes
     avg_launch_s = dom_ms / launches_per_kernel / 1e3
     achieved = kern_bytes / avg_launch_s / 1e9
-    path = la.la_last_path()
-    kname = f"{dom}_{path}" + ("_rope" if w.rope and path == "tc" else "")
 
     e2e = None
     if not args.no_e2e:
@@ -425,20 +445,22 @@ def main():
         import oracle as orc
 
         orc.build()
-        th, dt, desc = oracle_sample(w, 12.0, orc)
+        th, dt, desc = oracle_sample(w, 12.0, orc, backward=bwd)
         cpu = {"value": th / dt, "unit": UNIT, "cores": orc.get_threads(), "kind": "oracle", "sample": desc}
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "metric": METRIC_BWD if bwd else METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "strong" if args.shard == "heads" else "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-            "config": workload_config(w, {"parallelism": (f"heads of one problem split over {world} ranks"
+            "config": workload_config(w, {"pass": args.pass_,
+                                          "parallelism": (f"heads of one problem split over {world} ranks"
                                                           if args.shard == "heads" else
                                                           f"independent problem per rank x{world}")}),
             "achieved_hbm_gbs": step_gbs, "hbm_frac_of_" + peak_kind: step_gbs / peak,
-            "stage_ms_per_step": {"reduce": red_ms / K, "finish": fin_ms / K, "apply": app_ms / K},
+            "stage_ms_per_step": ({"forward_state": red_ms / K, "query_side": fin_ms / K, "key_side": app_ms / K}
+                                  if bwd else {"reduce": red_ms / K, "finish": fin_ms / K, "apply": app_ms / K}),
             "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": ncu_traffic(kname, per_call_th)},
@@ -462,7 +484,7 @@ def measure_e2e(runner, w, dev, world, dist, steps):
     reused by the next step only after this step is done with them."""
     from block_causal_linear_b200 import la  # noqa: F401
 
-    host_in = [tuple(t.cpu().pin_memory() for t in c[2:]) for c in runner.calls]
+    host_in = [tuple(t.cpu().pin_memory() for t in c) for c in runner.inputs]
     host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in runner.outs]
     h2d = sum(t.numel() * t.element_size() for c in host_in for t in c)
     d2h = sum(t.numel() * t.element_size() for t in host_out)
@@ -471,7 +493,7 @@ def measure_e2e(runner, w, dev, world, dist, steps):
     s_up, s_cmp, s_down = (torch.cuda.Stream(dev) for _ in range(3))
     ev_up = [torch.cuda.Event() for _ in range(n)]
     ev_cmp = [torch.cuda.Event() for _ in range(n)]
-    ev_down = [torch.cuda.Event() for _ in range(n)]
+    ev_down = [torch.cuda.Event() for _ in runner.outs]
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     state = {"first": True}
@@ -479,7 +501,9 @@ def measure_e2e(runner, w, dev, world, dist, steps):
     def before_call(i):
         s_cmp.wait_event(ev_up[i])
         if not state["first"]:
-            s_cmp.wait_event(ev_down[i])        # out i of the previous step is on the host
+            for j, c in enumerate(runner.out_call):
+                if c == i:
+                    s_cmp.wait_event(ev_down[j])   # call i's outputs of the previous step are on the host
 
     def after_call(i):
         ev_cmp[i].record(s_cmp)
@@ -487,19 +511,18 @@ def measure_e2e(runner, w, dev, world, dist, steps):
             before_call(i + 1)
 
     def one():
-        for i, ((q, k, v), c) in enumerate(zip(host_in, runner.calls)):
+        for i, (hs, ds) in enumerate(zip(host_in, runner.inputs)):
             if not state["first"]:
                 s_up.wait_event(ev_cmp[i])      # the previous step has read inputs i
             with torch.cuda.stream(s_up):
-                c[2].copy_(q, non_blocking=True)
-                c[3].copy_(k, non_blocking=True)
-                c[4].copy_(v, non_blocking=True)
+                for h_, d_ in zip(hs, ds):
+                    d_.copy_(h_, non_blocking=True)
             ev_up[i].record(s_up)
         before_call(0)
         with torch.cuda.stream(s_cmp):
             runner.step(after_call=after_call, stream=s_cmp)
         for i, (ho, o) in enumerate(zip(host_out, runner.outs)):
-            s_down.wait_event(ev_cmp[i])
+            s_down.wait_event(ev_cmp[runner.out_call[i]])
             with torch.cuda.stream(s_down):
                 ho.copy_(o, non_blocking=True)
             ev_down[i].record(s_down)

@@ -23,11 +23,6 @@
 namespace la {
 namespace {
 
-__device__ __forceinline__ float ldf(const float *p) { return *p; }
-__device__ __forceinline__ float ldf(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
-__device__ __forceinline__ void stf(float *p, float x) { *p = x; }
-__device__ __forceinline__ void stf(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
-
 // Angle of feature pair pr of token j of the call (numerator RoPE).
 __device__ __forceinline__ float pair_angle(const Plan &p, long long j, int pr) {
     const long long per_frame = (long long)p.Hg * p.Wg;
@@ -39,30 +34,82 @@ __device__ __forceinline__ float pair_angle(const Plan &p, long long j, int pr) 
     return (float)pos * p.theta[pr];
 }
 
-// (x0, x1) -> R(+/-angle) (x0, x1): sgn = +1 rotates (psi), -1 the transpose.
-__device__ __forceinline__ void rot_pair(float ang, float sgn, float &x0, float &x1) {
-    float s, c;
-    sincosf(ang, &s, &c);
-    s *= sgn;
-    const float a = x0, b = x1;
-    x0 = a * c - b * s;
-    x1 = a * s + b * c;
+constexpr int kBThreads = 256;   // bwd_finish_kernel
+
+// One token row (32 features of one head) between global memory and registers,
+// in 16-byte pieces.
+__device__ __forceinline__ void load_row(const float *p, float (&x)[kD]) {
+#pragma unroll
+    for (int i = 0; i < kD / 4; ++i) {
+        const float4 v = reinterpret_cast<const float4 *>(p)[i];
+        x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
+    }
+}
+__device__ __forceinline__ void load_row(const __nv_bfloat16 *p, float (&x)[kD]) {
+#pragma unroll
+    for (int i = 0; i < kD / 8; ++i) {
+        const uint4 v = reinterpret_cast<const uint4 *>(p)[i];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            x[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+            x[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+    }
+}
+__device__ __forceinline__ void store_row(float *p, const float (&x)[kD]) {
+#pragma unroll
+    for (int i = 0; i < kD / 4; ++i)
+        reinterpret_cast<float4 *>(p)[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+}
+__device__ __forceinline__ uint32_t bf2(float a, float b) {
+    const __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&t);
+}
+__device__ __forceinline__ void store_row(__nv_bfloat16 *p, const float (&x)[kD]) {
+#pragma unroll
+    for (int i = 0; i < kD / 8; ++i)
+        reinterpret_cast<uint4 *>(p)[i] = make_uint4(bf2(x[8 * i], x[8 * i + 1]), bf2(x[8 * i + 2], x[8 * i + 3]),
+                                                     bf2(x[8 * i + 4], x[8 * i + 5]), bf2(x[8 * i + 6], x[8 * i + 7]));
 }
 
-constexpr int kBThreads = 256;
-constexpr int kBRows = 64;       // token rows per staging round (4 threads per row)
+// cos, sin of the 16 feature pairs of token t (numerator RoPE).
+__device__ __forceinline__ void token_cs(const Plan &p, long long t, float (&c)[kD / 2], float (&s)[kD / 2]) {
+#pragma unroll
+    for (int pr = 0; pr < kD / 2; ++pr) sincosf(pair_angle(p, t, pr), &s[pr], &c[pr]);
+}
+// x <- R x (sgn = +1) or R^T x (sgn = -1), pair by pair.
+__device__ __forceinline__ void rotate_row(float (&x)[kD], const float (&c)[kD / 2], const float (&s)[kD / 2],
+                                           float sgn) {
+#pragma unroll
+    for (int pr = 0; pr < kD / 2; ++pr) {
+        const float a = x[2 * pr], b = x[2 * pr + 1], sn = sgn * s[pr];
+        x[2 * pr] = a * c[pr] - b * sn;
+        x[2 * pr + 1] = a * sn + b * c[pr];
+    }
+}
+
+constexpr int kQThreads = 128;
+constexpr int kQRows = 128;              // token rows per round: one per thread
+constexpr int kQStride = kD + 4;         // 36 floats: rows 16-byte aligned, 4 banks apart
+constexpr int kQSmem = (kKVZ + 3 * kQRows * kQStride + kQRows) * 4;
 
 // One CTA per (b, h, block n, split sp): dq of the split's tokens and the
 // split's [dS | dZ] sums.  seff: [B][H][nb][1056] inclusive prefix state.
+// Per round of 128 tokens: each thread takes one token (num, den, g, c, dq);
+// then [dS | dZ] += [psi(q) g^T | c phi(q)] over the round's rows, each thread
+// a 4 x 4 block of dS for half of the rows (the two halves are added in a
+// fixed order at the end).
 template <typename T>
-__global__ void __launch_bounds__(kBThreads)
+__global__ void __launch_bounds__(kQThreads)
 bwd_q_kernel(const T *__restrict__ q, const T *__restrict__ dout, const float *__restrict__ seff,
              T *__restrict__ dq, float *__restrict__ bpart, Plan p) {
-    __shared__ float Ss[kKVZ];                 // S_n (row = key feature), then Z_n
-    __shared__ float pq[kBRows][kD + 1];       // psi(q)
-    __shared__ float fq[kBRows][kD + 1];       // phi(q)
-    __shared__ float gg[kBRows][kD + 1];       // g = dout / den
-    __shared__ float cc[kBRows];               // c = -(dout . num) / den^2
+    extern __shared__ __align__(16) float qsm[];
+    float *Ss = qsm;                                  // S_n rows (key feature), then Z_n
+    float *pq = Ss + kKVZ;                            // psi(q)  [kQRows][kQStride]
+    float *fq = pq + kQRows * kQStride;               // phi(q)
+    float *gg = fq + kQRows * kQStride;               // g = dout / den
+    float *cc = gg + kQRows * kQStride;               // c = -(dout . num) / den^2
 
     long long id = blockIdx.x;
     const int sp = (int)(id % p.P); id /= p.P;
@@ -75,98 +122,149 @@ bwd_q_kernel(const T *__restrict__ q, const T *__restrict__ dout, const float *_
     const long long t1 = t0 + p.chunk < blk1 ? t0 + p.chunk : blk1;
     const int tid = threadIdx.x;
     const size_t bh = (size_t)b * p.H + h;
-
     const float *src = seff + (bh * p.nb + n) * kKVZ;
-    for (int e = tid; e < kKVZ; e += kBThreads) Ss[e] = src[e];
-    float acc[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
-    const int r4 = tid >> 2, part = tid & 3;   // row of the round, quarter of the features
-    const size_t row_stride = (size_t)p.H * kD;
+    for (int e = tid; e < kKVZ; e += kQThreads) Ss[e] = src[e];
+
+    const int gi = tid >> 6, j = tid & 63;            // accumulation: row half, 4 x 4 block
+    const int a0 = 4 * (j >> 3), c0 = 4 * (j & 7);
+    float acc[4][4], accz[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        accz[i] = 0.f;
+#pragma unroll
+        for (int k2 = 0; k2 < 4; ++k2) acc[i][k2] = 0.f;
+    }
     __syncthreads();
 
-    for (long long r0 = t0; r0 < t1; r0 += kBRows) {
-        const long long t = r0 + r4;
+    for (long long r0 = t0; r0 < t1; r0 += kQRows) {
+        const long long t = r0 + tid;
         const bool valid = t < t1;
-        const size_t off = ((size_t)b * p.N + (valid ? t : t0)) * row_stride + (size_t)h * kD;
-        // this thread's 8 features: phi, psi, and its 8 of the 32 num, dout terms
-        float f[8], ps[8], dd[8];
+        const size_t off = (((size_t)b * p.N + (valid ? t : t0)) * p.H + h) * kD;
+        float x[kD], ps[kD];
+        uint32_t pos = 0;                              // bit a: q_a > 0
+        if (valid) load_row(q + off, x);
 #pragma unroll
-        for (int a = 0; a < 8; ++a) {
-            const float x = valid ? ldf(q + off + 8 * part + a) : 0.f;
-            f[a] = fmaxf(x, 0.f);
-            ps[a] = f[a];
-            dd[a] = valid ? ldf(dout + off + 8 * part + a) : 0.f;
+        for (int a = 0; a < kD; ++a) {
+            const float v = valid ? x[a] : 0.f;
+            pos |= (v > 0.f ? 1u : 0u) << a;
+            x[a] = fmaxf(v, 0.f);                      // phi(q)
+            ps[a] = x[a];
         }
-        if (p.rope && valid)
-#pragma unroll
-            for (int a = 0; a < 8; a += 2) rot_pair(pair_angle(p, t, (8 * part + a) / 2), 1.f, ps[a], ps[a + 1]);
-#pragma unroll
-        for (int a = 0; a < 8; ++a) {
-            pq[r4][8 * part + a] = ps[a];
-            fq[r4][8 * part + a] = f[a];
+        float cs_c[kD / 2], cs_s[kD / 2];
+        if (p.rope && valid) {
+            token_cs(p, t, cs_c, cs_s);
+            rotate_row(ps, cs_c, cs_s, 1.f);
         }
-        __syncwarp();
-        // den = phi(q) . Z (4 threads of the row, fixed order), num_j for j in
-        // this thread's quarter, dn = dout . num
+#pragma unroll
+        for (int a = 0; a < kD; a += 4) {
+            *reinterpret_cast<float4 *>(pq + tid * kQStride + a) = make_float4(ps[a], ps[a + 1], ps[a + 2], ps[a + 3]);
+            *reinterpret_cast<float4 *>(fq + tid * kQStride + a) = make_float4(x[a], x[a + 1], x[a + 2], x[a + 3]);
+        }
         float den = 0.f;
 #pragma unroll
-        for (int a = 0; a < 8; ++a) den = fmaf(f[a], Ss[kD * kD + 8 * part + a], den);
-        den += __shfl_xor_sync(0xffffffffu, den, 1);
-        den += __shfl_xor_sync(0xffffffffu, den, 2);
+        for (int a = 0; a < kD; ++a) den = fmaf(x[a], Ss[kD * kD + a], den);
         den += p.eps;
+        // num = psi(q) S_n: one S row (8 broadcast 16-byte loads) per feature
+        float num[kD];
+#pragma unroll
+        for (int c = 0; c < kD; ++c) num[c] = 0.f;
+#pragma unroll 4
+        for (int a = 0; a < kD; ++a) {
+            const float4 *row = reinterpret_cast<const float4 *>(Ss + a * kD);
+#pragma unroll
+            for (int c4 = 0; c4 < kD / 4; ++c4) {
+                const float4 sv = row[c4];
+                num[4 * c4] = fmaf(ps[a], sv.x, num[4 * c4]);
+                num[4 * c4 + 1] = fmaf(ps[a], sv.y, num[4 * c4 + 1]);
+                num[4 * c4 + 2] = fmaf(ps[a], sv.z, num[4 * c4 + 2]);
+                num[4 * c4 + 3] = fmaf(ps[a], sv.w, num[4 * c4 + 3]);
+            }
+        }
+        float o[kD];
+        if (valid) load_row(dout + off, o);
         float dn = 0.f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int c = 8 * part + j;
-            float num = 0.f;
-#pragma unroll 8
-            for (int a = 0; a < kD; ++a) num = fmaf(pq[r4][a], Ss[a * kD + c], num);
-            dn = fmaf(dd[j], num, dn);
+        for (int c = 0; c < kD; ++c) {
+            if (!valid) o[c] = 0.f;
+            dn = fmaf(o[c], num[c], dn);
         }
-        dn += __shfl_xor_sync(0xffffffffu, dn, 1);
-        dn += __shfl_xor_sync(0xffffffffu, dn, 2);
         const float inv = 1.0f / den;
         const float cr = valid ? -dn * inv * inv : 0.f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) gg[r4][8 * part + j] = valid ? dd[j] * inv : 0.f;
-        if (part == 0) cc[r4] = cr;
-        __syncwarp();
-        // dq: R^T (S g) + c Z on this thread's 8 features, ReLU mask
-        if (valid) {
-            float dp[8];
+        for (int c = 0; c < kD; ++c) o[c] *= inv;      // g
 #pragma unroll
-            for (int a = 0; a < 8; ++a) {
+        for (int c = 0; c < kD; c += 4)
+            *reinterpret_cast<float4 *>(gg + tid * kQStride + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+        cc[tid] = cr;
+        if (valid) {
+            // dq = mask (R^T (S g) + c Z)
+            float dp[kD];
+#pragma unroll 4
+            for (int a = 0; a < kD; ++a) {
+                const float4 *row = reinterpret_cast<const float4 *>(Ss + a * kD);
                 float s = 0.f;
-#pragma unroll 8
-                for (int c = 0; c < kD; ++c) s = fmaf(Ss[(8 * part + a) * kD + c], gg[r4][c], s);
+#pragma unroll
+                for (int c4 = 0; c4 < kD / 4; ++c4) {
+                    const float4 sv = row[c4];
+                    s = fmaf(sv.x, o[4 * c4], s);
+                    s = fmaf(sv.y, o[4 * c4 + 1], s);
+                    s = fmaf(sv.z, o[4 * c4 + 2], s);
+                    s = fmaf(sv.w, o[4 * c4 + 3], s);
+                }
                 dp[a] = s;
             }
-            if (p.rope)
+            if (p.rope) rotate_row(dp, cs_c, cs_s, -1.f);
 #pragma unroll
-                for (int a = 0; a < 8; a += 2) rot_pair(pair_angle(p, t, (8 * part + a) / 2), -1.f, dp[a], dp[a + 1]);
-#pragma unroll
-            for (int a = 0; a < 8; ++a) {
-                const float g = fmaf(cr, Ss[kD * kD + 8 * part + a], dp[a]);
-                stf(dq + off + 8 * part + a, f[a] > 0.f ? g : 0.f);
-            }
+            for (int a = 0; a < kD; ++a) dp[a] = (pos >> a) & 1u ? fmaf(cr, Ss[kD * kD + a], dp[a]) : 0.f;
+            store_row(dq + off, dp);
         }
         __syncthreads();
-        // [dS | dZ] += [psi(q) g^T | c phi(q)] over the round's rows, row order
-        const int rows = t1 - r0 < kBRows ? (int)(t1 - r0) : kBRows;
-        for (int r = 0; r < rows; ++r) {
+        // [dS | dZ] over this thread's half of the round's rows, row order
+        const int nr = t1 - r0 < kQRows ? (int)(t1 - r0) : kQRows;
+        const int rb = gi * (kQRows / 2), re = rb + kQRows / 2 < nr ? rb + kQRows / 2 : nr;
+        for (int r = rb; r < re; ++r) {
+            const float4 pa = *reinterpret_cast<const float4 *>(pq + r * kQStride + a0);
+            const float4 gc = *reinterpret_cast<const float4 *>(gg + r * kQStride + c0);
+            const float pav[4] = {pa.x, pa.y, pa.z, pa.w}, gcv[4] = {gc.x, gc.y, gc.z, gc.w};
 #pragma unroll
-            for (int u = 0; u < 5; ++u) {
-                const int e = tid + u * kBThreads;
-                if (e < kD * kD) acc[u] = fmaf(pq[r][e / kD], gg[r][e % kD], acc[u]);
-                else if (e < kKVZ) acc[u] = fmaf(cc[r], fq[r][e - kD * kD], acc[u]);
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int k2 = 0; k2 < 4; ++k2) acc[i][k2] = fmaf(pav[i], gcv[k2], acc[i][k2]);
+            if (j < 8) {
+                const float4 fz = *reinterpret_cast<const float4 *>(fq + r * kQStride + 4 * j);
+                const float cr2 = cc[r];
+                accz[0] = fmaf(cr2, fz.x, accz[0]);
+                accz[1] = fmaf(cr2, fz.y, accz[1]);
+                accz[2] = fmaf(cr2, fz.z, accz[2]);
+                accz[3] = fmaf(cr2, fz.w, accz[3]);
             }
         }
         __syncthreads();
     }
-    float *dst = bpart + ((bh * p.nb + n) * p.P + sp) * kKVZ;
+    // the two row halves: first + second, in that order
+    float *comb = pq;
+    if (gi == 1) {
 #pragma unroll
-    for (int u = 0; u < 5; ++u) {
-        const int e = tid + u * kBThreads;
-        if (e < kKVZ) dst[e] = acc[u];
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int k2 = 0; k2 < 4; ++k2) comb[(a0 + i) * kD + c0 + k2] = acc[i][k2];
+        if (j < 8)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) comb[kD * kD + 4 * j + i] = accz[i];
+    }
+    __syncthreads();
+    if (gi == 0) {
+        float *dst = bpart + ((bh * p.nb + n) * p.P + sp) * kKVZ;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int k2 = 0; k2 < 4; ++k2) {
+                const int e = (a0 + i) * kD + c0 + k2;
+                dst[e] = acc[i][k2] + comb[e];
+            }
+        if (j < 8)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[kD * kD + 4 * j + i] = accz[i] + comb[kD * kD + 4 * j + i];
     }
 }
 
@@ -189,11 +287,13 @@ bwd_finish_kernel(const float *__restrict__ bpart, float *__restrict__ G, Plan p
 constexpr int kKThreads = 128;
 
 // One CTA per (b, block m, head h, tile of 128 tokens); one thread per token.
+// Each row a of G_m (8 broadcast 16-byte loads) serves both products:
+// dv += psi(k)_a G[a][:] and d psi(k)_a = G[a][:] . v.
 template <typename T>
 __global__ void __launch_bounds__(kKThreads)
 bwd_k_kernel(const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ G,
              T *__restrict__ dk, T *__restrict__ dv, Plan p) {
-    __shared__ float Gs[kKVZ];
+    __shared__ __align__(16) float Gs[kKVZ];
     const int tiles = (p.L + kKThreads - 1) / kKThreads;
     long long id = blockIdx.x;
     const int tile = (int)(id % tiles); id /= tiles;
@@ -208,39 +308,47 @@ bwd_k_kernel(const T *__restrict__ k, const T *__restrict__ v, const float *__re
     const long long blk1 = blk0 + p.L < p.N ? blk0 + p.L : (long long)p.N;
     const long long t = blk0 + (long long)tile * kKThreads + threadIdx.x;
     if (t >= blk1) return;
-    const size_t off = ((size_t)b * p.N + t) * (size_t)p.H * kD + (size_t)h * kD;
-    float f[kD], ps[kD], vv[kD];
+    const size_t off = (((size_t)b * p.N + t) * p.H + h) * kD;
+    float ps[kD], vv[kD];
+    load_row(k + off, ps);
+    load_row(v + off, vv);
+    uint32_t pos = 0;
 #pragma unroll
     for (int a = 0; a < kD; ++a) {
-        f[a] = fmaxf(ldf(k + off + a), 0.f);
-        ps[a] = f[a];
-        vv[a] = ldf(v + off + a);
+        pos |= (ps[a] > 0.f ? 1u : 0u) << a;
+        ps[a] = fmaxf(ps[a], 0.f);
     }
-    if (p.rope)
+    float cs_c[kD / 2], cs_s[kD / 2];
+    if (p.rope) {
+        token_cs(p, t, cs_c, cs_s);
+        rotate_row(ps, cs_c, cs_s, 1.f);
+    }
+    float dvv[kD], dp[kD];
 #pragma unroll
-        for (int a = 0; a < kD; a += 2) rot_pair(pair_angle(p, t, a / 2), 1.f, ps[a], ps[a + 1]);
-    // dv_c = sum_a G[a][c] psi(k)_a
+    for (int c = 0; c < kD; ++c) dvv[c] = 0.f;
 #pragma unroll 4
-    for (int c = 0; c < kD; ++c) {
-        float s = 0.f;
-#pragma unroll
-        for (int a = 0; a < kD; ++a) s = fmaf(Gs[a * kD + c], ps[a], s);
-        stf(dv + off + c, s);
-    }
-    // d psi(k)_a = sum_c G[a][c] v_c, then R^T, + Gz, ReLU mask
-    float dp[kD];
-#pragma unroll
     for (int a = 0; a < kD; ++a) {
+        const float4 *row = reinterpret_cast<const float4 *>(Gs + a * kD);
         float s = 0.f;
 #pragma unroll
-        for (int c = 0; c < kD; ++c) s = fmaf(Gs[a * kD + c], vv[c], s);
+        for (int c4 = 0; c4 < kD / 4; ++c4) {
+            const float4 gv = row[c4];
+            dvv[4 * c4] = fmaf(ps[a], gv.x, dvv[4 * c4]);
+            dvv[4 * c4 + 1] = fmaf(ps[a], gv.y, dvv[4 * c4 + 1]);
+            dvv[4 * c4 + 2] = fmaf(ps[a], gv.z, dvv[4 * c4 + 2]);
+            dvv[4 * c4 + 3] = fmaf(ps[a], gv.w, dvv[4 * c4 + 3]);
+            s = fmaf(gv.x, vv[4 * c4], s);
+            s = fmaf(gv.y, vv[4 * c4 + 1], s);
+            s = fmaf(gv.z, vv[4 * c4 + 2], s);
+            s = fmaf(gv.w, vv[4 * c4 + 3], s);
+        }
         dp[a] = s;
     }
-    if (p.rope)
+    if (p.rope) rotate_row(dp, cs_c, cs_s, -1.f);
 #pragma unroll
-        for (int a = 0; a < kD; a += 2) rot_pair(pair_angle(p, t, a / 2), -1.f, dp[a], dp[a + 1]);
-#pragma unroll
-    for (int a = 0; a < kD; ++a) stf(dk + off + a, f[a] > 0.f ? dp[a] + Gs[kD * kD + a] : 0.f);
+    for (int a = 0; a < kD; ++a) dp[a] = (pos >> a) & 1u ? dp[a] + Gs[kD * kD + a] : 0.f;
+    store_row(dk + off, dp);
+    store_row(dv + off, dvv);
 }
 
 }  // namespace
@@ -249,12 +357,17 @@ int launch_bwd_q(int is_bf16, const void *q, const void *dout, const float *seff
                  const Plan &p, cudaStream_t s) {
     const long long grid = (long long)p.B * p.H * p.nb * p.P;
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
+    static const bool attrs = cudaFuncSetAttribute((const void *)bwd_q_kernel<__nv_bfloat16>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem) == cudaSuccess &&
+                              cudaFuncSetAttribute((const void *)bwd_q_kernel<float>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem) == cudaSuccess;
+    if (!attrs) return -1;
     if (is_bf16)
-        bwd_q_kernel<__nv_bfloat16><<<(unsigned)grid, kBThreads, 0, s>>>(
+        bwd_q_kernel<__nv_bfloat16><<<(unsigned)grid, kQThreads, kQSmem, s>>>(
             static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(dout), seff,
             static_cast<__nv_bfloat16 *>(dq), bpart, p);
     else
-        bwd_q_kernel<float><<<(unsigned)grid, kBThreads, 0, s>>>(static_cast<const float *>(q),
+        bwd_q_kernel<float><<<(unsigned)grid, kQThreads, kQSmem, s>>>(static_cast<const float *>(q),
                                                                  static_cast<const float *>(dout), seff,
                                                                  static_cast<float *>(dq), bpart, p);
     return cudaGetLastError() == cudaSuccess ? 1 : -1;

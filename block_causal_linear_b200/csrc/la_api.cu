@@ -260,6 +260,9 @@ la_status la_full_backward(const void *q, const void *k, const void *v, const vo
     const bool tc = use_tc(dt, p);
     const int bf = dt == LA_BF16;
     int n = 0, r;
+    // stage events (la_set_stage_events): before the state pass, after it,
+    // after the query side, after the key side
+    if (!mark(0, s)) return LA_ECUDA;
     // the forward prefix state S_n, Z_n of every block, as the forward computes it
     r = tc ? la::launch_reduce_tc(k, v, partials, p, s) : la::launch_reduce_ffma(bf, k, v, partials, p, s);
     if (r < 0) return LA_ECUDA;
@@ -267,12 +270,15 @@ la_status la_full_backward(const void *q, const void *k, const void *v, const vo
     if ((r = la::launch_finish(partials, seff, base + w.fwd.bop, nullptr, nullptr, p, tc ? 1 : 0, s)) < 0)
         return LA_ECUDA;
     n += r;
+    if (!mark(1, s)) return LA_ECUDA;
     if ((r = la::launch_bwd_q(bf, q, dout, seff, dq, bpart, p, s)) < 0) return LA_ECUDA;
     n += r;
+    if (!mark(2, s)) return LA_ECUDA;
     if ((r = la::launch_bwd_finish(bpart, G, p, s)) < 0) return LA_ECUDA;
     n += r;
     if ((r = la::launch_bwd_k(bf, k, v, G, dk, dv, p, s)) < 0) return LA_ECUDA;
     n += r;
+    if (!mark(3, s)) return LA_ECUDA;
     g_last_launches = n;
     g_last_path = tc ? "bwd(tc state)" : "bwd";
     return LA_OK;

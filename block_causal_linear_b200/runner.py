@@ -33,6 +33,8 @@ class Runner:
             self.ws = la.alloc_workspace(w.B, w.n_blk, w.H, w.d, w.n_blk, device=self.device)
             self.tokens_per_block = w.n_blk
         self.outs = [torch.empty_like(c[2]) for c in self.calls]
+        self.inputs = [c[2:5] for c in self.calls]        # device inputs of each call
+        self.out_call = list(range(len(self.calls)))      # the call that writes each out
         self.state = la.State(w.B, w.H, w.d, device=self.device) if w.mode == "stream" else None
         self.rope = None
         if w.rope:
@@ -77,3 +79,41 @@ def host_heads(t: torch.Tensor, heads: Sequence[int]) -> torch.Tensor:
     """Copy the listed heads of a [B, N, H, d] device tensor to the host."""
     idx = torch.as_tensor(list(heads), device=t.device)
     return t.index_select(2, idx).contiguous().cpu()
+
+
+class BackwardRunner:
+    """One training backward pass (``la_full_backward``) over a workload's
+    whole sequence: its blocks concatenated (one pass per block), the same
+    block length and RoPE, a seeded upstream gradient dout; writes dq, dk, dv.
+    The same interface as Runner for the benchmark."""
+
+    def __init__(self, w: synth.Workload, device="cuda"):
+        self.w = w.shrink(passes=1)
+        w = self.w
+        self.device = torch.device(device)
+        q, k, v = synth.full_sequence(w, device=self.device)
+        dout = synth.upstream_grad(w, device=self.device)
+        self.calls = [(0, 0, q, k, v)]
+        self.inputs = [(q, k, v, dout)]
+        self.outs = [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
+        self.out_call = [0, 0, 0]
+        self.tokens_per_block = 0 if w.n_blocks == 1 else w.n_blk
+        self.ws = la.alloc_backward_workspace(w.B, w.n_total, w.H, w.d, self.tokens_per_block, device=self.device)
+        self.rope = (la.make_rope(Hg=w.Hg, Wg=w.Wg, T=w.frames, t_offset=0, dims=w.rope_dims, base=w.rope_base)
+                     if w.rope else None)
+        self._launches = 0
+
+    @property
+    def launches_per_step(self) -> int:
+        return self._launches
+
+    def step(self, after_call: Optional[Callable[[int], None]] = None, stream=None) -> None:
+        q, k, v, dout = self.inputs[0]
+        la.full_backward(q, k, v, dout, self.tokens_per_block, rope=self.rope, eps=self.w.eps, ws=self.ws,
+                         grads=tuple(self.outs), stream=stream)
+        self._launches = la.la_last_launch_count()
+        if after_call:
+            after_call(0)
+
+    def tokens_per_call(self, i: int) -> int:
+        return self.calls[i][2].shape[1]

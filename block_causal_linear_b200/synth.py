@@ -143,6 +143,15 @@ def full_sequence(w: Workload, device="cpu"):
     return torch.cat(qs, 1), torch.cat(ks, 1), torch.cat(vs, 1)
 
 
+def upstream_grad(w: Workload, device="cpu") -> torch.Tensor:
+    """dout for a backward pass over the whole sequence of a workload: the same
+    recipe as the inputs, from the workload's seed + 7919, drawn after nothing
+    else (so it does not change the inputs' draws)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed + 7919)
+    return _draw(w, g, w.n_blk * w.n_blocks, device)
+
+
 def random_qkv(B, N, H, d, seed, dtype=torch.float32, device="cpu", scale=1.0, bias=0.0):
     """Free-form seeded draw for edge-case tests (same recipe, any shape):
     fp64 normal draws rounded to fp32, then converted to ``dtype``."""
