@@ -209,3 +209,22 @@ def full_backward(q, k, v, dout, tokens_per_block=0, rope=None, eps=1e-6):
                                  int(tokens_per_block), _rope_ptr(rope), float(eps))
     _check(rc, "full_backward")
     return dq, dk, dv
+
+
+def e4m3_decode(codes: torch.Tensor, scale: float = 1.0) -> torch.Tensor:
+    """fp64 values of FP8 E4M3 codes (uint8) times a per-tensor scale.
+
+    The format (OCP 8-bit floating point, E4M3 variant): 1 sign bit, 4
+    exponent bits with bias 7, 3 mantissa bits; exponent field 0 encodes
+    subnormals m / 8 * 2^-6; S.1111.111 is NaN and there is no infinity, so
+    the largest finite magnitude is 1.75 * 2^8 = 448.  Every value times an
+    fp32 scale is exact in fp64 (4 + 24 significant bits)."""
+    c = codes.to(torch.int64)
+    sign = torch.where(c >= 128, -1.0, 1.0).to(torch.float64)
+    e = (c >> 3) & 15
+    m = (c & 7).to(torch.float64)
+    normal = (1.0 + m / 8.0) * torch.pow(torch.tensor(2.0, dtype=torch.float64), (e - 7).to(torch.float64))
+    sub = (m / 8.0) * 2.0 ** -6
+    mag = torch.where(e == 0, sub, normal)
+    mag = torch.where((e == 15) & ((c & 7) == 7), torch.tensor(float("nan"), dtype=torch.float64), mag)
+    return sign * mag * float(scale)
