@@ -30,6 +30,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -180,13 +182,15 @@ constexpr int kRRows = 32;                 // token rows per reduce pipeline sta
 constexpr int kRBox = kRRows * 128;        // [32 rows][64 bf16] = 4 KiB
 static_assert(kRRows == 32, "the ReLU pass below maps 128 threads x 4 chunks onto two 32-row boxes");
 
-template <bool ROPE>
+// F8: k and v are FP8 E4M3 codes; one TMA box per tensor and stage holds the
+// 4 heads' 128 codes of 32 tokens (4 KiB), and the MMAs are kind::f8f6f4.
+template <bool ROPE, bool F8 = false>
 struct RCfg {
-    static constexpr int kStages = ROPE ? 4 : 6;
+    static constexpr int kStages = F8 ? 12 : (ROPE ? 4 : 6);
     // stage: k boxes (becoming R phi(k) hi with RoPE), [lo boxes], v boxes
     static constexpr int kLoOff = 2 * kRBox;
-    static constexpr int kVOff = ROPE ? 4 * kRBox : 2 * kRBox;
-    static constexpr int kStageBytes = kVOff + 2 * kRBox;
+    static constexpr int kVOff = F8 ? kRRows * 128 : (ROPE ? 4 * kRBox : 2 * kRBox);
+    static constexpr int kStageBytes = F8 ? 2 * kRRows * 128 : kVOff + 2 * kRBox;
     static constexpr int kAuxOff = kStages * kStageBytes;          // ones (512 B) or RoPE table
     static constexpr int kAuxBytes = ROPE ? kTabMax * 8 : 512;
     static constexpr int kBarOff = kAuxOff + kAuxBytes;
@@ -199,11 +203,12 @@ struct RCfg {
     static constexpr int kThreadsR = 64 + kXform;
 };
 
-template <bool ROPE>
-__global__ void __launch_bounds__(RCfg<ROPE>::kThreadsR, 2)
+template <bool ROPE, bool F8 = false>
+__global__ void __launch_bounds__(RCfg<ROPE, F8>::kThreadsR, 2)
 reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  float *__restrict__ partials, const Plan p) {
-    using C = RCfg<ROPE>;
+    static_assert(!(ROPE && F8), "FP8 inputs take no RoPE");
+    using C = RCfg<ROPE, F8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     uint8_t *aux = smem + C::kAuxOff;
@@ -258,7 +263,9 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         build_rope_table(reinterpret_cast<float2 *>(aux), p, f_lo, nf, threadIdx.x, C::kThreadsR);
     } else {
         // B operand of the z contraction: 16 x 16 bf16 ones (any layout reads 1.0)
-        for (int i = threadIdx.x; i < 128; i += C::kThreadsR) reinterpret_cast<uint32_t *>(aux)[i] = 0x3F803F80u;
+        // (1.0 is 0x3F80 in bf16, 0x38 in E4M3)
+        for (int i = threadIdx.x; i < 128; i += C::kThreadsR)
+            reinterpret_cast<uint32_t *>(aux)[i] = F8 ? 0x38383838u : 0x3F803F80u;
     }
     if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, C::kTmemCols);
@@ -282,20 +289,27 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
                 if (!mbar_wait(&empty[s], ph ^ 1u, abort_word, &g_wait_flag, 1)) break;
                 uint8_t *st = smem + s * C::kStageBytes;
-                mbar_arrive_expect_tx(&full[s], 4 * kRBox);
                 const int row = (int)(t0 + (long long)kRRows * i);
-                const int c0 = g * 128;
-                tma_load_3d(st, &tm_k, &full[s], c0, row, b);
-                tma_load_3d(st + kRBox, &tm_k, &full[s], c0 + 64, row, b);
-                tma_load_3d(st + C::kVOff, &tm_v, &full[s], c0, row, b);
-                tma_load_3d(st + C::kVOff + kRBox, &tm_v, &full[s], c0 + 64, row, b);
+                const int c0 = g * 128;   // first feature of the group (a code = a byte with F8)
+                if constexpr (F8) {
+                    mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+                    tma_load_3d(st, &tm_k, &full[s], c0, row, b);
+                    tma_load_3d(st + C::kVOff, &tm_v, &full[s], c0, row, b);
+                } else {
+                    mbar_arrive_expect_tx(&full[s], 4 * kRBox);
+                    tma_load_3d(st, &tm_k, &full[s], c0, row, b);
+                    tma_load_3d(st + kRBox, &tm_k, &full[s], c0 + 64, row, b);
+                    tma_load_3d(st + C::kVOff, &tm_v, &full[s], c0, row, b);
+                    tma_load_3d(st + C::kVOff + kRBox, &tm_v, &full[s], c0 + 64, row, b);
+                }
                 issued = i + 1;
             }
         }
     } else if (warp == kWarpMma) {
         if (lane == 0) {
-            const uint32_t id_kv = idesc_bf16(128, 128, 1, 1);
-            const uint32_t id_z = idesc_bf16(128, 16, 1, 0);
+            const uint32_t id_kv = F8 ? idesc_e4m3(128, 128, 1, 1) : idesc_bf16(128, 128, 1, 1);
+            const uint32_t id_z = F8 ? idesc_e4m3(128, 16, 1, 0) : idesc_bf16(128, 16, 1, 0);
+            // ones: K-major, no swizzle, 32 bytes of K per row either way
             const uint64_t d_ones = smem_desc(smem_u32(aux), 128, 256, kLayoutNone);
             for (int i = 0; i < nst; ++i) {
                 const int s = i % C::kStages;
@@ -304,6 +318,17 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 tc_fence_after();
                 const uint32_t kaddr = smem_u32(smem + s * C::kStageBytes);
                 const uint32_t vaddr = kaddr + C::kVOff;
+                if constexpr (F8) {
+                    // MN-major, 128-byte swizzle: the 128 codes of a token are one
+                    // 128-byte row; K = 32 tokens = four 8-row groups 1024 B apart
+                    const uint64_t da = smem_desc(kaddr, 4096, 1024, kLayoutSw128);
+                    const uint64_t db = smem_desc(vaddr, 4096, 1024, kLayoutSw128);
+                    const uint32_t acc = i > 0 ? 1u : 0u;
+                    mma_f8(tmem, da, db, id_kv, acc);
+                    mma_f8(tmem + 128, da, d_ones, id_z, acc);
+                    mma_commit(&empty[s]);
+                    continue;
+                }
 #pragma unroll
                 for (int kk = 0; kk < kRRows / 16; ++kk) {
                     // MN-major, 128-byte swizzle: 64-wide MN atoms kRBox apart (LBO),
@@ -368,6 +393,23 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                         *reinterpret_cast<uint4 *>(kt + C::kLoOff + (size_t)c * 16) = lo;
                     }
                 }
+            } else if constexpr (F8) {
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {             // the k box: 256 chunks of 16 codes, 2 per thread
+                    const int c = wt + 128 * j;
+                    const int r = c >> 3;                 // token row (8 chunks of 16 B per 128-byte row)
+                    uint4 *ptr = reinterpret_cast<uint4 *>(kt + (size_t)c * 16);
+                    uint4 x = *ptr;
+                    if (row0 + r < t1) {
+                        // E4M3 codes as signed bytes: every negative value (sign bit
+                        // set, -0 included) is below 0, so a signed max with 0 is ReLU
+                        x.x = __vmaxs4(x.x, 0u); x.y = __vmaxs4(x.y, 0u);
+                        x.z = __vmaxs4(x.z, 0u); x.w = __vmaxs4(x.w, 0u);
+                    } else {
+                        x = make_uint4(0u, 0u, 0u, 0u);   // rows past the split contribute nothing
+                    }
+                    *ptr = x;
+                }
             } else {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {             // 512 chunks of 16 bytes: 4 per thread
@@ -419,6 +461,13 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             tmem_ld32(tmem + lane_off + 32 * qd, kv);
             if constexpr (!ROPE) z = tmem_ld1(tmem + lane_off + 128);
             tmem_wait_ld();
+            if constexpr (F8) {
+                // per-tensor scales: KV = sk sv sum phi(k^) v^T, z = sk sum phi(k^)
+                const float skv = p.sk * p.sv;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) kv[j] *= skv;
+                z *= p.sk;
+            }
             float *dst = partials + ((((size_t)b * p.H + h) * p.nb + n) * p.P + sp) * kKVZ;
             float4 *drow = reinterpret_cast<float4 *>(dst + lane * kD);
 #pragma unroll
@@ -452,11 +501,14 @@ constexpr int kAThreads = 320;                 // 10 warps
 constexpr int kAXform0 = 192;                  // first thread of the transform warps 6..9
 constexpr int kAWarpStg = 32 * 128;            // one epilogue warp's staging box: [32 rows][64 bf16]
 
-template <bool ROPE>
+template <bool ROPE, bool F8 = false>
 struct ACfg {
-    static constexpr int kStages = ROPE ? 2 : 4;
-    static constexpr int kStageBytes = ROPE ? 2 * kATile : kATile;   // [R phi(q) hi | lo] or phi(q)
-    static constexpr int kStgBufs = ROPE ? 1 : 2;                    // staging boxes per epilogue warp
+    // F8: a stage is the bf16 tile the MMA reads (16 KiB, 128-byte swizzle)
+    // followed by the tile's E4M3 codes as TMA lands them (8 KiB, no swizzle)
+    static constexpr int kStages = F8 ? 3 : (ROPE ? 2 : 4);
+    static constexpr int kCodeOff = kATile;
+    static constexpr int kStageBytes = F8 ? kATile + kATile / 2 : (ROPE ? 2 * kATile : kATile);
+    static constexpr int kStgBufs = (ROPE || F8) ? 1 : 2;             // staging boxes per epilogue warp
     static constexpr int kOutOff = kStages * kStageBytes;
     static constexpr int kBopOff = kOutOff + 4 * kStgBufs * kAWarpStg;
     static constexpr int kDenOff = kBopOff + kABopBytes;             // RoPE: [2][128 rows][2 heads] fp32
@@ -474,12 +526,13 @@ struct ACfg {
 // epilogue (warp w reads TMEM lanes 32*(w%4).. = token rows of the tile),
 // 6..9 apply phi (and RoPE) to the q tiles in shared memory.  The transform
 // of tile i+1 and the epilogue of tile i run at the same time.
-template <bool ROPE>
+template <bool ROPE, bool F8 = false>
 __global__ void __launch_bounds__(kAThreads, 2)
 apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_out,
                 __nv_bfloat16 *__restrict__ out, const uint8_t *__restrict__ bop, const float *__restrict__ seff,
                 const Plan p) {
-    using C = ACfg<ROPE>;
+    static_assert(!(ROPE && F8), "FP8 inputs take no RoPE");
+    using C = ACfg<ROPE, F8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     uint8_t *stg = smem + C::kOutOff;
@@ -561,8 +614,9 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // started: its first tiles are fetched while the state combine still runs
             const int pre = ntiles < C::kStages ? ntiles : C::kStages;
             for (int i = 0; i < pre; ++i) {
-                mbar_arrive_expect_tx(&full[i], kATile);
-                tma_load_3d(smem + i * C::kStageBytes, &tm_q, &full[i], hp * 64, (int)(ta0 + 128LL * i), b);
+                mbar_arrive_expect_tx(&full[i], F8 ? kATile / 2 : kATile);
+                tma_load_3d(smem + i * C::kStageBytes + (F8 ? C::kCodeOff : 0), &tm_q, &full[i], hp * 64,
+                            (int)(ta0 + 128LL * i), b);
                 issued = i + 1;
             }
             pdl_wait();   // the packed operand and Z_eff are written by the previous kernel
@@ -577,8 +631,9 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int s = i % C::kStages;
                 const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
                 if (!mbar_wait(&empty[s], ph ^ 1u, abort_word, &g_wait_flag, 11)) break;
-                mbar_arrive_expect_tx(&full[s], kATile);
-                tma_load_3d(smem + s * C::kStageBytes, &tm_q, &full[s], hp * 64, (int)(ta0 + 128LL * i), b);
+                mbar_arrive_expect_tx(&full[s], F8 ? kATile / 2 : kATile);
+                tma_load_3d(smem + s * C::kStageBytes + (F8 ? C::kCodeOff : 0), &tm_q, &full[s], hp * 64,
+                            (int)(ta0 + 128LL * i), b);
                 issued = i + 1;
             }
         }
@@ -699,6 +754,25 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         den_s[(i & 1) * 256 + rr * 2 + (h0 ^ 1)] = dp[1];
                     }
                 }
+            } else if (F8 && ok) {
+                // E4M3 codes [128 rows][64] -> phi(q) in bf16, exact (<= 4 significant
+                // bits), into the 128-byte swizzled tile the MMA reads
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int u = tt + 128 * j;
+                    const int rr = u >> 3, L = u & 7;       // token row, logical chunk of 8 features
+                    const uint2 c8 = *reinterpret_cast<const uint2 *>(qt + C::kCodeOff + rr * 64 + L * 8);
+                    const uint32_t w[2] = {__vmaxs4(c8.x, 0u), __vmaxs4(c8.y, 0u)};   // ReLU on the codes
+                    uint32_t o[4];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)(w[m >> 1] >> (16 * (m & 1)));
+                        const __half2 hv = __half2(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3));
+                        const float2 fv = __half22float2(hv);
+                        o[m] = pack_bf2(fv.x, fv.y);
+                    }
+                    *reinterpret_cast<uint4 *>(qt + rr * 128 + ((L ^ (rr & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
             } else if (ok) {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
@@ -756,7 +830,9 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (lane == 0) bulk_wait_read<C::kStgBufs - 1>();   // the last store from sb has read it
                 __syncwarp();
                 if (got) {
-                    const float inv0 = 1.0f / (den0 + p.eps), inv1 = 1.0f / (den1 + p.eps);
+                    // F8: out = sq num^ / (sq den^ + eps) with num^, den^ from the codes
+                    const float qs = F8 ? p.sq : 1.0f;
+                    const float inv0 = qs / (qs * den0 + p.eps), inv1 = qs / (qs * den1 + p.eps);
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {       // logical 16-byte chunk c: head c/4
                         const float *v = c < 4 ? num0 : num1;
@@ -776,7 +852,8 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             } else if (got && row0 + r < ta1) {
                 // a short last tile inside the tensor: the rows after ta1 belong to another block
-                const float inv0 = 1.0f / (den0 + p.eps), inv1 = 1.0f / (den1 + p.eps);
+                const float qs = F8 ? p.sq : 1.0f;
+                const float inv0 = qs / (qs * den0 + p.eps), inv1 = qs / (qs * den1 + p.eps);
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     const float *v = hh ? num1 : num0;
@@ -846,6 +923,21 @@ bool make_map(CUtensorMap *m, const void *base, int B, int N, int H, int box_row
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3D view of a [B][N][H*32] tensor of one-byte E4M3 codes: boxes of box_inner
+// codes x box_rows tokens, 128-byte swizzle or none.
+bool make_map_u8(CUtensorMap *m, const void *base, int B, int N, int H, int box_inner, int box_rows, bool sw128) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t row_bytes = (cuuint64_t)H * kD;
+    cuuint64_t dims[3] = {(cuuint64_t)H * kD, (cuuint64_t)N, (cuuint64_t)B};
+    cuuint64_t strides[2] = {row_bytes, row_bytes * (cuuint64_t)N};
+    cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Launch with programmatic stream serialization (the kernel may start while
 // the previous kernel of the stream drains; it orders itself with pdl_wait).
 template <typename... KArgs, typename... Args>
@@ -875,7 +967,9 @@ bool smem_ready() {
         ok = set_smem((const void *)reduce_tc_kernel<false>, RCfg<false>::kSmem) &&
              set_smem((const void *)reduce_tc_kernel<true>, RCfg<true>::kSmem) &&
              set_smem((const void *)apply_tc_kernel<false>, ACfg<false>::kSmem) &&
-             set_smem((const void *)apply_tc_kernel<true>, ACfg<true>::kSmem);
+             set_smem((const void *)apply_tc_kernel<true>, ACfg<true>::kSmem) &&
+             set_smem((const void *)reduce_tc_kernel<false, true>, RCfg<false, true>::kSmem) &&
+             set_smem((const void *)apply_tc_kernel<false, true>, ACfg<false, true>::kSmem);
     });
     return ok;
 }
@@ -907,9 +1001,18 @@ bool tc_rope_fits(const Plan &p) {
 int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &p, cudaStream_t s) {
     if (!smem_ready()) return -1;
     CUtensorMap mk, mv;
-    if (!make_map(&mk, k, p.B, p.N, p.H, kRRows) || !make_map(&mv, v, p.B, p.N, p.H, kRRows)) return -1;
     const long long grid = (long long)p.B * (p.H / 4) * p.nb * p.P;
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
+    if (p.f8) {
+        if (!make_map_u8(&mk, k, p.B, p.N, p.H, 128, kRRows, true) ||
+            !make_map_u8(&mv, v, p.B, p.N, p.H, 128, kRRows, true))
+            return -1;
+        return launch_pdl(reduce_tc_kernel<false, true>, (unsigned)grid, RCfg<false, true>::kThreadsR,
+                          RCfg<false, true>::kSmem, s, mk, mv, partials, p)
+                   ? 1
+                   : -1;
+    }
+    if (!make_map(&mk, k, p.B, p.N, p.H, kRRows) || !make_map(&mv, v, p.B, p.N, p.H, kRRows)) return -1;
     const bool ok = p.rope ? launch_pdl(reduce_tc_kernel<true>, (unsigned)grid, RCfg<true>::kThreadsR, RCfg<true>::kSmem, s, mk,
                                         mv, partials, p)
                            : launch_pdl(reduce_tc_kernel<false>, (unsigned)grid, RCfg<false>::kThreadsR, RCfg<false>::kSmem, s, mk,
@@ -920,11 +1023,19 @@ int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &
 int launch_apply_tc(const void *q, void *out, const void *bop, const float *seff, const Plan &p, cudaStream_t s) {
     if (!smem_ready()) return -1;
     CUtensorMap mq, mo;
-    if (!make_map(&mq, q, p.B, p.N, p.H, 128) || !make_map(&mo, out, p.B, p.N, p.H, 32)) return -1;
     const long long grid = (long long)p.B * p.nb * p.Pa * (p.H / 2);
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
     const uint8_t *bb = static_cast<const uint8_t *>(bop);
+    if (p.f8) {
+        // q codes: boxes of the 2 heads' 64 codes x 128 tokens, no swizzle; out bf16
+        if (!make_map_u8(&mq, q, p.B, p.N, p.H, 64, 128, false) || !make_map(&mo, out, p.B, p.N, p.H, 32)) return -1;
+        return launch_pdl(apply_tc_kernel<false, true>, (unsigned)grid, kAThreads, ACfg<false, true>::kSmem, s, mq,
+                          mo, o, bb, seff, p)
+                   ? 1
+                   : -1;
+    }
+    if (!make_map(&mq, q, p.B, p.N, p.H, 128) || !make_map(&mo, out, p.B, p.N, p.H, 32)) return -1;
     const bool ok = p.rope ? launch_pdl(apply_tc_kernel<true>, (unsigned)grid, kAThreads, ACfg<true>::kSmem, s, mq,
                                         mo, o, bb, seff, p)
                            : launch_pdl(apply_tc_kernel<false>, (unsigned)grid, kAThreads, ACfg<false>::kSmem, s, mq,

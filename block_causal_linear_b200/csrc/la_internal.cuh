@@ -30,6 +30,8 @@ struct Plan {
     int commit;           // write S_eff of the last block back to the state
     int has_state;        // S, Z hold a prior state (block_forward) or not (full_forward)
     int rope;             // numerator RoPE on phi(q), phi(k)
+    int f8;               // q, k, v are FP8 E4M3 codes with per-tensor scales sq, sk, sv
+    float sq, sk, sv;
     int Hg, Wg;           // latent grid of one frame
     int t_offset;         // frame of token 0 of the call
     float eps;

@@ -68,6 +68,11 @@ def lib() -> ctypes.CDLL:
         L.la_full_forward_static_ws.argtypes = [vp, vp, vp, vp, ip, ip, ip, ip, ip, ip,
                                                 ctypes.POINTER(la_rope), fp, vp]
         L.la_full_forward_static_ws.restype = ip
+        L.la_full_forward_e4m3.argtypes = [vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ip, fp, vp, sz, vp]
+        L.la_full_forward_e4m3.restype = ip
+        L.la_block_forward_e4m3.argtypes = [vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ctypes.POINTER(la_state), ip,
+                                            fp, vp, sz, vp]
+        L.la_block_forward_e4m3.restype = ip
         L.la_backward_workspace_size.argtypes = [ip, ip, ip, ip, ip]
         L.la_backward_workspace_size.restype = sz
         L.la_full_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip,
@@ -120,6 +125,16 @@ def la_full_forward_static_ws(q, k, v, out, dt, B, N, H, d, tokens_per_block, ro
 
 
 LA_STATIC_WS_BYTES = 16 << 20
+
+
+def la_full_forward_e4m3(q, k, v, sq, sk, sv, out, B, N, H, d, tokens_per_block, eps, ws, ws_bytes, stream) -> int:
+    return int(lib().la_full_forward_e4m3(q, k, v, sq, sk, sv, out, B, N, H, d, tokens_per_block, eps, ws, ws_bytes,
+                                          stream))
+
+
+def la_block_forward_e4m3(q, k, v, sq, sk, sv, out, B, N_blk, H, d, st, commit, eps, ws, ws_bytes, stream) -> int:
+    return int(lib().la_block_forward_e4m3(q, k, v, sq, sk, sv, out, B, N_blk, H, d, ctypes.byref(st), commit, eps,
+                                           ws, ws_bytes, stream))
 
 
 def la_backward_workspace_size(B, N, H, d, tokens_per_block) -> int:
@@ -254,6 +269,50 @@ def full_forward(q, k, v, tokens_per_block=0, rope: Optional[la_rope] = None, ep
                          ws.numel() * ws.element_size(), _stream_ptr(stream))
     if rc != LA_OK:
         raise LAError(rc, "la_full_forward")
+    return out
+
+
+def _check_codes(q, k, v):
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous() or t.dim() != 4 or t.dtype != torch.uint8:
+            raise ValueError("E4M3 q, k, v must be contiguous CUDA uint8 tensors [B, N, H, d]")
+    if not q.shape == k.shape == v.shape:
+        raise ValueError("q, k, v must agree in shape")
+
+
+def full_forward_e4m3(q, k, v, scales, tokens_per_block=0, eps=1e-6, ws: Optional[torch.Tensor] = None,
+                      out: Optional[torch.Tensor] = None, stream=None):
+    """la_full_forward on FP8 E4M3 codes (uint8 tensors) with per-tensor
+    scales (sq, sk, sv); out is bf16."""
+    _check_codes(q, k, v)
+    B, N, H, d = q.shape
+    if ws is None:
+        ws = alloc_workspace(B, N, H, d, tokens_per_block, device=q.device)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    sq, sk, sv = (float(x) for x in scales)
+    rc = la_full_forward_e4m3(q.data_ptr(), k.data_ptr(), v.data_ptr(), sq, sk, sv, out.data_ptr(), B, N, H, d,
+                              int(tokens_per_block), float(eps), ws.data_ptr(), ws.numel() * ws.element_size(),
+                              _stream_ptr(stream))
+    if rc != LA_OK:
+        raise LAError(rc, "la_full_forward_e4m3")
+    return out
+
+
+def block_forward_e4m3(q, k, v, scales, state: "State", commit=True, eps=1e-6, ws: Optional[torch.Tensor] = None,
+                       out: Optional[torch.Tensor] = None, stream=None):
+    _check_codes(q, k, v)
+    B, N, H, d = q.shape
+    if ws is None:
+        ws = alloc_workspace(B, N, H, d, N, device=q.device)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    sq, sk, sv = (float(x) for x in scales)
+    rc = la_block_forward_e4m3(q.data_ptr(), k.data_ptr(), v.data_ptr(), sq, sk, sv, out.data_ptr(), B, N, H, d,
+                               state.c, int(bool(commit)), float(eps), ws.data_ptr(), ws.numel() * ws.element_size(),
+                               _stream_ptr(stream))
+    if rc != LA_OK:
+        raise LAError(rc, "la_block_forward_e4m3")
     return out
 
 

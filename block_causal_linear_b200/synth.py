@@ -152,6 +152,18 @@ def upstream_grad(w: Workload, device="cpu") -> torch.Tensor:
     return _draw(w, g, w.n_blk * w.n_blocks, device)
 
 
+def to_e4m3(x: torch.Tensor):
+    """FP8 inputs for the E4M3 path: per-tensor amax scaling, scale =
+    max|x| / 448 in fp32 (448 is the largest E4M3 magnitude), codes = x / scale
+    rounded to nearest even E4M3 (torch float8_e4m3fn).  Returns (uint8 codes,
+    scale).  Input preparation only."""
+    xf = x.to(torch.float32)
+    amax = float(xf.abs().max()) if xf.numel() else 0.0
+    scale = float(torch.tensor(amax / 448.0 if amax > 0 else 1.0, dtype=torch.float32))
+    codes = (xf / scale).clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes, scale
+
+
 def random_qkv(B, N, H, d, seed, dtype=torch.float32, device="cpu", scale=1.0, bias=0.0):
     """Free-form seeded draw for edge-case tests (same recipe, any shape):
     fp64 normal draws rounded to fp32, then converted to ``dtype``."""

@@ -178,6 +178,33 @@ LA_API la_status la_full_backward(const void *q, const void *k, const void *v, c
                                   void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * FP8 inputs.  q, k, v as FP8 E4M3 codes (one byte each, [B][N][H][d], OCP
+ * 8-bit float E4M3: bias 7, 3 mantissa bits, max 448) with one fp32 scale per
+ * tensor: the values are q = scale_q * decode(q_code), and likewise k, v.
+ * Since ReLU commutes with a positive scale, the results are those of
+ * la_full_forward / la_block_forward on the decoded values:
+ *   KV_n = scale_k scale_v sum phi(k^) v^T,  z_n = scale_k sum phi(k^),
+ *   out = scale_q psi(q^) S_eff / (scale_q phi(q^) . Z_eff + eps),
+ * out in bf16.  The state (S, Z) is fp32 in real units, so e4m3 and bf16
+ * calls may share one stream of blocks.  The pages quantise the deployed
+ * model to NVFP4 ("Nvidia, MIT ve diğerleri video yapay zeka devrimini
+ * başlattı", section "Etkin eğitim ve çıkarım stratejileri": SVDQuant); FP8
+ * q, k, v here shrink the bytes this path moves (160 instead of 256 per token
+ * and head).
+ * Scales must be finite and > 0 (LA_EINVAL); H must be a multiple of 4 and
+ * the GPU must take the tensor-core path (else LA_EUNSUPPORTED); no RoPE.
+ * Workspace and every other argument as in the bf16 calls.
+ */
+LA_API la_status la_full_forward_e4m3(const void *q, const void *k, const void *v, float scale_q,
+                                      float scale_k, float scale_v, void *out, int B, int N, int H,
+                                      int d, int tokens_per_block, float eps, void *ws,
+                                      size_t ws_bytes, void *stream);
+LA_API la_status la_block_forward_e4m3(const void *q, const void *k, const void *v, float scale_q,
+                                       float scale_k, float scale_v, void *out, int B, int N_blk,
+                                       int H, int d, la_state *st, int commit, float eps, void *ws,
+                                       size_t ws_bytes, void *stream);
+
+/*
  * For callers that cannot allocate device memory at all.  Some code that
  * calls this library runs inside a host framework that owns every device
  * allocation and gives a plug-in no allocator and no way to size or keep a

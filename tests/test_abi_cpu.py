@@ -144,3 +144,38 @@ def test_backward_workspace_size(la):
     bwd = la.la_backward_workspace_size(1, 4 * 640, 8, 32, 640)
     assert bwd > fwd and bwd % 256 == 0
     assert la.la_backward_workspace_size(1, 0, 8, 32, 0) == 0
+
+
+def test_e4m3_validation(la):
+    def full(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, sq=0.01, sk=0.01, sv=0.01, out=FAKE, B=1, N=256, H=4, d=32, tpb=0,
+                 eps=1e-6, ws=FAKE, ws_bytes=1 << 30, stream=None)
+        a.update(kw)
+        return la.la_full_forward_e4m3(a["q"], a["k"], a["v"], a["sq"], a["sk"], a["sv"], a["out"], a["B"], a["N"],
+                                       a["H"], a["d"], a["tpb"], a["eps"], a["ws"], a["ws_bytes"], a["stream"])
+    assert full(q=None) == la.LA_EINVAL
+    assert full(out=FAKE + 4) == la.LA_EINVAL
+    assert full(sq=0.0) == la.LA_EINVAL
+    assert full(sk=-1.0) == la.LA_EINVAL
+    assert full(sv=float("nan")) == la.LA_EINVAL
+    assert full(d=16) == la.LA_EUNSUPPORTED
+    assert full(H=6) == la.LA_EUNSUPPORTED             # the E4M3 path takes 4-head groups
+    st = la.la_state()
+    assert la.la_block_forward_e4m3(FAKE, FAKE, FAKE, 1.0, 1.0, 1.0, FAKE, 1, 64, 4, 32, st, 1, 1e-6, FAKE,
+                                    1 << 30, None) in (la.LA_EINVAL, la.LA_EUNSUPPORTED)
+    assert st.blocks_committed == 0
+
+
+def test_e4m3_quantiser_round_trip():
+    import torch
+    from block_causal_linear_b200 import synth
+
+    x = torch.randn(3, 100, 2, 32, generator=torch.Generator().manual_seed(5))
+    codes, s = synth.to_e4m3(x)
+    assert codes.dtype == torch.uint8 and codes.shape == x.shape and s > 0
+    back = codes.view(torch.float8_e4m3fn).to(torch.float32) * s
+    # E4M3 keeps 4 significant bits: relative error <= 2^-4 for normal values
+    big = x.abs() > 2.0 ** -6 * s
+    assert bool(((back - x).abs() <= 2.0 ** -4 * x.abs() + 1e-30)[big].all())
+    # amax scaling: the largest magnitude lands on the largest code, 448
+    assert float(codes.view(torch.float8_e4m3fn).to(torch.float32).abs().max()) == 448.0
