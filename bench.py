@@ -64,6 +64,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "backward"],
                     help="backward: la_full_backward over the workload's whole sequence (dq, dk, dv)")
+    ap.add_argument("--input", default="native", choices=["native", "e4m3"],
+                    help="e4m3: q, k, v as FP8 E4M3 codes with per-tensor scales (la_*_forward_e4m3), bf16 out")
     ap.add_argument("--blocks", type=int, default=None,
                     help="streaming workloads: run only the first N blocks (small cases for profiling)")
     ap.add_argument("--shard", default="problem", choices=["problem", "heads"],
@@ -293,7 +295,10 @@ def main():
             raise SystemExit("--blocks needs a streaming workload and 1 <= N <= its block count")
         w = w.shrink(n_blocks=args.blocks)
     bwd = args.pass_ == "backward"
-    runner = BackwardRunner(w, dev) if bwd else Runner(w, dev)
+    f8 = args.input == "e4m3"
+    if f8 and bwd:
+        raise SystemExit("--input e4m3 is a forward path")
+    runner = BackwardRunner(w, dev) if bwd else Runner(w, dev, e4m3=f8)
     w = runner.w
     flush_w = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -415,7 +420,11 @@ def main():
     peak, peak_kind = measured_peaks()
     # algorithmic bytes: forward reads q, k, v and writes out (4 tensors);
     # backward reads q, k, v, dout and writes dq, dk, dv (7 tensors)
-    alg_bytes = w.token_heads * (7 if bwd else 4) * w.d * w.elem_bytes if bwd else w.alg_bytes
+    # E4M3 forward: q, k, v one byte per feature, out bf16
+    if f8:
+        alg_bytes = w.token_heads * w.d * (3 * 1 + 2) + (w.alg_bytes - w.token_heads * 4 * w.d * w.elem_bytes)
+    else:
+        alg_bytes = w.token_heads * (7 if bwd else 4) * w.d * w.elem_bytes if bwd else w.alg_bytes
     step_gbs = alg_bytes / (ms_per_step / 1e3) / 1e9
 
     launches_per_kernel = K * n_calls                # stage_ms is scaled to K steps
@@ -432,7 +441,10 @@ def main():
         dom, dom_ms = ("reduce", red_ms) if red_ms >= app_ms else ("apply", app_ms)
         ntens = 2
         kname = f"{dom}_{path}" + ("_rope" if w.rope and path == "tc" else "")
-    kern_bytes = per_call_th * ntens * w.d * w.elem_bytes
+    if f8:   # reduce: k, v codes; apply: q codes and bf16 out
+        kern_bytes = per_call_th * w.d * (2 if dom == "reduce" else 3)
+    else:
+        kern_bytes = per_call_th * ntens * w.d * w.elem_bytes
     avg_launch_s = dom_ms / launches_per_kernel / 1e3
     achieved = kern_bytes / avg_launch_s / 1e9
 
@@ -453,8 +465,8 @@ def main():
             "metric": METRIC_BWD if bwd else METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "strong" if args.shard == "heads" else "weak", "vs_baseline": None,
-            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-            "config": workload_config(w, {"pass": args.pass_,
+            "dtype": "e4m3 in, bf16 out" if f8 else ("bf16" if w.dtype == "bf16" else "f32"), "data": "synthetic",
+            "config": workload_config(w, {"pass": args.pass_, "input_dtype": "e4m3 (per-tensor scale)" if f8 else w.dtype,
                                           "parallelism": (f"heads of one problem split over {world} ranks"
                                                           if args.shard == "heads" else
                                                           f"independent problem per rank x{world}")}),

@@ -17,8 +17,9 @@ from . import la, synth
 
 
 class Runner:
-    def __init__(self, w: synth.Workload, device="cuda", blocks: Optional[int] = None):
+    def __init__(self, w: synth.Workload, device="cuda", blocks: Optional[int] = None, e4m3: bool = False):
         self.w = w
+        self.e4m3 = e4m3
         self.device = torch.device(device)
         self.calls: List[tuple] = []          # (block, pass, q, k, v) in call order
         if w.mode == "full":
@@ -33,6 +34,16 @@ class Runner:
             self.ws = la.alloc_workspace(w.B, w.n_blk, w.H, w.d, w.n_blk, device=self.device)
             self.tokens_per_block = w.n_blk
         self.outs = [torch.empty_like(c[2]) for c in self.calls]
+        self.scales = None
+        if e4m3:
+            # FP8 inputs: each call's q, k, v as E4M3 codes with per-tensor scales
+            if w.rope:
+                raise ValueError("the E4M3 path takes no RoPE")
+            self.scales = []
+            for i, c in enumerate(self.calls):
+                qk = [synth.to_e4m3(t) for t in c[2:5]]
+                self.calls[i] = (c[0], c[1], *[x for x, _ in qk])
+                self.scales.append([s_ for _, s_ in qk])
         self.inputs = [c[2:5] for c in self.calls]        # device inputs of each call
         self.out_call = list(range(len(self.calls)))      # the call that writes each out
         self.state = la.State(w.B, w.H, w.d, device=self.device) if w.mode == "stream" else None
@@ -52,8 +63,12 @@ class Runner:
         n = 0
         if w.mode == "full":
             _, _, q, k, v = self.calls[0]
-            la.full_forward(q, k, v, self.tokens_per_block, rope=self.rope, eps=w.eps, ws=self.ws,
-                            out=self.outs[0], stream=stream)
+            if self.e4m3:
+                la.full_forward_e4m3(q, k, v, self.scales[0], self.tokens_per_block, eps=w.eps, ws=self.ws,
+                                     out=self.outs[0], stream=stream)
+            else:
+                la.full_forward(q, k, v, self.tokens_per_block, rope=self.rope, eps=w.eps, ws=self.ws,
+                                out=self.outs[0], stream=stream)
             n += la.la_last_launch_count()
             if after_call:
                 after_call(0)
@@ -64,8 +79,12 @@ class Runner:
             if rc != la.LA_OK:
                 raise la.LAError(rc, "la_state_init")
             for i, (blk, p, q, k, v) in enumerate(self.calls):
-                la.block_forward(q, k, v, st, commit=(p == w.passes - 1), rope=self.rope, eps=w.eps,
-                                 ws=self.ws, out=self.outs[i], stream=stream)
+                if self.e4m3:
+                    la.block_forward_e4m3(q, k, v, self.scales[i], st, commit=(p == w.passes - 1), eps=w.eps,
+                                          ws=self.ws, out=self.outs[i], stream=stream)
+                else:
+                    la.block_forward(q, k, v, st, commit=(p == w.passes - 1), rope=self.rope, eps=w.eps,
+                                     ws=self.ws, out=self.outs[i], stream=stream)
                 n += la.la_last_launch_count()
                 if after_call:
                     after_call(i)
