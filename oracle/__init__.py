@@ -72,10 +72,11 @@ def lib():
         L.orc_block_forward.argtypes = [vp, vp, vp, ip, vp, ip, lp, ip, ip, vp, vp, ip, rp, lp, dp]
         L.orc_full_forward.argtypes = [vp, vp, vp, ip, vp, ip, lp, ip, ip, lp, rp, dp]
         L.orc_full_backward.argtypes = [vp, vp, vp, vp, ip, vp, vp, vp, ip, lp, ip, ip, lp, rp, dp]
+        L.orc_dwconv3d.argtypes = [vp, ip, vp, ip, ip, ip, ip, ip, ip, ip, ip, vp, vp]
         L.orc_set_threads.argtypes = [ip]
         L.orc_get_threads.restype = ip
         for f in ("orc_brute", "orc_block_kv", "orc_apply", "orc_block_forward", "orc_full_forward",
-                  "orc_full_backward"):
+                  "orc_full_backward", "orc_dwconv3d"):
             getattr(L, f).restype = ip
         _lib = L
     return _lib
@@ -228,3 +229,22 @@ def e4m3_decode(codes: torch.Tensor, scale: float = 1.0) -> torch.Tensor:
     mag = torch.where(e == 0, sub, normal)
     mag = torch.where((e == 15) & ((c & 7) == 7), torch.tensor(float("nan"), dtype=torch.float64), mag)
     return sign * mag * float(scale)
+
+
+def dwconv3d(x, weight, bias=None):
+    """Depthwise 3D convolution (Mix-FFN): x [B, T, Hg, Wg, C] (fp64/fp32/bf16
+    CPU tensor), weight [C, kt, kh, kw], bias [C] or None; zero padding of
+    (k-1)/2, fp64 numpy result [B, T, Hg, Wg, C]."""
+    if x.dim() != 5:
+        raise ValueError("expected [B, T, Hg, Wg, C]")
+    B, T, Hg, Wg, C = (int(s_) for s_ in x.shape)
+    xc, dt = _prep(x)
+    w = np.ascontiguousarray(np.asarray(weight, dtype=np.float64))
+    if w.ndim != 4 or w.shape[0] != C:
+        raise ValueError("weight must be [C, kt, kh, kw]")
+    bb = None if bias is None else np.ascontiguousarray(np.asarray(bias, dtype=np.float64))
+    y = np.zeros((B, T, Hg, Wg, C), dtype=np.float64)
+    rc = lib().orc_dwconv3d(xc.data_ptr(), dt, y.ctypes.data, B, T, Hg, Wg, C, *(int(k) for k in w.shape[1:]),
+                            w.ctypes.data, None if bb is None else bb.ctypes.data)
+    _check(rc, "dwconv3d")
+    return y

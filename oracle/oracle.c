@@ -485,3 +485,52 @@ int orc_full_backward(const void *q, const void *k, const void *v, const void *d
     }
     return bad;
 }
+
+/*
+ * Depthwise 3D convolution of the Spatial-Temporal Mix-FFN ("Nvidia, MIT ve
+ * diğerleri video yapay zeka devrimini başlattı", section "Verimli doğrusal
+ * DiT": the MLP alternates a 1x3x3 spatial and a 3x1x1 temporal convolution to
+ * add local information to each token).  x, y are [B][T][Hg][Wg][C] (tokens in
+ * frame, row, column order, channels last), w is [C][kt][kh][kw], bias [C] or
+ * NULL; odd kernel sizes, zero padding of (k-1)/2 on each side, within the
+ * call's frames:
+ *   y[b,t,h,w,c] = bias[c] + sum_{i,j,l} w[c][i][j][l] x[b, t+i-pt, h+j-ph, w+l-pw, c]
+ * with out-of-range taps reading 0.
+ */
+int orc_dwconv3d(const void *x, int dtype, double *y, int B, int T, int Hg, int Wg, int C,
+                 int kt, int kh, int kw, const double *w, const double *bias)
+{
+    if (B < 0 || T < 0 || Hg < 0 || Wg < 0 || C <= 0) return 1;
+    if (kt < 1 || kh < 1 || kw < 1 || !(kt & 1) || !(kh & 1) || !(kw & 1)) return 1;
+    int pt = kt / 2, ph = kh / 2, pw = kw / 2;
+    long ntok = (long)B * T * Hg * Wg;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static) ORC_THREADS
+#endif
+    for (long tok = 0; tok < ntok; ++tok) {
+        long r = tok;
+        int ww = (int)(r % Wg); r /= Wg;
+        int hh = (int)(r % Hg); r /= Hg;
+        int tt = (int)(r % T); r /= T;
+        int b = (int)r;
+        for (int c = 0; c < C; ++c) {
+            double acc = bias ? bias[c] : 0.0;
+            for (int i = 0; i < kt; ++i) {
+                int t2 = tt + i - pt;
+                if (t2 < 0 || t2 >= T) continue;
+                for (int j = 0; j < kh; ++j) {
+                    int h2 = hh + j - ph;
+                    if (h2 < 0 || h2 >= Hg) continue;
+                    for (int l = 0; l < kw; ++l) {
+                        int w2 = ww + l - pw;
+                        if (w2 < 0 || w2 >= Wg) continue;
+                        size_t src = ((((size_t)b * T + t2) * Hg + h2) * Wg + w2) * C + c;
+                        acc += w[(((size_t)c * kt + i) * kh + j) * kw + l] * elem(x, dtype, src);
+                    }
+                }
+            }
+            y[(size_t)tok * C + c] = acc;
+        }
+    }
+    return 0;
+}
