@@ -341,6 +341,22 @@ la_status la_block_forward_e4m3(const void *q, const void *k, const void *v, flo
     return LA_OK;
 }
 
+la_status la_dwconv3d(const void *x, void *y, la_dtype dt, int B, int T, int Hg, int Wg, int C, int kt, int kh,
+                      int kw, const float *weight, const float *bias, void *stream) {
+    if (!x || !y || !weight || !aligned16(x) || !aligned16(y)) return LA_EINVAL;
+    if (dt != LA_F32 && dt != LA_BF16) return LA_EINVAL;
+    if (B <= 0 || T <= 0 || Hg <= 0 || Wg <= 0 || C <= 0) return LA_EINVAL;
+    if ((long long)B * T * Hg * Wg * C >= (1LL << 40)) return LA_EINVAL;
+    if (C % 8 != 0) return LA_EUNSUPPORTED;
+    const int r = la::launch_dwconv(dt == LA_BF16, x, y, weight, bias, B, T, Hg, Wg, C, kt, kh, kw,
+                                    static_cast<cudaStream_t>(stream));
+    if (r == -2) return LA_EUNSUPPORTED;
+    if (r < 0) return LA_ECUDA;
+    g_last_launches = r;
+    g_last_path = "dwconv";
+    return LA_OK;
+}
+
 la_status la_device_status(void *stream) {
     unsigned flag = 0;
     if (la::read_and_clear_device_flag(static_cast<cudaStream_t>(stream), &flag) != 0)

@@ -137,6 +137,11 @@ inline BwdLayout bwd_layout(int B, int H, int nb, int P) {
     return w;
 }
 
+// Depthwise 3D convolution (Mix-FFN), kernel shapes 1x3x3 and 3x1x1; returns
+// -2 for any other shape.
+int launch_dwconv(int is_bf16, const void *x, void *y, const float *w, const float *bias, int B, int T, int Hg,
+                  int Wg, int C, int kt, int kh, int kw, cudaStream_t s);
+
 // Device flag raised by a bounded wait that gave up; read-and-clear.
 int read_and_clear_device_flag(cudaStream_t s, unsigned *flag_out);
 

@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.la_block_forward_e4m3.argtypes = [vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ctypes.POINTER(la_state), ip,
                                             fp, vp, sz, vp]
         L.la_block_forward_e4m3.restype = ip
+        L.la_dwconv3d.argtypes = [vp, vp, ip, ip, ip, ip, ip, ip, ip, ip, ip, vp, vp, vp]
+        L.la_dwconv3d.restype = ip
         L.la_backward_workspace_size.argtypes = [ip, ip, ip, ip, ip]
         L.la_backward_workspace_size.restype = sz
         L.la_full_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip,
@@ -135,6 +137,26 @@ def la_full_forward_e4m3(q, k, v, sq, sk, sv, out, B, N, H, d, tokens_per_block,
 def la_block_forward_e4m3(q, k, v, sq, sk, sv, out, B, N_blk, H, d, st, commit, eps, ws, ws_bytes, stream) -> int:
     return int(lib().la_block_forward_e4m3(q, k, v, sq, sk, sv, out, B, N_blk, H, d, ctypes.byref(st), commit, eps,
                                            ws, ws_bytes, stream))
+
+
+def la_dwconv3d(x, y, dt, B, T, Hg, Wg, C, kt, kh, kw, weight, bias, stream) -> int:
+    return int(lib().la_dwconv3d(x, y, dt, B, T, Hg, Wg, C, kt, kh, kw, weight, bias, stream))
+
+
+def dwconv3d(x, weight, bias=None, out=None, stream=None):
+    """Mix-FFN depthwise convolution: x [B, T, Hg, Wg, C] (bf16 or fp32 CUDA),
+    weight [C, kt, kh, kw] fp32 CUDA ((1,3,3) or (3,1,1)), bias [C] or None."""
+    if not x.is_cuda or not x.is_contiguous() or x.dim() != 5:
+        raise ValueError("x must be a contiguous CUDA tensor [B, T, Hg, Wg, C]")
+    if weight.dtype != torch.float32 or not weight.is_cuda or weight.dim() != 4 or not weight.is_contiguous():
+        raise ValueError("weight must be a contiguous fp32 CUDA tensor [C, kt, kh, kw]")
+    B, T, Hg, Wg, C = x.shape
+    out = torch.empty_like(x) if out is None else out
+    rc = la_dwconv3d(x.data_ptr(), out.data_ptr(), _dtype_code(x), B, T, Hg, Wg, C, *weight.shape[1:],
+                     weight.data_ptr(), None if bias is None else bias.data_ptr(), _stream_ptr(stream))
+    if rc != LA_OK:
+        raise LAError(rc, "la_dwconv3d")
+    return out
 
 
 def la_backward_workspace_size(B, N, H, d, tokens_per_block) -> int:

@@ -205,6 +205,24 @@ LA_API la_status la_block_forward_e4m3(const void *q, const void *k, const void 
                                        size_t ws_bytes, void *stream);
 
 /*
+ * Depthwise 3D convolution of the Spatial-Temporal Mix-FFN, the step after
+ * attention in a block ("Nvidia, MIT ve diğerleri video yapay zeka devrimini
+ * başlattı", section "Verimli doğrusal DiT": the MLP alternates a 1x3x3
+ * spatial and a 3x1x1 temporal convolution).  Reading: depthwise (one filter
+ * per channel), zero padding of one at the edges of the call's frames, rows
+ * and columns (a temporal tap never reaches another call's frames):
+ *   y[b,t,h,w,c] = bias[c] + sum_{i,j,l} weight[c][i][j][l] x[b, t+i-pt, h+j-ph, w+l-pw, c]
+ * x, y: DEVICE tensors [B][T][Hg][Wg][C] of type dt (channels last: the token
+ * layout of q, k, v), 16-byte aligned, caller-owned, not overlapping.
+ * weight: DEVICE fp32 [C][kt][kh][kw]; bias: DEVICE fp32 [C] or NULL.
+ * (kt, kh, kw) must be (1, 3, 3) or (3, 1, 1) and C a multiple of 8, else
+ * LA_EUNSUPPORTED; other argument errors LA_EINVAL.  fp32 accumulation.
+ */
+LA_API la_status la_dwconv3d(const void *x, void *y, la_dtype dt, int B, int T, int Hg, int Wg, int C,
+                             int kt, int kh, int kw, const float *weight, const float *bias,
+                             void *stream);
+
+/*
  * For callers that cannot allocate device memory at all.  Some code that
  * calls this library runs inside a host framework that owns every device
  * allocation and gives a plug-in no allocator and no way to size or keep a

@@ -179,3 +179,19 @@ def test_e4m3_quantiser_round_trip():
     assert bool(((back - x).abs() <= 2.0 ** -4 * x.abs() + 1e-30)[big].all())
     # amax scaling: the largest magnitude lands on the largest code, 448
     assert float(codes.view(torch.float8_e4m3fn).to(torch.float32).abs().max()) == 448.0
+
+
+def test_dwconv_validation(la):
+    def call(**kw):
+        a = dict(x=FAKE, y=FAKE, dt=la.LA_BF16, B=1, T=3, Hg=4, Wg=5, C=64, kt=1, kh=3, kw=3, w=FAKE, b=None)
+        a.update(kw)
+        return la.la_dwconv3d(a["x"], a["y"], a["dt"], a["B"], a["T"], a["Hg"], a["Wg"], a["C"], a["kt"], a["kh"],
+                              a["kw"], a["w"], a["b"], None)
+    assert call(x=None) == la.LA_EINVAL
+    assert call(w=None) == la.LA_EINVAL
+    assert call(y=FAKE + 2) == la.LA_EINVAL
+    assert call(T=0) == la.LA_EINVAL
+    assert call(dt=5) == la.LA_EINVAL
+    assert call(C=12) == la.LA_EUNSUPPORTED
+    assert call(kt=3, kh=3, kw=3) == la.LA_EUNSUPPORTED
+    assert call(kt=1, kh=1, kw=1) == la.LA_EUNSUPPORTED
