@@ -64,6 +64,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "backward"],
                     help="backward: la_full_backward over the workload's whole sequence (dq, dk, dv)")
+    ap.add_argument("--op", default="attention", choices=["attention", "dwconv"],
+                    help="dwconv: the Mix-FFN depthwise convolutions (1x3x3 then 3x1x1) on the workload's "
+                         "latent grid, DWCONV_C channels")
     ap.add_argument("--input", default="native", choices=["native", "e4m3"],
                     help="e4m3: q, k, v as FP8 E4M3 codes with per-tensor scales (la_*_forward_e4m3), bf16 out")
     ap.add_argument("--blocks", type=int, default=None,
@@ -255,6 +258,108 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- Mix-FFN convolutions
+
+DWCONV_C = 5120   # MLP channels: 2.5 x the 2048-wide attention (the pages give no width)
+
+
+def run_dwconv(args, w, world, rank, dist, dev, la):
+    """One step = the two depthwise convolutions of the Spatial-Temporal
+    Mix-FFN on one latent video: y1 = conv_1x3x3(x), y2 = conv_3x1x1(y1), bf16
+    activations, fp32 weights, over the workload's frames (one call's frames
+    for a streaming workload).  L2 flushed before every step.  Algorithmic
+    bytes: each convolution reads and writes its activation once."""
+    T = w.frames                  # one call's frames
+    B, Hg, Wg, C = w.B, w.Hg, w.Wg, DWCONV_C
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + 31)
+    x = torch.randn((B, T, Hg, Wg, C), generator=g, device=dev).to(torch.bfloat16)
+    w1 = (torch.randn((C, 1, 3, 3), generator=g, device=dev) / 3).contiguous()
+    w2 = (torch.randn((C, 3, 1, 1), generator=g, device=dev) / 2).contiguous()
+    b1 = torch.randn(C, generator=g, device=dev)
+    b2 = torch.randn(C, generator=g, device=dev)
+    y1, y2 = torch.empty_like(x), torch.empty_like(x)
+    flush_w = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    acc = torch.empty(1, dtype=torch.float32, device=dev)
+
+    def flush(v):
+        flush_w.fill_(v)
+        torch.sum(flush_r, dim=0, out=acc)
+
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+
+    def step(record=False):
+        if record:
+            ev[0].record()
+        la.dwconv3d(x, w1, b1, out=y1)
+        if record:
+            ev[1].record()
+        la.dwconv3d(y1, w2, b2, out=y2)
+        if record:
+            ev[2].record()
+
+    for i in range(max(3, args.warmup)):
+        flush(float(i))
+        step()
+    torch.cuda.synchronize()
+    K = args.steps or 200
+    K = ranks.agree_steps(K, dist, dev)
+    sampler = ClockSampler()
+    if rank == 0:
+        sampler.start(dev)
+        time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_all, t1, t2 = 0.0, 0.0, 0.0
+    for i in range(K):
+        flush(float(i))
+        step(record=True)
+        ev[2].synchronize()
+        t_all += ev[0].elapsed_time(ev[2])
+        t1 += ev[0].elapsed_time(ev[1])
+        t2 += ev[1].elapsed_time(ev[2])
+    torch.cuda.synchronize()
+    clocks = sampler.stop(dev.index or 0) if rank == 0 else None
+    t_all, t1, t2 = ranks.max_over_ranks([t_all, t1, t2], dist, dev)
+    tokens = B * T * Hg * Wg
+    value = ranks.job_throughput(tokens, world, K, t_all)
+    peak, peak_kind = measured_peaks()
+    conv_bytes = tokens * C * 2 * 2                     # read + write, bf16
+    dom, dom_ms = ("dwconv_1x3x3", t1) if t1 >= t2 else ("dwconv_3x1x1", t2)
+    achieved = conv_bytes / (dom_ms / K / 1e3) / 1e9
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle as orc
+
+        orc.build()
+        nc = 64
+        xs = x[..., :nc].contiguous().cpu()
+        t0 = time.perf_counter()
+        orc.dwconv3d(xs, w1[:nc].double().cpu().numpy(), b1[:nc].double().cpu().numpy())
+        dt = time.perf_counter() - t0
+        cpu = {"value": tokens * nc / C / dt, "unit": "tokens/s", "cores": orc.get_threads(), "kind": "oracle",
+               "sample": f"the 1x3x3 convolution of the same grid on {nc} of {C} channels, fp64, scaled to {C}"}
+    if rank == 0:
+        line = {"metric": "Mix-FFN depthwise convolutions (1x3x3 then 3x1x1) tokens/s", "value": value,
+                "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": max(3, args.warmup),
+                "ms_per_step": t_all / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16 activations, fp32 weights and accumulation", "data": "synthetic",
+                "config": {"workload": f"{w.name} latent grid", "B": B, "T": T, "Hg": Hg, "Wg": Wg, "C": C,
+                           "l2": "flushed before every step (256 MiB write then 256 MiB read)"},
+                "achieved_hbm_gbs": 2 * conv_bytes / (t_all / K / 1e3) / 1e9,
+                "hbm_frac_of_" + peak_kind: 2 * conv_bytes / (t_all / K / 1e3) / 1e9 / peak,
+                "stage_ms_per_step": {"dwconv_1x3x3": t1 / K, "dwconv_3x1x1": t2 / K},
+                "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                             "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None},
+                "cpu_baseline": cpu, "e2e": None, "gpu_launches": 2 * K, "path": "dwconv", "clocks": clocks}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 # ---------------------------------------------------------------- our arm
 
 def main():
@@ -290,6 +395,8 @@ def main():
     else:
         w = ranks.rank_workload(base, rank)
     dev = torch.device("cuda", local_rank)
+    if args.op == "dwconv":
+        return run_dwconv(args, w, world, rank, dist, dev, la)
     if args.blocks is not None:
         if w.mode != "stream" or not 1 <= args.blocks <= w.n_blocks:
             raise SystemExit("--blocks needs a streaming workload and 1 <= N <= its block count")
