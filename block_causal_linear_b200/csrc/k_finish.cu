@@ -38,7 +38,7 @@ constexpr int kPerBH = kKVZ + kZeroRows * kD;   // numbers + zero-padding entrie
 __global__ void __launch_bounds__(kFinThreads)
 finish_kernel(const float *__restrict__ partials, float *__restrict__ seff,
               unsigned char *__restrict__ bop, float *__restrict__ S, float *__restrict__ Z,
-              Plan p, int write_bop) {
+              Plan p, int write_bop, long long part_bh, long long part_sp) {
     // let the apply be scheduled now (it prefetches its q tiles), then wait
     // for the reduce before reading its partials
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -65,11 +65,12 @@ finish_kernel(const float *__restrict__ partials, float *__restrict__ seff,
     const int nrow = e < kD * kD ? (e % kD) : kD;     // value column, or the Z column
     const int kcol = e < kD * kD ? (e / kD) : (e - kD * kD);
     for (int n = 0; n < p.nb; ++n) {
-        const float *src = partials + ((size_t)bh * p.nb + n) * p.P * kKVZ + e;
+        // split sp of (bh, n) at partials + (bh * nb + n) * part_bh + sp * part_sp
+        const float *src = partials + ((size_t)bh * p.nb + n) * part_bh + e;
         for (int s0 = 0; s0 < p.P; s0 += kBatch) {
             float v[kBatch];
 #pragma unroll
-            for (int j = 0; j < kBatch; ++j) v[j] = s0 + j < p.P ? __ldg(src + (size_t)(s0 + j) * kKVZ) : 0.f;
+            for (int j = 0; j < kBatch; ++j) v[j] = s0 + j < p.P ? __ldg(src + (size_t)(s0 + j) * part_sp) : 0.f;
 #pragma unroll
             for (int j = 0; j < kBatch; ++j)
                 if (s0 + j < p.P) run += v[j];
@@ -91,8 +92,9 @@ finish_kernel(const float *__restrict__ partials, float *__restrict__ seff,
 
 }  // namespace
 
-int launch_finish(const float *partials, float *seff, void *bop, float *S, float *Z, const Plan &p,
-                  int write_bop, cudaStream_t s) {
+namespace {
+int launch_finish_strided(const float *partials, float *seff, void *bop, float *S, float *Z, const Plan &p,
+                          int write_bop, long long part_bh, long long part_sp, cudaStream_t s) {
     const long long threads = (long long)p.B * p.H * kPerBH;
     const long long grid = (threads + kFinThreads - 1) / kFinThreads;
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
@@ -108,9 +110,23 @@ int launch_finish(const float *partials, float *seff, void *bop, float *S, float
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, finish_kernel, partials, seff, static_cast<unsigned char *>(bop), S, Z, p,
-                              write_bop) == cudaSuccess
+                              write_bop, part_bh, part_sp) == cudaSuccess
                ? 1
                : -1;
+}
+}  // namespace
+
+int launch_finish(const float *partials, float *seff, void *bop, float *S, float *Z, const Plan &p,
+                  int write_bop, cudaStream_t s) {
+    return launch_finish_strided(partials, seff, bop, S, Z, p, write_bop, (long long)p.P * kKVZ, kKVZ, s);
+}
+
+int launch_finish_ranks(const float *gathered, int R, float *seff, void *bop, float *S, float *Z, const Plan &p,
+                        int write_bop, cudaStream_t s) {
+    if (p.nb != 1 || R < 1) return -1;
+    Plan q = p;
+    q.P = R;   // the ranks' partial sums play the splits, in rank order
+    return launch_finish_strided(gathered, seff, bop, S, Z, q, write_bop, kKVZ, (long long)p.B * p.H * kKVZ, s);
 }
 
 }  // namespace la

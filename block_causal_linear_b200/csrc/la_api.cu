@@ -357,6 +357,77 @@ la_status la_dwconv3d(const void *x, void *y, la_dtype dt, int B, int T, int Hg,
     return LA_OK;
 }
 
+size_t la_split_partial_bytes(int B, int H, int d) {
+    if (B <= 0 || H <= 0 || d != la::kD) return 0;
+    return size_t(B) * H * la::kKVZ * sizeof(float);
+}
+
+la_status la_block_reduce(const void *k, const void *v, la_dtype dt, int B, int N_slice, int H, int d,
+                          const la_rope *rope, float *partial, void *ws, size_t ws_bytes, void *stream) {
+    la_status e = common_checks(k, k, v, partial, dt, B, N_slice, H, d, 0.0f);
+    if (e != LA_OK) return e;
+    if ((e = check_rope(rope, d, false)) != LA_OK) return e;
+    const size_t need = la_workspace_size(B, N_slice, H, d, N_slice);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return LA_EWORKSPACE;
+    la::Plan p{};
+    p.B = B; p.N = N_slice; p.H = H; p.L = N_slice; p.nb = 1;
+    make_splits(p);
+    fill_rope(p, rope, rope ? rope->t_offset : 0);
+    const la::WsLayout w = la::ws_layout(B, H, 1, p.P);
+    char *base = static_cast<char *>(ws);
+    float *partials = reinterpret_cast<float *>(base + w.partials);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool tc = use_tc(dt, p);
+    int n = 0, r;
+    r = tc ? la::launch_reduce_tc(k, v, partials, p, s) : la::launch_reduce_ffma(dt == LA_BF16, k, v, partials, p, s);
+    if (r < 0) return LA_ECUDA;
+    n += r;
+    // the slice's split sums, in split order, straight into the caller's partial
+    if ((r = la::launch_finish(partials, partial, base + w.bop, nullptr, nullptr, p, 0, s)) < 0) return LA_ECUDA;
+    n += r;
+    g_last_launches = n;
+    g_last_path = tc ? "tc" : "ffma";
+    return LA_OK;
+}
+
+la_status la_block_apply(const void *q, void *out, la_dtype dt, int B, int N_slice, int H, int d,
+                         const float *gathered, int R, la_state *st, int commit, const la_rope *rope, float eps,
+                         void *ws, size_t ws_bytes, void *stream) {
+    la_status e = common_checks(q, q, q, out, dt, B, N_slice, H, d, eps);
+    if (e != LA_OK) return e;
+    if (!gathered || !aligned16(gathered) || R < 1 || R > 32) return LA_EINVAL;
+    if (!st || !st->S || !st->Z || st->B != B || st->H != H || st->d != d) return LA_EINVAL;
+    if ((e = check_rope(rope, d, true)) != LA_OK) return e;
+    const size_t need = la_workspace_size(B, N_slice, H, d, N_slice);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return LA_EWORKSPACE;
+    la::Plan p{};
+    p.B = B; p.N = N_slice; p.H = H; p.L = N_slice; p.nb = 1;
+    p.commit = commit != 0;
+    p.has_state = 1;
+    p.eps = eps;
+    make_splits(p);
+    fill_rope(p, rope, rope ? (rope->t_offset < 0 ? st->t_next : rope->t_offset) : 0);
+    const la::WsLayout w = la::ws_layout(B, H, 1, p.P);
+    char *base = static_cast<char *>(ws);
+    float *seff = reinterpret_cast<float *>(base + w.seff);
+    void *bop = base + w.bop;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool tc = use_tc(dt, p);
+    int n = 0, r;
+    if ((r = la::launch_finish_ranks(gathered, R, seff, bop, st->S, st->Z, p, tc ? 1 : 0, s)) < 0) return LA_ECUDA;
+    n += r;
+    r = tc ? la::launch_apply_tc(q, out, bop, seff, p, s) : la::launch_apply_ffma(dt == LA_BF16, q, out, seff, p, s);
+    if (r < 0) return LA_ECUDA;
+    n += r;
+    g_last_launches = n;
+    g_last_path = tc ? "tc" : "ffma";
+    if (commit) {
+        st->blocks_committed += 1;
+        if (rope) st->t_next += rope->T;
+    }
+    return LA_OK;
+}
+
 la_status la_device_status(void *stream) {
     unsigned flag = 0;
     if (la::read_and_clear_device_flag(static_cast<cudaStream_t>(stream), &flag) != 0)

@@ -100,6 +100,11 @@ int launch_apply_ffma(int is_bf16, const void *q, void *out, const float *seff,
 int launch_finish(const float *partials, float *seff, void *bop, float *S, float *Z,
                   const Plan &p, int write_bop, cudaStream_t s);
 
+// The same for a block whose tokens were split over R ranks: gathered is
+// [R][B][H][kKVZ], the ranks' partial sums in rank order; p.nb must be 1.
+int launch_finish_ranks(const float *gathered, int R, float *seff, void *bop, float *S, float *Z, const Plan &p,
+                        int write_bop, cudaStream_t s);
+
 // Tensor-core path (bf16, H % 4 == 0): tcgen05 MMAs, TMA tiles.
 // The three kernels of a call (reduce, finish above, apply) order themselves
 // by grid through programmatic dependent launch.

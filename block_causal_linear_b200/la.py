@@ -75,6 +75,13 @@ def lib() -> ctypes.CDLL:
         L.la_block_forward_e4m3.restype = ip
         L.la_dwconv3d.argtypes = [vp, vp, ip, ip, ip, ip, ip, ip, ip, ip, ip, vp, vp, vp]
         L.la_dwconv3d.restype = ip
+        L.la_split_partial_bytes.argtypes = [ip, ip, ip]
+        L.la_split_partial_bytes.restype = sz
+        L.la_block_reduce.argtypes = [vp, vp, ip, ip, ip, ip, ip, ctypes.POINTER(la_rope), vp, vp, sz, vp]
+        L.la_block_reduce.restype = ip
+        L.la_block_apply.argtypes = [vp, vp, ip, ip, ip, ip, ip, vp, ip, ctypes.POINTER(la_state), ip,
+                                     ctypes.POINTER(la_rope), fp, vp, sz, vp]
+        L.la_block_apply.restype = ip
         L.la_backward_workspace_size.argtypes = [ip, ip, ip, ip, ip]
         L.la_backward_workspace_size.restype = sz
         L.la_full_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip,
@@ -156,6 +163,54 @@ def dwconv3d(x, weight, bias=None, out=None, stream=None):
                      weight.data_ptr(), None if bias is None else bias.data_ptr(), _stream_ptr(stream))
     if rc != LA_OK:
         raise LAError(rc, "la_dwconv3d")
+    return out
+
+
+def la_split_partial_bytes(B, H, d) -> int:
+    return int(lib().la_split_partial_bytes(B, H, d))
+
+
+def la_block_reduce(k, v, dt, B, N, H, d, rope, partial, ws, ws_bytes, stream) -> int:
+    return int(lib().la_block_reduce(k, v, dt, B, N, H, d, ctypes.byref(rope) if rope is not None else None,
+                                     partial, ws, ws_bytes, stream))
+
+
+def la_block_apply(q, out, dt, B, N, H, d, gathered, R, st, commit, rope, eps, ws, ws_bytes, stream) -> int:
+    return int(lib().la_block_apply(q, out, dt, B, N, H, d, gathered, R, ctypes.byref(st), commit,
+                                    ctypes.byref(rope) if rope is not None else None, eps, ws, ws_bytes, stream))
+
+
+def block_reduce(k, v, rope=None, ws=None, partial=None, stream=None):
+    """This rank's [KV | z] partial sums of a token slice: fp32 [B, H, 1056]."""
+    _check_qkv(k, k, v)
+    B, N, H, d = k.shape
+    if ws is None:
+        ws = alloc_workspace(B, N, H, d, N, device=k.device)
+    if partial is None:
+        partial = torch.empty((B, H, d * d + d), dtype=torch.float32, device=k.device)
+    rc = la_block_reduce(k.data_ptr(), v.data_ptr(), _dtype_code(k), B, N, H, d, rope, partial.data_ptr(),
+                         ws.data_ptr(), ws.numel() * ws.element_size(), _stream_ptr(stream))
+    if rc != LA_OK:
+        raise LAError(rc, "la_block_reduce")
+    return partial
+
+
+def block_apply(q, gathered, state: "State", commit=True, rope=None, eps=1e-6, ws=None, out=None, stream=None):
+    """out for this rank's token slice from the gathered partials [R, B, H, 1056]
+    (rank order) and the state; commits on every rank alike."""
+    _check_qkv(q, q, q)
+    B, N, H, d = q.shape
+    if gathered.dtype != torch.float32 or not gathered.is_contiguous() or gathered.dim() != 4:
+        raise ValueError("gathered must be a contiguous fp32 tensor [R, B, H, d*d + d]")
+    if ws is None:
+        ws = alloc_workspace(B, N, H, d, N, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    rc = la_block_apply(q.data_ptr(), out.data_ptr(), _dtype_code(q), B, N, H, d, gathered.data_ptr(),
+                        gathered.shape[0], state.c, int(bool(commit)), rope, float(eps), ws.data_ptr(),
+                        ws.numel() * ws.element_size(), _stream_ptr(stream))
+    if rc != LA_OK:
+        raise LAError(rc, "la_block_apply")
     return out
 
 

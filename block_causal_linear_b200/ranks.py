@@ -64,6 +64,38 @@ def agree_steps(steps: int, dist=None, device="cpu") -> int:
     return int(_reduce([float(steps)], dist, device, op)[0])
 
 
+def token_slice(N: int, world: int, rank: int, align: int = 1) -> Tuple[int, int]:
+    """Tokens [t0, t1) of rank `rank` when one block of N tokens is split over
+    `world` ranks: contiguous, in whole units of `align` tokens (a frame, for
+    RoPE), as even as possible."""
+    if world < 1 or not 0 <= rank < world or N < 0 or align < 1:
+        raise ValueError("need N >= 0, align >= 1 and 0 <= rank < world")
+    units = (N + align - 1) // align
+    base, extra = divmod(units, world)
+    u0 = rank * base + min(rank, extra)
+    u1 = u0 + base + (1 if rank < extra else 0)
+    return min(u0 * align, N), min(u1 * align, N)
+
+
+def token_split_block(q, k, v, reduce_fn, gather_fn, apply_fn):
+    """One block whose tokens are split over the ranks: this rank's q, k, v
+    slice -> its partial sums (reduce_fn) -> every rank's partials in rank
+    order (gather_fn, the one collective) -> this rank's outputs (apply_fn,
+    which adds the partials to the state in rank order and commits).  The
+    steps are passed in so that the exchange can run with any backend."""
+    partial = reduce_fn(k, v)
+    gathered = gather_fn(partial)
+    return apply_fn(q, gathered)
+
+
+def nccl_gather(partial, dist):
+    """All-gather of the partial sums, stacked in rank order: [R, *partial.shape]."""
+    world = dist.get_world_size()
+    out = partial.new_empty((world,) + tuple(partial.shape))
+    dist.all_gather_into_tensor(out, partial.contiguous())
+    return out
+
+
 def job_throughput(units_per_rank_step: int, world: int, steps: int, total_ms: float) -> float:
     """Whole-job units per second: every rank's units over the slowest rank's
     time."""

@@ -223,6 +223,38 @@ LA_API la_status la_dwconv3d(const void *x, void *y, la_dtype dt, int B, int T, 
                              void *stream);
 
 /*
+ * Token split of one block over R GPUs (one process per GPU), for blocks
+ * whose (batch, head) pairs are too few to fill the GPUs: rank r holds a
+ * contiguous slice of the block's tokens (q, k, v [B][N_slice][H][d]).  The
+ * block's KV_n and z_n are sums over its tokens ("Nvidia, MIT ve diğerleri
+ * video yapay zeka devrimini başlattı", section "Sabit Bellekli KV önbelleğe
+ * alma mekanizması"), so each rank reduces its slice, the ranks exchange the
+ * B*H*(d*d + d) fp32 partial sums (an all-gather, the caller's collective,
+ * e.g. NCCL), and each rank adds them to the state in rank order and applies
+ * its own queries:
+ *   la_block_reduce: partial[b][h] = [sum_{t in slice} psi(k_t)^T v_t | sum phi(k_t)]
+ *     (fp32 DEVICE buffer of la_split_partial_bytes(B, H, d) bytes, layout of
+ *     one [S | Z] per (b, h): 1024 + 32 floats);
+ *   la_block_apply: gathered = the R ranks' partials, [R][B][H][d*d + d] in
+ *     rank order (DEVICE, caller-owned); S_eff = S + partial_0 + ... +
+ *     partial_{R-1} (that order), out for this rank's tokens, and on commit
+ *     S <- S_eff on every rank alike (identical bits on all ranks).
+ * With RoPE every slice must start at a frame boundary, rope->t_offset being
+ * the frame of the slice's first token (la_block_apply: < 0 means the state's
+ * t_next, which on commit advances by rope->T, the block's frames).  ws as
+ * la_workspace_size(B, N_slice, H, d, N_slice).  R in [1, 32].  Errors as in
+ * la_block_forward.
+ */
+LA_API size_t la_split_partial_bytes(int B, int H, int d);
+LA_API la_status la_block_reduce(const void *k, const void *v, la_dtype dt, int B, int N_slice, int H,
+                                 int d, const la_rope *rope, float *partial, void *ws,
+                                 size_t ws_bytes, void *stream);
+LA_API la_status la_block_apply(const void *q, void *out, la_dtype dt, int B, int N_slice, int H, int d,
+                                const float *gathered, int R, la_state *st, int commit,
+                                const la_rope *rope, float eps, void *ws, size_t ws_bytes,
+                                void *stream);
+
+/*
  * For callers that cannot allocate device memory at all.  Some code that
  * calls this library runs inside a host framework that owns every device
  * allocation and gives a plug-in no allocator and no way to size or keep a

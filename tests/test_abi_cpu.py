@@ -195,3 +195,26 @@ def test_dwconv_validation(la):
     assert call(C=12) == la.LA_EUNSUPPORTED
     assert call(kt=3, kh=3, kw=3) == la.LA_EUNSUPPORTED
     assert call(kt=1, kh=1, kw=1) == la.LA_EUNSUPPORTED
+
+
+def test_token_split_validation(la):
+    assert la.la_split_partial_bytes(1, 4, 32) == 4 * 1056 * 4
+    assert la.la_split_partial_bytes(0, 4, 32) == 0
+    # reduce: null / misaligned partial, bad sizes, small workspace
+    assert la.la_block_reduce(FAKE, FAKE, la.LA_BF16, 1, 64, 4, 32, None, None, FAKE, 1 << 30, None) == la.LA_EINVAL
+    assert la.la_block_reduce(FAKE, FAKE, la.LA_BF16, 1, 64, 4, 32, None, FAKE + 4, FAKE, 1 << 30, None) == la.LA_EINVAL
+    assert la.la_block_reduce(FAKE, FAKE, la.LA_BF16, 1, 0, 4, 32, None, FAKE, FAKE, 1 << 30, None) == la.LA_EINVAL
+    assert la.la_block_reduce(FAKE, FAKE, la.LA_BF16, 1, 64, 4, 32, None, FAKE, FAKE, 8, None) == la.LA_EWORKSPACE
+    # apply: rank count, unbound state, gathered pointer
+    st = la.la_state()
+    assert la.la_block_apply(FAKE, FAKE, la.LA_BF16, 1, 64, 4, 32, FAKE, 2, st, 1, None, 1e-6, FAKE, 1 << 30,
+                             None) == la.LA_EINVAL
+    st.S, st.Z, st.B, st.H, st.d = FAKE, FAKE, 1, 4, 32
+    for R in (0, 33):
+        assert la.la_block_apply(FAKE, FAKE, la.LA_BF16, 1, 64, 4, 32, FAKE, R, st, 1, None, 1e-6, FAKE, 1 << 30,
+                                 None) == la.LA_EINVAL
+    assert la.la_block_apply(FAKE, FAKE, la.LA_BF16, 1, 64, 4, 32, None, 2, st, 1, None, 1e-6, FAKE, 1 << 30,
+                             None) == la.LA_EINVAL
+    assert la.la_block_apply(FAKE, FAKE, la.LA_BF16, 1, 64, 4, 32, FAKE, 2, st, 1, None, 1e-6, FAKE, 8,
+                             None) == la.LA_EWORKSPACE
+    assert st.blocks_committed == 0

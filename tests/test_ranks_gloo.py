@@ -128,3 +128,95 @@ def test_head_slice_partitions():
     assert ranks.head_slice(64, 8, 3) == (24, 32)
     with pytest.raises(ValueError):
         ranks.head_slice(64, 2, 2)
+
+
+def _split_worker(rank, world, port, errfile):
+    """Token split of one block over `world` gloo ranks with oracle steps:
+    reduce the slice, all-gather the partial sums in rank order, add them to
+    the state in that order, apply the slice's queries."""
+    try:
+        sys.path.insert(0, ROOT)
+        os.environ["MASTER_ADDR"] = "127.0.0.1"
+        os.environ["MASTER_PORT"] = str(port)
+        from datetime import timedelta
+
+        dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+        import oracle as orc
+        from block_causal_linear_b200 import ranks, synth
+
+        B, N, H, d = 1, 23, 3, 32
+        q, k, v = synth.random_qkv(B, N, H, d, seed=17)
+        prior = synth.random_qkv(B, 9, H, d, seed=18)
+        st = orc.State(B, H, d)
+        orc.block_forward(*prior, st, commit=True)
+        t0, t1 = ranks.token_slice(N, world, rank)
+
+        def reduce_fn(kk, vv):
+            KV, z = orc.block_kv(kk, vv)
+            return torch.from_numpy(np.concatenate([KV.reshape(B, H, d * d), z], -1))
+
+        def gather_fn(partial):
+            parts = [torch.empty_like(partial) for _ in range(world)]
+            dist.all_gather(parts, partial)
+            return torch.stack(parts)
+
+        def apply_fn(qq, gathered):
+            S, Z = st.S.copy(), st.Z.copy()
+            for r in range(world):                       # rank order
+                S += gathered[r, :, :, : d * d].numpy().reshape(B, H, d, d)
+                Z += gathered[r, :, :, d * d:].numpy()
+            st.S, st.Z = S, Z                            # commit
+            return orc.apply(qq, S, Z)
+
+        out = ranks.token_split_block(q[:, t0:t1].contiguous(), k[:, t0:t1].contiguous(),
+                                      v[:, t0:t1].contiguous(), reduce_fn, gather_fn, apply_fn)
+        got = [None] * world
+        dist.all_gather_object(got, (t0, out, st.S, st.Z))
+        if rank == 0:
+            ref_st = orc.State(B, H, d)
+            orc.block_forward(*prior, ref_st, commit=True)
+            ref = orc.block_forward(q, k, v, ref_st, commit=True)
+            got.sort(key=lambda x: x[0])
+            assert np.abs(np.concatenate([x[1] for x in got], 1) - ref).max() <= 1e-12 * np.abs(ref).max()
+            assert all(np.array_equal(x[2], got[0][2]) and np.array_equal(x[3], got[0][3]) for x in got)
+            assert np.abs(got[0][2] - ref_st.S).max() <= 1e-12 * np.abs(ref_st.S).max()
+        dist.barrier()
+        dist.destroy_process_group()
+    except BaseException as e:
+        import traceback
+
+        with open(errfile, "a") as f:
+            f.write(f"rank {rank}: {e!r}\n{traceback.format_exc()}\n")
+        raise
+
+
+def test_token_split_two_ranks_gloo(orc, tmp_path):
+    errfile = str(tmp_path / "errors.txt")
+    world = 2
+    ctx = mp.get_context("spawn")
+    port = _free_port()
+    procs = [ctx.Process(target=_split_worker, args=(r, world, port, errfile)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    alive = [p for p in procs if p.is_alive()]
+    for p in alive:
+        p.kill()
+        p.join()
+    err = open(errfile).read() if os.path.exists(errfile) else ""
+    assert not alive, "a rank did not finish"
+    assert all(p.exitcode == 0 for p in procs), err
+
+
+def test_token_slice_partitions():
+    sys.path.insert(0, ROOT)
+    from block_causal_linear_b200 import ranks
+
+    for N in (0, 1, 7, 100, 8190):
+        for world in (1, 2, 3, 8):
+            for align in (1, 15, 390):
+                sl = [ranks.token_slice(N, world, r, align) for r in range(world)]
+                assert sl[0][0] == 0 and sl[-1][1] == N
+                assert all(a[1] == b[0] for a, b in zip(sl, sl[1:]))
+                assert all(a[0] % align == 0 for a in sl if a[0] < N)
