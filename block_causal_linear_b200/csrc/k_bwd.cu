@@ -271,7 +271,10 @@ bwd_q_kernel(const T *__restrict__ q, const T *__restrict__ dout, const float *_
 // One thread per (b, h, number e of [dS | dZ]): suffix sums over blocks, last
 // block first, the P splits of a block in split order.
 __global__ void __launch_bounds__(kBThreads)
-bwd_finish_kernel(const float *__restrict__ bpart, float *__restrict__ G, Plan p) {
+bwd_finish_kernel(const float *__restrict__ bpart, float *__restrict__ G, unsigned char *__restrict__ gop, Plan p) {
+    // the key-side kernel may be scheduled now (it prefetches its k, v tiles);
+    // it waits for this grid before reading G
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const long long w = (long long)blockIdx.x * kBThreads + threadIdx.x;
     if (w >= (long long)p.B * p.H * kKVZ) return;
     const size_t bh = (size_t)(w / kKVZ);
@@ -281,6 +284,18 @@ bwd_finish_kernel(const float *__restrict__ bpart, float *__restrict__ G, Plan p
         const float *src = bpart + (bh * p.nb + n) * p.P * kKVZ + e;
         for (int s = 0; s < p.P; ++s) run += src[(size_t)s * kKVZ];
         G[(bh * p.nb + n) * kKVZ + e] = run;
+        if (gop && e < kD * kD) {
+            // bf16 hi + lo of G[a][c] as the B operands of the key side:
+            // G (row c, K a) and G^T (row a, K c)
+            const int a = e / kD, c = e % kD;
+            unsigned char *o = gop + (bh * p.nb + n) * 4 * (size_t)kGopBytes;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(run);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(run - __bfloat162float(hi));
+            *reinterpret_cast<__nv_bfloat16 *>(o + op_offset(c, a)) = hi;
+            *reinterpret_cast<__nv_bfloat16 *>(o + kGopBytes + op_offset(c, a)) = lo;
+            *reinterpret_cast<__nv_bfloat16 *>(o + 2 * kGopBytes + op_offset(a, c)) = hi;
+            *reinterpret_cast<__nv_bfloat16 *>(o + 3 * kGopBytes + op_offset(a, c)) = lo;
+        }
     }
 }
 
@@ -373,11 +388,11 @@ int launch_bwd_q(int is_bf16, const void *q, const void *dout, const float *seff
     return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }
 
-int launch_bwd_finish(const float *bpart, float *G, const Plan &p, cudaStream_t s) {
+int launch_bwd_finish(const float *bpart, float *G, void *gop, const Plan &p, cudaStream_t s) {
     const long long threads = (long long)p.B * p.H * kKVZ;
     const long long grid = (threads + kBThreads - 1) / kBThreads;
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
-    bwd_finish_kernel<<<(unsigned)grid, kBThreads, 0, s>>>(bpart, G, p);
+    bwd_finish_kernel<<<(unsigned)grid, kBThreads, 0, s>>>(bpart, G, static_cast<unsigned char *>(gop), p);
     return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }
 

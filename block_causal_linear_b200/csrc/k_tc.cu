@@ -53,35 +53,6 @@ constexpr int kWarpTma = 0;
 constexpr int kWarpMma = 1;
 constexpr int kWork = 128;      // threads of warps 2..5
 
-__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
-    const uint32_t a = smem_u32(p);
-    return p + ((1024u - (a & 1023u)) & 1023u);
-}
-
-__device__ __forceinline__ uint32_t relu2(uint32_t x) {
-    // two bf16 in one word: as signed 16-bit integers every negative bf16
-    // (sign bit set, including -0) is below 0, so a signed max with 0 is ReLU
-    return __vmaxs2(x, 0u);
-}
-
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-__device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
-    const __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<const uint32_t *>(&t);
-}
-
-// Drain at exit after an abort: wait (briefly, ignoring the abort word) for
-// anything still writing this CTA's shared memory or TMEM.
-__device__ __forceinline__ void final_wait(uint64_t *bar, uint32_t parity) {
-    const uint64_t t0 = global_timer_ns();
-    for (uint32_t i = 0; i < (1u << 24); ++i) {
-        if (mbar_try_wait(bar, parity)) return;
-        if ((i & 255u) == 0 && global_timer_ns() - t0 > 200000000ull) return;
-    }
-}
-
 // ---------------------------------------------------------------- RoPE table
 // (cos, sin) of every feature pair at every position a CTA can meet: pair p of
 // the frame axis at frames [f_lo, f_lo + nf) of the call, of the row axis at
@@ -938,28 +909,6 @@ bool make_map_u8(CUtensorMap *m, const void *base, int B, int N, int H, int box_
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Launch with programmatic stream serialization (the kernel may start while
-// the previous kernel of the stream drains; it orders itself with pdl_wait).
-template <typename... KArgs, typename... Args>
-bool launch_pdl(void (*kernel)(KArgs...), unsigned grid, int threads, int smem, cudaStream_t s,
-                Args &&...args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(threads);
-    cfg.dynamicSmemBytes = (size_t)smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess;
-}
-
-bool set_smem(const void *kernel, int bytes) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
-}
-
 bool smem_ready() {
     static std::once_flag once;
     static bool ok = false;
@@ -992,6 +941,10 @@ bool tc_available() {
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
     if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return false;
     return major == 10 && minor == 0 && encode_fn() != nullptr;
+}
+
+bool make_bf16_map(CUtensorMap *m, const void *base, int B, int N, int H, int box_rows) {
+    return make_map(m, base, B, N, H, box_rows);
 }
 
 bool tc_rope_fits(const Plan &p) {

@@ -269,6 +269,7 @@ la_status la_full_backward(const void *q, const void *k, const void *v, const vo
     float *seff = reinterpret_cast<float *>(base + w.fwd.seff);
     float *bpart = reinterpret_cast<float *>(base + w.bpart);
     float *G = reinterpret_cast<float *>(base + w.G);
+    void *gop = base + w.gop;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool tc = use_tc(dt, p);
     const int bf = dt == LA_BF16;
@@ -287,13 +288,15 @@ la_status la_full_backward(const void *q, const void *k, const void *v, const vo
     if ((r = la::launch_bwd_q(bf, q, dout, seff, dq, bpart, p, s)) < 0) return LA_ECUDA;
     n += r;
     if (!mark(2, s)) return LA_ECUDA;
-    if ((r = la::launch_bwd_finish(bpart, G, p, s)) < 0) return LA_ECUDA;
+    const bool ktc = bf && la::bwd_k_tc_available(p);
+    if ((r = la::launch_bwd_finish(bpart, G, ktc ? gop : nullptr, p, s)) < 0) return LA_ECUDA;
     n += r;
-    if ((r = la::launch_bwd_k(bf, k, v, G, dk, dv, p, s)) < 0) return LA_ECUDA;
+    r = ktc ? la::launch_bwd_k_tc(k, v, G, gop, dk, dv, p, s) : la::launch_bwd_k(bf, k, v, G, dk, dv, p, s);
+    if (r < 0) return LA_ECUDA;
     n += r;
     if (!mark(3, s)) return LA_ECUDA;
     g_last_launches = n;
-    g_last_path = tc ? "bwd(tc state)" : "bwd";
+    g_last_path = ktc ? "bwd(tc state, tc keys)" : (tc ? "bwd(tc state)" : "bwd");
     return LA_OK;
 }
 

@@ -6,7 +6,9 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <utility>
 
 namespace la {
 
@@ -121,7 +123,12 @@ bool tc_rope_fits(const Plan &p);
 // over blocks; dk and dv from k, v and those sums.
 int launch_bwd_q(int is_bf16, const void *q, const void *dout, const float *seff, void *dq, float *bpart,
                  const Plan &p, cudaStream_t s);
-int launch_bwd_finish(const float *bpart, float *G, const Plan &p, cudaStream_t s);
+int launch_bwd_finish(const float *bpart, float *G, void *gop, const Plan &p, cudaStream_t s);
+// Key side on the tensor cores (bf16, H % 4 == 0, no RoPE): dk, dv from k, v
+// and the packed G operands; Gz from G.
+bool bwd_k_tc_available(const Plan &p);
+int launch_bwd_k_tc(const void *k, const void *v, const float *G, const void *gop, void *dk, void *dv,
+                    const Plan &p, cudaStream_t s);
 int launch_bwd_k(int is_bf16, const void *k, const void *v, const float *G, void *dk, void *dv, const Plan &p,
                  cudaStream_t s);
 
@@ -129,8 +136,14 @@ int launch_bwd_k(int is_bf16, const void *k, const void *v, const float *G, void
 // ([B][H][nb][P][kKVZ]) and their suffix sums G ([B][H][nb][kKVZ]), fp32.
 struct BwdLayout {
     WsLayout fwd;
-    size_t bpart, G, total;
+    size_t bpart, G, gop, total;
 };
+
+// Packed bf16 operands of the key-side tensor-core backward, per (b, h,
+// block): G (rows = value column c, K = key feature a) and G^T (rows = a,
+// K = c), each as a hi and a lo part, 32 rows of the K-major core-matrix
+// layout of op_offset: 4 x 2048 bytes.
+constexpr int kGopBytes = 2048;
 
 inline BwdLayout bwd_layout(int B, int H, int nb, int P) {
     BwdLayout w;
@@ -138,7 +151,8 @@ inline BwdLayout bwd_layout(int B, int H, int nb, int P) {
     const size_t bhn = size_t(B) * H * nb;
     w.bpart = w.fwd.total;
     w.G = align256(w.bpart + bhn * P * kKVZ * sizeof(float));
-    w.total = align256(w.G + bhn * kKVZ * sizeof(float));
+    w.gop = align256(w.G + bhn * kKVZ * sizeof(float));
+    w.total = align256(w.gop + bhn * 4 * size_t(kGopBytes));
     return w;
 }
 
@@ -146,6 +160,32 @@ inline BwdLayout bwd_layout(int B, int H, int nb, int P) {
 // -2 for any other shape.
 int launch_dwconv(int is_bf16, const void *x, void *y, const float *w, const float *bias, int B, int T, int Hg,
                   int Wg, int C, int kt, int kh, int kw, cudaStream_t s);
+
+// Launch with programmatic stream serialization (the kernel may start while
+// the previous kernel of the stream drains; it orders itself with pdl_wait).
+template <typename... KArgs, typename... Args>
+bool launch_pdl(void (*kernel)(KArgs...), unsigned grid, int threads, int smem, cudaStream_t s,
+                Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess;
+}
+
+inline bool set_smem(const void *kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+// 3D TMA map of a [B][N][H*32] bf16 tensor: boxes of 64 features x box_rows
+// tokens, 128-byte swizzle.
+bool make_bf16_map(CUtensorMap *m, const void *base, int B, int N, int H, int box_rows);
 
 // Device flag raised by a bounded wait that gave up; read-and-clear.
 int read_and_clear_device_flag(cudaStream_t s, unsigned *flag_out);

@@ -5,6 +5,7 @@
 
 #include <cstdint>
 #include <cuda.h>
+#include <cuda_bf16.h>
 
 namespace la {
 namespace sm100 {
@@ -248,6 +249,37 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// ---------------------------------------------------------------- small shared pieces
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    const uint32_t a = smem_u32(p);
+    return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+__device__ __forceinline__ uint32_t relu2(uint32_t x) {
+    // two bf16 in one word: as signed 16-bit integers every negative bf16
+    // (sign bit set, including -0) is below 0, so a signed max with 0 is ReLU
+    return __vmaxs2(x, 0u);
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
+    const __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&t);
+}
+
+// Drain at exit after an abort: wait (briefly, ignoring the abort word) for
+// anything still writing this CTA's shared memory or TMEM.
+__device__ __forceinline__ void final_wait(uint64_t *bar, uint32_t parity) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 0; i < (1u << 24); ++i) {
+        if (mbar_try_wait(bar, parity)) return;
+        if ((i & 255u) == 0 && global_timer_ns() - t0 > 200000000ull) return;
+    }
 }
 
 }  // namespace sm100
