@@ -28,9 +28,11 @@ namespace la {
 
 using namespace sm100;
 
-extern __device__ unsigned int g_wait_flag;
-
 namespace {
+
+// Raised by a bounded wait of this file's kernel that gave up (0x100 | where);
+// read by la_device_status through read_and_clear_bwd_k_flag.
+__device__ unsigned int g_wait_flag = 0;
 
 constexpr int kKTThreads = 320;
 constexpr int kKTWarpTma = 0, kKTWarpMma = 1, kKTXform0 = 192, kKTWork = 128;
@@ -346,6 +348,13 @@ int launch_bwd_k_tc(const void *k, const void *v, const float *G, const void *go
                       static_cast<const uint8_t *>(gop), p)
                ? 1
                : -1;
+}
+
+int read_and_clear_bwd_k_flag(unsigned *flag_out) {
+    unsigned zero = 0;
+    if (cudaMemcpyFromSymbol(flag_out, g_wait_flag, sizeof(unsigned)) != cudaSuccess) return -1;
+    if (*flag_out && cudaMemcpyToSymbol(g_wait_flag, &zero, sizeof(unsigned)) != cudaSuccess) return -1;
+    return 0;
 }
 
 }  // namespace la

@@ -281,22 +281,31 @@ la_status la_full_backward(const void *q, const void *k, const void *v, const vo
     r = tc ? la::launch_reduce_tc(k, v, partials, p, s) : la::launch_reduce_ffma(bf, k, v, partials, p, s);
     if (r < 0) return LA_ECUDA;
     n += r;
-    if ((r = la::launch_finish(partials, seff, base + w.fwd.bop, nullptr, nullptr, p, tc ? 1 : 0, s)) < 0)
-        return LA_ECUDA;
+    // the query side on the tensor cores needs the packed [S|Z|0] and S^T operands
+    const bool qtc = bf && tc && la::bwd_q_tc_available(p);
+    void *stop = base + w.stop;
+    r = qtc ? la::launch_finish_with_st(partials, seff, base + w.fwd.bop, stop, p, s)
+            : la::launch_finish(partials, seff, base + w.fwd.bop, nullptr, nullptr, p, tc ? 1 : 0, s);
+    if (r < 0) return LA_ECUDA;
     n += r;
     if (!mark(1, s)) return LA_ECUDA;
-    if ((r = la::launch_bwd_q(bf, q, dout, seff, dq, bpart, p, s)) < 0) return LA_ECUDA;
+    // the query side takes its own split plan; the suffix sums below read its splits
+    la::Plan pq = p;
+    if (qtc) la::bwd_q_tc_plan(pq);
+    r = qtc ? la::launch_bwd_q_tc(q, dout, dq, seff, base + w.fwd.bop, stop, bpart, pq, s)
+            : la::launch_bwd_q(bf, q, dout, seff, dq, bpart, p, s);
+    if (r < 0) return LA_ECUDA;
     n += r;
     if (!mark(2, s)) return LA_ECUDA;
     const bool ktc = bf && la::bwd_k_tc_available(p);
-    if ((r = la::launch_bwd_finish(bpart, G, ktc ? gop : nullptr, p, s)) < 0) return LA_ECUDA;
+    if ((r = la::launch_bwd_finish(bpart, G, ktc ? gop : nullptr, qtc ? pq : p, s)) < 0) return LA_ECUDA;
     n += r;
     r = ktc ? la::launch_bwd_k_tc(k, v, G, gop, dk, dv, p, s) : la::launch_bwd_k(bf, k, v, G, dk, dv, p, s);
     if (r < 0) return LA_ECUDA;
     n += r;
     if (!mark(3, s)) return LA_ECUDA;
     g_last_launches = n;
-    g_last_path = ktc ? "bwd(tc state, tc keys)" : (tc ? "bwd(tc state)" : "bwd");
+    g_last_path = qtc && ktc ? "bwd_tc" : (ktc ? "bwd(tc state, tc keys)" : (tc ? "bwd(tc state)" : "bwd"));
     return LA_OK;
 }
 
@@ -432,10 +441,11 @@ la_status la_block_apply(const void *q, void *out, la_dtype dt, int B, int N_sli
 }
 
 la_status la_device_status(void *stream) {
-    unsigned flag = 0;
-    if (la::read_and_clear_device_flag(static_cast<cudaStream_t>(stream), &flag) != 0)
-        return LA_ECUDA;
-    return flag ? LA_ETIMEOUT : LA_OK;
+    unsigned flag = 0, fk = 0, fq = 0;
+    // (synchronises the stream first)
+    if (la::read_and_clear_device_flag(static_cast<cudaStream_t>(stream), &flag) != 0) return LA_ECUDA;
+    if (la::read_and_clear_bwd_k_flag(&fk) != 0 || la::read_and_clear_bwd_q_flag(&fq) != 0) return LA_ECUDA;
+    return (flag | fk | fq) ? LA_ETIMEOUT : LA_OK;
 }
 
 const char *la_status_string(la_status s) {
