@@ -20,7 +20,9 @@
 // are bf16 hi + lo (~16 bits).  All sums have one fixed order.
 //
 // Warp roles: 0 TMA, 1 TMEM + MMAs, 2..5 ReLU on the q tile and its sign
-// bytes, 6..9 epilogue (M1 -> g, c; M2 -> dq; at the end dS, dZ).  Every
+// bytes, then the dq epilogue one tile behind (M2 -> dq), 6..9 the g epilogue
+// (M1 -> g, c; at the end dS, dZ).  c passes between the two epilogues in a
+// double buffer.  Every
 // wait is bounded; a wait that gives up raises the device flag.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -53,8 +55,8 @@ constexpr int kQTOpsOff = kQTCOff + kQTCBytes;       // per head: [S|Z|0] hi, lo
 constexpr int kQTOpsHead = 2 * kOpBytes + 2 * kStOpBytes;
 constexpr int kQTStgOff = kQTOpsOff + 4 * kQTOpsHead;   // 4 epilogue warps x 2 boxes [32 rows][64 bf16]
 constexpr int kQTZOff = kQTStgOff + 4 * 2 * 4096;       // Z_n of the 4 heads
-constexpr int kQTCValOff = kQTZOff + 4 * kD * 4;        // c per row and head, fp32
-constexpr int kQTMaskOff = kQTCValOff + 128 * 4 * 4;    // sign bytes [2 buffers][128 rows][16 logical chunks]
+constexpr int kQTCValOff = kQTZOff + 4 * kD * 4;        // c per row and head, fp32, [2 buffers][128][4]
+constexpr int kQTMaskOff = kQTCValOff + 2 * 128 * 4 * 4;  // sign bytes [2 buffers][128 rows][16 logical chunks]
 constexpr int kQTBarOff = kQTMaskOff + 2 * 128 * 16;
 constexpr int kQTNumBars = 3 * kQTStages + 14;
 constexpr int kQTSmem = kQTBarOff + kQTNumBars * 8 + 16 + 1024;
@@ -99,9 +101,9 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint64_t *ops_full = accS_full + 1;
     uint64_t *dep_ready = ops_full + 1;
     uint64_t *drain = dep_ready + 1;
-    uint64_t *mask_ready = drain + 1;          // [2] a tile's sign bytes are written
-    uint64_t *mask_free = mask_ready + 2;      // [2] ... and read by the dq epilogue
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mask_free + 2);
+    uint64_t *c_ready = drain + 1;             // [2] a tile's c values are written (g epilogue)
+    uint64_t *c_free = c_ready + 2;            // [2] ... and read by the dq epilogue
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c_free + 2);
     volatile int *abort_word = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int G4 = p.H / 4;
@@ -140,8 +142,8 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(dep_ready, 1);
         mbar_init(drain, 1);
         for (int a = 0; a < 2; ++a) {
-            mbar_init(&mask_ready[a], kQTWork);
-            mbar_init(&mask_free[a], kQTWork);
+            mbar_init(&c_ready[a], kQTWork);
+            mbar_init(&c_free[a], kQTWork);
         }
         *abort_word = 0;
         fence_barrier_init();
@@ -271,18 +273,24 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mma_commit(accS_full);
         }
     } else if (warp < 6) {
-        // ------------------------------------------------ ReLU on the q tile, sign bytes, rows past the split
+        // ------------------------------------------------ warps 2..5: ReLU on the q tile and its sign
+        // bytes for tile i + 1, then the dq epilogue of tile i (one tile behind warps 6..9)
         const int tt = threadIdx.x - kQTXform0;
-        bool ok = true;
-        for (int i = 0; i < ntiles; ++i) {
+        const int qd = warp & 3;                // TMEM lane quarter
+        const int r = 32 * qd + lane;           // token row of this thread in a tile
+        const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
+        uint8_t *sb = stg + qd * 2 * 4096;      // this warp's two staging boxes
+        bool ok = mbar_wait(dep_ready, 0, abort_word, &g_wait_flag, 69);
+        {   // Z_n of the 4 heads
+            const size_t bh = (size_t)b * p.H + 4 * g + (tt >> 5);
+            zs[tt] = ok ? __ldcg(seff + (bh * p.nb + n) * kKVZ + kD * kD + (tt & 31)) : 0.f;
+        }
+        auto transform = [&](int i) {
             const int s = i % kQTStages;
             const uint32_t ph = (uint32_t)(i / kQTStages) & 1u;
             if (ok && !mbar_wait(&full[s], ph, abort_word, &g_wait_flag, 67)) ok = false;
-            // sign-byte buffer i % 2 is free once the epilogue of tile i-2 has formed dq
-            const int mb = i & 1;
-            const uint32_t mph = (uint32_t)(i >> 1) & 1u;
-            if (ok && !mbar_wait(&mask_free[mb], mph ^ 1u, abort_word, &g_wait_flag, 68)) ok = false;
             uint8_t *qt = smem + s * kQTTile;
+            uint8_t *mk = mask8 + (i & 1) * 2048;
             const long long row0 = t0 + 128LL * i;
             if (ok) {
 #pragma unroll 4
@@ -300,29 +308,95 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         bits |= (((w[m] & 0x8000u) == 0u && (w[m] & 0x7FFFu) != 0u) ? 1u : 0u) << (2 * m);
                         bits |= (((w[m] & 0x80000000u) == 0u && (w[m] & 0x7FFF0000u) != 0u) ? 1u : 0u) << (2 * m + 1);
                     }
-                    mask8[mb * 2048 + row * 16 + bx * 8 + L] = (uint8_t)bits;
+                    mk[row * 16 + bx * 8 + L] = (uint8_t)bits;
                     *ptr = make_uint4(relu2(x.x), relu2(x.y), relu2(x.z), relu2(x.w));
                 }
             }
             fence_proxy_async_smem();
             mbar_arrive(&xform_done[s]);
-            mbar_arrive(&mask_ready[mb]);
+        };
+        transform(0);
+        for (int i = 0; i < ntiles; ++i) {
+            // sign-byte buffer (i + 1) % 2 was last read by this group's dq epilogue of tile i - 1
+            // (and every sign byte of tile i, and Z_n, is written)
+            named_bar_sync(5, kQTWork);
+            if (i + 1 < ntiles) transform(i + 1);
+            // ---- E2: dq = mask (S g + c Z) from M2
+            const int cb = i & 1;
+            const uint32_t cph = (uint32_t)(i >> 1) & 1u;
+            bool got2 = ok && mbar_wait(acc2_full, (uint32_t)i & 1u, abort_word, &g_wait_flag, 72);
+            got2 = got2 && mbar_wait(&c_ready[cb], cph, abort_word, &g_wait_flag, 73);
+            got2 = __all_sync(0xffffffffu, got2);
+            if (!got2) ok = false;
+            const long long row0 = t0 + 128LL * i;
+            const long long t = row0 + r;
+            const bool valid = t < t1;
+            const long long wrow0 = row0 + 32 * qd;
+            const bool boxed = wrow0 + 32 <= t1 || t1 == p.N;   // TMA clips rows >= N
+            if (boxed) {
+                if (lane == 0) bulk_wait_read<0>();   // the previous tile's stores have read sb
+                __syncwarp();
+            }
+#pragma unroll 1
+            for (int hh = 0; hh < 4; ++hh) {
+                float pre[32];
+                uint32_t m = 0;
+                float cr = 0.f;
+                if (got2) {
+                    tc_fence_after();
+                    tmem_ld32(tmem + lane_off + kQTAcc2 + hh * kD, pre);
+                    tmem_wait_ld();
+                    m = *reinterpret_cast<const uint32_t *>(mask8 + (i & 1) * 2048 + r * 16 + (hh >> 1) * 8 +
+                                                            (hh & 1) * 4);
+                    cr = cval[cb * 512 + r * 4 + hh];
+                }
+                if (hh == 3) {   // the M2 result and the c values are read
+                    tc_fence_before();
+                    mbar_arrive(acc2_empty);
+                    mbar_arrive(&c_free[cb]);
+                }
+                if (!got2) continue;
+#pragma unroll
+                for (int a = 0; a < 32; ++a) pre[a] = (m >> a) & 1u ? fmaf(cr, zs[hh * kD + a], pre[a]) : 0.f;
+                if (boxed) {
+                    uint8_t *bx = sb + (hh >> 1) * 4096 + lane * 128;
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const int pc = (4 * (hh & 1) + c4) ^ (lane & 7);   // 128-byte swizzle
+                        *reinterpret_cast<uint4 *>(bx + pc * 16) =
+                            make_uint4(pack_bf2(pre[8 * c4], pre[8 * c4 + 1]), pack_bf2(pre[8 * c4 + 2], pre[8 * c4 + 3]),
+                                       pack_bf2(pre[8 * c4 + 4], pre[8 * c4 + 5]),
+                                       pack_bf2(pre[8 * c4 + 6], pre[8 * c4 + 7]));
+                    }
+                } else if (valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(dq + (((size_t)b * p.N + t) * p.H + 4 * g + hh) * kD);
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4)
+                        dst[c4] = make_uint4(pack_bf2(pre[8 * c4], pre[8 * c4 + 1]), pack_bf2(pre[8 * c4 + 2], pre[8 * c4 + 3]),
+                                             pack_bf2(pre[8 * c4 + 4], pre[8 * c4 + 5]),
+                                             pack_bf2(pre[8 * c4 + 6], pre[8 * c4 + 7]));
+                }
+            }
+            if (boxed) {
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && ok) {
+                    tma_store_3d(&tm_dq, sb, g * 128, (int)wrow0, b);
+                    tma_store_3d(&tm_dq, sb + 4096, g * 128 + 64, (int)wrow0, b);
+                    bulk_commit();
+                }
+            }
         }
+        if (lane == 0) bulk_wait_all();
     } else {
-        // ------------------------------------------------ epilogue warps 6..9
-        const int ew = threadIdx.x - kQTEpi0;   // 0..127
+        // ------------------------------------------------ epilogue warps 6..9: g and c from M1
         const int qd = warp & 3;                // TMEM lane quarter
         const int r = 32 * qd + lane;           // token row of this thread in a tile
         const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
-        uint8_t *sb = stg + qd * 2 * 4096;      // this warp's two staging boxes
-        bool ok = mbar_wait(dep_ready, 0, abort_word, &g_wait_flag, 69);
-        {   // Z_n of the 4 heads
-            const size_t bh = (size_t)b * p.H + 4 * g + (ew >> 5);
-            zs[ew] = ok ? __ldcg(seff + (bh * p.nb + n) * kKVZ + kD * kD + (ew & 31)) : 0.f;
-        }
-        named_bar_sync(4, kQTWork);
+        bool ok = true;
         for (int i = 0; i < ntiles; ++i) {
             const uint32_t tph = (uint32_t)i & 1u;
+            const int cb = i & 1;
             const long long row0 = t0 + 128LL * i;
             const long long t = row0 + r;
             const bool valid = t < t1;
@@ -334,9 +408,9 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int j = 0; j < 16; ++j) dv[j] = valid ? __ldg(src + j) : make_uint4(0u, 0u, 0u, 0u);
             }
-            // ---- E1: g = dout / den, c = -(dout . num) / den^2 from M1
             bool got = ok && mbar_wait(acc1_full, tph, abort_word, &g_wait_flag, 70);
             got = got && mbar_wait(g_free, tph ^ 1u, abort_word, &g_wait_flag, 71);   // M2..M4 of tile i-1 are done
+            got = got && mbar_wait(&c_free[cb], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_word, &g_wait_flag, 75);
             got = __all_sync(0xffffffffu, got);
             if (!got) ok = false;
 #pragma unroll
@@ -392,69 +466,11 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 *reinterpret_cast<__nv_bfloat16 *>(cop + c_offset(2 * hh, r)) = ch;
                 *reinterpret_cast<__nv_bfloat16 *>(cop + c_offset(2 * hh + 1, r)) =
                     __float2bfloat16_rn(cr - __bfloat162float(ch));
-                cval[r * 4 + hh] = cr;
+                cval[cb * 512 + r * 4 + hh] = cr;
             }
             fence_proxy_async_smem();   // g and c are read by the tensor cores
             mbar_arrive(g_ready);
-            // ---- E2: dq = mask (S g + c Z) from M2
-            bool got2 = ok && mbar_wait(acc2_full, tph, abort_word, &g_wait_flag, 72);
-            const int mb = i & 1;
-            got2 = got2 && mbar_wait(&mask_ready[mb], (uint32_t)(i >> 1) & 1u, abort_word, &g_wait_flag, 73);
-            got2 = __all_sync(0xffffffffu, got2);
-            if (!got2) ok = false;
-            const long long wrow0 = row0 + 32 * qd;
-            const bool boxed = wrow0 + 32 <= t1 || t1 == p.N;   // TMA clips rows >= N
-            if (boxed) {
-                if (lane == 0) bulk_wait_read<0>();   // the previous tile's stores have read sb
-                __syncwarp();
-            }
-#pragma unroll 1
-            for (int hh = 0; hh < 4; ++hh) {
-                float pre[32];
-                uint32_t m = 0;
-                if (got2) {
-                    tc_fence_after();
-                    tmem_ld32(tmem + lane_off + kQTAcc2 + hh * kD, pre);
-                    tmem_wait_ld();
-                    m = *reinterpret_cast<const uint32_t *>(mask8 + mb * 2048 + r * 16 + (hh >> 1) * 8 + (hh & 1) * 4);
-                }
-                if (hh == 3) {   // the M2 result and the sign bytes are read
-                    tc_fence_before();
-                    mbar_arrive(acc2_empty);
-                    mbar_arrive(&mask_free[mb]);
-                }
-                if (!got2) continue;
-                const float cr = cval[r * 4 + hh];
-#pragma unroll
-                for (int a = 0; a < 32; ++a) pre[a] = (m >> a) & 1u ? fmaf(cr, zs[hh * kD + a], pre[a]) : 0.f;
-                if (boxed) {
-                    uint8_t *bx = sb + (hh >> 1) * 4096 + lane * 128;
-#pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        const int pc = (4 * (hh & 1) + c4) ^ (lane & 7);   // 128-byte swizzle
-                        *reinterpret_cast<uint4 *>(bx + pc * 16) =
-                            make_uint4(pack_bf2(pre[8 * c4], pre[8 * c4 + 1]), pack_bf2(pre[8 * c4 + 2], pre[8 * c4 + 3]),
-                                       pack_bf2(pre[8 * c4 + 4], pre[8 * c4 + 5]),
-                                       pack_bf2(pre[8 * c4 + 6], pre[8 * c4 + 7]));
-                    }
-                } else if (valid) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(dq + (((size_t)b * p.N + t) * p.H + 4 * g + hh) * kD);
-#pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4)
-                        dst[c4] = make_uint4(pack_bf2(pre[8 * c4], pre[8 * c4 + 1]), pack_bf2(pre[8 * c4 + 2], pre[8 * c4 + 3]),
-                                             pack_bf2(pre[8 * c4 + 4], pre[8 * c4 + 5]),
-                                             pack_bf2(pre[8 * c4 + 6], pre[8 * c4 + 7]));
-                }
-            }
-            if (boxed) {
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0 && ok) {
-                    tma_store_3d(&tm_dq, sb, g * 128, (int)wrow0, b);
-                    tma_store_3d(&tm_dq, sb + 4096, g * 128 + 64, (int)wrow0, b);
-                    bulk_commit();
-                }
-            }
+            mbar_arrive(&c_ready[cb]);
         }
         // ---- the split's [dS | dZ]: lane quarter qd = the key features of head 4g + qd
         bool gs = ok && mbar_wait(accS_full, 0, abort_word, &g_wait_flag, 74);
