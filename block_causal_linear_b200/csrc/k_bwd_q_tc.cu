@@ -16,14 +16,21 @@
 // ReLU in place).  g is written by the epilogue as a bf16 hi and a lo tile in
 // the same layout: the K-major A operand of M2 and the MN-major B operand of
 // M3.  c goes into a [16 rows][128 tokens] operand (rows 2h, 2h + 1: c hi and
-// c lo of head h) so that M4 gives dZ of head h as the sum of two columns.  The state operands S, S^T
-// are bf16 hi + lo (~16 bits).  All sums have one fixed order.
+// c lo of head h) so that M4 gives dZ of head h as the sum of two columns.
+// The state operands S, S^T are bf16 hi + lo (~16 bits).  All sums have one
+// fixed order.
+//
+// The work of a tile is cut at its two 64-feature boxes (2 heads each): M1
+// of box 0, the g epilogue of box 0 and the MMAs that read it (M2 of its heads,
+// M3 against its g columns) run while the epilogue works on box 1, and M1 of
+// the next tile is issued between them, so that the tensor cores and the
+// epilogue overlap.
 //
 // Warp roles: 0 TMA, 1 TMEM + MMAs, 2..5 ReLU on the q tile and its sign
-// bytes, then the dq epilogue one tile behind (M2 -> dq), 6..9 the g epilogue
-// (M1 -> g, c; at the end dS, dZ).  c passes between the two epilogues in a
-// double buffer.  Every
-// wait is bounded; a wait that gives up raises the device flag.
+// bytes, 6..9 the g epilogue (M1 -> g, c; at the end dS, dZ), 10..13 the dq
+// epilogue (M2 -> dq, staged for TMA stores).  c passes between the two
+// epilogues in a double buffer, the sign bytes in a ring of four.  Every wait
+// is bounded; a wait that gives up raises the device flag.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -43,25 +50,28 @@ namespace {
 // read by la_device_status through read_and_clear_bwd_q_flag.
 __device__ unsigned int g_wait_flag = 0;
 
-constexpr int kQTThreads = 320;
-constexpr int kQTWarpTma = 0, kQTWarpMma = 1, kQTXform0 = 64, kQTEpi0 = 192, kQTWork = 128;
+constexpr int kQTThreads = 448;
+constexpr int kQTWarpTma = 0, kQTWarpMma = 1, kQTWork = 128;
+constexpr int kQTXform0 = 64, kQTDq0 = 320;   // first thread of the transform and the dq warps
 constexpr int kQTBox = 128 * 128;                    // [128 rows][64 bf16] = 16 KiB: 2 heads
 constexpr int kQTTile = 2 * kQTBox;                  // 4 heads
 constexpr int kQTStages = 2;
+constexpr int kQTMaskBufs = 4;
 constexpr int kQTGOff = kQTStages * kQTTile;         // g hi tile, then g lo tile
 constexpr int kQTCOff = kQTGOff + 2 * kQTTile;       // c operand: [16 rows][128 tokens] bf16
 constexpr int kQTCBytes = 2 * 2048;
 constexpr int kQTOpsOff = kQTCOff + kQTCBytes;       // per head: [S|Z|0] hi, lo; S^T hi, lo
 constexpr int kQTOpsHead = 2 * kOpBytes + 2 * kStOpBytes;
-constexpr int kQTStgOff = kQTOpsOff + 4 * kQTOpsHead;   // 4 epilogue warps x 2 boxes [32 rows][64 bf16]
-constexpr int kQTZOff = kQTStgOff + 4 * 2 * 4096;       // Z_n of the 4 heads
-constexpr int kQTCValOff = kQTZOff + 4 * kD * 4;        // c per row and head, fp32, [2 buffers][128][4]
-constexpr int kQTMaskOff = kQTCValOff + 2 * 128 * 4 * 4;  // sign bytes [2 buffers][128 rows][16 logical chunks]
-constexpr int kQTBarOff = kQTMaskOff + 2 * 128 * 16;
-constexpr int kQTNumBars = 3 * kQTStages + 14;
+constexpr int kQTStgOff = kQTOpsOff + 4 * kQTOpsHead;   // 4 dq warps x 2 boxes [32 rows][64 bf16]
+constexpr int kQTAcOff = kQTStgOff + 4 * 2 * 4096;      // c as the K = 16 extension of M2's A: [128 tokens][16]
+constexpr int kQTBcOff = kQTAcOff + 4096;               // Z_n as that extension of B, per head [32][16]
+constexpr int kQTMaskOff = kQTBcOff + 4096;             // sign bytes [4 buffers][128 rows][16 logical chunks]
+constexpr int kQTBarOff = kQTMaskOff + kQTMaskBufs * 128 * 16;
+constexpr int kQTNumBars = 3 * kQTStages + 2 * kQTMaskBufs + 14;
 constexpr int kQTSmem = kQTBarOff + kQTNumBars * 8 + 16 + 1024;
+static_assert(kQTSmem <= 232448, "shared memory of the query-side kernel");
 // TMEM columns
-constexpr uint32_t kQTAcc1 = 0;      // num | den per head: 4 x 48
+constexpr uint32_t kQTAcc1 = 0;      // num | den per head: 4 x 48 (box b: heads 2b, 2b + 1)
 constexpr uint32_t kQTAcc2 = 192;    // S g per head: 4 x 32
 constexpr uint32_t kQTAccS = 320;    // dS: 128 x 128 (4 diagonal 32 x 32 blocks used)
 constexpr uint32_t kQTAccZ = 448;    // dZ: columns 0 (c hi) and 1 (c lo) of 16
@@ -74,36 +84,48 @@ __device__ __forceinline__ int c_offset(int n, int t) {
     return (n >> 3) * 2048 + (t >> 3) * 128 + (n & 7) * 16 + (t & 7) * 2;
 }
 
+// The product c_t Z_n of dq is folded into M2 as one more K = 16 step per
+// head.  Its A operand holds, per token t, the columns 3h, 3h + 1, 3h + 2 =
+// c hi, c lo, c hi of head h (12..15 zero); the B operand of head h holds,
+// per key feature f, the rows 3h, 3h + 1, 3h + 2 = Z hi, Z hi, Z lo (others
+// zero), so the step adds (c hi + c lo) Z hi + c hi Z lo.  Both are K-major
+// without swizzle: core matrices of 8 rows x 8 columns, the two column halves
+// 128 B apart, 8-row groups 256 B apart.
+__device__ __forceinline__ int ac_offset(int t, int k) {
+    return (t >> 3) * 256 + (k >> 3) * 128 + (t & 7) * 16 + (k & 7) * 2;
+}
+
 __global__ void __launch_bounds__(kQTThreads, 1)
 bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_dq,
-                const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ dout,
-                __nv_bfloat16 *__restrict__ dq, const float *__restrict__ seff, const uint8_t *__restrict__ bop,
-                const uint8_t *__restrict__ stop, float *__restrict__ bpart, const Plan p) {
+                const __nv_bfloat16 *__restrict__ dout, __nv_bfloat16 *__restrict__ dq,
+                const float *__restrict__ seff, const uint8_t *__restrict__ bop, const uint8_t *__restrict__ stop,
+                float *__restrict__ bpart, const Plan p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     uint8_t *gtile = smem + kQTGOff;
     uint8_t *cop = smem + kQTCOff;
     uint8_t *ops = smem + kQTOpsOff;
     uint8_t *stg = smem + kQTStgOff;
-    float *zs = reinterpret_cast<float *>(smem + kQTZOff);
-    float *cval = reinterpret_cast<float *>(smem + kQTCValOff);
+    uint8_t *acx = smem + kQTAcOff;
+    uint8_t *bcx = smem + kQTBcOff;
     uint8_t *mask8 = smem + kQTMaskOff;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + kQTBarOff);
     uint64_t *xform_done = full + kQTStages;
     uint64_t *empty = xform_done + kQTStages;
-    uint64_t *acc1_full = empty + kQTStages;
-    uint64_t *acc1_empty = acc1_full + 1;
-    uint64_t *g_ready = acc1_empty + 1;
-    uint64_t *g_free = g_ready + 1;
+    uint64_t *mask_ready = empty + kQTStages;      // [4] a tile's sign bytes are written
+    uint64_t *mask_free = mask_ready + kQTMaskBufs; // [4] ... and read by the dq epilogue
+    uint64_t *acc1_full = mask_free + kQTMaskBufs;  // [2] per box: M1 done
+    uint64_t *acc1_empty = acc1_full + 2;           // [2] per box: the g epilogue has read it
+    uint64_t *g_ready = acc1_empty + 2;             // [2] per box: g (and at box 1, c) written
+    uint64_t *g_free = g_ready + 2;                 // M2, M3, M4 of a tile are done with g and c
     uint64_t *acc2_full = g_free + 1;
     uint64_t *acc2_empty = acc2_full + 1;
-    uint64_t *accS_full = acc2_empty + 1;
+    uint64_t *bc_ready = acc2_empty + 1;            // the Z_n operand is written
+    uint64_t *accS_full = bc_ready + 1;
     uint64_t *ops_full = accS_full + 1;
     uint64_t *dep_ready = ops_full + 1;
     uint64_t *drain = dep_ready + 1;
-    uint64_t *c_ready = drain + 1;             // [2] a tile's c values are written (g epilogue)
-    uint64_t *c_free = c_ready + 2;            // [2] ... and read by the dq epilogue
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c_free + 2);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_word = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int G4 = p.H / 4;
@@ -131,26 +153,31 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&xform_done[s], kQTWork);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(acc1_full, 1);
-        mbar_init(acc1_empty, kQTWork);
-        mbar_init(g_ready, kQTWork);
+        for (int a = 0; a < kQTMaskBufs; ++a) {
+            mbar_init(&mask_ready[a], kQTWork);
+            mbar_init(&mask_free[a], kQTWork);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&acc1_full[a], 1);
+            mbar_init(&acc1_empty[a], kQTWork);
+            mbar_init(&g_ready[a], kQTWork);
+        }
         mbar_init(g_free, 1);
         mbar_init(acc2_full, 1);
         mbar_init(acc2_empty, kQTWork);
+        mbar_init(bc_ready, kQTWork);
         mbar_init(accS_full, 1);
         mbar_init(ops_full, 1);
         mbar_init(dep_ready, 1);
         mbar_init(drain, 1);
-        for (int a = 0; a < 2; ++a) {
-            mbar_init(&c_ready[a], kQTWork);
-            mbar_init(&c_free[a], kQTWork);
-        }
         *abort_word = 0;
         fence_barrier_init();
     }
-    // rows 8..15 of the c operand stay zero
+    // rows 8..15 of the c operand and columns 12..15 of its M2 form stay zero
     for (int i = threadIdx.x; i < kQTCBytes / 16; i += kQTThreads)
         reinterpret_cast<uint4 *>(cop)[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = threadIdx.x; i < 4096 / 16; i += kQTThreads)
+        reinterpret_cast<uint4 *>(acx)[i] = make_uint4(0u, 0u, 0u, 0u);
     if (warp == kQTWarpMma) {
         tmem_alloc(tmem_slot, kQTTmemCols);
         tmem_relinquish();
@@ -207,54 +234,79 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t id_m3 = idesc_bf16(128, 128, 1, 1);         // phi(Q)^T x g
             const uint32_t id_m4 = idesc_bf16(128, 16, 1, 0);          // phi(Q)^T x [c hi | c lo | 0]
             const uint32_t oaddr = smem_u32(ops), gaddr = smem_u32(gtile), caddr = smem_u32(cop);
-            bool ok = mbar_wait(ops_full, 0, abort_word, &g_wait_flag, 62);
-            for (int i = 0; i < ntiles && ok; ++i) {
-                const int s = i % kQTStages;
-                const uint32_t ph = (uint32_t)(i / kQTStages) & 1u;
-                const uint32_t tph = (uint32_t)i & 1u;
-                if (!mbar_wait(&xform_done[s], ph, abort_word, &g_wait_flag, 63)) break;
-                if (!mbar_wait(acc1_empty, tph ^ 1u, abort_word, &g_wait_flag, 64)) break;
-                tc_fence_after();
-                const uint32_t qaddr = smem_u32(smem + s * kQTTile);
-                // M1: per head, num | den from the packed [S | Z | 0] (hi, lo)
+            const uint32_t acaddr = smem_u32(acx), bcaddr = smem_u32(bcx);
+            // M1 of box bx (heads 2bx, 2bx + 1) of tile i: num | den from the packed [S | Z | 0] (hi, lo)
+            auto m1 = [&](int i, int bx) {
+                const uint32_t qaddr = smem_u32(smem + (i % kQTStages) * kQTTile) + bx * kQTBox;
 #pragma unroll
-                for (int hh = 0; hh < 4; ++hh) {
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int hh = 2 * bx + h2;
 #pragma unroll
                     for (int part = 0; part < 2; ++part)
 #pragma unroll
                         for (int kk = 0; kk < 2; ++kk) {
-                            const uint64_t da = smem_desc(qaddr + (hh >> 1) * kQTBox + (hh & 1) * 64 + kk * 32, 16,
-                                                          1024, kLayoutSw128);
+                            const uint64_t da = smem_desc(qaddr + h2 * 64 + kk * 32, 16, 1024, kLayoutSw128);
                             const uint64_t db = smem_desc(oaddr + hh * kQTOpsHead + part * kOpBytes + kk * 256, 128,
                                                           512, kLayoutNone);
                             mma_bf16(tmem + kQTAcc1 + hh * kOpRows, da, db, id_m1, (part | kk) ? 1u : 0u);
                         }
                 }
-                mma_commit(acc1_full);
-                // M2..M4 once the epilogue has turned M1 into g and c
-                if (!mbar_wait(g_ready, tph, abort_word, &g_wait_flag, 65)) break;
-                if (!mbar_wait(acc2_empty, tph ^ 1u, abort_word, &g_wait_flag, 66)) break;
-                tc_fence_after();
-                // M2: per head, g S^T as g_hi.ST_hi + g_hi.ST_lo + g_lo.ST_hi
+                mma_commit(&acc1_full[bx]);
+            };
+            // M2 of box bx: per head, g S^T as g_hi.ST_hi + g_hi.ST_lo + g_lo.ST_hi
+            auto m2 = [&](int bx) {
 #pragma unroll
-                for (int hh = 0; hh < 4; ++hh) {
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int hh = 2 * bx + h2;
 #pragma unroll
                     for (int prod = 0; prod < 3; ++prod) {
                         const int gp = prod == 2 ? 1 : 0, sp2 = prod == 1 ? 1 : 0;
 #pragma unroll
                         for (int kk = 0; kk < 2; ++kk) {
-                            const uint64_t da = smem_desc(gaddr + gp * kQTTile + (hh >> 1) * kQTBox + (hh & 1) * 64 +
-                                                              kk * 32,
-                                                          16, 1024, kLayoutSw128);
+                            const uint64_t da = smem_desc(gaddr + gp * kQTTile + bx * kQTBox + h2 * 64 + kk * 32, 16,
+                                                          1024, kLayoutSw128);
                             const uint64_t db = smem_desc(oaddr + hh * kQTOpsHead + 2 * kOpBytes + sp2 * kStOpBytes +
                                                               kk * 256,
                                                           128, 512, kLayoutNone);
                             mma_bf16(tmem + kQTAcc2 + hh * kD, da, db, id_m2, (prod | kk) ? 1u : 0u);
                         }
                     }
+                    // + c_t Z_n: the K = 16 extension
+                    mma_bf16(tmem + kQTAcc2 + hh * kD, smem_desc(acaddr, 128, 256, kLayoutNone),
+                             smem_desc(bcaddr + hh * 1024, 128, 256, kLayoutNone), id_m2, 1u);
                 }
+            };
+            bool ok = mbar_wait(ops_full, 0, abort_word, &g_wait_flag, 62);
+            ok = ok && mbar_wait(&xform_done[0], 0, abort_word, &g_wait_flag, 63);
+            if (ok) {
+                tc_fence_after();
+                m1(0, 0);
+                m1(0, 1);
+            }
+            ok = ok && mbar_wait(bc_ready, 0, abort_word, &g_wait_flag, 78);
+            // per tile i: M2 of box 0, M1 of box 0 of tile i + 1, M2 of box 1 with M3 and
+            // M4, M1 of box 1 of tile i + 1
+            for (int i = 0; i < ntiles && ok; ++i) {
+                const int s = i % kQTStages;
+                const uint32_t tph = (uint32_t)i & 1u;
+                const bool next = i + 1 < ntiles;
+                if (!mbar_wait(&g_ready[0], tph, abort_word, &g_wait_flag, 65)) break;
+                if (!mbar_wait(acc2_empty, tph ^ 1u, abort_word, &g_wait_flag, 66)) break;
+                tc_fence_after();
+                m2(0);
+                if (next) {
+                    const uint32_t ph1 = (uint32_t)((i + 1) / kQTStages) & 1u;
+                    if (!mbar_wait(&xform_done[(i + 1) % kQTStages], ph1, abort_word, &g_wait_flag, 63)) break;
+                    if (!mbar_wait(&acc1_empty[0], tph, abort_word, &g_wait_flag, 64)) break;
+                    tc_fence_after();
+                    m1(i + 1, 0);
+                }
+                if (!mbar_wait(&g_ready[1], tph, abort_word, &g_wait_flag, 67)) break;
+                tc_fence_after();
+                m2(1);
                 // M3, M4: over the tile's 128 tokens, 16 per MMA; MN-major, the two
                 // 64-feature boxes kQTBox apart (LBO), 8-token groups 1024 B apart (SBO)
+                const uint32_t qaddr = smem_u32(smem + s * kQTTile);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint64_t da = smem_desc(qaddr + kk * 2048, kQTBox, 1024, kLayoutSw128);
@@ -269,28 +321,26 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mma_commit(&empty[s]);   // the q tile is read
                 mma_commit(g_free);      // g and c are read
                 mma_commit(acc2_full);
+                if (next) {
+                    if (!mbar_wait(&acc1_empty[1], tph, abort_word, &g_wait_flag, 68)) break;
+                    tc_fence_after();
+                    m1(i + 1, 1);
+                }
             }
             mma_commit(accS_full);
         }
     } else if (warp < 6) {
-        // ------------------------------------------------ warps 2..5: ReLU on the q tile and its sign
-        // bytes for tile i + 1, then the dq epilogue of tile i (one tile behind warps 6..9)
+        // ------------------------------------------------ warps 2..5: ReLU on the q tile, its sign bytes
         const int tt = threadIdx.x - kQTXform0;
-        const int qd = warp & 3;                // TMEM lane quarter
-        const int r = 32 * qd + lane;           // token row of this thread in a tile
-        const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
-        uint8_t *sb = stg + qd * 2 * 4096;      // this warp's two staging boxes
-        bool ok = mbar_wait(dep_ready, 0, abort_word, &g_wait_flag, 69);
-        {   // Z_n of the 4 heads
-            const size_t bh = (size_t)b * p.H + 4 * g + (tt >> 5);
-            zs[tt] = ok ? __ldcg(seff + (bh * p.nb + n) * kKVZ + kD * kD + (tt & 31)) : 0.f;
-        }
-        auto transform = [&](int i) {
+        bool ok = true;
+        for (int i = 0; i < ntiles; ++i) {
             const int s = i % kQTStages;
-            const uint32_t ph = (uint32_t)(i / kQTStages) & 1u;
-            if (ok && !mbar_wait(&full[s], ph, abort_word, &g_wait_flag, 67)) ok = false;
+            const int mb = i % kQTMaskBufs;
+            if (ok && !mbar_wait(&full[s], (uint32_t)(i / kQTStages) & 1u, abort_word, &g_wait_flag, 76)) ok = false;
+            if (ok && !mbar_wait(&mask_free[mb], ((uint32_t)(i / kQTMaskBufs) & 1u) ^ 1u, abort_word, &g_wait_flag, 77))
+                ok = false;
             uint8_t *qt = smem + s * kQTTile;
-            uint8_t *mk = mask8 + (i & 1) * 2048;
+            uint8_t *mk = mask8 + mb * 2048;
             const long long row0 = t0 + 128LL * i;
             if (ok) {
 #pragma unroll 4
@@ -314,25 +364,166 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             fence_proxy_async_smem();
             mbar_arrive(&xform_done[s]);
+            mbar_arrive(&mask_ready[mb]);
+        }
+    } else if (warp < 10) {
+        // ------------------------------------------------ warps 6..9: the g epilogue, from M1
+        const int qd = warp & 3;                // TMEM lane quarter
+        const int r = 32 * qd + lane;           // token row of this thread in a tile
+        const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
+        // dout of (tile i, box bx) for this thread's row: 2 heads, 128 bytes; zero past the split
+        auto load_dout = [&](int i, int bx, uint4 (&v)[8]) {
+            const long long t = t0 + 128LL * i + r;
+            if (t < t1) {
+                const uint4 *src =
+                    reinterpret_cast<const uint4 *>(dout + (((size_t)b * p.N + t) * p.H + 4 * g + 2 * bx) * kD);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = __ldg(src + j);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = make_uint4(0u, 0u, 0u, 0u);
+            }
         };
-        transform(0);
+        bool ok = true;
+        uint4 cur[8];
+        load_dout(0, 0, cur);
         for (int i = 0; i < ntiles; ++i) {
-            // sign-byte buffer (i + 1) % 2 was last read by this group's dq epilogue of tile i - 1
-            // (and every sign byte of tile i, and Z_n, is written)
-            named_bar_sync(5, kQTWork);
-            if (i + 1 < ntiles) transform(i + 1);
-            // ---- E2: dq = mask (S g + c Z) from M2
-            const int cb = i & 1;
-            const uint32_t cph = (uint32_t)(i >> 1) & 1u;
-            bool got2 = ok && mbar_wait(acc2_full, (uint32_t)i & 1u, abort_word, &g_wait_flag, 72);
-            got2 = got2 && mbar_wait(&c_ready[cb], cph, abort_word, &g_wait_flag, 73);
-            got2 = __all_sync(0xffffffffu, got2);
-            if (!got2) ok = false;
+            const uint32_t tph = (uint32_t)i & 1u;
+            const long long t = t0 + 128LL * i + r;
+            const bool valid = t < t1;
+            if (t + 128 < t1) {   // the next tile's dout row into L2
+                const uint8_t *nx =
+                    reinterpret_cast<const uint8_t *>(dout + (((size_t)b * p.N + t + 128) * p.H + 4 * g) * kD);
+                prefetch_l2(nx);
+                prefetch_l2(nx + 128);
+            }
+#pragma unroll 1
+            for (int bx = 0; bx < 2; ++bx) {
+                uint4 nxt[8];   // one box ahead; zeros past the last tile
+                if (bx == 0) load_dout(i, 1, nxt);
+                else load_dout(i + 1, 0, nxt);
+                bool got = ok && mbar_wait(&acc1_full[bx], tph, abort_word, &g_wait_flag, 70);
+                if (bx == 0)   // M2, M3, M4 of tile i - 1 are done with g and c
+                    got = got && mbar_wait(g_free, tph ^ 1u, abort_word, &g_wait_flag, 71);
+                got = __all_sync(0xffffffffu, got);
+                if (!got) ok = false;
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int hh = 2 * bx + h2;
+                    float num[32], den = 0.f;
+                    if (got) {
+                        tc_fence_after();
+                        tmem_ld32(tmem + lane_off + kQTAcc1 + hh * kOpRows, num);
+                        den = tmem_ld1(tmem + lane_off + kQTAcc1 + hh * kOpRows + kD);
+                        tmem_wait_ld();
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) num[c] = 0.f;
+                    }
+                    if (h2 == 1) {   // both heads of the box are read
+                        tc_fence_before();
+                        mbar_arrive(&acc1_empty[bx]);
+                    }
+                    const float inv = 1.0f / (den + p.eps);
+                    float dn = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint4 u = cur[4 * h2 + j];
+                        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            dn = fmaf(bf_lo(w[m]), num[8 * j + 2 * m], dn);
+                            dn = fmaf(bf_hi(w[m]), num[8 * j + 2 * m + 1], dn);
+                        }
+                    }
+                    const bool live = valid && got;
+                    const float cr = live ? -dn * inv * inv : 0.f;
+                    const float sc = live ? inv : 0.f;
+                    // g hi and lo into the two g tiles: box bx, logical chunks 4 h2 + c4
+                    uint8_t *gbox = gtile + bx * kQTBox + r * 128;
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const uint4 u = cur[4 * h2 + c4];
+                        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+                        uint32_t hi[4], lo[4];
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            const float g0 = bf_lo(w[m]) * sc;
+                            const float g1 = bf_hi(w[m]) * sc;
+                            const __nv_bfloat162 hv = __floats2bfloat162_rn(g0, g1);
+                            hi[m] = *reinterpret_cast<const uint32_t *>(&hv);
+                            lo[m] = pack_bf2(g0 - __low2float(hv), g1 - __high2float(hv));
+                        }
+                        const int pc = (4 * h2 + c4) ^ (r & 7);
+                        *reinterpret_cast<uint4 *>(gbox + pc * 16) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                        *reinterpret_cast<uint4 *>(gbox + kQTTile + pc * 16) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    }
+                    const __nv_bfloat16 ch = __float2bfloat16_rn(cr);
+                    *reinterpret_cast<__nv_bfloat16 *>(cop + c_offset(2 * hh, r)) = ch;
+                    *reinterpret_cast<__nv_bfloat16 *>(cop + c_offset(2 * hh + 1, r)) =
+                        __float2bfloat16_rn(cr - __bfloat162float(ch));
+                    *reinterpret_cast<__nv_bfloat16 *>(acx + ac_offset(r, 3 * hh)) = ch;
+                    *reinterpret_cast<__nv_bfloat16 *>(acx + ac_offset(r, 3 * hh + 1)) =
+                        __float2bfloat16_rn(cr - __bfloat162float(ch));
+                    *reinterpret_cast<__nv_bfloat16 *>(acx + ac_offset(r, 3 * hh + 2)) = ch;
+                }
+                fence_proxy_async_smem();   // the box's g (and its c) is read by the tensor cores
+                mbar_arrive(&g_ready[bx]);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) cur[j] = nxt[j];
+            }
+        }
+        // ---- the split's [dS | dZ]: lane quarter qd = the key features of head 4g + qd
+        bool gs = ok && mbar_wait(accS_full, 0, abort_word, &g_wait_flag, 74);
+        gs = __all_sync(0xffffffffu, gs);
+        if (gs) {
+            tc_fence_after();
+            float kv[32];
+            tmem_ld32(tmem + lane_off + kQTAccS + 32 * qd, kv);
+            const float z0 = tmem_ld1(tmem + lane_off + kQTAccZ + 2 * qd);
+            const float z1 = tmem_ld1(tmem + lane_off + kQTAccZ + 2 * qd + 1);
+            tmem_wait_ld();
+            float *dst = bpart + ((((size_t)b * p.H + 4 * g + qd) * p.nb + n) * p.P + sp) * kKVZ;
+            float4 *drow = reinterpret_cast<float4 *>(dst + lane * kD);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) drow[j] = make_float4(kv[4 * j], kv[4 * j + 1], kv[4 * j + 2], kv[4 * j + 3]);
+            dst[kD * kD + lane] = z0 + z1;
+        }
+    } else {
+        // ------------------------------------------------ warps 10..13: the dq epilogue, from M2
+        const int tt = threadIdx.x - kQTDq0;
+        const int qd = warp & 3;                // TMEM lane quarter
+        const int r = 32 * qd + lane;           // token row of this thread in a tile
+        const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
+        bool ok = mbar_wait(dep_ready, 0, abort_word, &g_wait_flag, 69);
+        {   // the Z_n operand of the folded c Z step: head tt / 32, key feature tt % 32
+            const int h = tt >> 5, f = tt & 31;
+            const size_t bh = (size_t)b * p.H + 4 * g + h;
+            const float z = ok ? __ldcg(seff + (bh * p.nb + n) * kKVZ + kD * kD + f) : 0.f;
+            const __nv_bfloat16 zh = __float2bfloat16_rn(z);
+            const __nv_bfloat16 zl = __float2bfloat16_rn(z - __bfloat162float(zh));
+            uint4 row[2];
+            __nv_bfloat16 *e = reinterpret_cast<__nv_bfloat16 *>(row);
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                e[k] = (k == 3 * h || k == 3 * h + 1) ? zh : (k == 3 * h + 2 ? zl : __float2bfloat16_rn(0.f));
+            *reinterpret_cast<uint4 *>(bcx + h * 1024 + ac_offset(f, 0)) = row[0];
+            *reinterpret_cast<uint4 *>(bcx + h * 1024 + ac_offset(f, 8)) = row[1];
+            fence_proxy_async_smem();
+            mbar_arrive(bc_ready);
+        }
+        for (int i = 0; i < ntiles; ++i) {
+            const int mb = i % kQTMaskBufs;
+            bool got = ok && mbar_wait(acc2_full, (uint32_t)i & 1u, abort_word, &g_wait_flag, 72);
+            got = got && mbar_wait(&mask_ready[mb], (uint32_t)(i / kQTMaskBufs) & 1u, abort_word, &g_wait_flag, 73);
+            got = __all_sync(0xffffffffu, got);
+            if (!got) ok = false;
             const long long row0 = t0 + 128LL * i;
             const long long t = row0 + r;
             const bool valid = t < t1;
             const long long wrow0 = row0 + 32 * qd;
             const bool boxed = wrow0 + 32 <= t1 || t1 == p.N;   // TMA clips rows >= N
+            uint8_t *sb = stg + qd * 2 * 4096;                 // this warp's two staging boxes
             if (boxed) {
                 if (lane == 0) bulk_wait_read<0>();   // the previous tile's stores have read sb
                 __syncwarp();
@@ -341,23 +532,20 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int hh = 0; hh < 4; ++hh) {
                 float pre[32];
                 uint32_t m = 0;
-                float cr = 0.f;
-                if (got2) {
+                if (got) {
                     tc_fence_after();
                     tmem_ld32(tmem + lane_off + kQTAcc2 + hh * kD, pre);
                     tmem_wait_ld();
-                    m = *reinterpret_cast<const uint32_t *>(mask8 + (i & 1) * 2048 + r * 16 + (hh >> 1) * 8 +
-                                                            (hh & 1) * 4);
-                    cr = cval[cb * 512 + r * 4 + hh];
+                    m = *reinterpret_cast<const uint32_t *>(mask8 + mb * 2048 + r * 16 + (hh >> 1) * 8 + (hh & 1) * 4);
                 }
-                if (hh == 3) {   // the M2 result and the c values are read
+                if (hh == 3) {   // the M2 result and the sign bytes are read
                     tc_fence_before();
                     mbar_arrive(acc2_empty);
-                    mbar_arrive(&c_free[cb]);
+                    mbar_arrive(&mask_free[mb]);
                 }
-                if (!got2) continue;
+                if (!got) continue;
 #pragma unroll
-                for (int a = 0; a < 32; ++a) pre[a] = (m >> a) & 1u ? fmaf(cr, zs[hh * kD + a], pre[a]) : 0.f;
+                for (int a = 0; a < 32; ++a) pre[a] = (m >> a) & 1u ? pre[a] : 0.f;
                 if (boxed) {
                     uint8_t *bx = sb + (hh >> 1) * 4096 + lane * 128;
 #pragma unroll
@@ -388,107 +576,6 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
         if (lane == 0) bulk_wait_all();
-    } else {
-        // ------------------------------------------------ epilogue warps 6..9: g and c from M1
-        const int qd = warp & 3;                // TMEM lane quarter
-        const int r = 32 * qd + lane;           // token row of this thread in a tile
-        const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
-        bool ok = true;
-        for (int i = 0; i < ntiles; ++i) {
-            const uint32_t tph = (uint32_t)i & 1u;
-            const int cb = i & 1;
-            const long long row0 = t0 + 128LL * i;
-            const long long t = row0 + r;
-            const bool valid = t < t1;
-            // dout of this token, 4 heads (256 bytes), loaded before the waits
-            uint4 dv[16];
-            {
-                const uint4 *src = reinterpret_cast<const uint4 *>(
-                    dout + (((size_t)b * p.N + (valid ? t : t0)) * p.H + 4 * g) * kD);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) dv[j] = valid ? __ldg(src + j) : make_uint4(0u, 0u, 0u, 0u);
-            }
-            bool got = ok && mbar_wait(acc1_full, tph, abort_word, &g_wait_flag, 70);
-            got = got && mbar_wait(g_free, tph ^ 1u, abort_word, &g_wait_flag, 71);   // M2..M4 of tile i-1 are done
-            got = got && mbar_wait(&c_free[cb], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_word, &g_wait_flag, 75);
-            got = __all_sync(0xffffffffu, got);
-            if (!got) ok = false;
-#pragma unroll
-            for (int hh = 0; hh < 4; ++hh) {
-                float num[32], den = 0.f;
-                if (got) {
-                    tc_fence_after();
-                    tmem_ld32(tmem + lane_off + kQTAcc1 + hh * kOpRows, num);
-                    den = tmem_ld1(tmem + lane_off + kQTAcc1 + hh * kOpRows + kD);
-                    tmem_wait_ld();
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) num[c] = 0.f;
-                }
-                if (hh == 3) {   // every head's M1 result is read
-                    tc_fence_before();
-                    mbar_arrive(acc1_empty);
-                }
-                float o[32];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint4 u = dv[4 * hh + j];
-                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        o[8 * j + 2 * m] = __uint_as_float(w[m] << 16);
-                        o[8 * j + 2 * m + 1] = __uint_as_float(w[m] & 0xFFFF0000u);
-                    }
-                }
-                const float inv = 1.0f / (den + p.eps);
-                float dn = 0.f;
-#pragma unroll
-                for (int c = 0; c < 32; ++c) dn = fmaf(o[c], num[c], dn);
-                const float cr = valid && got ? -dn * inv * inv : 0.f;
-                // g hi and lo into the two g tiles: box hh/2, logical chunks 4 (hh%2) + c4
-                uint8_t *gbox = gtile + (hh >> 1) * kQTBox + r * 128;
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    uint32_t hi[4], lo[4];
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        const float g0 = valid && got ? o[8 * c4 + 2 * m] * inv : 0.f;
-                        const float g1 = valid && got ? o[8 * c4 + 2 * m + 1] * inv : 0.f;
-                        const __nv_bfloat162 hv = __floats2bfloat162_rn(g0, g1);
-                        hi[m] = *reinterpret_cast<const uint32_t *>(&hv);
-                        lo[m] = pack_bf2(g0 - __low2float(hv), g1 - __high2float(hv));
-                    }
-                    const int pc = (4 * (hh & 1) + c4) ^ (r & 7);
-                    *reinterpret_cast<uint4 *>(gbox + pc * 16) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                    *reinterpret_cast<uint4 *>(gbox + kQTTile + pc * 16) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                }
-                const __nv_bfloat16 ch = __float2bfloat16_rn(cr);
-                *reinterpret_cast<__nv_bfloat16 *>(cop + c_offset(2 * hh, r)) = ch;
-                *reinterpret_cast<__nv_bfloat16 *>(cop + c_offset(2 * hh + 1, r)) =
-                    __float2bfloat16_rn(cr - __bfloat162float(ch));
-                cval[cb * 512 + r * 4 + hh] = cr;
-            }
-            fence_proxy_async_smem();   // g and c are read by the tensor cores
-            mbar_arrive(g_ready);
-            mbar_arrive(&c_ready[cb]);
-        }
-        // ---- the split's [dS | dZ]: lane quarter qd = the key features of head 4g + qd
-        bool gs = ok && mbar_wait(accS_full, 0, abort_word, &g_wait_flag, 74);
-        gs = __all_sync(0xffffffffu, gs);
-        if (gs) {
-            tc_fence_after();
-            float kv[32];
-            tmem_ld32(tmem + lane_off + kQTAccS + 32 * qd, kv);
-            const float z0 = tmem_ld1(tmem + lane_off + kQTAccZ + 2 * qd);
-            const float z1 = tmem_ld1(tmem + lane_off + kQTAccZ + 2 * qd + 1);
-            tmem_wait_ld();
-            float *dst = bpart + ((((size_t)b * p.H + 4 * g + qd) * p.nb + n) * p.P + sp) * kKVZ;
-            float4 *drow = reinterpret_cast<float4 *>(dst + lane * kD);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) drow[j] = make_float4(kv[4 * j], kv[4 * j + 1], kv[4 * j + 2], kv[4 * j + 3]);
-            dst[kD * kD + lane] = z0 + z1;
-        }
-        if (lane == 0) bulk_wait_all();
     }
 
     // teardown: nothing may still write this CTA's shared memory or TMEM
@@ -514,7 +601,7 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
 bool bwd_q_tc_available(const Plan &p) { return tc_available() && p.H % 4 == 0 && !p.rope && !p.f8; }
 
-// One CTA per SM (the kernel takes 512 TMEM columns and ~210 KiB of shared
+// One CTA per SM (the kernel takes 512 TMEM columns and ~218 KiB of shared
 // memory): the split plan aims at one wave of 148 CTAs.
 void bwd_q_tc_plan(Plan &p) {
     const long long groups = (long long)p.B * (p.H / 4) * p.nb;
@@ -539,9 +626,8 @@ int launch_bwd_q_tc(const void *q, const void *dout, void *dq, const float *seff
     const long long grid = (long long)p.B * (p.H / 4) * p.nb * p.P;
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
     return launch_pdl(bwd_q_tc_kernel, (unsigned)grid, kQTThreads, kQTSmem, s, mq, mdq,
-                      static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(dout),
-                      static_cast<__nv_bfloat16 *>(dq), seff, static_cast<const uint8_t *>(bop),
-                      static_cast<const uint8_t *>(stop), bpart, p)
+                      static_cast<const __nv_bfloat16 *>(dout), static_cast<__nv_bfloat16 *>(dq), seff,
+                      static_cast<const uint8_t *>(bop), static_cast<const uint8_t *>(stop), bpart, p)
                ? 1
                : -1;
 }
