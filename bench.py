@@ -99,10 +99,22 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_sources_sha():
-    h = hashlib.sha256()
+# the source files each timed kernel is built from (the shared headers too)
+KERNEL_SOURCES = {
+    "reduce": ["k_tc.cu"], "apply": ["k_tc.cu"], "finish": ["k_finish.cu"],
+    "bwd_q": ["k_bwd_q_tc.cu"], "bwd_k": ["k_bwd_tc.cu"], "dwconv": ["k_conv.cu"],
+}
+SHARED_SOURCES = ["la_internal.cuh", "la_sm100.cuh"]
+
+
+def kernel_sources_sha(kernel: str) -> str:
+    """Hash of the sources of `kernel` (by its name's first part), so that a
+    stored ncu figure is dropped when, and only when, that kernel changed."""
     csrc = os.path.join(ROOT, "block_causal_linear_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    key = next((k for k in KERNEL_SOURCES if kernel.startswith(k)), None)
+    files = sorted(os.listdir(csrc)) if key is None else KERNEL_SOURCES[key] + SHARED_SOURCES
+    h = hashlib.sha256()
+    for f in files:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -110,16 +122,17 @@ def kernel_sources_sha():
 
 def ncu_traffic(kernel: str, units_per_launch: int):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, scaled
-    to this launch by token-heads, or None when the kernels changed since."""
+    to this launch by its units (token-heads, or elements for the convolution),
+    or None when the kernel changed since."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         j = json.load(f)
     e = j.get(kernel)
-    if not e or e.get("sources_sha") != kernel_sources_sha():
+    if not e or e.get("sources_sha") != kernel_sources_sha(kernel):
         return None
-    return e["dram_bytes_per_token_head"] * units_per_launch
+    return e["dram_bytes_per_unit"] * units_per_launch
 
 
 class ClockSampler:
@@ -352,7 +365,8 @@ def run_dwconv(args, w, world, rank, dist, dev, la):
                 "hbm_frac_of_" + peak_kind: 2 * conv_bytes / (t_all / K / 1e3) / 1e9 / peak,
                 "stage_ms_per_step": {"dwconv_1x3x3": t1 / K, "dwconv_3x1x1": t2 / K},
                 "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
-                             "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None},
+                             "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                             "traffic": ncu_traffic(dom, tokens * C)},
                 "cpu_baseline": cpu, "e2e": None, "gpu_launches": 2 * K, "path": "dwconv", "clocks": clocks}
         print(json.dumps(line), flush=True)
     if dist is not None:

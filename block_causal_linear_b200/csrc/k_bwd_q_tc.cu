@@ -58,16 +58,17 @@ constexpr int kQTTile = 2 * kQTBox;                  // 4 heads
 constexpr int kQTStages = 2;
 constexpr int kQTMaskBufs = 4;
 constexpr int kQTGOff = kQTStages * kQTTile;         // g hi tile, then g lo tile
-constexpr int kQTCOff = kQTGOff + 2 * kQTTile;       // c operand: [16 rows][128 tokens] bf16
+constexpr int kQTDoOff = kQTGOff + 2 * kQTTile;      // the dout tile, laid out as the q tile
+constexpr int kQTCOff = kQTDoOff + kQTTile;          // c operand: [16 rows][128 tokens] bf16
 constexpr int kQTCBytes = 2 * 2048;
-constexpr int kQTOpsOff = kQTCOff + kQTCBytes;       // per head: [S|Z|0] hi, lo; S^T hi, lo
-constexpr int kQTOpsHead = 2 * kOpBytes + 2 * kStOpBytes;
-constexpr int kQTStgOff = kQTOpsOff + 4 * kQTOpsHead;   // 4 dq warps x 2 boxes [32 rows][64 bf16]
-constexpr int kQTAcOff = kQTStgOff + 4 * 2 * 4096;      // c as the K = 16 extension of M2's A: [128 tokens][16]
+constexpr int kQTOpsOff = kQTCOff + kQTCBytes;       // per head: [S|Z|0] hi, lo
+constexpr int kQTOpsHead = 2 * kOpBytes;
+constexpr int kQTStgOff = kQTOpsOff + 4 * kQTOpsHead;   // 4 dq warps x one box [32 rows][64 bf16]
+constexpr int kQTAcOff = kQTStgOff + 4 * 4096;          // c as the K = 16 extension of M2's A: [128 tokens][16]
 constexpr int kQTBcOff = kQTAcOff + 4096;               // Z_n as that extension of B, per head [32][16]
 constexpr int kQTMaskOff = kQTBcOff + 4096;             // sign bytes [4 buffers][128 rows][16 logical chunks]
 constexpr int kQTBarOff = kQTMaskOff + kQTMaskBufs * 128 * 16;
-constexpr int kQTNumBars = 3 * kQTStages + 2 * kQTMaskBufs + 14;
+constexpr int kQTNumBars = 3 * kQTStages + 2 * kQTMaskBufs + 16;
 constexpr int kQTSmem = kQTBarOff + kQTNumBars * 8 + 16 + 1024;
 static_assert(kQTSmem <= 232448, "shared memory of the query-side kernel");
 // TMEM columns
@@ -96,16 +97,17 @@ __device__ __forceinline__ int ac_offset(int t, int k) {
 }
 
 __global__ void __launch_bounds__(kQTThreads, 1)
-bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_dq,
-                const __nv_bfloat16 *__restrict__ dout, __nv_bfloat16 *__restrict__ dq,
-                const float *__restrict__ seff, const uint8_t *__restrict__ bop, const uint8_t *__restrict__ stop,
-                float *__restrict__ bpart, const Plan p) {
+bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                const __grid_constant__ CUtensorMap tm_dq, __nv_bfloat16 *__restrict__ dq,
+                const float *__restrict__ seff, const uint8_t *__restrict__ bop, float *__restrict__ bpart,
+                const Plan p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     uint8_t *gtile = smem + kQTGOff;
     uint8_t *cop = smem + kQTCOff;
     uint8_t *ops = smem + kQTOpsOff;
     uint8_t *stg = smem + kQTStgOff;
+    uint8_t *dot = smem + kQTDoOff;
     uint8_t *acx = smem + kQTAcOff;
     uint8_t *bcx = smem + kQTBcOff;
     uint8_t *mask8 = smem + kQTMaskOff;
@@ -125,7 +127,9 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint64_t *ops_full = accS_full + 1;
     uint64_t *dep_ready = ops_full + 1;
     uint64_t *drain = dep_ready + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *dout_full = drain + 1;                // the dout tile is loaded
+    uint64_t *dout_free = dout_full + 1;            // ... and read by the g epilogue
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(dout_free + 1);
     volatile int *abort_word = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int G4 = p.H / 4;
@@ -170,6 +174,8 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(ops_full, 1);
         mbar_init(dep_ready, 1);
         mbar_init(drain, 1);
+        mbar_init(dout_full, 1);
+        mbar_init(dout_free, kQTWork);
         *abort_word = 0;
         fence_barrier_init();
     }
@@ -184,6 +190,7 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     if (warp == kQTWarpTma && lane == 0) {
         prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_do);
         prefetch_tmap(&tm_dq);
     }
     fence_proxy_async_smem();
@@ -191,46 +198,56 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    int issued = 0;
+    int issued = 0, do_issued = 0;
     bool ops_issued = false;
 
     if (warp == kQTWarpTma) {
         if (lane == 0) {
-            // q is an input of the call: its first tiles come in before the
-            // dependency on the state combine resolves
-            const int pre = ntiles < kQTStages ? ntiles : kQTStages;
-            for (int i = 0; i < pre; ++i) {
-                mbar_arrive_expect_tx(&full[i], kQTTile);
+            auto load_q = [&](int i) {
+                const int s = i % kQTStages;
                 const int row = (int)(t0 + 128LL * i);
-                tma_load_3d(smem + i * kQTTile, &tm_q, &full[i], g * 128, row, b);
-                tma_load_3d(smem + i * kQTTile + kQTBox, &tm_q, &full[i], g * 128 + 64, row, b);
+                mbar_arrive_expect_tx(&full[s], kQTTile);
+                tma_load_3d(smem + s * kQTTile, &tm_q, &full[s], g * 128, row, b);
+                tma_load_3d(smem + s * kQTTile + kQTBox, &tm_q, &full[s], g * 128 + 64, row, b);
                 issued = i + 1;
-            }
+            };
+            auto load_dout = [&](int i) {
+                const int row = (int)(t0 + 128LL * i);
+                mbar_arrive_expect_tx(dout_full, kQTTile);
+                tma_load_3d(dot, &tm_do, dout_full, g * 128, row, b);
+                tma_load_3d(dot + kQTBox, &tm_do, dout_full, g * 128 + 64, row, b);
+                do_issued = i + 1;
+            };
+            // q and dout are inputs of the call: their first tiles come in before
+            // the dependency on the state combine resolves
+            const int pre = ntiles < kQTStages ? ntiles : kQTStages;
+            for (int i = 0; i < pre; ++i) load_q(i);
+            load_dout(0);
             pdl_wait();
             mbar_arrive(dep_ready);
             mbar_arrive_expect_tx(ops_full, 4 * kQTOpsHead);
             for (int hh = 0; hh < 4; ++hh) {
                 const size_t bh = (size_t)b * p.H + 4 * g + hh;
                 bulk_load(ops + hh * kQTOpsHead, bop + (bh * p.nb + n) * 2 * kOpBytes, 2 * kOpBytes, ops_full);
-                bulk_load(ops + hh * kQTOpsHead + 2 * kOpBytes, stop + (bh * p.nb + n) * 2 * kStOpBytes,
-                          2 * kStOpBytes, ops_full);
             }
             ops_issued = true;
-            for (int i = pre; i < ntiles; ++i) {
-                const int s = i % kQTStages;
-                const uint32_t ph = (uint32_t)(i / kQTStages) & 1u;
-                if (!mbar_wait(&empty[s], ph ^ 1u, abort_word, &g_wait_flag, 61)) break;
-                mbar_arrive_expect_tx(&full[s], kQTTile);
-                const int row = (int)(t0 + 128LL * i);
-                tma_load_3d(smem + s * kQTTile, &tm_q, &full[s], g * 128, row, b);
-                tma_load_3d(smem + s * kQTTile + kQTBox, &tm_q, &full[s], g * 128 + 64, row, b);
-                issued = i + 1;
+            // per tile: its q tile once a stage is free, then its dout tile once the
+            // g epilogue has read the previous one (q first: it is needed earlier)
+            for (int i = 1; i < ntiles; ++i) {
+                if (i >= pre) {
+                    const uint32_t ph = (uint32_t)(i / kQTStages) & 1u;
+                    if (!mbar_wait(&empty[i % kQTStages], ph ^ 1u, abort_word, &g_wait_flag, 61)) break;
+                    load_q(i);
+                }
+                if (!mbar_wait(dout_free, (uint32_t)(i - 1) & 1u, abort_word, &g_wait_flag, 60)) break;
+                load_dout(i);
             }
         }
     } else if (warp == kQTWarpMma) {
         if (lane == 0) {
             const uint32_t id_m1 = idesc_bf16(128, kOpRows, 0, 0);     // phi(Q) x [S|Z|0]
-            const uint32_t id_m2 = idesc_bf16(128, kD, 0, 0);          // g x S^T
+            const uint32_t id_m2 = idesc_bf16(128, kD, 0, 1);          // g x S^T, S^T read MN-major
+            const uint32_t id_m2c = idesc_bf16(128, kD, 0, 0);         // [c] x [Z], both K-major
             const uint32_t id_m3 = idesc_bf16(128, 128, 1, 1);         // phi(Q)^T x g
             const uint32_t id_m4 = idesc_bf16(128, 16, 1, 0);          // phi(Q)^T x [c hi | c lo | 0]
             const uint32_t oaddr = smem_u32(ops), gaddr = smem_u32(gtile), caddr = smem_u32(cop);
@@ -253,7 +270,10 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 mma_commit(&acc1_full[bx]);
             };
-            // M2 of box bx: per head, g S^T as g_hi.ST_hi + g_hi.ST_lo + g_lo.ST_hi
+            // M2 of box bx: per head, g S^T as g_hi.ST_hi + g_hi.ST_lo + g_lo.ST_hi.  S^T is
+            // the packed [S|Z|0] operand of M1 read MN-major: its value columns are
+            // the K rows of S^T (8-row groups 512 B apart: LBO), its key features
+            // the N columns (8-column chunks 128 B apart: SBO)
             auto m2 = [&](int bx) {
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
@@ -265,15 +285,14 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         for (int kk = 0; kk < 2; ++kk) {
                             const uint64_t da = smem_desc(gaddr + gp * kQTTile + bx * kQTBox + h2 * 64 + kk * 32, 16,
                                                           1024, kLayoutSw128);
-                            const uint64_t db = smem_desc(oaddr + hh * kQTOpsHead + 2 * kOpBytes + sp2 * kStOpBytes +
-                                                              kk * 256,
-                                                          128, 512, kLayoutNone);
+                            const uint64_t db = smem_desc(oaddr + hh * kQTOpsHead + sp2 * kOpBytes + kk * 1024, 512,
+                                                          128, kLayoutNone);
                             mma_bf16(tmem + kQTAcc2 + hh * kD, da, db, id_m2, (prod | kk) ? 1u : 0u);
                         }
                     }
                     // + c_t Z_n: the K = 16 extension
                     mma_bf16(tmem + kQTAcc2 + hh * kD, smem_desc(acaddr, 128, 256, kLayoutNone),
-                             smem_desc(bcaddr + hh * 1024, 128, 256, kLayoutNone), id_m2, 1u);
+                             smem_desc(bcaddr + hh * 1024, 128, 256, kLayoutNone), id_m2c, 1u);
                 }
             };
             bool ok = mbar_wait(ops_full, 0, abort_word, &g_wait_flag, 62);
@@ -371,42 +390,26 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int qd = warp & 3;                // TMEM lane quarter
         const int r = 32 * qd + lane;           // token row of this thread in a tile
         const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
-        // dout of (tile i, box bx) for this thread's row: 2 heads, 128 bytes; zero past the split
-        auto load_dout = [&](int i, int bx, uint4 (&v)[8]) {
-            const long long t = t0 + 128LL * i + r;
-            if (t < t1) {
-                const uint4 *src =
-                    reinterpret_cast<const uint4 *>(dout + (((size_t)b * p.N + t) * p.H + 4 * g + 2 * bx) * kD);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = __ldg(src + j);
-            } else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = make_uint4(0u, 0u, 0u, 0u);
-            }
-        };
         bool ok = true;
-        uint4 cur[8];
-        load_dout(0, 0, cur);
         for (int i = 0; i < ntiles; ++i) {
             const uint32_t tph = (uint32_t)i & 1u;
             const long long t = t0 + 128LL * i + r;
             const bool valid = t < t1;
-            if (t + 128 < t1) {   // the next tile's dout row into L2
-                const uint8_t *nx =
-                    reinterpret_cast<const uint8_t *>(dout + (((size_t)b * p.N + t + 128) * p.H + 4 * g) * kD);
-                prefetch_l2(nx);
-                prefetch_l2(nx + 128);
-            }
 #pragma unroll 1
             for (int bx = 0; bx < 2; ++bx) {
-                uint4 nxt[8];   // one box ahead; zeros past the last tile
-                if (bx == 0) load_dout(i, 1, nxt);
-                else load_dout(i + 1, 0, nxt);
                 bool got = ok && mbar_wait(&acc1_full[bx], tph, abort_word, &g_wait_flag, 70);
-                if (bx == 0)   // M2, M3, M4 of tile i - 1 are done with g and c
+                if (bx == 0) {   // M2, M3, M4 of tile i - 1 are done with g and c; this tile's dout is in
                     got = got && mbar_wait(g_free, tph ^ 1u, abort_word, &g_wait_flag, 71);
+                    got = got && mbar_wait(dout_full, tph, abort_word, &g_wait_flag, 75);
+                }
                 got = __all_sync(0xffffffffu, got);
                 if (!got) ok = false;
+                // this row's dout of the box's 2 heads (rows past the split are not used)
+                uint4 cur[8];
+                const uint8_t *drow = dot + bx * kQTBox + r * 128;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) cur[j] = *reinterpret_cast<const uint4 *>(drow + ((j ^ (r & 7)) * 16));
+                if (bx == 1) mbar_arrive(dout_free);   // the dout tile is read
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
                     const int hh = 2 * bx + h2;
@@ -469,8 +472,6 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 fence_proxy_async_smem();   // the box's g (and its c) is read by the tensor cores
                 mbar_arrive(&g_ready[bx]);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) cur[j] = nxt[j];
             }
         }
         // ---- the split's [dS | dZ]: lane quarter qd = the key features of head 4g + qd
@@ -523,13 +524,25 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const bool valid = t < t1;
             const long long wrow0 = row0 + 32 * qd;
             const bool boxed = wrow0 + 32 <= t1 || t1 == p.N;   // TMA clips rows >= N
-            uint8_t *sb = stg + qd * 2 * 4096;                 // this warp's two staging boxes
+            uint8_t *sb = stg + qd * 4096;                     // this warp's staging box
             if (boxed) {
                 if (lane == 0) bulk_wait_read<0>();   // the previous tile's stores have read sb
                 __syncwarp();
             }
 #pragma unroll 1
             for (int hh = 0; hh < 4; ++hh) {
+                if (hh == 2 && boxed) {   // heads 0, 1 go out; the box then takes heads 2, 3
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (ok) {
+                            tma_store_3d(&tm_dq, sb, g * 128, (int)wrow0, b);
+                            bulk_commit();
+                        }
+                        bulk_wait_read<0>();
+                    }
+                    __syncwarp();
+                }
                 float pre[32];
                 uint32_t m = 0;
                 if (got) {
@@ -547,7 +560,7 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int a = 0; a < 32; ++a) pre[a] = (m >> a) & 1u ? pre[a] : 0.f;
                 if (boxed) {
-                    uint8_t *bx = sb + (hh >> 1) * 4096 + lane * 128;
+                    uint8_t *bx = sb + lane * 128;
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
                         const int pc = (4 * (hh & 1) + c4) ^ (lane & 7);   // 128-byte swizzle
@@ -569,8 +582,7 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0 && ok) {
-                    tma_store_3d(&tm_dq, sb, g * 128, (int)wrow0, b);
-                    tma_store_3d(&tm_dq, sb + 4096, g * 128 + 64, (int)wrow0, b);
+                    tma_store_3d(&tm_dq, sb, g * 128 + 64, (int)wrow0, b);
                     bulk_commit();
                 }
             }
@@ -583,6 +595,7 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (ops_issued) final_wait(ops_full, 0);
         for (int i = issued - kQTStages < 0 ? 0 : issued - kQTStages; i < issued; ++i)
             final_wait(&full[i % kQTStages], (uint32_t)(i / kQTStages) & 1u);
+        if (do_issued > 0) final_wait(dout_full, (uint32_t)(do_issued - 1) & 1u);
     }
     if (warp == kQTWarpMma && lane == 0 && *abort_word) {
         mma_commit(drain);
@@ -615,19 +628,20 @@ void bwd_q_tc_plan(Plan &p) {
     p.P = (int)((p.L + chunk - 1) / chunk);
 }
 
-int launch_bwd_q_tc(const void *q, const void *dout, void *dq, const float *seff, const void *bop, const void *stop,
-                    float *bpart, const Plan &p, cudaStream_t s) {
+int launch_bwd_q_tc(const void *q, const void *dout, void *dq, const float *seff, const void *bop, float *bpart,
+                    const Plan &p, cudaStream_t s) {
     static std::once_flag once;
     static bool attr_ok = false;
     std::call_once(once, [] { attr_ok = set_smem((const void *)bwd_q_tc_kernel, kQTSmem); });
     if (!attr_ok) return -1;
-    CUtensorMap mq, mdq;
-    if (!make_bf16_map(&mq, q, p.B, p.N, p.H, 128) || !make_bf16_map(&mdq, dq, p.B, p.N, p.H, 32)) return -1;
+    CUtensorMap mq, mdo, mdq;
+    if (!make_bf16_map(&mq, q, p.B, p.N, p.H, 128) || !make_bf16_map(&mdo, dout, p.B, p.N, p.H, 128) ||
+        !make_bf16_map(&mdq, dq, p.B, p.N, p.H, 32))
+        return -1;
     const long long grid = (long long)p.B * (p.H / 4) * p.nb * p.P;
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
-    return launch_pdl(bwd_q_tc_kernel, (unsigned)grid, kQTThreads, kQTSmem, s, mq, mdq,
-                      static_cast<const __nv_bfloat16 *>(dout), static_cast<__nv_bfloat16 *>(dq), seff,
-                      static_cast<const uint8_t *>(bop), static_cast<const uint8_t *>(stop), bpart, p)
+    return launch_pdl(bwd_q_tc_kernel, (unsigned)grid, kQTThreads, kQTSmem, s, mq, mdo, mdq,
+                      static_cast<__nv_bfloat16 *>(dq), seff, static_cast<const uint8_t *>(bop), bpart, p)
                ? 1
                : -1;
 }

@@ -38,7 +38,7 @@ constexpr int kPerBH = kKVZ + kZeroRows * kD;   // numbers + zero-padding entrie
 __global__ void __launch_bounds__(kFinThreads)
 finish_kernel(const float *__restrict__ partials, float *__restrict__ seff,
               unsigned char *__restrict__ bop, float *__restrict__ S, float *__restrict__ Z,
-              Plan p, int write_bop, long long part_bh, long long part_sp, unsigned char *__restrict__ stop) {
+              Plan p, int write_bop, long long part_bh, long long part_sp) {
     // let the apply be scheduled now (it prefetches its q tiles), then wait
     // for the reduce before reading its partials
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -76,13 +76,6 @@ finish_kernel(const float *__restrict__ partials, float *__restrict__ seff,
                 if (s0 + j < p.P) run += v[j];
         }
         seff[((size_t)bh * p.nb + n) * kKVZ + e] = run;
-        if (stop && e < kD * kD) {
-            // S^T as a bf16 hi + lo operand (rows = key feature, K = value column)
-            unsigned char *o = stop + ((size_t)bh * p.nb + n) * 2 * kStOpBytes + op_offset(e / kD, e % kD);
-            const __nv_bfloat16 hi = __float2bfloat16_rn(run);
-            *reinterpret_cast<__nv_bfloat16 *>(o) = hi;
-            *reinterpret_cast<__nv_bfloat16 *>(o + kStOpBytes) = __float2bfloat16_rn(run - __bfloat162float(hi));
-        }
         if (write_bop) {
             unsigned char *dst = bop + ((size_t)bh * p.nb + n) * 2 * kOpBytes + op_offset(nrow, kcol);
             const __nv_bfloat16 hi = __float2bfloat16_rn(run);
@@ -101,7 +94,7 @@ finish_kernel(const float *__restrict__ partials, float *__restrict__ seff,
 
 namespace {
 int launch_finish_strided(const float *partials, float *seff, void *bop, float *S, float *Z, const Plan &p,
-                          int write_bop, long long part_bh, long long part_sp, unsigned char *stop, cudaStream_t s) {
+                          int write_bop, long long part_bh, long long part_sp, cudaStream_t s) {
     const long long threads = (long long)p.B * p.H * kPerBH;
     const long long grid = (threads + kFinThreads - 1) / kFinThreads;
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
@@ -117,7 +110,7 @@ int launch_finish_strided(const float *partials, float *seff, void *bop, float *
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, finish_kernel, partials, seff, static_cast<unsigned char *>(bop), S, Z, p,
-                              write_bop, part_bh, part_sp, stop) == cudaSuccess
+                              write_bop, part_bh, part_sp) == cudaSuccess
                ? 1
                : -1;
 }
@@ -125,20 +118,17 @@ int launch_finish_strided(const float *partials, float *seff, void *bop, float *
 
 int launch_finish(const float *partials, float *seff, void *bop, float *S, float *Z, const Plan &p,
                   int write_bop, cudaStream_t s) {
-    return launch_finish_strided(partials, seff, bop, S, Z, p, write_bop, (long long)p.P * kKVZ, kKVZ, nullptr, s);
+    return launch_finish_strided(partials, seff, bop, S, Z, p, write_bop, (long long)p.P * kKVZ, kKVZ, s);
 }
 
-int launch_finish_with_st(const float *partials, float *seff, void *bop, void *stop, const Plan &p, cudaStream_t s) {
-    return launch_finish_strided(partials, seff, bop, nullptr, nullptr, p, 1, (long long)p.P * kKVZ, kKVZ,
-                                 static_cast<unsigned char *>(stop), s);
-}
+
 
 int launch_finish_ranks(const float *gathered, int R, float *seff, void *bop, float *S, float *Z, const Plan &p,
                         int write_bop, cudaStream_t s) {
     if (p.nb != 1 || R < 1) return -1;
     Plan q = p;
     q.P = R;   // the ranks' partial sums play the splits, in rank order
-    return launch_finish_strided(gathered, seff, bop, S, Z, q, write_bop, kKVZ, (long long)p.B * p.H * kKVZ, nullptr,
+    return launch_finish_strided(gathered, seff, bop, S, Z, q, write_bop, kKVZ, (long long)p.B * p.H * kKVZ,
                                  s);
 }
 

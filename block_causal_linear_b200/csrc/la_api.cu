@@ -281,18 +281,16 @@ la_status la_full_backward(const void *q, const void *k, const void *v, const vo
     r = tc ? la::launch_reduce_tc(k, v, partials, p, s) : la::launch_reduce_ffma(bf, k, v, partials, p, s);
     if (r < 0) return LA_ECUDA;
     n += r;
-    // the query side on the tensor cores needs the packed [S|Z|0] and S^T operands
+    // the query side on the tensor cores needs the packed [S|Z|0] operand
     const bool qtc = bf && tc && la::bwd_q_tc_available(p);
-    void *stop = base + w.stop;
-    r = qtc ? la::launch_finish_with_st(partials, seff, base + w.fwd.bop, stop, p, s)
-            : la::launch_finish(partials, seff, base + w.fwd.bop, nullptr, nullptr, p, tc ? 1 : 0, s);
+    r = la::launch_finish(partials, seff, base + w.fwd.bop, nullptr, nullptr, p, tc ? 1 : 0, s);
     if (r < 0) return LA_ECUDA;
     n += r;
     if (!mark(1, s)) return LA_ECUDA;
     // the query side takes its own split plan; the suffix sums below read its splits
     la::Plan pq = p;
     if (qtc) la::bwd_q_tc_plan(pq);
-    r = qtc ? la::launch_bwd_q_tc(q, dout, dq, seff, base + w.fwd.bop, stop, bpart, pq, s)
+    r = qtc ? la::launch_bwd_q_tc(q, dout, dq, seff, base + w.fwd.bop, bpart, pq, s)
             : la::launch_bwd_q(bf, q, dout, seff, dq, bpart, p, s);
     if (r < 0) return LA_ECUDA;
     n += r;

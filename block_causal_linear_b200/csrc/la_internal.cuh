@@ -103,7 +103,6 @@ int launch_finish(const float *partials, float *seff, void *bop, float *S, float
                   const Plan &p, int write_bop, cudaStream_t s);
 
 // The same, also packing S^T (hi, lo) for the query-side backward; no state.
-int launch_finish_with_st(const float *partials, float *seff, void *bop, void *stop, const Plan &p, cudaStream_t s);
 
 // The same for a block whose tokens were split over R ranks: gathered is
 // [R][B][H][kKVZ], the ranks' partial sums in rank order; p.nb must be 1.
@@ -139,7 +138,7 @@ int launch_bwd_k(int is_bf16, const void *k, const void *v, const float *G, void
 // ([B][H][nb][P][kKVZ]) and their suffix sums G ([B][H][nb][kKVZ]), fp32.
 struct BwdLayout {
     WsLayout fwd;
-    size_t bpart, G, gop, stop, total;
+    size_t bpart, G, gop, total;
 };
 
 // Packed bf16 operands of the key-side tensor-core backward, per (b, h,
@@ -147,9 +146,6 @@ struct BwdLayout {
 // K = c), each as a hi and a lo part, 32 rows of the K-major core-matrix
 // layout of op_offset: 4 x 2048 bytes.
 constexpr int kGopBytes = 2048;
-// S^T operand of the query-side tensor-core backward (rows = key feature a,
-// K = value column c), per (b, h, block), hi and lo: 2 x 2048 bytes.
-constexpr int kStOpBytes = 2048;
 
 inline BwdLayout bwd_layout(int B, int H, int nb, int P) {
     BwdLayout w;
@@ -158,8 +154,7 @@ inline BwdLayout bwd_layout(int B, int H, int nb, int P) {
     w.bpart = w.fwd.total;
     w.G = align256(w.bpart + bhn * P * kKVZ * sizeof(float));
     w.gop = align256(w.G + bhn * kKVZ * sizeof(float));
-    w.stop = align256(w.gop + bhn * 4 * size_t(kGopBytes));
-    w.total = align256(w.stop + bhn * 2 * size_t(kStOpBytes));
+    w.total = align256(w.gop + bhn * 4 * size_t(kGopBytes));
     return w;
 }
 
@@ -196,11 +191,11 @@ bool make_bf16_map(CUtensorMap *m, const void *base, int B, int N, int H, int bo
 
 // Query side on the tensor cores (bf16, H % 4 == 0, no RoPE): its own split
 // plan (one CTA per SM), dq and the split sums of [dS | dZ] from q, dout, the
-// state S_eff (seff) and its packed operands [S|Z|0] (bop) and S^T (stop).
+// state S_eff (seff) and its packed operand [S|Z|0] (bop), which also gives S^T.
 bool bwd_q_tc_available(const Plan &p);
 void bwd_q_tc_plan(Plan &p);
-int launch_bwd_q_tc(const void *q, const void *dout, void *dq, const float *seff, const void *bop, const void *stop,
-                    float *bpart, const Plan &p, cudaStream_t s);
+int launch_bwd_q_tc(const void *q, const void *dout, void *dq, const float *seff, const void *bop, float *bpart,
+                    const Plan &p, cudaStream_t s);
 int read_and_clear_bwd_k_flag(unsigned *flag_out);
 int read_and_clear_bwd_q_flag(unsigned *flag_out);
 
