@@ -35,10 +35,15 @@ constexpr int kBatch = 32;         // partial loads in flight per thread (one ro
 constexpr int kZeroRows = kOpRows - kD - 1;
 constexpr int kPerBH = kKVZ + kZeroRows * kD;   // numbers + zero-padding entries per (b, h)
 
+// STRIDED: the split sums sit at runtime strides (the ranks' gathered sums);
+// otherwise at the workspace's own: split sp of (bh, n) at ((bh nb + n) P + sp) kKVZ.
+template <bool STRIDED>
 __global__ void __launch_bounds__(kFinThreads)
 finish_kernel(const float *__restrict__ partials, float *__restrict__ seff,
               unsigned char *__restrict__ bop, float *__restrict__ S, float *__restrict__ Z,
-              Plan p, int write_bop, long long part_bh, long long part_sp) {
+              Plan p, int write_bop, long long part_bh_rt, long long part_sp_rt) {
+    const long long part_bh = STRIDED ? part_bh_rt : (long long)p.P * kKVZ;
+    const long long part_sp = STRIDED ? part_sp_rt : (long long)kKVZ;
     // let the apply be scheduled now (it prefetches its q tiles), then wait
     // for the reduce before reading its partials
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -109,8 +114,9 @@ int launch_finish_strided(const float *partials, float *seff, void *bop, float *
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, finish_kernel, partials, seff, static_cast<unsigned char *>(bop), S, Z, p,
-                              write_bop, part_bh, part_sp) == cudaSuccess
+    const bool strided = part_bh != (long long)p.P * kKVZ || part_sp != kKVZ;
+    return cudaLaunchKernelEx(&cfg, strided ? finish_kernel<true> : finish_kernel<false>, partials, seff,
+                              static_cast<unsigned char *>(bop), S, Z, p, write_bop, part_bh, part_sp) == cudaSuccess
                ? 1
                : -1;
 }

@@ -174,12 +174,73 @@ struct RCfg {
     static constexpr int kThreadsR = 64 + kXform;
 };
 
+// Fused state combine: the split sums of the CTA's 4 heads ([4][kKVZ] fp32)
+// in shared memory, past the z scratch of the RoPE epilogue.
+constexpr int kFusePartOff = 16384;
+constexpr int kZeroRowsOp = kOpRows - kD - 1;   // zero rows 33..47 of the packed operand
+
+// The cluster's share of one head group's combine, in the order of the
+// separate combine kernel: S_eff = prior state (with one) + the split sums in
+// split order; then the packed bf16 hi + lo operand and (commit) the state.
+// The splits of the group are the cluster's CTAs, rank = split.
+__device__ void fused_combine(const Plan &p, const Fuse &fz, const float *part, int b, int g, int n, int nthr) {
+    const int rank = (int)cluster_ctarank(), P = (int)cluster_nctarank();
+    constexpr int kU = 3;   // entries per thread whose remote loads are in flight together
+    for (int u0 = rank * nthr + (int)threadIdx.x; u0 < 4 * kKVZ; u0 += kU * P * nthr) {
+        float v[kU][kFuseMaxSplits];
+#pragma unroll
+        for (int j = 0; j < kU; ++j) {
+            const int u = u0 + j * P * nthr;
+#pragma unroll
+            for (int c = 0; c < kFuseMaxSplits; ++c)
+                v[j][c] = (c < P && u < 4 * kKVZ) ? ld_dsmem_f32(part + u, (unsigned)c) : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < kU; ++j) {
+            const int u = u0 + j * P * nthr;
+            if (u >= 4 * kKVZ) break;
+            const int hh = u / kKVZ, e = u - hh * kKVZ;
+            const size_t bh = (size_t)b * p.H + 4 * g + hh;
+            float run = 0.f;
+            if (p.has_state) run = e < kD * kD ? fz.S[bh * kD * kD + e] : fz.Z[bh * kD + e - kD * kD];
+#pragma unroll
+            for (int c = 0; c < kFuseMaxSplits; ++c)
+                if (c < P) run += v[j][c];
+            fz.seff[(bh * p.nb + n) * kKVZ + e] = run;
+            if (fz.write_bop) {
+                const int nrow = e < kD * kD ? (e % kD) : kD;   // value column, or the Z column
+                const int kcol = e < kD * kD ? (e / kD) : (e - kD * kD);
+                unsigned char *dst = fz.bop + (bh * p.nb + n) * 2 * kOpBytes + op_offset(nrow, kcol);
+                const __nv_bfloat16 hi = __float2bfloat16_rn(run);
+                *reinterpret_cast<__nv_bfloat16 *>(dst) = hi;
+                *reinterpret_cast<__nv_bfloat16 *>(dst + kOpBytes) = __float2bfloat16_rn(run - __bfloat162float(hi));
+            }
+            if (p.commit) {
+                if (e < kD * kD) fz.S[bh * kD * kD + e] = run;
+                else fz.Z[bh * kD + e - kD * kD] = run;
+            }
+        }
+    }
+    if (fz.write_bop) {
+        for (int u = rank * nthr + (int)threadIdx.x; u < 4 * kZeroRowsOp * kD; u += P * nthr) {
+            const int hh = u / (kZeroRowsOp * kD), z = u - hh * (kZeroRowsOp * kD);
+            const size_t bh = (size_t)b * p.H + 4 * g + hh;
+            unsigned char *dst = fz.bop + (bh * p.nb + n) * 2 * kOpBytes + op_offset(kD + 1 + z / kD, z % kD);
+            *reinterpret_cast<unsigned short *>(dst) = 0;
+            *reinterpret_cast<unsigned short *>(dst + kOpBytes) = 0;
+        }
+    }
+}
+
 template <bool ROPE, bool F8 = false>
 __global__ void __launch_bounds__(RCfg<ROPE, F8>::kThreadsR, 2)
 reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                 float *__restrict__ partials, const Plan p) {
+                 float *__restrict__ partials, const Plan p, const Fuse fz) {
     static_assert(!(ROPE && F8), "FP8 inputs take no RoPE");
     using C = RCfg<ROPE, F8>;
+    static_assert(C::kXform * 16 * 4 <= kFusePartOff &&
+                      kFusePartOff + 4 * kKVZ * 4 <= C::kStages * C::kStageBytes,
+                  "the fused split sums sit past the z scratch, inside the stages");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     uint8_t *aux = smem + C::kAuxOff;
@@ -190,10 +251,11 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_ready + 1);
     volatile int *abort_word = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
+    // the splits of a head group are consecutive CTAs (one cluster when fused)
     const int G = p.H / 4;
     long long id = blockIdx.x;
-    const int g = (int)(id % G); id /= G;
     const int sp = (int)(id % p.P); id /= p.P;
+    const int g = (int)(id % G); id /= G;
     const int n = (int)(id % p.nb); id /= p.nb;
     const int b = (int)id;
     const long long blk0 = (long long)n * p.L;
@@ -202,12 +264,21 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     const long long t1 = t0 + p.chunk < blk1 ? t0 + p.chunk : blk1;
     const int nst = t1 > t0 ? (int)((t1 - t0 + kRRows - 1) / kRRows) : 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float *fpart = reinterpret_cast<float *>(smem + kFusePartOff);
 
-    // k, v may come from the kernel just before this one: wait for it, then let
-    // the next kernel (the state combine) be scheduled
+    // k, v (and the prior state) may come from the kernel just before this one:
+    // wait for it, then let the next kernel be scheduled
     pdl_wait();
     pdl_trigger();
 
+    if (nst == 0 && fz.on) {   // a split past the end of a short block: zero sums, still in the cluster
+        for (int e = threadIdx.x; e < 4 * kKVZ; e += C::kThreadsR) fpart[e] = 0.f;
+        __syncthreads();
+        cluster_sync();
+        fused_combine(p, fz, fpart, b, g, n, C::kThreadsR);
+        cluster_sync();
+        return;
+    }
     if (nst == 0) {   // a split past the end of a short last block: its sums are zero
         for (int e = threadIdx.x; e < 4 * kKVZ; e += C::kThreadsR) {
             const int h = g * 4 + e / kKVZ;
@@ -255,13 +326,13 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 
     if (warp == kWarpTma) {
         if (lane == 0) {
+            const int c0 = g * 128;   // first feature of the group (a code = a byte with F8)
             for (int i = 0; i < nst; ++i) {
                 const int s = i % C::kStages;
                 const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
                 if (!mbar_wait(&empty[s], ph ^ 1u, abort_word, &g_wait_flag, 1)) break;
                 uint8_t *st = smem + s * C::kStageBytes;
                 const int row = (int)(t0 + (long long)kRRows * i);
-                const int c0 = g * 128;   // first feature of the group (a code = a byte with F8)
                 if constexpr (F8) {
                     mbar_arrive_expect_tx(&full[s], C::kStageBytes);
                     tma_load_3d(st, &tm_k, &full[s], c0, row, b);
@@ -439,7 +510,7 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 for (int j = 0; j < 32; ++j) kv[j] *= skv;
                 z *= p.sk;
             }
-            float *dst = partials + ((((size_t)b * p.H + h) * p.nb + n) * p.P + sp) * kKVZ;
+            float *dst = fz.on ? fpart + qd * kKVZ : partials + ((((size_t)b * p.H + h) * p.nb + n) * p.P + sp) * kKVZ;
             float4 *drow = reinterpret_cast<float4 *>(dst + lane * kD);
 #pragma unroll
             for (int j = 0; j < 8; ++j) drow[j] = make_float4(kv[4 * j], kv[4 * j + 1], kv[4 * j + 2], kv[4 * j + 3]);
@@ -461,6 +532,11 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
+    }
+    if (fz.on) {   // every split's sums are in its CTA's shared memory: combine them
+        cluster_sync();
+        fused_combine(p, fz, fpart, b, g, n, C::kThreadsR);
+        cluster_sync();   // no CTA leaves while another still reads its shared memory
     }
 }
 
@@ -951,25 +1027,27 @@ bool tc_rope_fits(const Plan &p) {
     return rope_table_entries(p, p.chunk) <= kTabMax && rope_table_entries(p, p.chunka) <= kTabMax;
 }
 
-int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &p, cudaStream_t s) {
+int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &p, cudaStream_t s, const Fuse *fz) {
     if (!smem_ready()) return -1;
     CUtensorMap mk, mv;
     const long long grid = (long long)p.B * (p.H / 4) * p.nb * p.P;
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
+    const Fuse off = {nullptr, nullptr, nullptr, nullptr, 0, 0};
+    const Fuse f = fz ? *fz : off;
+    if (f.on && (p.nb != 1 || p.P < 1 || p.P > kFuseMaxSplits)) return -1;
+    auto go = [&](auto kernel, int threads, int smem) {
+        return f.on ? launch_pdl_cluster(kernel, (unsigned)grid, threads, smem, (unsigned)p.P, s, mk, mv, partials, p, f)
+                    : launch_pdl(kernel, (unsigned)grid, threads, smem, s, mk, mv, partials, p, f);
+    };
     if (p.f8) {
         if (!make_map_u8(&mk, k, p.B, p.N, p.H, 128, kRRows, true) ||
             !make_map_u8(&mv, v, p.B, p.N, p.H, 128, kRRows, true))
             return -1;
-        return launch_pdl(reduce_tc_kernel<false, true>, (unsigned)grid, RCfg<false, true>::kThreadsR,
-                          RCfg<false, true>::kSmem, s, mk, mv, partials, p)
-                   ? 1
-                   : -1;
+        return go(reduce_tc_kernel<false, true>, RCfg<false, true>::kThreadsR, RCfg<false, true>::kSmem) ? 1 : -1;
     }
     if (!make_map(&mk, k, p.B, p.N, p.H, kRRows) || !make_map(&mv, v, p.B, p.N, p.H, kRRows)) return -1;
-    const bool ok = p.rope ? launch_pdl(reduce_tc_kernel<true>, (unsigned)grid, RCfg<true>::kThreadsR, RCfg<true>::kSmem, s, mk,
-                                        mv, partials, p)
-                           : launch_pdl(reduce_tc_kernel<false>, (unsigned)grid, RCfg<false>::kThreadsR, RCfg<false>::kSmem, s, mk,
-                                        mv, partials, p);
+    const bool ok = p.rope ? go(reduce_tc_kernel<true>, RCfg<true>::kThreadsR, RCfg<true>::kSmem)
+                           : go(reduce_tc_kernel<false>, RCfg<false>::kThreadsR, RCfg<false>::kSmem);
     return ok ? 1 : -1;
 }
 

@@ -55,6 +55,14 @@ void make_splits(la::Plan &p) {
     p.Pa = (int)ceil_div(p.L, chunka);
 }
 
+// The fused plan (the reduce combines its own splits): one block per call and
+// a default plan of at most kFuseMaxSplits splits per head group, which then
+// run as one cluster.  (Cutting a longer plan down to that many splits slows
+// the reduce by more than the separate combine kernel costs.)
+bool fuse_plan(const la::Plan &p) {
+    return p.nb == 1 && p.H % 4 == 0 && p.P >= 1 && p.P <= la::kFuseMaxSplits;
+}
+
 bool sizes_ok(int B, int N, int H, int d) {
     return B > 0 && N > 0 && H > 0 && d > 0 &&
            (long long)B * N * H * d < (1LL << 40);
@@ -136,13 +144,21 @@ la_status run(const void *q, const void *k, const void *v, void *out, la_dtype d
     int n = 0, r;
 
     if (!mark(0, s)) return LA_ECUDA;
-    r = tc ? la::launch_reduce_tc(k, v, partials, p, s)
-           : la::launch_reduce_ffma(dt == LA_BF16, k, v, partials, p, s);
-    if (r < 0 || !mark(1, s)) return LA_ECUDA;
-    n += r;
-    r = la::launch_finish(partials, seff, bop, S, Z, p, tc ? 1 : 0, s);
-    if (r < 0 || !mark(2, s)) return LA_ECUDA;
-    n += r;
+    if (tc && fuse_plan(p)) {
+        // one block: the reduce combines its splits itself (no combine kernel)
+        const la::Fuse fz = {seff, static_cast<unsigned char *>(bop), S, Z, 1, 1};
+        r = la::launch_reduce_tc(k, v, partials, p, s, &fz);
+        if (r < 0 || !mark(1, s) || !mark(2, s)) return LA_ECUDA;
+        n += r;
+    } else {
+        r = tc ? la::launch_reduce_tc(k, v, partials, p, s)
+               : la::launch_reduce_ffma(dt == LA_BF16, k, v, partials, p, s);
+        if (r < 0 || !mark(1, s)) return LA_ECUDA;
+        n += r;
+        r = la::launch_finish(partials, seff, bop, S, Z, p, tc ? 1 : 0, s);
+        if (r < 0 || !mark(2, s)) return LA_ECUDA;
+        n += r;
+    }
     r = tc ? la::launch_apply_tc(q, out, bop, seff, p, s)
            : la::launch_apply_ffma(dt == LA_BF16, q, out, seff, p, s);
     if (r < 0 || !mark(3, s)) return LA_ECUDA;

@@ -14,6 +14,7 @@ namespace la {
 
 constexpr int kD = 32;                 // head dim supported by this build
 constexpr int kKVZ = kD * kD + kD;     // floats per (b, h) of [KV | z]: KV[dk][dv] then z[dk]
+constexpr int kSmCount = 148;          // SMs of a B200
 constexpr int kTargetCtas = 296;       // 2 resident CTAs on each of the 148 SMs of a B200
 constexpr int kReduceRows = 64;        // token rows per reduce pipeline stage
 constexpr int kApplyRows = 128;        // token rows per apply tile (= MMA M)
@@ -112,7 +113,19 @@ int launch_finish_ranks(const float *gathered, int R, float *seff, void *bop, fl
 // Tensor-core path (bf16, H % 4 == 0): tcgen05 MMAs, TMA tiles.
 // The three kernels of a call (reduce, finish above, apply) order themselves
 // by grid through programmatic dependent launch.
-int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &p, cudaStream_t s);
+// The state combine done by the reduce itself (one block per call, P <= 8):
+// the P splits of a head group run as one cluster, add their split sums
+// through distributed shared memory in split order, and write S_eff, the
+// packed operand and (commit) the state, as launch_finish does.
+struct Fuse {
+    float *seff;
+    unsigned char *bop;
+    float *S, *Z;
+    int on, write_bop;
+};
+constexpr int kFuseMaxSplits = 8;
+int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &p, cudaStream_t s,
+                     const Fuse *fz = nullptr);
 int launch_apply_tc(const void *q, void *out, const void *bop, const float *seff, const Plan &p,
                     cudaStream_t s);
 bool tc_available();
@@ -178,6 +191,27 @@ bool launch_pdl(void (*kernel)(KArgs...), unsigned grid, int threads, int smem, 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess;
+}
+
+// The same, launched as clusters of `cluster` consecutive CTAs (portable sizes: <= 8).
+template <typename... KArgs, typename... Args>
+bool launch_pdl_cluster(void (*kernel)(KArgs...), unsigned grid, int threads, int smem, unsigned cluster,
+                        cudaStream_t s, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess;
 }
 
