@@ -1023,6 +1023,16 @@ bool make_bf16_map(CUtensorMap *m, const void *base, int B, int N, int H, int bo
     return make_map(m, base, B, N, H, box_rows);
 }
 
+bool make_bf16_map_nd(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims,
+                      const cuuint64_t *strides, const cuuint32_t *box) {
+    auto fn = encode_fn();
+    if (!fn || rank < 1 || rank > 5) return false;
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool tc_rope_fits(const Plan &p) {
     return rope_table_entries(p, p.chunk) <= kTabMax && rope_table_entries(p, p.chunka) <= kTabMax;
 }

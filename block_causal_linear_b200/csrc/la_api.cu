@@ -455,11 +455,13 @@ la_status la_block_apply(const void *q, void *out, la_dtype dt, int B, int N_sli
 }
 
 la_status la_device_status(void *stream) {
-    unsigned flag = 0, fk = 0, fq = 0;
+    unsigned flag = 0, fk = 0, fq = 0, fc = 0;
     // (synchronises the stream first)
     if (la::read_and_clear_device_flag(static_cast<cudaStream_t>(stream), &flag) != 0) return LA_ECUDA;
-    if (la::read_and_clear_bwd_k_flag(&fk) != 0 || la::read_and_clear_bwd_q_flag(&fq) != 0) return LA_ECUDA;
-    return (flag | fk | fq) ? LA_ETIMEOUT : LA_OK;
+    if (la::read_and_clear_bwd_k_flag(&fk) != 0 || la::read_and_clear_bwd_q_flag(&fq) != 0 ||
+        la::read_and_clear_conv_flag(&fc) != 0)
+        return LA_ECUDA;
+    return (flag | fk | fq | fc) ? LA_ETIMEOUT : LA_OK;
 }
 
 const char *la_status_string(la_status s) {

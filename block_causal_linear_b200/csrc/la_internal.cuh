@@ -223,6 +223,11 @@ inline bool set_smem(const void *kernel, int bytes) {
 // tokens, 128-byte swizzle.
 bool make_bf16_map(CUtensorMap *m, const void *base, int B, int N, int H, int box_rows);
 
+// A rank-dimensional TMA map of a bf16 tensor (dims innermost first, byte
+// strides of dims 1.., box extents), no swizzle, zero fill out of range.
+bool make_bf16_map_nd(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims,
+                      const cuuint64_t *strides, const cuuint32_t *box);
+
 // Query side on the tensor cores (bf16, H % 4 == 0, no RoPE): its own split
 // plan (one CTA per SM), dq and the split sums of [dS | dZ] from q, dout, the
 // state S_eff (seff) and its packed operand [S|Z|0] (bop), which also gives S^T.
@@ -232,6 +237,7 @@ int launch_bwd_q_tc(const void *q, const void *dout, void *dq, const float *seff
                     const Plan &p, cudaStream_t s);
 int read_and_clear_bwd_k_flag(unsigned *flag_out);
 int read_and_clear_bwd_q_flag(unsigned *flag_out);
+int read_and_clear_conv_flag(unsigned *flag_out);
 
 // Device flag raised by a bounded wait that gave up; read-and-clear.
 int read_and_clear_device_flag(cudaStream_t s, unsigned *flag_out);

@@ -1,6 +1,6 @@
 """GPU parity of the Mix-FFN depthwise convolution (la_dwconv3d) against the
 fp64 oracle: both kernel shapes (1x3x3 spatial, 3x1x1 temporal), bf16 and fp32,
-ragged grids, with and without bias, element by element (fp32: per-element
+ragged grids, tiled and untiled TMA shapes, with and without bias, element by element (fp32: per-element
 relative 1e-4 with an RMS floor; bf16: max error / RMS 2e-2); a full-size
 latent grid checked on sampled channels; bitwise determinism."""
 import numpy as np
@@ -39,6 +39,11 @@ CASES = [  # shape [B, T, Hg, Wg, C], kernel, dtype, bias
     ((1, 7, 4, 5, 2056), (3, 1, 1), torch.float32, True),
     ((1, 2, 1, 1, 16), (1, 3, 3), torch.float32, True),          # 1x1 frames: only the centre tap
     ((1, 1, 6, 6, 16), (3, 1, 1), torch.bfloat16, True),         # one frame: only the centre tap
+    # bf16 with C >= 64 runs on TMA tiles (64 channels, halo zero-filled by the copy):
+    ((2, 7, 4, 5, 2056), (3, 1, 1), torch.bfloat16, True),      # ragged last channel tile, two batches
+    ((2, 3, 300, 5, 64), (1, 3, 3), torch.bfloat16, True),      # frame split into row tiles
+    ((1, 2, 3, 300, 128), (1, 3, 3), torch.bfloat16, False),    # rows split into column tiles
+    ((2, 300, 2, 40, 64), (3, 1, 1), torch.bfloat16, True),     # frame tiles and column tiles
 ]
 
 
