@@ -187,17 +187,6 @@ constexpr int kTThreads = 256;
 constexpr int kTSmemMax = 96 * 1024;   // tile budget: two CTAs per SM
 constexpr int kTSeg = 8;            // outputs one thread slides through
 
-// Two fp32 fused multiply-adds in one instruction (each lane rounded as fmaf).
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
-
 // 8 bf16 channels from shared memory as 4 fp32 pairs (channels 2m, 2m + 1).
 __device__ __forceinline__ void lds8x2(const uint8_t *p, float2 (&v)[4]) {
     const uint4 u = *reinterpret_cast<const uint4 *>(p);
