@@ -300,10 +300,12 @@ LA_API const char *la_status_string(la_status s);
  * created on the current device), every following forward call records
  * before_reduce before its first kernel, after_reduce after the state
  * reduction, after_finish after the state combine and after_apply after its
- * last kernel, all on its stream.  la_full_backward records the same four
- * events before its first kernel, after the forward state (reduction and
- * combine), after the query side (dq and the state-gradient sums) and after
- * the key side (suffix sums, dk, dv).  Pass four NULLs to stop.
+ * last kernel, all on its stream (when the reduction combines its own splits,
+ * after_reduce and after_finish are recorded back to back).  la_full_backward
+ * records the same four events before its first kernel, after the forward
+ * state (reduction and combine), after the query side (dq and the
+ * state-gradient sums) and after the key side (suffix sums, dk, dv).  Pass
+ * four NULLs to stop.
  * Process-global; not thread-safe.  Changes no result.
  */
 LA_API void la_set_stage_events(void *before_reduce, void *after_reduce, void *after_finish,
