@@ -1084,6 +1084,27 @@ int launch_apply_tc(const void *q, void *out, const void *bop, const float *seff
     return ok ? 1 : -1;
 }
 
+namespace {
+// One CTA waits on an mbarrier that nothing arrives at: the bounded wait gives
+// up after its time limit, raises the device flag and the kernel returns.
+__global__ void bounded_wait_selftest_kernel() {
+    __shared__ uint64_t bar;
+    __shared__ int abort_word;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_word = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, &abort_word, &g_wait_flag, 99);
+}
+}  // namespace
+
+int launch_bounded_wait_selftest(cudaStream_t s) {
+    bounded_wait_selftest_kernel<<<1, 32, 0, s>>>();
+    return cudaGetLastError() == cudaSuccess ? 1 : -1;
+}
+
 int read_and_clear_device_flag(cudaStream_t s, unsigned *flag_out) {
     unsigned zero = 0;
     if (cudaStreamSynchronize(s) != cudaSuccess) return -1;

@@ -464,6 +464,10 @@ la_status la_device_status(void *stream) {
     return (flag | fk | fq | fc) ? LA_ETIMEOUT : LA_OK;
 }
 
+la_status la_selftest_bounded_wait(void *stream) {
+    return la::launch_bounded_wait_selftest(static_cast<cudaStream_t>(stream)) < 0 ? LA_ECUDA : LA_OK;
+}
+
 const char *la_status_string(la_status s) {
     switch (s) {
         case LA_OK: return "LA_OK";

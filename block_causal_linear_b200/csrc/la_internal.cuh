@@ -238,6 +238,7 @@ int launch_bwd_q_tc(const void *q, const void *dout, void *dq, const float *seff
 int read_and_clear_bwd_k_flag(unsigned *flag_out);
 int read_and_clear_bwd_q_flag(unsigned *flag_out);
 int read_and_clear_conv_flag(unsigned *flag_out);
+int launch_bounded_wait_selftest(cudaStream_t s);
 
 // Device flag raised by a bounded wait that gave up; read-and-clear.
 int read_and_clear_device_flag(cudaStream_t s, unsigned *flag_out);

@@ -89,6 +89,8 @@ def lib() -> ctypes.CDLL:
         L.la_full_backward.restype = ip
         L.la_device_status.argtypes = [vp]
         L.la_device_status.restype = ip
+        L.la_selftest_bounded_wait.argtypes = [vp]
+        L.la_selftest_bounded_wait.restype = ip
         L.la_status_string.argtypes = [ip]
         L.la_status_string.restype = ctypes.c_char_p
         L.la_set_stage_events.argtypes = [vp, vp, vp, vp]
@@ -415,6 +417,14 @@ def full_backward(q, k, v, dout, tokens_per_block=0, rope: Optional[la_rope] = N
     if rc != LA_OK:
         raise LAError(rc, "la_full_backward")
     return dq, dk, dv
+
+
+def selftest_bounded_wait(stream=None) -> None:
+    """Enqueue the bounded-wait self-test kernel (la_selftest_bounded_wait):
+    the next device_status raises LAError(LA_ETIMEOUT)."""
+    rc = lib().la_selftest_bounded_wait(_stream_ptr(stream))
+    if rc != LA_OK:
+        raise LAError(rc, "la_selftest_bounded_wait")
 
 
 def device_status(stream=None) -> None:

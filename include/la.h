@@ -292,6 +292,16 @@ LA_API la_status la_full_forward_static_ws(const void *q, const void *k, const v
  */
 LA_API la_status la_device_status(void *stream);
 
+/*
+ * Self-test of the bounded waits: enqueues on `stream` one small kernel whose
+ * wait on a barrier that nothing arrives at gives up after the waits' time
+ * limit (2 s) and raises the device flag, as a kernel's wait would after a
+ * lost copy or a stalled partner.  The following la_device_status returns
+ * LA_ETIMEOUT (and clears the flag).  No fault, no trap, the context stays
+ * usable.  Returns LA_ECUDA if the launch failed, else LA_OK.
+ */
+LA_API la_status la_selftest_bounded_wait(void *stream);
+
 /* Static, human-readable name of a status. */
 LA_API const char *la_status_string(la_status s);
 
