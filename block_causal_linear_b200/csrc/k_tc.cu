@@ -157,7 +157,7 @@ static_assert(kRRows == 32, "the ReLU pass below maps 128 threads x 4 chunks ont
 // 4 heads' 128 codes of 32 tokens (4 KiB), and the MMAs are kind::f8f6f4.
 template <bool ROPE, bool F8 = false>
 struct RCfg {
-    static constexpr int kStages = F8 ? 12 : (ROPE ? 4 : 4);
+    static constexpr int kStages = F8 ? 6 : 4;   // 6 x 8 KiB with FP8 codes, 4 x 16 (24 with RoPE) KiB with bf16
     // stage: k boxes (becoming R phi(k) hi with RoPE), [lo boxes], v boxes
     static constexpr int kLoOff = 2 * kRBox;
     static constexpr int kVOff = F8 ? kRRows * 128 : (ROPE ? 4 * kRBox : 2 * kRBox);
