@@ -34,7 +34,9 @@ def decoded(orc, qkv):
     return [orc.e4m3_decode(c, s) for c, s in qkv]
 
 
-@pytest.mark.parametrize("B,N,H,L", [(1, 517, 4, 0), (2, 300, 8, 128), (1, 1000, 12, 250), (1, 4099, 64, 0)])
+# (2, 300, 8, 0): one block of 5 splits per head group, combined inside the reduce (a cluster)
+@pytest.mark.parametrize("B,N,H,L", [(1, 517, 4, 0), (2, 300, 8, 128), (1, 1000, 12, 250), (1, 4099, 64, 0),
+                                     (2, 300, 8, 0)])
 def test_full_forward_e4m3_matches_oracle(la, orc, B, N, H, L):
     qkv = fp8_inputs(B, N, H, seed=60 + N)
     codes = [c.cuda() for c, _ in qkv]
