@@ -164,6 +164,43 @@ def to_e4m3(x: torch.Tensor):
     return codes, scale
 
 
+_E2M1_GRID = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)   # magnitudes of E2M1 codes 0..7
+
+
+def to_nvfp4(x: torch.Tensor):
+    """NVFP4 inputs (two-level scaling, the usual recipe): a per-tensor fp32
+    scale s = max|x| / (6 * 448); per 16 consecutive elements of the last axis
+    an E4M3 block scale, max|block| / 6 / s rounded to nearest even E4M3; each
+    element x / (s * block scale) rounded to the nearest E2M1 value (ties to
+    the even code), saturated at 6.  Returns (uint8 codes [..., d/2] with
+    element 2i in the low nibble, uint8 block scales [..., d/16], s).  Input
+    preparation only."""
+    d = x.shape[-1]
+    if d % 16:
+        raise ValueError("the last axis must be a multiple of 16")
+    xf = x.to(torch.float64)
+    amax = float(xf.abs().max()) if xf.numel() else 0.0
+    s = float(torch.tensor(amax / (6.0 * 448.0) if amax > 0 else 1.0, dtype=torch.float32))
+    blocks = xf.reshape(*xf.shape[:-1], d // 16, 16)
+    bmax = blocks.abs().amax(dim=-1)
+    sf = (bmax / 6.0 / s).to(torch.float32).clamp(max=448.0).to(torch.float8_e4m3fn)
+    sfv = sf.to(torch.float64)
+    denom = (sfv * s).unsqueeze(-1)
+    y = torch.where(denom > 0, blocks / torch.where(denom > 0, denom, torch.ones_like(denom)),
+                    torch.zeros_like(blocks))
+    mag = y.abs().clamp(max=6.0)
+    grid = torch.tensor(_E2M1_GRID, dtype=torch.float64, device=x.device)
+    up = torch.searchsorted(grid, mag.contiguous(), right=False).clamp(max=7)   # first grid value >= mag
+    lo = (up - 1).clamp(min=0)
+    dl, du = mag - grid[lo], grid[up] - mag
+    pick_up = (du < dl) | ((du == dl) & (up % 2 == 0))
+    code = torch.where(pick_up, up, lo)
+    code = code | torch.where((y < 0) & (code > 0), 8, 0)
+    code = code.reshape(*xf.shape[:-1], d).to(torch.uint8)
+    packed = code[..., 0::2] | (code[..., 1::2] << 4)
+    return packed.contiguous(), sf.view(torch.uint8).contiguous(), s
+
+
 def random_qkv(B, N, H, d, seed, dtype=torch.float32, device="cpu", scale=1.0, bias=0.0):
     """Free-form seeded draw for edge-case tests (same recipe, any shape):
     fp64 normal draws rounded to fp32, then converted to ``dtype``."""

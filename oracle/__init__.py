@@ -231,6 +231,39 @@ def e4m3_decode(codes: torch.Tensor, scale: float = 1.0) -> torch.Tensor:
     return sign * mag * float(scale)
 
 
+def e2m1_decode(codes: torch.Tensor) -> torch.Tensor:
+    """fp64 values of FP4 E2M1 codes (integers 0..15, one code per element).
+
+    The format (OCP Microscaling Formats, FP4 E2M1 element type): bit 3 the
+    sign, bits 2..1 the exponent with bias 1, bit 0 the mantissa; exponent
+    field 0 encodes the subnormals m * 0.5 (0 and 0.5); no infinity, no NaN,
+    so the magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6."""
+    c = codes.to(torch.int64)
+    sign = torch.where((c & 8) != 0, -1.0, 1.0).to(torch.float64)
+    e = (c >> 1) & 3
+    m = (c & 1).to(torch.float64)
+    normal = (1.0 + m / 2.0) * torch.pow(torch.tensor(2.0, dtype=torch.float64), (e - 1).to(torch.float64))
+    mag = torch.where(e == 0, m * 0.5, normal)
+    return sign * mag
+
+
+def nvfp4_decode(codes: torch.Tensor, block_scales: torch.Tensor, scale: float = 1.0) -> torch.Tensor:
+    """fp64 values of an NVFP4 tensor: ``codes`` uint8 [..., d/2] holding two
+    E2M1 codes per byte (element 2i in the low nibble, 2i+1 in the high
+    nibble), ``block_scales`` uint8 [..., d/16] holding one E4M3 scale per 16
+    consecutive elements of the last axis, and one fp32 per-tensor scale:
+        x[..., i] = e2m1(code i) * e4m3(block_scales[..., i // 16]) * scale.
+    Every such product is exact in fp64 (2 + 4 + 24 significant bits)."""
+    c = codes.to(torch.int64)
+    lo, hi = c & 15, (c >> 4) & 15
+    elems = torch.stack((lo, hi), dim=-1).reshape(*c.shape[:-1], 2 * c.shape[-1])
+    d = elems.shape[-1]
+    if block_scales.shape[-1] * 16 != d or block_scales.shape[:-1] != codes.shape[:-1]:
+        raise ValueError("block_scales must be [..., d/16] for codes [..., d/2]")
+    sf = e4m3_decode(block_scales).repeat_interleave(16, dim=-1)
+    return e2m1_decode(elems) * sf * float(scale)
+
+
 def dwconv3d(x, weight, bias=None):
     """Depthwise 3D convolution (Mix-FFN): x [B, T, Hg, Wg, C] (fp64/fp32/bf16
     CPU tensor), weight [C, kt, kh, kw], bias [C] or None; zero padding of
