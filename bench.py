@@ -67,8 +67,10 @@ def parse():
     ap.add_argument("--op", default="attention", choices=["attention", "dwconv"],
                     help="dwconv: the Mix-FFN depthwise convolutions (1x3x3 then 3x1x1) on the workload's "
                          "latent grid, DWCONV_C channels")
-    ap.add_argument("--input", default="native", choices=["native", "e4m3"],
-                    help="e4m3: q, k, v as FP8 E4M3 codes with per-tensor scales (la_*_forward_e4m3), bf16 out")
+    ap.add_argument("--input", default="native", choices=["native", "e4m3", "nvfp4"],
+                    help="e4m3: q, k, v as FP8 E4M3 codes with per-tensor scales (la_*_forward_e4m3); nvfp4: "
+                         "E2M1 codes with an E4M3 scale per 16 features and a per-tensor scale "
+                         "(la_*_forward_nvfp4); bf16 out")
     ap.add_argument("--blocks", type=int, default=None,
                     help="streaming workloads: run only the first N blocks (small cases for profiling)")
     ap.add_argument("--shard", default="problem", choices=["problem", "heads"],
@@ -417,9 +419,10 @@ def main():
         w = w.shrink(n_blocks=args.blocks)
     bwd = args.pass_ == "backward"
     f8 = args.input == "e4m3"
-    if f8 and bwd:
-        raise SystemExit("--input e4m3 is a forward path")
-    runner = BackwardRunner(w, dev) if bwd else Runner(w, dev, e4m3=f8)
+    f4 = args.input == "nvfp4"
+    if (f8 or f4) and bwd:
+        raise SystemExit(f"--input {args.input} is a forward path")
+    runner = BackwardRunner(w, dev) if bwd else Runner(w, dev, e4m3=f8, nvfp4=f4)
     w = runner.w
     flush_w = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -541,9 +544,12 @@ def main():
     peak, peak_kind = measured_peaks()
     # algorithmic bytes: forward reads q, k, v and writes out (4 tensors);
     # backward reads q, k, v, dout and writes dq, dk, dv (7 tensors)
-    # E4M3 forward: q, k, v one byte per feature, out bf16
+    # E4M3 forward: q, k, v one byte per feature, out bf16; NVFP4 forward: q,
+    # k, v half a byte per feature plus one scale byte per 16 features, out bf16
     if f8:
         alg_bytes = w.token_heads * w.d * (3 * 1 + 2) + (w.alg_bytes - w.token_heads * 4 * w.d * w.elem_bytes)
+    elif f4:
+        alg_bytes = w.token_heads * (3 * (w.d // 2 + w.d // 16) + 2 * w.d)
     else:
         alg_bytes = w.token_heads * (7 if bwd else 4) * w.d * w.elem_bytes if bwd else w.alg_bytes
     step_gbs = alg_bytes / (ms_per_step / 1e3) / 1e9
@@ -564,6 +570,9 @@ def main():
         kname = f"{dom}_{path}" + ("_rope" if w.rope and path == "tc" else "")
     if f8:   # reduce: k, v codes; apply: q codes and bf16 out
         kern_bytes = per_call_th * w.d * (2 if dom == "reduce" else 3)
+    elif f4:   # reduce: k, v codes and block scales; apply: q codes and scales, bf16 out
+        per_t = w.d // 2 + w.d // 16
+        kern_bytes = per_call_th * (2 * per_t if dom == "reduce" else per_t + 2 * w.d)
     else:
         kern_bytes = per_call_th * ntens * w.d * w.elem_bytes
     avg_launch_s = dom_ms / launches_per_kernel / 1e3
@@ -586,8 +595,12 @@ def main():
             "metric": METRIC_BWD if bwd else METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "strong" if args.shard == "heads" else "weak", "vs_baseline": None,
-            "dtype": "e4m3 in, bf16 out" if f8 else ("bf16" if w.dtype == "bf16" else "f32"), "data": "synthetic",
-            "config": workload_config(w, {"pass": args.pass_, "input_dtype": "e4m3 (per-tensor scale)" if f8 else w.dtype,
+            "dtype": ("e4m3 in, bf16 out" if f8 else "nvfp4 in, bf16 out" if f4 else
+                      ("bf16" if w.dtype == "bf16" else "f32")), "data": "synthetic",
+            "config": workload_config(w, {"pass": args.pass_,
+                                          "input_dtype": ("e4m3 (per-tensor scale)" if f8 else
+                                                          "nvfp4 (e2m1, e4m3 scale per 16, per-tensor scale)" if f4
+                                                          else w.dtype),
                                           "parallelism": (f"heads of one problem split over {world} ranks"
                                                           if args.shard == "heads" else
                                                           f"independent problem per rank x{world}")}),

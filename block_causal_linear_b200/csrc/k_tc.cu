@@ -31,6 +31,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
@@ -147,6 +148,43 @@ __device__ __forceinline__ void relu_rotate_chunk(uint4 x, const RowCS &cs, uint
     rotate_pair(x.w, cs.c3, f[6], f[7], hi.w, lo.w);
 }
 
+// ---------------------------------------------------------------- NVFP4
+// ReLU on 8 packed E2M1 codes: a code with its sign bit (bit 3 of the nibble)
+// set is negative or -0, and becomes +0.
+__device__ __forceinline__ uint32_t relu_e2m1x8(uint32_t w) {
+    const uint32_t neg = (w >> 3) & 0x11111111u;
+    return w & ~(neg * 15u);
+}
+
+// 16 E2M1 codes (8 bytes, element 2i in the low nibble) times their E4M3 block
+// scale, as 16 f16 (features 0-7 in `a`, 8-15 in `b`).  Exact: a code value
+// has 2 significant bits and a scale 4, so every product (0 or 2^-10 .. 2688)
+// is an f16.
+__device__ __forceinline__ void decode_nvfp4_16(uint2 c, uint8_t sf, uint4 &a, uint4 &b) {
+    const __half2 s2 = __half2half2(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)sf, __NV_E4M3)));
+    uint32_t o[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const uint32_t w = m < 4 ? c.x : c.y;
+        const __nv_fp4x2_storage_t pair = (__nv_fp4x2_storage_t)((w >> (8 * (m & 3))) & 0xFFu);
+        const __half2 h = __hmul2(__half2(__nv_cvt_fp4x2_to_halfraw2(pair, __NV_E2M1)), s2);
+        o[m] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    a = make_uint4(o[0], o[1], o[2], o[3]);
+    b = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// 8 f16 -> 8 bf16, for values with at most 8 significant bits (exact).
+__device__ __forceinline__ uint4 f16x8_to_bf16x8(uint4 h) {
+    uint32_t w[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[m]));
+        w[m] = pack_bf2(f.x, f.y);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // ================================================================ reduce
 
 constexpr int kRRows = 32;                 // token rows per reduce pipeline stage
@@ -155,23 +193,41 @@ static_assert(kRRows == 32, "the ReLU pass below maps 128 threads x 4 chunks ont
 
 // F8: k and v are FP8 E4M3 codes; one TMA box per tensor and stage holds the
 // 4 heads' 128 codes of 32 tokens (4 KiB), and the MMAs are kind::f8f6f4.
-template <bool ROPE, bool F8 = false>
+// F4: k and v are NVFP4; a raw stage holds the 4 heads' E2M1 codes of 32
+// tokens (2 KiB per tensor, 64 bytes a row) and their E4M3 block scales (a
+// 16-byte box per row, of which the group's 8 bytes are used); the transform
+// warps decode them into f16 boxes laid out as the bf16 path's tiles (a ring
+// of kDec decoded stages, shorter than the raw ring that covers the memory
+// latency), and the MMAs are kind::f16 on f16.
+template <bool ROPE, int IN = kInBf16>
 struct RCfg {
-    static constexpr int kStages = F8 ? 6 : 4;   // 6 x 8 KiB with FP8 codes, 4 x 16 (24 with RoPE) KiB with bf16
+    static constexpr bool F8 = IN == kInE4m3, F4 = IN == kInNvfp4;
+    // 6 x 8 KiB with FP8 codes, 4 x 16 (24 with RoPE) KiB with bf16, 8 x 5 KiB raw with NVFP4
+    static constexpr int kStages = F8 ? 6 : (F4 ? 8 : 4);
     // stage: k boxes (becoming R phi(k) hi with RoPE), [lo boxes], v boxes
     static constexpr int kLoOff = 2 * kRBox;
     static constexpr int kVOff = F8 ? kRRows * 128 : (ROPE ? 4 * kRBox : 2 * kRBox);
-    static constexpr int kStageBytes = F8 ? 2 * kRRows * 128 : kVOff + 2 * kRBox;
-    static constexpr int kAuxOff = kStages * kStageBytes;          // ones (512 B) or RoPE table
+    static constexpr int kStageBytes = F8 ? 2 * kRRows * 128 : (F4 ? 5 * 1024 : kVOff + 2 * kRBox);
+    // F4: decoded ring first (1024-byte aligned for the swizzled boxes), then the raw ring
+    static constexpr int kDec = F4 ? 3 : 0;
+    static constexpr int kDecBytes = 4 * kRBox;
+    static constexpr int kRawOff = kDec * kDecBytes;
+    static constexpr int kCodeBytes = kRRows * 64;                  // F4: one tensor's codes in a raw stage
+    static constexpr int kSfOff = 2 * kCodeBytes;                   // F4: k scales, then v scales (512 B each)
+    static constexpr int kRawTx = 2 * kCodeBytes + 2 * kRRows * 16;
+    static constexpr int kAuxOff = kRawOff + kStages * kStageBytes; // ones (512 B) or RoPE table
     static constexpr int kAuxBytes = ROPE ? kTabMax * 8 : 512;
     static constexpr int kBarOff = kAuxOff + kAuxBytes;
-    static constexpr int kSmem = kBarOff + (3 * kStages + 1) * 8 + 16 + 1024;
+    static constexpr int kNumBars = F4 ? 2 * kStages + 2 * kDec + 1 : 3 * kStages + 1;
+    static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
     static constexpr uint32_t kTmemCols = ROPE ? 128 : 256;
     // threads that transform the k boxes (warps 2..): RoPE has 8 such warps,
     // one token row per thread and stage, to hide the latency of its longer
-    // per-chunk work; without RoPE 4 warps, 4 chunks per thread
-    static constexpr int kXform = ROPE ? 256 : 128;
+    // per-chunk work; NVFP4 8 warps, one 16-feature block of k and one of v per
+    // thread and stage; otherwise 4 warps, 4 chunks per thread
+    static constexpr int kXform = (ROPE || F4) ? 256 : 128;
     static constexpr int kThreadsR = 64 + kXform;
+    static_assert(!F4 || kStageBytes >= kRawTx, "the raw stage holds codes and scales");
 };
 
 // Fused state combine: the split sums of the CTA's 4 heads ([4][kKVZ] fp32)
@@ -232,23 +288,29 @@ __device__ void fused_combine(const Plan &p, const Fuse &fz, const float *part, 
     }
 }
 
-template <bool ROPE, bool F8 = false>
-__global__ void __launch_bounds__(RCfg<ROPE, F8>::kThreadsR, 2)
+// tm_ks, tm_vs: the NVFP4 block scales of k and v (unused otherwise).
+template <bool ROPE, int IN = kInBf16>
+__global__ void __launch_bounds__(RCfg<ROPE, IN>::kThreadsR, 2)
 reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                 const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                  float *__restrict__ partials, const Plan p, const Fuse fz) {
-    static_assert(!(ROPE && F8), "FP8 inputs take no RoPE");
-    using C = RCfg<ROPE, F8>;
+    constexpr bool F8 = IN == kInE4m3, F4 = IN == kInNvfp4;
+    static_assert(!(ROPE && (F8 || F4)), "FP8 and NVFP4 inputs take no RoPE");
+    using C = RCfg<ROPE, IN>;
     static_assert(C::kXform * 16 * 4 <= kFusePartOff &&
                       kFusePartOff + 4 * kKVZ * 4 <= C::kStages * C::kStageBytes,
                   "the fused split sums sit past the z scratch, inside the stages");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     uint8_t *aux = smem + C::kAuxOff;
+    // F4: full / raw_free guard the raw ring, relu_done / empty the decoded ring
+    constexpr int kRing = F4 ? C::kDec : C::kStages;   // stages the MMAs read
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
     uint64_t *relu_done = full + C::kStages;
-    uint64_t *empty = relu_done + C::kStages;
-    uint64_t *acc_ready = empty + C::kStages;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_ready + 1);
+    uint64_t *empty = relu_done + kRing;
+    uint64_t *acc_ready = empty + kRing;
+    uint64_t *raw_free = acc_ready + 1;   // F4 only: [kStages], the raw stage has been decoded
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kBarOff + C::kNumBars * 8);
     volatile int *abort_word = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     // the splits of a head group are consecutive CTAs (one cluster when fused)
@@ -292,11 +354,13 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     const int nf = ROPE ? (int)((t1 - 1) / hw) - f_lo + 1 : 0;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&full[s], 1);
+        for (int s = 0; s < C::kStages; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < kRing; ++s) {
             mbar_init(&relu_done[s], C::kXform);
             mbar_init(&empty[s], 1);
         }
+        if constexpr (F4)
+            for (int s = 0; s < C::kStages; ++s) mbar_init(&raw_free[s], C::kXform);
         mbar_init(acc_ready, 1);
         *abort_word = 0;
         fence_barrier_init();
@@ -304,10 +368,10 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     if constexpr (ROPE) {
         build_rope_table(reinterpret_cast<float2 *>(aux), p, f_lo, nf, threadIdx.x, C::kThreadsR);
     } else {
-        // B operand of the z contraction: 16 x 16 bf16 ones (any layout reads 1.0)
-        // (1.0 is 0x3F80 in bf16, 0x38 in E4M3)
+        // B operand of the z contraction: 16 x 16 ones (any layout reads 1.0)
+        // (1.0 is 0x3F80 in bf16, 0x38 in E4M3, 0x3C00 in f16)
         for (int i = threadIdx.x; i < 128; i += C::kThreadsR)
-            reinterpret_cast<uint32_t *>(aux)[i] = F8 ? 0x38383838u : 0x3F803F80u;
+            reinterpret_cast<uint32_t *>(aux)[i] = F8 ? 0x38383838u : (F4 ? 0x3C003C00u : 0x3F803F80u);
     }
     if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, C::kTmemCols);
@@ -316,6 +380,10 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     if (warp == kWarpTma && lane == 0) {
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
+        if constexpr (F4) {
+            prefetch_tmap(&tm_ks);
+            prefetch_tmap(&tm_vs);
+        }
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -330,10 +398,18 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             for (int i = 0; i < nst; ++i) {
                 const int s = i % C::kStages;
                 const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
-                if (!mbar_wait(&empty[s], ph ^ 1u, abort_word, &g_wait_flag, 1)) break;
-                uint8_t *st = smem + s * C::kStageBytes;
+                if (!mbar_wait(F4 ? &raw_free[s] : &empty[s], ph ^ 1u, abort_word, &g_wait_flag, 1)) break;
+                uint8_t *st = smem + C::kRawOff + s * C::kStageBytes;
                 const int row = (int)(t0 + (long long)kRRows * i);
-                if constexpr (F8) {
+                if constexpr (F4) {
+                    // codes: the group's 4 x 16 bytes of a row; scales: the 16-byte
+                    // aligned box holding the group's 8 bytes
+                    mbar_arrive_expect_tx(&full[s], C::kRawTx);
+                    tma_load_3d(st, &tm_k, &full[s], g * 64, row, b);
+                    tma_load_3d(st + C::kCodeBytes, &tm_v, &full[s], g * 64, row, b);
+                    tma_load_3d(st + C::kSfOff, &tm_ks, &full[s], (g >> 1) * 16, row, b);
+                    tma_load_3d(st + C::kSfOff + kRRows * 16, &tm_vs, &full[s], (g >> 1) * 16, row, b);
+                } else if constexpr (F8) {
                     mbar_arrive_expect_tx(&full[s], C::kStageBytes);
                     tma_load_3d(st, &tm_k, &full[s], c0, row, b);
                     tma_load_3d(st + C::kVOff, &tm_v, &full[s], c0, row, b);
@@ -349,16 +425,16 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
     } else if (warp == kWarpMma) {
         if (lane == 0) {
-            const uint32_t id_kv = F8 ? idesc_e4m3(128, 128, 1, 1) : idesc_bf16(128, 128, 1, 1);
-            const uint32_t id_z = F8 ? idesc_e4m3(128, 16, 1, 0) : idesc_bf16(128, 16, 1, 0);
+            const uint32_t id_kv = F8 ? idesc_e4m3(128, 128, 1, 1) : (F4 ? idesc_f16(128, 128, 1, 1) : idesc_bf16(128, 128, 1, 1));
+            const uint32_t id_z = F8 ? idesc_e4m3(128, 16, 1, 0) : (F4 ? idesc_f16(128, 16, 1, 0) : idesc_bf16(128, 16, 1, 0));
             // ones: K-major, no swizzle, 32 bytes of K per row either way
             const uint64_t d_ones = smem_desc(smem_u32(aux), 128, 256, kLayoutNone);
             for (int i = 0; i < nst; ++i) {
-                const int s = i % C::kStages;
-                const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
+                const int s = i % kRing;
+                const uint32_t ph = (uint32_t)(i / kRing) & 1u;
                 if (!mbar_wait(&relu_done[s], ph, abort_word, &g_wait_flag, 2)) break;
                 tc_fence_after();
-                const uint32_t kaddr = smem_u32(smem + s * C::kStageBytes);
+                const uint32_t kaddr = smem_u32(smem + s * (F4 ? C::kDecBytes : C::kStageBytes));
                 const uint32_t vaddr = kaddr + C::kVOff;
                 if constexpr (F8) {
                     // MN-major, 128-byte swizzle: the 128 codes of a token are one
@@ -408,9 +484,38 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             const int s = i % C::kStages;
             const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
             if (!mbar_wait(&full[s], ph, abort_word, &g_wait_flag, 3)) break;
-            uint8_t *kt = smem + s * C::kStageBytes;
+            const int ds = F4 ? i % kRing : s;   // the stage the MMAs read
+            uint8_t *kt = smem + (F4 ? ds * C::kDecBytes : s * C::kStageBytes);
             const long long row0 = t0 + (long long)kRRows * i;
-            if constexpr (ROPE) {
+            if constexpr (F4) {
+                // the decoded stage is free once the MMAs of stage i - kDec are done
+                if (!mbar_wait(&empty[ds], ((uint32_t)(i / kRing) & 1u) ^ 1u, abort_word, &g_wait_flag, 5)) break;
+                const uint8_t *raw = smem + C::kRawOff + s * C::kStageBytes;
+                // this thread: block u of k and of v, u = (row, head, 16-feature half)
+                const int u = wt;
+                const int r = u >> 3, hd = (u >> 1) & 3, fb = u & 1;
+                const int L0 = (hd & 1) * 4 + fb * 2;   // logical chunks L0, L0 + 1 of box hd / 2
+                uint8_t *drow = kt + (hd >> 1) * kRBox + r * 128;
+                const int p0 = (L0 ^ (r & 7)) << 4, p1 = ((L0 + 1) ^ (r & 7)) << 4;
+                const int cb = r * 64 + hd * 16 + fb * 8;                        // code bytes in the raw boxes
+                const int sb = C::kSfOff + r * 16 + (g & 1) * 8 + hd * 2 + fb;   // scale byte
+                uint2 ck = *reinterpret_cast<const uint2 *>(raw + cb);
+                const uint2 cv = *reinterpret_cast<const uint2 *>(raw + C::kCodeBytes + cb);
+                const uint8_t sk = raw[sb], sv = raw[sb + kRRows * 16];
+                if (row0 + r < t1) {
+                    ck.x = relu_e2m1x8(ck.x);
+                    ck.y = relu_e2m1x8(ck.y);
+                } else {
+                    ck = make_uint2(0u, 0u);   // rows past the split contribute nothing
+                }
+                uint4 a, bq;
+                decode_nvfp4_16(ck, sk, a, bq);
+                *reinterpret_cast<uint4 *>(drow + p0) = a;
+                *reinterpret_cast<uint4 *>(drow + p1) = bq;
+                decode_nvfp4_16(cv, sv, a, bq);
+                *reinterpret_cast<uint4 *>(drow + C::kVOff + p0) = a;
+                *reinterpret_cast<uint4 *>(drow + C::kVOff + p1) = bq;
+            } else if constexpr (ROPE) {
                 // the thread's chunks: token row r (and r + 16 with 4 warps), each
                 // in both boxes (heads 0-1 and 2-3), all with the same 8 features,
                 // so one position and one set of cos/sin per row
@@ -467,8 +572,11 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     *ptr = x;
                 }
             }
+            // the generic reads and writes of this stage before the tensor cores
+            // read the decoded boxes and TMA refills the raw stage (async proxy)
             fence_proxy_async_smem();
-            mbar_arrive(&relu_done[s]);
+            if constexpr (F4) mbar_arrive(&raw_free[s]);
+            mbar_arrive(&relu_done[ds]);
         }
         // epilogue: warp quarter q reads TMEM lanes 32q.. = key features of head 4g+q.
         // Every work thread reaches the named barrier, and the TMEM read is
@@ -503,7 +611,7 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             tmem_ld32(tmem + lane_off + 32 * qd, kv);
             if constexpr (!ROPE) z = tmem_ld1(tmem + lane_off + 128);
             tmem_wait_ld();
-            if constexpr (F8) {
+            if constexpr (F8 || F4) {
                 // per-tensor scales: KV = sk sv sum phi(k^) v^T, z = sk sum phi(k^)
                 const float skv = p.sk * p.sv;
 #pragma unroll
@@ -548,13 +656,18 @@ constexpr int kAThreads = 320;                 // 10 warps
 constexpr int kAXform0 = 192;                  // first thread of the transform warps 6..9
 constexpr int kAWarpStg = 32 * 128;            // one epilogue warp's staging box: [32 rows][64 bf16]
 
-template <bool ROPE, bool F8 = false>
+template <bool ROPE, int IN = kInBf16>
 struct ACfg {
+    static constexpr bool F8 = IN == kInE4m3, F4 = IN == kInNvfp4;
     // F8: a stage is the bf16 tile the MMA reads (16 KiB, 128-byte swizzle)
-    // followed by the tile's E4M3 codes as TMA lands them (8 KiB, no swizzle)
-    static constexpr int kStages = F8 ? 3 : (ROPE ? 2 : 4);
+    // followed by the tile's E4M3 codes as TMA lands them (8 KiB, no swizzle).
+    // F4: the bf16 tile, the tile's E2M1 codes (4 KiB: 32 bytes a row) and
+    // the 16-byte box of E4M3 block scales of each row (2 KiB)
+    static constexpr int kStages = (F8 || F4) ? 3 : (ROPE ? 2 : 4);
     static constexpr int kCodeOff = kATile;
-    static constexpr int kStageBytes = F8 ? kATile + kATile / 2 : (ROPE ? 2 * kATile : kATile);
+    static constexpr int kSfOff = kATile + kATile / 4;   // F4
+    static constexpr int kQTx = F8 ? kATile / 2 : (F4 ? kATile / 4 + 128 * 16 : kATile);   // bytes TMA lands per tile
+    static constexpr int kStageBytes = F8 ? kATile + kATile / 2 : (F4 ? kSfOff + 128 * 16 : (ROPE ? 2 * kATile : kATile));
     static constexpr int kStgBufs = (ROPE || F8) ? 1 : 2;             // staging boxes per epilogue warp
     static constexpr int kOutOff = kStages * kStageBytes;
     static constexpr int kBopOff = kOutOff + 4 * kStgBufs * kAWarpStg;
@@ -573,13 +686,15 @@ struct ACfg {
 // epilogue (warp w reads TMEM lanes 32*(w%4).. = token rows of the tile),
 // 6..9 apply phi (and RoPE) to the q tiles in shared memory.  The transform
 // of tile i+1 and the epilogue of tile i run at the same time.
-template <bool ROPE, bool F8 = false>
+// tm_qs: the NVFP4 block scales of q (unused otherwise).
+template <bool ROPE, int IN = kInBf16>
 __global__ void __launch_bounds__(kAThreads, 2)
-apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_out,
-                __nv_bfloat16 *__restrict__ out, const uint8_t *__restrict__ bop, const float *__restrict__ seff,
-                const Plan p) {
-    static_assert(!(ROPE && F8), "FP8 inputs take no RoPE");
-    using C = ACfg<ROPE, F8>;
+apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qs,
+                const __grid_constant__ CUtensorMap tm_out, __nv_bfloat16 *__restrict__ out,
+                const uint8_t *__restrict__ bop, const float *__restrict__ seff, const Plan p) {
+    constexpr bool F8 = IN == kInE4m3, F4 = IN == kInNvfp4;
+    static_assert(!(ROPE && (F8 || F4)), "FP8 and NVFP4 inputs take no RoPE");
+    using C = ACfg<ROPE, IN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     uint8_t *stg = smem + C::kOutOff;
@@ -647,6 +762,7 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (warp == kWarpTma && lane == 0) {
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_out);
+        if constexpr (F4) prefetch_tmap(&tm_qs);
     }
     tc_fence_before();
     __syncthreads();
@@ -657,15 +773,23 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     if (warp == kWarpTma) {
         if (lane == 0) {
+            auto load_q = [&](int i, int s) {
+                uint8_t *st = smem + s * C::kStageBytes;
+                const int row = (int)(ta0 + 128LL * i);
+                mbar_arrive_expect_tx(&full[s], C::kQTx);
+                if constexpr (F4) {
+                    // the pair's 2 x 16 code bytes; the 16-byte aligned box holding its 4 scale bytes
+                    tma_load_3d(st + C::kCodeOff, &tm_q, &full[s], hp * 32, row, b);
+                    tma_load_3d(st + C::kSfOff, &tm_qs, &full[s], (hp >> 2) * 16, row, b);
+                } else {
+                    tma_load_3d(st + (F8 ? C::kCodeOff : 0), &tm_q, &full[s], hp * 64, row, b);
+                }
+                issued = i + 1;
+            };
             // q is an input of the call, complete before the reduce of this call
             // started: its first tiles are fetched while the state combine still runs
             const int pre = ntiles < C::kStages ? ntiles : C::kStages;
-            for (int i = 0; i < pre; ++i) {
-                mbar_arrive_expect_tx(&full[i], F8 ? kATile / 2 : kATile);
-                tma_load_3d(smem + i * C::kStageBytes + (F8 ? C::kCodeOff : 0), &tm_q, &full[i], hp * 64,
-                            (int)(ta0 + 128LL * i), b);
-                issued = i + 1;
-            }
+            for (int i = 0; i < pre; ++i) load_q(i, i);
             pdl_wait();   // the packed operand and Z_eff are written by the previous kernel
             mbar_arrive(dep_ready);
             mbar_arrive_expect_tx(bop_full, kABopBytes);
@@ -678,10 +802,7 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int s = i % C::kStages;
                 const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
                 if (!mbar_wait(&empty[s], ph ^ 1u, abort_word, &g_wait_flag, 11)) break;
-                mbar_arrive_expect_tx(&full[s], F8 ? kATile / 2 : kATile);
-                tma_load_3d(smem + s * C::kStageBytes + (F8 ? C::kCodeOff : 0), &tm_q, &full[s], hp * 64,
-                            (int)(ta0 + 128LL * i), b);
-                issued = i + 1;
+                load_q(i, s);
             }
         }
     } else if (warp == kWarpMma) {
@@ -801,6 +922,24 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         den_s[(i & 1) * 256 + rr * 2 + (h0 ^ 1)] = dp[1];
                     }
                 }
+            } else if (F4 && ok) {
+                // NVFP4 [128 rows][2 heads][32 codes] -> phi(q) in bf16, exact (<= 6
+                // significant bits), into the 128-byte swizzled tile the MMA reads:
+                // 4 blocks of 16 features per thread
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int u = tt + 128 * j;
+                    const int rr = u >> 2, hd = (u >> 1) & 1, fb = u & 1;
+                    uint2 c = *reinterpret_cast<const uint2 *>(qt + C::kCodeOff + rr * 32 + hd * 16 + fb * 8);
+                    const uint8_t sf = qt[C::kSfOff + rr * 16 + (hp & 3) * 4 + hd * 2 + fb];
+                    c.x = relu_e2m1x8(c.x);
+                    c.y = relu_e2m1x8(c.y);
+                    uint4 a, bq;
+                    decode_nvfp4_16(c, sf, a, bq);
+                    const int L0 = hd * 4 + fb * 2;
+                    *reinterpret_cast<uint4 *>(qt + rr * 128 + ((L0 ^ (rr & 7)) << 4)) = f16x8_to_bf16x8(a);
+                    *reinterpret_cast<uint4 *>(qt + rr * 128 + (((L0 + 1) ^ (rr & 7)) << 4)) = f16x8_to_bf16x8(bq);
+                }
             } else if (F8 && ok) {
                 // E4M3 codes [128 rows][64] -> phi(q) in bf16, exact (<= 4 significant
                 // bits), into the 128-byte swizzled tile the MMA reads
@@ -877,8 +1016,8 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (lane == 0) bulk_wait_read<C::kStgBufs - 1>();   // the last store from sb has read it
                 __syncwarp();
                 if (got) {
-                    // F8: out = sq num^ / (sq den^ + eps) with num^, den^ from the codes
-                    const float qs = F8 ? p.sq : 1.0f;
+                    // F8, F4: out = sq num^ / (sq den^ + eps) with num^, den^ from the codes
+                    const float qs = (F8 || F4) ? p.sq : 1.0f;
                     const float inv0 = qs / (qs * den0 + p.eps), inv1 = qs / (qs * den1 + p.eps);
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {       // logical 16-byte chunk c: head c/4
@@ -899,7 +1038,7 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             } else if (got && row0 + r < ta1) {
                 // a short last tile inside the tensor: the rows after ta1 belong to another block
-                const float qs = F8 ? p.sq : 1.0f;
+                const float qs = (F8 || F4) ? p.sq : 1.0f;
                 const float inv0 = qs / (qs * den0 + p.eps), inv1 = qs / (qs * den1 + p.eps);
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
@@ -970,14 +1109,15 @@ bool make_map(CUtensorMap *m, const void *base, int B, int N, int H, int box_row
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3D view of a [B][N][H*32] tensor of one-byte E4M3 codes: boxes of box_inner
-// codes x box_rows tokens, 128-byte swizzle or none.
-bool make_map_u8(CUtensorMap *m, const void *base, int B, int N, int H, int box_inner, int box_rows, bool sw128) {
+// 3D view of a [B][N][row_bytes] tensor of bytes (E4M3 codes: H*32 bytes a
+// row; NVFP4 codes: H*16; NVFP4 block scales: H*2): boxes of box_inner bytes
+// x box_rows tokens, 128-byte swizzle or none.
+bool make_map_bytes(CUtensorMap *m, const void *base, int B, int N, long long row_bytes, int box_inner,
+                    int box_rows, bool sw128) {
     auto fn = encode_fn();
     if (!fn) return false;
-    const cuuint64_t row_bytes = (cuuint64_t)H * kD;
-    cuuint64_t dims[3] = {(cuuint64_t)H * kD, (cuuint64_t)N, (cuuint64_t)B};
-    cuuint64_t strides[2] = {row_bytes, row_bytes * (cuuint64_t)N};
+    cuuint64_t dims[3] = {(cuuint64_t)row_bytes, (cuuint64_t)N, (cuuint64_t)B};
+    cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)row_bytes * (cuuint64_t)N};
     cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
     cuuint32_t es[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, es,
@@ -993,8 +1133,10 @@ bool smem_ready() {
              set_smem((const void *)reduce_tc_kernel<true>, RCfg<true>::kSmem) &&
              set_smem((const void *)apply_tc_kernel<false>, ACfg<false>::kSmem) &&
              set_smem((const void *)apply_tc_kernel<true>, ACfg<true>::kSmem) &&
-             set_smem((const void *)reduce_tc_kernel<false, true>, RCfg<false, true>::kSmem) &&
-             set_smem((const void *)apply_tc_kernel<false, true>, ACfg<false, true>::kSmem);
+             set_smem((const void *)reduce_tc_kernel<false, kInE4m3>, RCfg<false, kInE4m3>::kSmem) &&
+             set_smem((const void *)apply_tc_kernel<false, kInE4m3>, ACfg<false, kInE4m3>::kSmem) &&
+             set_smem((const void *)reduce_tc_kernel<false, kInNvfp4>, RCfg<false, kInNvfp4>::kSmem) &&
+             set_smem((const void *)apply_tc_kernel<false, kInNvfp4>, ACfg<false, kInNvfp4>::kSmem);
     });
     return ok;
 }
@@ -1039,21 +1181,33 @@ bool tc_rope_fits(const Plan &p) {
 
 int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &p, cudaStream_t s, const Fuse *fz) {
     if (!smem_ready()) return -1;
-    CUtensorMap mk, mv;
+    CUtensorMap mk, mv, mks{}, mvs{};
     const long long grid = (long long)p.B * (p.H / 4) * p.nb * p.P;
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
     const Fuse off = {nullptr, nullptr, nullptr, nullptr, 0, 0};
     const Fuse f = fz ? *fz : off;
     if (f.on && (p.nb != 1 || p.P < 1 || p.P > kFuseMaxSplits)) return -1;
     auto go = [&](auto kernel, int threads, int smem) {
-        return f.on ? launch_pdl_cluster(kernel, (unsigned)grid, threads, smem, (unsigned)p.P, s, mk, mv, partials, p, f)
-                    : launch_pdl(kernel, (unsigned)grid, threads, smem, s, mk, mv, partials, p, f);
+        return f.on ? launch_pdl_cluster(kernel, (unsigned)grid, threads, smem, (unsigned)p.P, s, mk, mv, mks, mvs,
+                                         partials, p, f)
+                    : launch_pdl(kernel, (unsigned)grid, threads, smem, s, mk, mv, mks, mvs, partials, p, f);
     };
-    if (p.f8) {
-        if (!make_map_u8(&mk, k, p.B, p.N, p.H, 128, kRRows, true) ||
-            !make_map_u8(&mv, v, p.B, p.N, p.H, 128, kRRows, true))
+    if (p.f4) {
+        // codes: the group's 64 bytes of a row; scales: 16-byte boxes (H % 8 == 0)
+        if (p.H % 8 != 0 || !make_map_bytes(&mk, k, p.B, p.N, (long long)p.H * kD / 2, 64, kRRows, false) ||
+            !make_map_bytes(&mv, v, p.B, p.N, (long long)p.H * kD / 2, 64, kRRows, false) ||
+            !make_map_bytes(&mks, p.sfk, p.B, p.N, (long long)p.H * kD / 16, 16, kRRows, false) ||
+            !make_map_bytes(&mvs, p.sfv, p.B, p.N, (long long)p.H * kD / 16, 16, kRRows, false))
             return -1;
-        return go(reduce_tc_kernel<false, true>, RCfg<false, true>::kThreadsR, RCfg<false, true>::kSmem) ? 1 : -1;
+        using C4 = RCfg<false, kInNvfp4>;
+        return go(reduce_tc_kernel<false, kInNvfp4>, C4::kThreadsR, C4::kSmem) ? 1 : -1;
+    }
+    if (p.f8) {
+        if (!make_map_bytes(&mk, k, p.B, p.N, (long long)p.H * kD, 128, kRRows, true) ||
+            !make_map_bytes(&mv, v, p.B, p.N, (long long)p.H * kD, 128, kRRows, true))
+            return -1;
+        using C8 = RCfg<false, kInE4m3>;
+        return go(reduce_tc_kernel<false, kInE4m3>, C8::kThreadsR, C8::kSmem) ? 1 : -1;
     }
     if (!make_map(&mk, k, p.B, p.N, p.H, kRRows) || !make_map(&mv, v, p.B, p.N, p.H, kRRows)) return -1;
     const bool ok = p.rope ? go(reduce_tc_kernel<true>, RCfg<true>::kThreadsR, RCfg<true>::kSmem)
@@ -1063,24 +1217,35 @@ int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &
 
 int launch_apply_tc(const void *q, void *out, const void *bop, const float *seff, const Plan &p, cudaStream_t s) {
     if (!smem_ready()) return -1;
-    CUtensorMap mq, mo;
+    CUtensorMap mq, mqs{}, mo;
     const long long grid = (long long)p.B * p.nb * p.Pa * (p.H / 2);
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
     const uint8_t *bb = static_cast<const uint8_t *>(bop);
-    if (p.f8) {
-        // q codes: boxes of the 2 heads' 64 codes x 128 tokens, no swizzle; out bf16
-        if (!make_map_u8(&mq, q, p.B, p.N, p.H, 64, 128, false) || !make_map(&mo, out, p.B, p.N, p.H, 32)) return -1;
-        return launch_pdl(apply_tc_kernel<false, true>, (unsigned)grid, kAThreads, ACfg<false, true>::kSmem, s, mq,
-                          mo, o, bb, seff, p)
+    if (!make_map(&mo, out, p.B, p.N, p.H, 32)) return -1;
+    if (p.f4) {
+        // q codes: the pair's 32 bytes x 128 tokens; scales: 16-byte boxes (H % 8 == 0)
+        if (p.H % 8 != 0 || !make_map_bytes(&mq, q, p.B, p.N, (long long)p.H * kD / 2, 32, 128, false) ||
+            !make_map_bytes(&mqs, p.sfq, p.B, p.N, (long long)p.H * kD / 16, 16, 128, false))
+            return -1;
+        return launch_pdl(apply_tc_kernel<false, kInNvfp4>, (unsigned)grid, kAThreads, ACfg<false, kInNvfp4>::kSmem,
+                          s, mq, mqs, mo, o, bb, seff, p)
                    ? 1
                    : -1;
     }
-    if (!make_map(&mq, q, p.B, p.N, p.H, 128) || !make_map(&mo, out, p.B, p.N, p.H, 32)) return -1;
+    if (p.f8) {
+        // q codes: boxes of the 2 heads' 64 codes x 128 tokens, no swizzle; out bf16
+        if (!make_map_bytes(&mq, q, p.B, p.N, (long long)p.H * kD, 64, 128, false)) return -1;
+        return launch_pdl(apply_tc_kernel<false, kInE4m3>, (unsigned)grid, kAThreads, ACfg<false, kInE4m3>::kSmem,
+                          s, mq, mqs, mo, o, bb, seff, p)
+                   ? 1
+                   : -1;
+    }
+    if (!make_map(&mq, q, p.B, p.N, p.H, 128)) return -1;
     const bool ok = p.rope ? launch_pdl(apply_tc_kernel<true>, (unsigned)grid, kAThreads, ACfg<true>::kSmem, s, mq,
-                                        mo, o, bb, seff, p)
+                                        mqs, mo, o, bb, seff, p)
                            : launch_pdl(apply_tc_kernel<false>, (unsigned)grid, kAThreads, ACfg<false>::kSmem, s, mq,
-                                        mo, o, bb, seff, p);
+                                        mqs, mo, o, bb, seff, p);
     return ok ? 1 : -1;
 }
 

@@ -117,6 +117,7 @@ la_status common_checks(const void *q, const void *k, const void *v, void *out, 
 // their shared memory; the rest runs on the CUDA cores.
 bool use_tc(la_dtype dt, const la::Plan &p) {
     if (p.f8) return (p.H % 4) == 0 && !p.rope && la::tc_available();
+    if (p.f4) return (p.H % 8) == 0 && !p.rope && la::tc_available();
     return dt == LA_BF16 && (p.H % 4) == 0 && (!p.rope || la::tc_rope_fits(p)) && la::tc_available();
 }
 
@@ -129,6 +130,22 @@ la_status e4m3_checks(const void *q, const void *k, const void *v, void *out, in
     for (float x : {sq, sk, sv})
         if (!(x > 0.0f) || !std::isfinite(x)) return LA_EINVAL;
     if (H % 4 != 0 || !la::tc_available()) return LA_EUNSUPPORTED;
+    return LA_OK;
+}
+
+// NVFP4 calls: q, k, v E2M1 codes [B][N][H][16] bytes, E4M3 block scales
+// [B][N][H][2] bytes, per-tensor scales; bf16 out; tensor cores only (H a
+// multiple of 8: the scale rows are then whole 16-byte units), no RoPE.
+la_status nvfp4_checks(const void *q, const void *k, const void *v, const void *sq_blk, const void *sk_blk,
+                       const void *sv_blk, void *out, int B, int N, int H, int d, float eps, float sq, float sk,
+                       float sv) {
+    la_status e = common_checks(q, k, v, out, LA_BF16, B, N, H, d, eps);
+    if (e != LA_OK) return e;
+    if (!sq_blk || !sk_blk || !sv_blk) return LA_EINVAL;
+    if (!aligned16(sq_blk) || !aligned16(sk_blk) || !aligned16(sv_blk)) return LA_EINVAL;
+    for (float x : {sq, sk, sv})
+        if (!(x > 0.0f) || !std::isfinite(x)) return LA_EINVAL;
+    if (H % 8 != 0 || !la::tc_available()) return LA_EUNSUPPORTED;
     return LA_OK;
 }
 
@@ -164,7 +181,7 @@ la_status run(const void *q, const void *k, const void *v, void *out, la_dtype d
     if (r < 0 || !mark(3, s)) return LA_ECUDA;
     n += r;
     g_last_launches = n;
-    g_last_path = tc ? (p.f8 ? "tc_e4m3" : "tc") : "ffma";
+    g_last_path = tc ? (p.f8 ? "tc_e4m3" : (p.f4 ? "tc_nvfp4" : "tc")) : "ffma";
     return LA_OK;
 }
 
@@ -359,6 +376,56 @@ la_status la_block_forward_e4m3(const void *q, const void *k, const void *v, flo
     p.eps = eps;
     p.f8 = 1;
     p.sq = scale_q; p.sk = scale_k; p.sv = scale_v;
+    make_splits(p);
+    fill_rope(p, nullptr, 0);
+    e = run(q, k, v, out, LA_BF16, p, st->S, st->Z, ws, static_cast<cudaStream_t>(stream));
+    if (e != LA_OK) return e;
+    if (commit) st->blocks_committed += 1;
+    return LA_OK;
+}
+
+la_status la_full_forward_nvfp4(const void *q, const void *k, const void *v, const void *q_blk_scale,
+                                const void *k_blk_scale, const void *v_blk_scale, float scale_q, float scale_k,
+                                float scale_v, void *out, int B, int N, int H, int d, int tokens_per_block,
+                                float eps, void *ws, size_t ws_bytes, void *stream) {
+    la_status e = nvfp4_checks(q, k, v, q_blk_scale, k_blk_scale, v_blk_scale, out, B, N, H, d, eps, scale_q,
+                               scale_k, scale_v);
+    if (e != LA_OK) return e;
+    if (tokens_per_block < 0) return LA_EINVAL;
+    const size_t need = la_workspace_size(B, N, H, d, tokens_per_block);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return LA_EWORKSPACE;
+    la::Plan p{};
+    p.B = B; p.N = N; p.H = H;
+    p.L = tokens_per_block > 0 && tokens_per_block < N ? tokens_per_block : N;
+    p.nb = (int)ceil_div(N, p.L);
+    p.eps = eps;
+    p.f4 = 1;
+    p.sq = scale_q; p.sk = scale_k; p.sv = scale_v;
+    p.sfq = q_blk_scale; p.sfk = k_blk_scale; p.sfv = v_blk_scale;
+    make_splits(p);
+    fill_rope(p, nullptr, 0);
+    return run(q, k, v, out, LA_BF16, p, nullptr, nullptr, ws, static_cast<cudaStream_t>(stream));
+}
+
+la_status la_block_forward_nvfp4(const void *q, const void *k, const void *v, const void *q_blk_scale,
+                                 const void *k_blk_scale, const void *v_blk_scale, float scale_q, float scale_k,
+                                 float scale_v, void *out, int B, int N_blk, int H, int d, la_state *st, int commit,
+                                 float eps, void *ws, size_t ws_bytes, void *stream) {
+    la_status e = nvfp4_checks(q, k, v, q_blk_scale, k_blk_scale, v_blk_scale, out, B, N_blk, H, d, eps, scale_q,
+                               scale_k, scale_v);
+    if (e != LA_OK) return e;
+    if (!st || !st->S || !st->Z) return LA_EINVAL;
+    if (st->B != B || st->H != H || st->d != d) return LA_EINVAL;
+    const size_t need = la_workspace_size(B, N_blk, H, d, N_blk);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return LA_EWORKSPACE;
+    la::Plan p{};
+    p.B = B; p.N = N_blk; p.H = H; p.L = N_blk; p.nb = 1;
+    p.commit = commit != 0;
+    p.has_state = 1;
+    p.eps = eps;
+    p.f4 = 1;
+    p.sq = scale_q; p.sk = scale_k; p.sv = scale_v;
+    p.sfq = q_blk_scale; p.sfk = k_blk_scale; p.sfv = v_blk_scale;
     make_splits(p);
     fill_rope(p, nullptr, 0);
     e = run(q, k, v, out, LA_BF16, p, st->S, st->Z, ws, static_cast<cudaStream_t>(stream));

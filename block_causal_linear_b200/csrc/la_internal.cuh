@@ -22,6 +22,11 @@ constexpr int kOpRows = 48;            // N of the apply MMA: 32 S columns, Z, 1
 constexpr int kOpBytes = kOpRows * kD * 2;   // one bf16 operand (hi or lo) = 3072 B
 
 // Everything a kernel needs to know about one call, passed by value.
+// Input kinds of the tensor-core kernels: bf16 q, k, v; FP8 E4M3 codes with
+// per-tensor scales; NVFP4 (E2M1 codes, an E4M3 scale per 16 features, a
+// per-tensor scale).
+constexpr int kInBf16 = 0, kInE4m3 = 1, kInNvfp4 = 2;
+
 struct Plan {
     int B, N, H;          // batch, tokens in the call, heads
     int L;                // tokens per block (the last block may be shorter)
@@ -34,7 +39,9 @@ struct Plan {
     int has_state;        // S, Z hold a prior state (block_forward) or not (full_forward)
     int rope;             // numerator RoPE on phi(q), phi(k)
     int f8;               // q, k, v are FP8 E4M3 codes with per-tensor scales sq, sk, sv
+    int f4;               // q, k, v are NVFP4: E2M1 codes, E4M3 block scales sfq, sfk, sfv, per-tensor sq, sk, sv
     float sq, sk, sv;
+    const void *sfq, *sfk, *sfv;   // NVFP4 block scales [B][N][H][2] (host-side, for the tensor maps)
     int Hg, Wg;           // latent grid of one frame
     int t_offset;         // frame of token 0 of the call
     float eps;

@@ -17,9 +17,13 @@ from . import la, synth
 
 
 class Runner:
-    def __init__(self, w: synth.Workload, device="cuda", blocks: Optional[int] = None, e4m3: bool = False):
+    def __init__(self, w: synth.Workload, device="cuda", blocks: Optional[int] = None, e4m3: bool = False,
+                 nvfp4: bool = False):
         self.w = w
         self.e4m3 = e4m3
+        self.nvfp4 = nvfp4
+        if e4m3 and nvfp4:
+            raise ValueError("one input format")
         self.device = torch.device(device)
         self.calls: List[tuple] = []          # (block, pass, q, k, v) in call order
         if w.mode == "full":
@@ -44,7 +48,18 @@ class Runner:
                 qk = [synth.to_e4m3(t) for t in c[2:5]]
                 self.calls[i] = (c[0], c[1], *[x for x, _ in qk])
                 self.scales.append([s_ for _, s_ in qk])
+        self.fp4 = None
+        if nvfp4:
+            # NVFP4 inputs: each call's q, k, v as (E2M1 codes, E4M3 block scales, per-tensor scale)
+            if w.rope:
+                raise ValueError("the NVFP4 path takes no RoPE")
+            self.fp4 = []
+            for i, c in enumerate(self.calls):
+                self.fp4.append([synth.to_nvfp4(t) for t in c[2:5]])
+                self.calls[i] = (c[0], c[1], *[x[0] for x in self.fp4[-1]])
         self.inputs = [c[2:5] for c in self.calls]        # device inputs of each call
+        if nvfp4:
+            self.inputs = [tuple(x[0] for x in f) + tuple(x[1] for x in f) for f in self.fp4]
         self.out_call = list(range(len(self.calls)))      # the call that writes each out
         self.state = la.State(w.B, w.H, w.d, device=self.device) if w.mode == "stream" else None
         self.rope = None
@@ -63,7 +78,10 @@ class Runner:
         n = 0
         if w.mode == "full":
             _, _, q, k, v = self.calls[0]
-            if self.e4m3:
+            if self.nvfp4:
+                la.full_forward_nvfp4(*self.fp4[0], self.tokens_per_block, eps=w.eps, ws=self.ws,
+                                      out=self.outs[0], stream=stream)
+            elif self.e4m3:
                 la.full_forward_e4m3(q, k, v, self.scales[0], self.tokens_per_block, eps=w.eps, ws=self.ws,
                                      out=self.outs[0], stream=stream)
             else:
@@ -79,7 +97,10 @@ class Runner:
             if rc != la.LA_OK:
                 raise la.LAError(rc, "la_state_init")
             for i, (blk, p, q, k, v) in enumerate(self.calls):
-                if self.e4m3:
+                if self.nvfp4:
+                    la.block_forward_nvfp4(*self.fp4[i], st, commit=(p == w.passes - 1), eps=w.eps,
+                                           ws=self.ws, out=self.outs[i], stream=stream)
+                elif self.e4m3:
                     la.block_forward_e4m3(q, k, v, self.scales[i], st, commit=(p == w.passes - 1), eps=w.eps,
                                           ws=self.ws, out=self.outs[i], stream=stream)
                 else:

@@ -205,6 +205,42 @@ LA_API la_status la_block_forward_e4m3(const void *q, const void *k, const void 
                                        size_t ws_bytes, void *stream);
 
 /*
+ * NVFP4 inputs, the format the pages deploy the model in ("Nvidia, MIT ve
+ * diğerleri video yapay zeka devrimini başlattı", section "Etkin eğitim ve
+ * çıkarım stratejileri": SVDQuant NVFP4).  Each of q, k, v is three parts:
+ *   codes:       DEVICE uint8 [B][N][H][d/2], two FP4 E2M1 codes per byte
+ *                (element 2i in the low nibble, 2i+1 in the high nibble;
+ *                E2M1: sign, 2 exponent bits with bias 1, 1 mantissa bit,
+ *                magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6);
+ *   block scale: DEVICE uint8 [B][N][H][d/16], one FP8 E4M3 scale per 16
+ *                consecutive features, sign bit clear (not NaN);
+ *   scale_x:     one fp32 per-tensor scale, finite and > 0;
+ * value = e2m1(code) * e4m3(block scale) * scale_x.  A positive scale
+ * commutes with ReLU, so the results are those of la_full_forward /
+ * la_block_forward on the decoded values (out = scale_q psi(q^) S_eff /
+ * (scale_q phi(q^) . Z_eff + eps), KV and z carry scale_k scale_v and
+ * scale_k), out in bf16, the state fp32 in real units.  q, k, v move 18
+ * bytes per token and head each instead of 64.
+ * Errors: null or not 16-byte aligned pointers, or a scale_x not finite and
+ * > 0, LA_EINVAL; H not a multiple of 8 or no tensor-core path,
+ * LA_EUNSUPPORTED; no RoPE.  A block scale with the sign bit set or NaN gives
+ * unspecified values (no fault).  Workspace and every other argument as in
+ * the bf16 calls.
+ */
+LA_API la_status la_full_forward_nvfp4(const void *q, const void *k, const void *v,
+                                       const void *q_blk_scale, const void *k_blk_scale,
+                                       const void *v_blk_scale, float scale_q, float scale_k,
+                                       float scale_v, void *out, int B, int N, int H, int d,
+                                       int tokens_per_block, float eps, void *ws, size_t ws_bytes,
+                                       void *stream);
+LA_API la_status la_block_forward_nvfp4(const void *q, const void *k, const void *v,
+                                        const void *q_blk_scale, const void *k_blk_scale,
+                                        const void *v_blk_scale, float scale_q, float scale_k,
+                                        float scale_v, void *out, int B, int N_blk, int H, int d,
+                                        la_state *st, int commit, float eps, void *ws,
+                                        size_t ws_bytes, void *stream);
+
+/*
  * Depthwise 3D convolution of the Spatial-Temporal Mix-FFN, the step after
  * attention in a block ("Nvidia, MIT ve diğerleri video yapay zeka devrimini
  * başlattı", section "Verimli doğrusal DiT": the MLP alternates a 1x3x3
