@@ -409,7 +409,12 @@ bwd_q_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const uint8_t *drow = dot + bx * kQTBox + r * 128;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) cur[j] = *reinterpret_cast<const uint4 *>(drow + ((j ^ (r & 7)) * 16));
-                if (bx == 1) mbar_arrive(dout_free);   // the dout tile is read
+                if (bx == 1) {
+                    // the dout tile is read: order these generic loads before TMA
+                    // (async proxy) refills the tile
+                    fence_proxy_async_smem();
+                    mbar_arrive(dout_free);
+                }
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
                     const int hh = 2 * bx + h2;

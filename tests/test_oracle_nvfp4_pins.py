@@ -79,3 +79,15 @@ def test_quantiser_error_bound_and_idempotence(orc):
     assert torch.equal(torch.sign(dec[dec != 0]), torch.sign(x[dec != 0]))
     c2, sf2, s2 = synth.to_nvfp4(dec)
     assert torch.equal(c2, codes) and torch.equal(sf2, sf) and s2 == s
+
+
+def test_quantiser_zero_and_sign_cases(orc):
+    codes, sf, s = synth.to_nvfp4(torch.zeros(2, 32, dtype=torch.float64))
+    assert s == 1.0 and int(codes.sum()) == 0 and int(sf.sum()) == 0
+    # one block of +-10.5 = 6 * 448 * 2^-8 (the tensor scale is then exactly 2^-8): element
+    # codes 0x7 and 0xF (6, -6) at the largest block scale; an all-zero block gets scale 0
+    x = torch.tensor([[10.5, -10.5] * 8 + [0.0] * 16], dtype=torch.float64)
+    codes, sf, s = synth.to_nvfp4(x)
+    assert s == 2.0 ** -8
+    assert codes[0, :8].tolist() == [0xF7] * 8 and sf[0, 0] == 0x7E and sf[0, 1] == 0x00
+    assert torch.equal(orc.nvfp4_decode(codes, sf, s), x)
