@@ -3,10 +3,14 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
 
-One step is one of the workloads (default: configuration 2, the 5 s 480p
-latent as a single bidirectional block, 8190 tokens x 64 heads x d 32, bf16)
-run once through the library from a zero state, with every input already
-resident in HBM.  L2 is flushed before every timed step: a 256 MiB device
+One step is one of the workloads run once through the library from a zero
+state, with every input already resident in HBM.  The default is the largest
+one that fits a GPU: batched 720p block-autoregressive streaming, B 4 x 64
+heads x d 32, 7 blocks of 3 latent frames x 45 x 80 = 10,800 tokens, 4
+denoising passes per block (the last one commits), 3D RoPE, bf16 (28
+la_block_forward calls per step).  --config 2 is the 5 s 480p latent as one
+bidirectional block (8190 tokens), 3 the 720p latent as one block, 4 the
+minute-long 480p stream.  L2 is flushed before every timed step: a 256 MiB device
 write, then a read of another 256 MiB buffer, so that no input line is in L2
 and the flush's own dirty lines are written back before the step starts (a
 write alone leaves ~126 MB of them to be written back inside the step); the
@@ -58,7 +62,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--config", type=int, default=5, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

@@ -214,6 +214,36 @@ la_status la_state_init(la_state *st, float *S, float *Z, int B, int H, int d, v
     return LA_OK;
 }
 
+// A bound state: what la_state_init leaves behind.
+static bool state_bound(const la_state *st) {
+    return st && st->S && st->Z && st->B > 0 && st->H > 0 && st->d == la::kD;
+}
+
+la_status la_state_save(const la_state *st, float *S_dst, float *Z_dst, la_state_counters *counters,
+                        void *stream) {
+    if (!state_bound(st) || !S_dst || !Z_dst || !counters) return LA_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t nS = size_t(st->B) * st->H * st->d * st->d, nZ = size_t(st->B) * st->H * st->d;
+    if (cudaMemcpyAsync(S_dst, st->S, nS * sizeof(float), cudaMemcpyDefault, s) != cudaSuccess) return LA_ECUDA;
+    if (cudaMemcpyAsync(Z_dst, st->Z, nZ * sizeof(float), cudaMemcpyDefault, s) != cudaSuccess) return LA_ECUDA;
+    counters->blocks_committed = st->blocks_committed;
+    counters->t_next = st->t_next;
+    return LA_OK;
+}
+
+la_status la_state_restore(la_state *st, const float *S_src, const float *Z_src,
+                           const la_state_counters *counters, void *stream) {
+    if (!state_bound(st) || !S_src || !Z_src || !counters) return LA_EINVAL;
+    if (counters->blocks_committed < 0 || counters->t_next < 0) return LA_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t nS = size_t(st->B) * st->H * st->d * st->d, nZ = size_t(st->B) * st->H * st->d;
+    if (cudaMemcpyAsync(st->S, S_src, nS * sizeof(float), cudaMemcpyDefault, s) != cudaSuccess) return LA_ECUDA;
+    if (cudaMemcpyAsync(st->Z, Z_src, nZ * sizeof(float), cudaMemcpyDefault, s) != cudaSuccess) return LA_ECUDA;
+    st->blocks_committed = counters->blocks_committed;
+    st->t_next = counters->t_next;
+    return LA_OK;
+}
+
 la_status la_block_forward(const void *q, const void *k, const void *v, void *out, la_dtype dt,
                            int B, int N_blk, int H, int d, la_state *st, int commit,
                            const la_rope *rope, float eps, void *ws, size_t ws_bytes,

@@ -43,6 +43,10 @@ class la_state(ctypes.Structure):
                 ("t_next", ctypes.c_int)]
 
 
+class la_state_counters(ctypes.Structure):
+    _fields_ = [("blocks_committed", ctypes.c_longlong), ("t_next", ctypes.c_int)]
+
+
 _lib = None
 
 
@@ -59,6 +63,10 @@ def lib() -> ctypes.CDLL:
         L.la_workspace_size.restype = sz
         L.la_state_init.argtypes = [ctypes.POINTER(la_state), vp, vp, ip, ip, ip, vp]
         L.la_state_init.restype = ip
+        L.la_state_save.argtypes = [ctypes.POINTER(la_state), vp, vp, ctypes.POINTER(la_state_counters), vp]
+        L.la_state_save.restype = ip
+        L.la_state_restore.argtypes = [ctypes.POINTER(la_state), vp, vp, ctypes.POINTER(la_state_counters), vp]
+        L.la_state_restore.restype = ip
         L.la_block_forward.argtypes = [vp, vp, vp, vp, ip, ip, ip, ip, ip, ctypes.POINTER(la_state), ip,
                                        ctypes.POINTER(la_rope), fp, vp, sz, vp]
         L.la_block_forward.restype = ip
@@ -118,6 +126,16 @@ def la_workspace_size(B, N, H, d, tokens_per_block) -> int:
 
 def la_state_init(st, S, Z, B, H, d, stream) -> int:
     return int(lib().la_state_init(ctypes.byref(st), S, Z, B, H, d, stream))
+
+
+def la_state_save(st, S_dst, Z_dst, counters, stream) -> int:
+    return int(lib().la_state_save(ctypes.byref(st), S_dst, Z_dst,
+                                   ctypes.byref(counters) if counters is not None else None, stream))
+
+
+def la_state_restore(st, S_src, Z_src, counters, stream) -> int:
+    return int(lib().la_state_restore(ctypes.byref(st), S_src, Z_src,
+                                      ctypes.byref(counters) if counters is not None else None, stream))
 
 
 def la_block_forward(q, k, v, out, dt, B, N_blk, H, d, st, commit, rope, eps, ws, ws_bytes, stream) -> int:
@@ -322,6 +340,27 @@ class State:
 
     def nbytes(self) -> int:
         return self.S.numel() * 4 + self.Z.numel() * 4
+
+    def save(self, S_dst: torch.Tensor, Z_dst: torch.Tensor, stream=None) -> la_state_counters:
+        """la_state_save into caller tensors (host, pinned host or device) of
+        S's and Z's shapes and dtype; returns the counters."""
+        if S_dst.shape != self.S.shape or Z_dst.shape != self.Z.shape or S_dst.dtype != torch.float32 \
+                or Z_dst.dtype != torch.float32 or not S_dst.is_contiguous() or not Z_dst.is_contiguous():
+            raise ValueError("checkpoint buffers must be contiguous fp32 tensors of S's and Z's shapes")
+        c = la_state_counters()
+        rc = la_state_save(self.c, S_dst.data_ptr(), Z_dst.data_ptr(), c, _stream_ptr(stream))
+        if rc != LA_OK:
+            raise LAError(rc, "la_state_save")
+        return c
+
+    def restore(self, S_src: torch.Tensor, Z_src: torch.Tensor, counters: la_state_counters, stream=None):
+        """la_state_restore from caller tensors saved by ``save``."""
+        if S_src.shape != self.S.shape or Z_src.shape != self.Z.shape or S_src.dtype != torch.float32 \
+                or Z_src.dtype != torch.float32 or not S_src.is_contiguous() or not Z_src.is_contiguous():
+            raise ValueError("checkpoint buffers must be contiguous fp32 tensors of S's and Z's shapes")
+        rc = la_state_restore(self.c, S_src.data_ptr(), Z_src.data_ptr(), counters, _stream_ptr(stream))
+        if rc != LA_OK:
+            raise LAError(rc, "la_state_restore")
 
 
 def block_forward(q, k, v, state: State, commit=True, rope: Optional[la_rope] = None, eps=1e-6,

@@ -111,18 +111,63 @@ typedef struct {
  * the split partial sums, the per-block effective state and the packed
  * tensor-core operand; its size never depends on how many blocks were
  * streamed before.  Its base must be 256-byte aligned.
+ * The pages have no counterpart of this call: they describe the block sum
+ * KV_n as one reduction ("Nvidia, MIT ve diğerleri video yapay zeka
+ * devrimini başlattı", section "Sabit Bellekli KV önbelleğe alma
+ * mekanizması"); the workspace is where this library keeps the pieces of
+ * that reduction when it cuts a block's tokens into splits to fill the GPU.
  */
 LA_API size_t la_workspace_size(int B, int N, int H, int d, int tokens_per_block);
 
 /*
- * Bind the caller's S, Z buffers to *st, zero them (cudaMemsetAsync on
- * `stream`) and reset blocks_committed and t_next to 0.
+ * Start a stream: bind the caller's S, Z buffers to *st, zero them
+ * (cudaMemsetAsync on `stream`) and reset blocks_committed and t_next to 0.
+ * Source: "Nvidia, MIT ve diğerleri video yapay zeka devrimini başlattı"
+ * (aihaber.org), section "Sabit Bellekli KV önbelleğe alma mekanizması": the
+ * cache is empty before block 1 and receives block 1's KV first; sd114.wiki
+ * SANA-Video summary, section "两大核心技术突破", item 2: the only context a
+ * chunk sees is one cumulative state of constant size.  Zero S, Z is that
+ * empty cache, so block 1 sees only itself.
+ * Errors: null st, S or Z, or S, Z not 16-byte aligned, or B, H <= 0:
+ * LA_EINVAL; d != 32: LA_EUNSUPPORTED; a failed memset: LA_ECUDA.
  */
 LA_API la_status la_state_init(la_state *st, float *S, float *Z, int B, int H, int d, void *stream);
 
 /*
- * One block of the streaming method ("each block computes only KVsum plus its
- * own KV"): for the N_blk tokens of this block,
+ * Checkpoint and resume of a stream.  All the method keeps of the past is the
+ * fixed-size state ("Nvidia, MIT ve diğerleri video yapay zeka devrimini
+ * başlattı", section "Sabit Bellekli KV önbelleğe alma mekanizması": the cache
+ * holds only the running sum of the blocks' KV; sd114.wiki, section
+ * "两大核心技术突破", item 2: one cumulative state of constant size), so S, Z
+ * and the two host counters are a complete checkpoint of any stream.
+ * la_state_save: copies st's S and Z to S_dst (B*H*d*d floats) and Z_dst
+ *   (B*H*d floats), host or device memory, with one cudaMemcpyAsync each
+ *   (cudaMemcpyDefault) on `stream`, and stores the counters in *counters at
+ *   once.  The copies are complete when `stream` reaches them (pinned host
+ *   memory keeps them asynchronous).
+ * la_state_restore: copies S_src, Z_src into st's S, Z the same way and sets
+ *   st's counters from *counters.  st must be bound by la_state_init with the
+ *   checkpoint's B, H, d.
+ * Streaming blocks after a restore gives bitwise the results of streaming on
+ * from the saved point.  Errors: a null or unbound st, a null buffer or
+ * counters pointer, or negative counters: LA_EINVAL; a failed copy: LA_ECUDA.
+ */
+typedef struct {
+    long long blocks_committed;
+    int t_next;
+} la_state_counters;
+LA_API la_status la_state_save(const la_state *st, float *S_dst, float *Z_dst, la_state_counters *counters,
+                               void *stream);
+LA_API la_status la_state_restore(la_state *st, const float *S_src, const float *Z_src,
+                                  const la_state_counters *counters, void *stream);
+
+/*
+ * One block of the streaming method.  Source: "Nvidia, MIT ve diğerleri video
+ * yapay zeka devrimini başlattı" (aihaber.org), section "Sabit Bellekli KV
+ * önbelleğe alma mekanizması": a block needs only the cached sum of the
+ * earlier blocks' KV plus its own KV, and its KV is then added to the cache;
+ * later blocks never reach back into earlier tokens.  For the N_blk tokens of
+ * this block:
  *   S_eff = S + KV_n,  Z_eff = Z + z_n,  out = psi(q) S_eff / (phi(q).Z_eff + eps),
  * every token of the block attending to every other token of it
  * (bidirectional inside the block) and to all committed blocks.
@@ -132,6 +177,13 @@ LA_API la_status la_state_init(la_state *st, float *S, float *Z, int B, int H, i
  *   stay bitwise unchanged.
  * rope may be NULL.  st must have been set up by la_state_init with the same
  * B, H, d.  ws must hold la_workspace_size(B, N_blk, H, d, N_blk) bytes.
+ * The host counters advance when the call is enqueued.  If a later
+ * la_device_status reports LA_ETIMEOUT, a committing call enqueued since the
+ * last successful la_device_status may have left S, Z partly updated while
+ * the counters say it committed: restore the last checkpoint
+ * (la_state_restore) or start over with la_state_init before streaming on.
+ * Errors: as la_full_forward, plus LA_EINVAL for a null or unbound st or one
+ * of other shapes.
  */
 LA_API la_status la_block_forward(const void *q, const void *k, const void *v, void *out, la_dtype dt,
                            int B, int N_blk, int H, int d, la_state *st, int commit,
@@ -139,12 +191,20 @@ LA_API la_status la_block_forward(const void *q, const void *k, const void *v, v
                            void *stream);
 
 /*
- * The whole sequence from a zero state in one call: blocks of tokens_per_block
- * tokens (0 = a single bidirectional block of all N tokens; the last block may
- * be shorter), block n seeing blocks 0..n.  Equal to la_state_init followed by
+ * The whole sequence from a zero state in one call.  Source: "Nvidia, MIT ve
+ * diğerleri video yapay zeka devrimini başlattı" (aihaber.org), section
+ * "Sabit Bellekli KV önbelleğe alma mekanizması": block 1's KV is cached,
+ * block 2 adds its KV to the cache (KV_{1-2} = KV_1 + KV_2), and so on until
+ * the last block's sum is the KV of the whole video; every block sees the
+ * cached sum plus its own KV.  Blocks of tokens_per_block tokens (0 = a
+ * single bidirectional block of all N tokens; the last block may be
+ * shorter), block n seeing blocks 0..n.  Equal to la_state_init followed by
  * la_block_forward(commit=1) on each block, up to the order of fp32 sums.
  * rope may be NULL; positions run over the whole sequence (t_offset >= 0).
  * ws must hold la_workspace_size(B, N, H, d, tokens_per_block) bytes.
+ * Errors: null or not 16-byte aligned q, k, v, out, a bad dtype, size, eps
+ * or RoPE: LA_EINVAL; d != 32: LA_EUNSUPPORTED; ws null, too small or not
+ * 256-byte aligned: LA_EWORKSPACE; a failed launch: LA_ECUDA.
  */
 LA_API la_status la_full_forward(const void *q, const void *k, const void *v, void *out, la_dtype dt,
                           int B, int N, int H, int d, int tokens_per_block,
@@ -324,7 +384,11 @@ LA_API la_status la_full_forward_static_ws(const void *q, const void *k, const v
  * wait inside a kernel is bounded; one that gives up records the fact in a
  * device flag and the kernel returns early.  This call synchronises `stream`,
  * reads and clears the flag, and returns LA_ETIMEOUT if it was set, LA_ECUDA
- * on a CUDA error, else LA_OK.
+ * on a CUDA error, else LA_OK.  After LA_ETIMEOUT the outputs of the calls
+ * enqueued since the last LA_OK are not valid, and a stream with committing
+ * calls among them must be restored from a checkpoint (la_state_restore) or
+ * restarted (la_state_init): their host counters advanced when they were
+ * enqueued.
  */
 LA_API la_status la_device_status(void *stream);
 
@@ -338,7 +402,9 @@ LA_API la_status la_device_status(void *stream);
  */
 LA_API la_status la_selftest_bounded_wait(void *stream);
 
-/* Static, human-readable name of a status. */
+/* Static, human-readable name of a status (never NULL; "unknown status" for
+ * a value outside la_status).  The pages have no counterpart: it belongs to
+ * the library's error reporting. */
 LA_API const char *la_status_string(la_status s);
 
 /*

@@ -239,3 +239,68 @@ def test_token_split_validation(la):
     assert la.la_block_apply(FAKE, FAKE, la.LA_BF16, 1, 64, 4, 32, FAKE, 2, st, 1, None, 1e-6, FAKE, 8,
                              None) == la.LA_EWORKSPACE
     assert st.blocks_committed == 0
+
+
+def test_static_ws_validation(la):
+    """The allocation-free variant rejects bad arguments, and shapes whose
+    scratch exceeds its static array, before it looks up the array."""
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, dt=la.LA_BF16, B=1, N=256, H=4, d=32, tpb=0, rope=None,
+                 eps=1e-6)
+        a.update(kw)
+        return la.la_full_forward_static_ws(a["q"], a["k"], a["v"], a["out"], a["dt"], a["B"], a["N"], a["H"],
+                                            a["d"], a["tpb"], a["rope"], a["eps"], None)
+    assert call(q=None) == la.LA_EINVAL
+    assert call(v=FAKE + 4) == la.LA_EINVAL
+    assert call(eps=-1.0) == la.LA_EINVAL
+    assert call(eps=float("nan")) == la.LA_EINVAL
+    assert call(tpb=-1) == la.LA_EINVAL
+    assert call(d=16) == la.LA_EUNSUPPORTED
+    assert call(rope=la.make_rope(Hg=2, Wg=2, t_offset=-1)) == la.LA_EINVAL
+    # 64 x 2000 tokens x 64 heads in blocks of 100 needs far more than the array
+    assert la.la_workspace_size(64, 2000, 64, 32, 100) > la.LA_STATIC_WS_BYTES
+    assert call(B=64, N=2000, H=64, tpb=100) == la.LA_EWORKSPACE
+
+
+def test_state_checkpoint_validation(la):
+    st = la.la_state()
+    c = la.la_state_counters()
+    # an unbound state
+    assert la.la_state_save(st, FAKE, FAKE, c, None) == la.LA_EINVAL
+    assert la.la_state_restore(st, FAKE, FAKE, c, None) == la.LA_EINVAL
+    st.S, st.Z, st.B, st.H, st.d = FAKE, FAKE, 1, 4, 32
+    st.blocks_committed, st.t_next = 5, 15
+    assert la.la_state_save(st, None, FAKE, c, None) == la.LA_EINVAL
+    assert la.la_state_save(st, FAKE, None, c, None) == la.LA_EINVAL
+    assert la.la_state_save(st, FAKE, FAKE, None, None) == la.LA_EINVAL
+    assert la.la_state_restore(st, None, FAKE, c, None) == la.LA_EINVAL
+    assert la.la_state_restore(st, FAKE, FAKE, None, None) == la.LA_EINVAL
+    c.blocks_committed, c.t_next = -1, 0
+    assert la.la_state_restore(st, FAKE, FAKE, c, None) == la.LA_EINVAL
+    # nothing was enqueued, so the counters are untouched
+    assert (st.blocks_committed, st.t_next) == (5, 15)
+
+
+PAGE_TITLES = ("Nvidia, MIT ve diğerleri video yapay zeka devrimini başlattı", "sd114.wiki")
+
+
+def _decl_comment(text, name):
+    """The comment block right before the LA_API declaration of `name`."""
+    m = re.search(r"/\*((?:(?!\*/).)*)\*/\s*(?:typedef\s+struct\s*\{[^}]*\}\s*\w+;\s*)*(?:LA_API[^;]*;\s*)*LA_API[^;]*?\b" + name + r"\s*\(",
+                  text, re.S)
+    assert m, name
+    # one line of prose: drop the comment's line breaks and leading stars
+    return " ".join(re.sub(r"^\s*\*\s?", "", ln) for ln in m.group(1).splitlines()).replace("  ", " ")
+
+
+def test_boundary_calls_cite_their_passages():
+    """Each call of the boundary names the page and section that defines it,
+    or says that the pages have none."""
+    text = open(os.path.join(ROOT, "include", "la.h"), encoding="utf-8").read()
+    for name in ("la_state_init", "la_block_forward", "la_full_forward", "la_workspace_size",
+                 "la_state_save", "la_state_restore"):
+        c = _decl_comment(text, name)
+        assert any(t in c for t in PAGE_TITLES), name
+        assert "section" in c, name
+    assert "no counterpart" in _decl_comment(text, "la_status_string")
+    assert "no counterpart" in _decl_comment(text, "la_workspace_size")
