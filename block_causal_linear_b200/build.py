@@ -14,7 +14,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libla_b200.so")
-SOURCES = ["la_api.cu", "k_ffma.cu", "k_finish.cu", "k_tc.cu", "k_bwd.cu", "k_bwd_tc.cu", "k_bwd_q_tc.cu", "k_conv.cu"]
+SOURCES = ["la_api.cu", "k_ffma.cu", "k_finish.cu", "k_tc.cu", "k_rope_tc.cu", "k_bwd.cu", "k_bwd_tc.cu", "k_bwd_q_tc.cu", "k_conv.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

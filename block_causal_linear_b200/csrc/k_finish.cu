@@ -42,7 +42,9 @@ __global__ void __launch_bounds__(kFinThreads)
 finish_kernel(const float *__restrict__ partials, float *__restrict__ seff,
               unsigned char *__restrict__ bop, float *__restrict__ S, float *__restrict__ Z,
               Plan p, int write_bop, long long part_bh_rt, long long part_sp_rt) {
-    const long long part_bh = STRIDED ? part_bh_rt : (long long)p.P * kKVZ;
+    // the split sums of (bh, block n) start at part_bh * (bh nb + n): P slots of
+    // the split plan, or skP slots of the RoPE kernels' stream-K plan
+    const long long part_bh = STRIDED ? part_bh_rt : (long long)(p.sk_layout ? p.skP : p.P) * kKVZ;
     const long long part_sp = STRIDED ? part_sp_rt : (long long)kKVZ;
     // let the apply be scheduled now (it prefetches its q tiles), then wait
     // for the reduce before reading its partials
@@ -72,13 +74,20 @@ finish_kernel(const float *__restrict__ partials, float *__restrict__ seff,
     for (int n = 0; n < p.nb; ++n) {
         // split sp of (bh, n) at partials + (bh * nb + n) * part_bh + sp * part_sp
         const float *src = partials + ((size_t)bh * p.nb + n) * part_bh + e;
-        for (int s0 = 0; s0 < p.P; s0 += kBatch) {
+        int P = p.P;
+        if (!STRIDED && p.sk_layout) {
+            // the CTAs of the stream-K plan that met unit (b, head group, n), in order
+            const int b = (int)(bh / p.H), g = (int)(bh % p.H) / 4;
+            const long long first = sk_unit_first(p.skr, b, n, g);
+            P = sk_cta_of(p.skr, first + sk_len(p.skr, n) - 1) - sk_cta_of(p.skr, first) + 1;
+        }
+        for (int s0 = 0; s0 < P; s0 += kBatch) {
             float v[kBatch];
 #pragma unroll
-            for (int j = 0; j < kBatch; ++j) v[j] = s0 + j < p.P ? __ldg(src + (size_t)(s0 + j) * part_sp) : 0.f;
+            for (int j = 0; j < kBatch; ++j) v[j] = s0 + j < P ? __ldg(src + (size_t)(s0 + j) * part_sp) : 0.f;
 #pragma unroll
             for (int j = 0; j < kBatch; ++j)
-                if (s0 + j < p.P) run += v[j];
+                if (s0 + j < P) run += v[j];
         }
         seff[((size_t)bh * p.nb + n) * kKVZ + e] = run;
         if (write_bop) {
@@ -114,7 +123,7 @@ int launch_finish_strided(const float *partials, float *seff, void *bop, float *
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const bool strided = part_bh != (long long)p.P * kKVZ || part_sp != kKVZ;
+    const bool strided = part_bh != (long long)(p.sk_layout ? p.skP : p.P) * kKVZ || part_sp != kKVZ;
     return cudaLaunchKernelEx(&cfg, strided ? finish_kernel<true> : finish_kernel<false>, partials, seff,
                               static_cast<unsigned char *>(bop), S, Z, p, write_bop, part_bh, part_sp) == cudaSuccess
                ? 1
@@ -124,7 +133,8 @@ int launch_finish_strided(const float *partials, float *seff, void *bop, float *
 
 int launch_finish(const float *partials, float *seff, void *bop, float *S, float *Z, const Plan &p,
                   int write_bop, cudaStream_t s) {
-    return launch_finish_strided(partials, seff, bop, S, Z, p, write_bop, (long long)p.P * kKVZ, kKVZ, s);
+    return launch_finish_strided(partials, seff, bop, S, Z, p, write_bop,
+                                 (long long)(p.sk_layout ? p.skP : p.P) * kKVZ, kKVZ, s);
 }
 
 
@@ -134,6 +144,7 @@ int launch_finish_ranks(const float *gathered, int R, float *seff, void *bop, fl
     if (p.nb != 1 || R < 1) return -1;
     Plan q = p;
     q.P = R;   // the ranks' partial sums play the splits, in rank order
+    q.sk_layout = 0;
     return launch_finish_strided(gathered, seff, bop, S, Z, q, write_bop, kKVZ, (long long)p.B * p.H * kKVZ,
                                  s);
 }

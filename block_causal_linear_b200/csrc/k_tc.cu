@@ -1175,9 +1175,6 @@ bool make_bf16_map_nd(CUtensorMap *m, const void *base, int rank, const cuuint64
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool tc_rope_fits(const Plan &p) {
-    return rope_table_entries(p, p.chunk) <= kTabMax && rope_table_entries(p, p.chunka) <= kTabMax;
-}
 
 int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &p, cudaStream_t s, const Fuse *fz) {
     if (!smem_ready()) return -1;

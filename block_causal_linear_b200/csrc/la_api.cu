@@ -53,6 +53,8 @@ void make_splits(la::Plan &p) {
     const long long chunka = ceil_div(ceil_div(p.L, wanta), la::kApplyRows) * la::kApplyRows;
     p.chunka = (int)chunka;
     p.Pa = (int)ceil_div(p.L, chunka);
+    // the stream-K plans of the RoPE kernels (the workspace holds their split sums too)
+    la::plan_rope_sk(p);
 }
 
 // The fused plan (the reduce combines its own splits): one block per call and
@@ -99,6 +101,7 @@ void fill_rope(la::Plan &p, const la_rope *r, int t_offset) {
         p.theta[pr] = (float)std::pow((double)r->base, -2.0 * (double)i / (double)D);
         p.axis[pr] = ax;
     }
+    la::plan_rope_table(p);
 }
 
 la_status common_checks(const void *q, const void *k, const void *v, void *out, la_dtype dt,
@@ -152,7 +155,7 @@ la_status nvfp4_checks(const void *q, const void *k, const void *v, const void *
 // Enqueue reduce -> finish -> apply for a prepared plan.
 la_status run(const void *q, const void *k, const void *v, void *out, la_dtype dt,
               la::Plan &p, float *S, float *Z, void *ws, cudaStream_t s) {
-    la::WsLayout w = la::ws_layout(p.B, p.H, p.nb, p.P);
+    la::WsLayout w = la::ws_layout(p.B, p.H, p.nb, la::ws_slots(p));
     char *base = static_cast<char *>(ws);
     float *partials = reinterpret_cast<float *>(base + w.partials);
     float *seff = reinterpret_cast<float *>(base + w.seff);
@@ -161,6 +164,22 @@ la_status run(const void *q, const void *k, const void *v, void *out, la_dtype d
     int n = 0, r;
 
     if (!mark(0, s)) return LA_ECUDA;
+    if (tc && p.rope) {
+        // RoPE: stream-K reduce, the combine over its slots, stream-K apply
+        p.sk_layout = 1;
+        r = la::launch_reduce_rope_tc(k, v, partials, p, s);
+        if (r < 0 || !mark(1, s)) return LA_ECUDA;
+        n += r;
+        r = la::launch_finish(partials, seff, bop, S, Z, p, 1, s);
+        if (r < 0 || !mark(2, s)) return LA_ECUDA;
+        n += r;
+        r = la::launch_apply_rope_tc(q, out, bop, seff, p, s);
+        if (r < 0 || !mark(3, s)) return LA_ECUDA;
+        n += r;
+        g_last_launches = n;
+        g_last_path = "tc";
+        return LA_OK;
+    }
     if (tc && fuse_plan(p)) {
         // one block: the reduce combines its splits itself (no combine kernel)
         const la::Fuse fz = {seff, static_cast<unsigned char *>(bop), S, Z, 1, 1};
@@ -196,7 +215,7 @@ size_t la_workspace_size(int B, int N, int H, int d, int tokens_per_block) {
     p.L = tokens_per_block > 0 && tokens_per_block < N ? tokens_per_block : N;
     p.nb = (int)ceil_div(N, p.L);
     make_splits(p);
-    return la::ws_layout(B, H, p.nb, p.P).total;
+    return la::ws_layout(B, H, p.nb, la::ws_slots(p)).total;
 }
 
 la_status la_state_init(la_state *st, float *S, float *Z, int B, int H, int d, void *stream) {
@@ -302,7 +321,7 @@ size_t la_backward_workspace_size(int B, int N, int H, int d, int tokens_per_blo
     p.L = tokens_per_block > 0 && tokens_per_block < N ? tokens_per_block : N;
     p.nb = (int)ceil_div(N, p.L);
     make_splits(p);
-    return la::bwd_layout(B, H, p.nb, p.P).total;
+    return la::bwd_layout(B, H, p.nb, la::ws_slots(p)).total;
 }
 
 la_status la_full_backward(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk,
@@ -326,7 +345,7 @@ la_status la_full_backward(const void *q, const void *k, const void *v, const vo
     make_splits(p);
     fill_rope(p, rope, rope ? rope->t_offset : 0);
 
-    const la::BwdLayout w = la::bwd_layout(B, H, p.nb, p.P);
+    const la::BwdLayout w = la::bwd_layout(B, H, p.nb, la::ws_slots(p));
     char *base = static_cast<char *>(ws);
     float *partials = reinterpret_cast<float *>(base + w.fwd.partials);
     float *seff = reinterpret_cast<float *>(base + w.fwd.seff);
@@ -341,7 +360,9 @@ la_status la_full_backward(const void *q, const void *k, const void *v, const vo
     // after the query side, after the key side
     if (!mark(0, s)) return LA_ECUDA;
     // the forward prefix state S_n, Z_n of every block, as the forward computes it
-    r = tc ? la::launch_reduce_tc(k, v, partials, p, s) : la::launch_reduce_ffma(bf, k, v, partials, p, s);
+    if (tc && p.rope) p.sk_layout = 1;
+    r = tc ? (p.rope ? la::launch_reduce_rope_tc(k, v, partials, p, s) : la::launch_reduce_tc(k, v, partials, p, s))
+           : la::launch_reduce_ffma(bf, k, v, partials, p, s);
     if (r < 0) return LA_ECUDA;
     n += r;
     // the query side on the tensor cores needs the packed [S|Z|0] operand
@@ -496,13 +517,15 @@ la_status la_block_reduce(const void *k, const void *v, la_dtype dt, int B, int 
     p.B = B; p.N = N_slice; p.H = H; p.L = N_slice; p.nb = 1;
     make_splits(p);
     fill_rope(p, rope, rope ? rope->t_offset : 0);
-    const la::WsLayout w = la::ws_layout(B, H, 1, p.P);
+    const la::WsLayout w = la::ws_layout(B, H, 1, la::ws_slots(p));
     char *base = static_cast<char *>(ws);
     float *partials = reinterpret_cast<float *>(base + w.partials);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool tc = use_tc(dt, p);
     int n = 0, r;
-    r = tc ? la::launch_reduce_tc(k, v, partials, p, s) : la::launch_reduce_ffma(dt == LA_BF16, k, v, partials, p, s);
+    if (tc && p.rope) p.sk_layout = 1;
+    r = tc ? (p.rope ? la::launch_reduce_rope_tc(k, v, partials, p, s) : la::launch_reduce_tc(k, v, partials, p, s))
+           : la::launch_reduce_ffma(dt == LA_BF16, k, v, partials, p, s);
     if (r < 0) return LA_ECUDA;
     n += r;
     // the slice's split sums, in split order, straight into the caller's partial
@@ -530,7 +553,7 @@ la_status la_block_apply(const void *q, void *out, la_dtype dt, int B, int N_sli
     p.eps = eps;
     make_splits(p);
     fill_rope(p, rope, rope ? (rope->t_offset < 0 ? st->t_next : rope->t_offset) : 0);
-    const la::WsLayout w = la::ws_layout(B, H, 1, p.P);
+    const la::WsLayout w = la::ws_layout(B, H, 1, la::ws_slots(p));
     char *base = static_cast<char *>(ws);
     float *seff = reinterpret_cast<float *>(base + w.seff);
     void *bop = base + w.bop;
@@ -539,7 +562,8 @@ la_status la_block_apply(const void *q, void *out, la_dtype dt, int B, int N_sli
     int n = 0, r;
     if ((r = la::launch_finish_ranks(gathered, R, seff, bop, st->S, st->Z, p, tc ? 1 : 0, s)) < 0) return LA_ECUDA;
     n += r;
-    r = tc ? la::launch_apply_tc(q, out, bop, seff, p, s) : la::launch_apply_ffma(dt == LA_BF16, q, out, seff, p, s);
+    r = tc ? (p.rope ? la::launch_apply_rope_tc(q, out, bop, seff, p, s) : la::launch_apply_tc(q, out, bop, seff, p, s))
+           : la::launch_apply_ffma(dt == LA_BF16, q, out, seff, p, s);
     if (r < 0) return LA_ECUDA;
     n += r;
     g_last_launches = n;
@@ -552,13 +576,13 @@ la_status la_block_apply(const void *q, void *out, la_dtype dt, int B, int N_sli
 }
 
 la_status la_device_status(void *stream) {
-    unsigned flag = 0, fk = 0, fq = 0, fc = 0;
+    unsigned flag = 0, fk = 0, fq = 0, fc = 0, fr = 0;
     // (synchronises the stream first)
     if (la::read_and_clear_device_flag(static_cast<cudaStream_t>(stream), &flag) != 0) return LA_ECUDA;
     if (la::read_and_clear_bwd_k_flag(&fk) != 0 || la::read_and_clear_bwd_q_flag(&fq) != 0 ||
-        la::read_and_clear_conv_flag(&fc) != 0)
+        la::read_and_clear_conv_flag(&fc) != 0 || la::read_and_clear_rope_flag(&fr) != 0)
         return LA_ECUDA;
-    return (flag | fk | fq | fc) ? LA_ETIMEOUT : LA_OK;
+    return (flag | fk | fq | fc | fr) ? LA_ETIMEOUT : LA_OK;
 }
 
 la_status la_selftest_bounded_wait(void *stream) {

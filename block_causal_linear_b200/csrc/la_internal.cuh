@@ -21,6 +21,51 @@ constexpr int kApplyRows = 128;        // token rows per apply tile (= MMA M)
 constexpr int kOpRows = 48;            // N of the apply MMA: 32 S columns, Z, 15 zero rows
 constexpr int kOpBytes = kOpRows * kD * 2;   // one bf16 operand (hi or lo) = 3072 B
 
+// A stream-K plan: a call's work as units (a head group or a head pair of one
+// batch element and block) in the order (b, block, unit), each unit cut into
+// granules of a fixed number of tokens; CTA c takes granules
+// [c * total / C, (c + 1) * total / C) of that order, so every CTA gets the
+// same amount of work whatever the shapes.  A function of the shapes only.
+struct Sk {
+    long long total;   // granules in the call
+    int C;             // CTAs
+    int units;         // units per (b, block)
+    int g_full;        // granules of a full block
+    int g_last;        // granules of the last block
+    int nb;            // blocks
+};
+
+__host__ __device__ inline long long sk_per_b(const Sk &s) {
+    return (long long)s.units * ((long long)(s.nb - 1) * s.g_full + s.g_last);
+}
+// First granule of CTA c (c = C gives the end).
+__host__ __device__ inline long long sk_cta_start(const Sk &s, int c) { return (long long)c * s.total / s.C; }
+// The CTA whose range holds granule x.
+__host__ __device__ inline int sk_cta_of(const Sk &s, long long x) {
+    return (int)(((x + 1) * (long long)s.C - 1) / s.total);
+}
+// Granules of a unit of block n, and the first granule of unit (b, n, u).
+__host__ __device__ inline int sk_len(const Sk &s, int n) { return n < s.nb - 1 ? s.g_full : s.g_last; }
+__host__ __device__ inline long long sk_unit_first(const Sk &s, int b, int n, int u) {
+    return (long long)b * sk_per_b(s) + (long long)n * s.units * s.g_full + (long long)u * sk_len(s, n);
+}
+// The unit (b, n, u) that holds granule x.
+__host__ __device__ inline void sk_locate(const Sk &s, long long x, int &b, int &n, int &u) {
+    const long long pb = sk_per_b(s);
+    b = (int)(x / pb);
+    long long r = x - (long long)b * pb;
+    const long long full = (long long)(s.nb - 1) * s.units * s.g_full;
+    if (r < full) {
+        const long long blk = (long long)s.units * s.g_full;
+        n = (int)(r / blk);
+        r -= (long long)n * blk;
+        u = (int)(r / s.g_full);
+    } else {
+        n = s.nb - 1;
+        u = (int)((r - full) / s.g_last);
+    }
+}
+
 // Everything a kernel needs to know about one call, passed by value.
 // Input kinds of the tensor-core kernels: bf16 q, k, v; FP8 E4M3 codes with
 // per-tensor scales; NVFP4 (E2M1 codes, an E4M3 scale per 16 features, a
@@ -51,6 +96,20 @@ struct Plan {
     // invariant integer through a multiply, Granlund & Montgomery 1994)
     unsigned long long hw_m, wg_m;
     int hw_s, wg_s;
+    // The RoPE tensor-core kernels (k_rope_tc.cu): stream-K plans of the
+    // reduce (head groups x 16-token granules) and of the apply (head pairs x
+    // 128-token tiles); the reduce's split sums then sit in skP slots per
+    // (b, h, block), slot j holding the sums of the j-th CTA that met the unit.
+    int sk_layout;        // the split sums are in the stream-K layout
+    int skP;              // slots per (b, h, block) of that layout (a bound)
+    Sk skr, ska;
+    // Their cos/sin table: the 8 groups of 4 features ("half chunks": 2 pairs
+    // each, one axis) read records of (cos a, cos b, sin a, sin b) at byte
+    // hc_base[m] + position * hc_stride[m] of the table, position along axis
+    // hc_axis[m] (0 frame relative to token 0 of the call, 1 row, 2 column).
+    int hc_base[8], hc_stride[8], hc_axis[8];
+    int tab_frames;       // frames the table covers (all frames of the call)
+    int tab_bytes;        // table size; 0 if the RoPE sections do not fit this layout
 };
 
 // m, s with floor(n / d) == (n * m) >> s for every 0 <= n < 2^31 (1 <= d < 2^31):
@@ -84,6 +143,10 @@ struct WsLayout {
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Split-sum slots per (b, h, block) that the workspace holds for a plan: the
+// split plan's P, or the stream-K layout's, whichever is larger.
+inline int ws_slots(const Plan &p) { return p.P > p.skP ? p.P : p.skP; }
 
 inline WsLayout ws_layout(int B, int H, int nb, int P) {
     WsLayout w;
@@ -136,9 +199,19 @@ int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &
 int launch_apply_tc(const void *q, void *out, const void *bop, const float *seff, const Plan &p,
                     cudaStream_t s);
 bool tc_available();
-// The RoPE variants keep a per-CTA (cos, sin) table in shared memory; true if
-// it fits for this plan (else the call takes the CUDA-core kernels).
+// RoPE on the tensor cores (k_rope_tc.cu): the stream-K plans of a call and
+// the layout of its cos/sin table (shape-only; sets skr, ska, skP and the
+// table fields), whether the table fits the kernels' shared memory, and the
+// two kernels.  The reduce writes its split sums in the stream-K layout
+// (p.sk must be set for the combine), the apply reads the packed operand and
+// Z_eff the combine wrote.
+void plan_rope_sk(Plan &p);
+void plan_rope_table(Plan &p);
 bool tc_rope_fits(const Plan &p);
+int launch_reduce_rope_tc(const void *k, const void *v, float *partials, const Plan &p, cudaStream_t s);
+int launch_apply_rope_tc(const void *q, void *out, const void *bop, const float *seff, const Plan &p,
+                         cudaStream_t s);
+int read_and_clear_rope_flag(unsigned *flag_out);
 
 // Backward pass (CUDA cores, fp32 or bf16 tensors): dq and the per-split
 // [dS | dZ] sums from q, dout and the forward prefix state; the suffix sums

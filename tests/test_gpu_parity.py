@@ -76,6 +76,9 @@ CASES = [  # B, N, H, tokens_per_block, dtype, rope
     (1, 900, 4, 250, torch.bfloat16, True),
     (1, 500, 6, 0, torch.bfloat16, False),       # H not a multiple of 4
     (1, 333, 2, 100, torch.bfloat16, True),
+    (1, 3000, 64, 0, torch.bfloat16, True),      # RoPE: every head group split over many CTAs
+    (3, 2000, 12, 700, torch.bfloat16, True),    # RoPE: 3 blocks, the last one short, B 3
+    (2, 2100, 16, 1000, torch.bfloat16, True),   # RoPE: a last block of 100 tokens
     (2, 300, 3, 64, torch.float32, False),
     (1, 257, 4, 0, torch.float32, True),
 ]
