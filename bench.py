@@ -538,9 +538,41 @@ def main():
             for j in range(3):
                 stage_ms[j] += e[j].elapsed_time(e[j + 1])
     stage_ms = [x * K / Ks for x in stage_ms]      # scaled to K steps like total_ms
+
+    # The step's last writes can still sit dirty in L2 when its last kernel
+    # ends; they reach DRAM during the next (untimed) flush.  A second timing
+    # counts them: the step followed by a read of a buffer twice the size of
+    # L2 (which evicts every dirty line) between event nodes of one graph,
+    # minus the same read alone after a flush.
+    wb_start = torch.cuda.Event(enable_timing=True, external=True)
+    wb_end = torch.cuda.Event(enable_timing=True, external=True)
+    rd_start = torch.cuda.Event(enable_timing=True, external=True)
+    rd_end = torch.cuda.Event(enable_timing=True, external=True)
+    evict = torch.empty(1, dtype=torch.float32, device=dev)
+    graph_wb, graph_rd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_wb):
+        wb_start.record()
+        runner.step()
+        torch.sum(flush_r, dim=0, out=evict)
+        wb_end.record()
+    with torch.cuda.graph(graph_rd):
+        rd_start.record()
+        torch.sum(flush_r, dim=0, out=evict)
+        rd_end.record()
+    Kw = min(K, 100)
+    wb_ms = rd_ms = 0.0
+    for kk in range(Kw):
+        flush.fill_(float(kk))
+        graph_wb.replay()
+        flush.fill_(float(kk))
+        graph_rd.replay()
+        torch.cuda.synchronize()
+        wb_ms += wb_start.elapsed_time(wb_end)
+        rd_ms += rd_start.elapsed_time(rd_end)
+    wb_step_ms = (wb_ms - rd_ms) / Kw
     total_ms = sum(step_ms)
-    total_ms, outer_total_ms, red_ms, fin_ms, app_ms = ranks.max_over_ranks(
-        [total_ms, sum(outer_ms)] + stage_ms, dist, dev)
+    total_ms, outer_total_ms, red_ms, fin_ms, app_ms, wb_step_ms = ranks.max_over_ranks(
+        [total_ms, sum(outer_ms)] + stage_ms + [wb_step_ms], dist, dev)
 
     th_step = w.token_heads                          # per rank per step
     value = ranks.job_throughput(th_step, world, K, total_ms)
@@ -609,6 +641,8 @@ def main():
                                                           if args.shard == "heads" else
                                                           f"independent problem per rank x{world}")}),
             "achieved_hbm_gbs": step_gbs, "hbm_frac_of_" + peak_kind: step_gbs / peak,
+            "ms_per_step_incl_writeback": wb_step_ms,
+            "hbm_frac_incl_writeback_of_" + peak_kind: alg_bytes / (wb_step_ms / 1e3) / 1e9 / peak,
             "stage_ms_per_step": ({"forward_state": red_ms / K, "query_side": fin_ms / K, "key_side": app_ms / K}
                                   if bwd else {"reduce": red_ms / K, "finish": fin_ms / K, "apply": app_ms / K}),
             "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,

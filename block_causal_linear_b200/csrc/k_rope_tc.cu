@@ -29,7 +29,7 @@
 // reproducible.
 //
 // Shared memory is laid out for depth: the TMA tiles land in a ring of raw
-// stages (160 KiB in the reduce, 112 KiB in the apply) separate from the
+// stages (176 KiB in the reduce, 144 KiB in the apply) separate from the
 // transformed operands the tensor cores read, so that a raw q stage is free
 // as soon as the transform has read it.  The cos/sin table holds records of
 // two feature pairs (cos a, cos b, sin a, sin b) per position of each axis;
@@ -37,8 +37,10 @@
 // phase read 8 consecutive rows: distinct 16-byte chunks of the swizzled
 // tiles, and for the column axis distinct consecutive records.
 //
-// Warp roles (448 threads): 0 TMA, 1 TMEM owner and MMA issue, 2..5 epilogue
-// (warp w reads TMEM lanes 32 (w % 4) ..), 6..13 transform.  Every wait is
+// Warp roles (736 threads): 0 and 6 TMA (even and odd stages), 1 TMEM owner
+// and MMA issue, 2..5 epilogue (warp w reads TMEM lanes 32 (w % 4) ..), 7..22
+// transform.  The transform is latency-bound (long dependent chains per
+// chunk), so it gets 16 warps: 4 per scheduler.  Every wait is
 // bounded (la_sm100.cuh): one that gives up raises this file's device flag,
 // read by la_device_status, and the CTA drains its copies and MMAs, frees
 // its TMEM and returns.
@@ -62,14 +64,30 @@ namespace {
 
 constexpr int kTabBytes = 8192;          // cos/sin table of a call
 constexpr int kMinGranules = 8;          // fewest 16-token granules a reduce CTA takes
+
 constexpr int kBox = 32 * 128;           // 32 token rows x 64 bf16 features (2 heads): 4 KiB
-constexpr int kThreads = 448;
-constexpr int kWarpTma = 0, kWarpMma = 1;
-constexpr int kXf0 = 192;                // first transform thread (warp 6)
-constexpr int kNXf = 256;                // transform threads
+constexpr int kThreads = 736;
+// Two warps issue the TMA loads, even and odd stages: one issuing warp moves
+// at most ~27 GB/s per SM of 4-16 KiB tiles (about 4.0 TB/s over the GPU,
+// measured), two reach the copy bandwidth.
+constexpr int kWarpTma0 = 0, kWarpMma = 1, kWarpTma1 = 6;
+constexpr int kXf0 = 224;                // first transform thread (warp 7)
+constexpr int kNXf = 512;                // transform threads (warps 7..22)
 constexpr int kNEpi = 128;               // epilogue threads (warps 2..5)
+// Barriers that several warps release take one arrival per warp (lane 0,
+// after __syncwarp orders the warp's shared-memory work before it): hundreds
+// of per-thread arrivals on one barrier word serialise in shared memory.
+constexpr int kXfWarps = kNXf / 32, kEpiWarps = kNEpi / 32;
+
+// One arrival for the whole warp, after every lane's preceding work.
+__device__ __forceinline__ void warp_arrive(uint64_t *bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
 
 // ---------------------------------------------------------------- reduce layout
+// The raw ring is as deep as shared memory allows: under load a copy takes
+// ~4 us from issue to arrival, and only the stages in flight move data.
 constexpr int kRRaw = 10;                // raw stages: k (2 boxes) and v (2 boxes) of 32 tokens x 4 heads
 constexpr int kROp = 3;                  // transformed stages: R phi(k) hi (2 boxes), lo (2 boxes)
 constexpr int kRStage = 4 * kBox;        // 16 KiB, raw and transformed alike
@@ -79,23 +97,34 @@ constexpr int kRZOff = kRTabOff + kTabBytes;             // z sums [2][4 heads][
 constexpr int kRBarOff = kRZOff + 2 * 128 * 4;
 constexpr int kRNumBars = 2 * kRRaw + 2 * kROp + 2 * 4 + 1;
 constexpr int kRSmem = kRBarOff + kRNumBars * 8 + 16 + 1024;
-constexpr uint32_t kRTmemCols = 256;     // two accumulators of 128 columns
+// Per 16 tokens one M=128 x N=256 MMA: A = V of the 4 heads (value features
+// as rows), B = [R phi(K) hi | R phi(K) lo] (key features as columns), so the
+// V tile is read once, not once per part; D = [V^T R phi(K)_hi | V^T R phi(K)_lo],
+// the 4 diagonal 32x32 blocks of each half used.  Two accumulators.
+constexpr uint32_t kRTmemCols = 256;
 static_assert(kRSmem <= 232448, "reduce shared memory");
 
 // ---------------------------------------------------------------- apply layout
 constexpr int kATile = 128 * 128;        // 128 tokens x 64 bf16 features (2 heads): 16 KiB
-constexpr int kARaw = 7;                 // raw q stages
-constexpr int kAOp = 2;                  // transformed tiles: R phi(q) hi, then lo
-constexpr int kAOpOff = kARaw * kATile;
-constexpr int kAStgOff = kAOpOff + kAOp * 2 * kATile;   // one [32 rows][64 bf16] staging box per epilogue warp
+// The apply is bound by shared-memory bandwidth, so the rotated phi(q) (hi and
+// lo parts) goes to the tensor cores through tensor memory, not shared
+// memory: the transform stores it with tcgen05.st and the MMA reads A from
+// TMEM.  That leaves shared memory to the raw ring.
+constexpr int kARaw = 11;                // raw q stages
+constexpr int kAOp = 4;                  // transformed tiles in TMEM (hi, lo of 2 heads: 64 columns each)
+constexpr int kAStgOff = kARaw * kATile; // one [32 rows][64 bf16] staging box per epilogue warp
 constexpr int kABopBytes = 4 * 2048 + 256;              // S rows hi, lo of 2 heads, then Z_eff of 2 heads
 constexpr int kABopOff = kAStgOff + 4 * kBox;
-constexpr int kADenOff = kABopOff + 2 * kABopBytes;     // denominators [2][2 heads][128 rows] fp32
-constexpr int kATabOff = kADenOff + 2 * 256 * 4;
+constexpr int kADenOff = kABopOff + 2 * kABopBytes;     // denominator halves [2][2 heads][2][128 rows] fp32
+constexpr int kATabOff = kADenOff + 2 * 512 * 4;
 constexpr int kABarOff = kATabOff + kTabBytes;
 constexpr int kANumBars = 2 * kARaw + 2 * kAOp + 2 * 2 + 2 * 2 + 2 * 2 + 1;
 constexpr int kASmem = kABarOff + kANumBars * 8 + 16 + 1024;
-constexpr uint32_t kATmemCols = 128;     // two accumulators of 2 heads x 32 columns
+// TMEM: two accumulators of 2 heads x 32 columns (columns 0..127), then the
+// transformed tiles (columns 128..255): head hh at + 32 hh, hi at + 0, lo at
+// + 16, the 16-feature K step kk at + 8 kk
+constexpr uint32_t kATmemCols = 512;
+constexpr uint32_t kATmemA = 128;
 static_assert(kASmem <= 232448, "apply shared memory");
 static_assert(kABopBytes % 16 == 0 && kABopOff % 16 == 0, "bulk copies need 16-byte alignment");
 
@@ -168,7 +197,9 @@ __device__ __forceinline__ void rope_chunk(uint4 x, float4 t0, float4 t1, uint4 
 // group's axis (frames of the call, rows, columns), at the byte offsets the
 // host planned.
 __device__ void build_table(uint8_t *tab, const Plan &p, int tid, int nthr) {
-#pragma unroll 1
+    // (unrolled: the plan's arrays are then read at fixed offsets of the
+    // kernel parameters, never copied to local memory)
+#pragma unroll
     for (int m = 0; m < 8; ++m) {
         const int ax = p.hc_axis[m];
         const int len = ax == 0 ? p.tab_frames : (ax == 1 ? p.Hg : p.Wg);
@@ -197,13 +228,32 @@ __device__ __forceinline__ Pos token_pos(const Plan &p, int jg) {
     return q;
 }
 
+// The position d tokens further on (d >= 0): columns wrap into rows, rows
+// into frames.
+__device__ __forceinline__ void pos_step(const Plan &p, Pos &q, int d) {
+    q.w += d;
+    while (q.w >= p.Wg) {
+        q.w -= p.Wg;
+        if (++q.h == p.Hg) {
+            q.h = 0;
+            ++q.f;
+        }
+    }
+}
+
 // Where the records of feature group m sit in the table.
 struct GroupRec {
     int base, stride, axis;
 };
 
 __device__ __forceinline__ GroupRec group_rec(const Plan &p, int m) {
-    return GroupRec{p.hc_base[m], p.hc_stride[m], p.hc_axis[m]};
+    // select by an unrolled compare, so that the parameter arrays are never
+    // indexed at run time (which would copy them to local memory)
+    GroupRec g{0, 0, 0};
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        if (k == m) g = GroupRec{p.hc_base[k], p.hc_stride[k], p.hc_axis[k]};
+    return g;
 }
 
 __device__ __forceinline__ float4 tab_rec(const uint8_t *tab, const GroupRec &g, const Pos &q) {
@@ -280,25 +330,24 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             mbar_init(&raw_empty[s], 1);
         }
         for (int o = 0; o < kROp; ++o) {
-            mbar_init(&op_full[o], kNXf);
+            mbar_init(&op_full[o], kXfWarps);
             mbar_init(&op_empty[o], 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&acc_full[a], 1);
-            mbar_init(&acc_empty[a], kNEpi);
-            mbar_init(&z_full[a], kNXf);
-            mbar_init(&z_empty[a], kNEpi);
+            mbar_init(&acc_empty[a], kEpiWarps);
+            mbar_init(&z_full[a], kXfWarps);
+            mbar_init(&z_empty[a], kEpiWarps);
         }
         mbar_init(drain, 1);
         *abort_word = 0;
         fence_barrier_init();
     }
-    build_table(tab, p, threadIdx.x, kThreads);
     if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, kRTmemCols);
         tmem_relinquish();
     }
-    if (warp == kWarpTma && lane == 0) {
+    if ((warp == kWarpTma0 || warp == kWarpTma1) && lane == 0) {
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
     }
@@ -325,9 +374,10 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         sg.slot = cta - sk_cta_of(S, w.first);
         return sg;
     };
-    int issued = 0;
+    int issued = 0;   // stages issued by this TMA warp: the last one + 1
+    const int ti = warp == kWarpTma0 ? 0 : 1;
 
-    if (warp == kWarpTma) {
+    if (warp == kWarpTma0 || warp == kWarpTma1) {
         if (lane == 0) {
             UnitWalk w;
             w.start(S, x_begin);
@@ -338,6 +388,7 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 const Seg sg = seg_of(w, x);
                 const int nst = (sg.tok1 - sg.tok0 + 31) / 32;
                 for (int st = 0; st < nst; ++st, ++i) {
+                    if ((i & 1) != ti) continue;   // the other TMA warp's stage
                     const int s = i % kRRaw;
                     if (!mbar_wait(&raw_empty[s], ((uint32_t)(i / kRRaw) & 1u) ^ 1u, abort_word, &g_rope_wait_flag,
                                    1)) {
@@ -385,8 +436,9 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                     const uint32_t va = smem_u32(smem + s * kRStage + 2 * kBox);
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk) {
-                        // MN-major, 128-byte swizzle: the two 64-feature boxes are the
-                        // MN atoms (kBox apart), 8-token groups 1024 B apart
+                        // MN-major, 128-byte swizzle: the 64-feature boxes are the MN
+                        // atoms (kBox apart: v box 0, 1 for A; hi box 0, 1, lo box 0, 1
+                        // for B), 8-token groups 1024 B apart, 16 tokens = 2048 B per step
                         const uint64_t dh = smem_desc(hi + kk * 2048, kBox, 1024, kLayoutSw128);
                         const uint64_t dl = smem_desc(hi + 2 * kBox + kk * 2048, kBox, 1024, kLayoutSw128);
                         const uint64_t dv = smem_desc(va + kk * 2048, kBox, 1024, kLayoutSw128);
@@ -407,7 +459,8 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         }
     } else if (warp < 6) {
         // ------------------------------------------------ epilogue: warp quarter q
-        // reads TMEM lanes 32q.. = key features of head 4g + q
+        // reads TMEM lanes 32q.. = value features of head 4g + q; its key
+        // features are columns 32q.. of the hi half and 128 + 32q.. of the lo half
         const int q = warp & 3;
         UnitWalk w;
         w.start(S, x_begin);
@@ -427,8 +480,8 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             tmem_wait_ld();
             const float z = zbuf[a * 128 + q * 32 + lane];
             tc_fence_before();
-            mbar_arrive(&acc_empty[a]);
-            mbar_arrive(&z_empty[a]);
+            warp_arrive(&acc_empty[a]);
+            warp_arrive(&z_empty[a]);
             const int h = 4 * sg.g + q;
             float *dst = partials + ((((size_t)sg.b * p.H + h) * p.nb + sg.n) * p.skP + sg.slot) * kKVZ;
             float4 *drow = reinterpret_cast<float4 *>(dst + lane * kD);
@@ -438,16 +491,19 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         }
     } else {
         // ------------------------------------------------ transform: one token row
-        // (lane) per stage, feature chunk j of head hl (box 0) and of head 2 + hl
-        // (box 1): the same 8 features, so one position and one pair of records
+        // (lane) per stage, feature chunk j of one head of the group.  The
+        // transform warps build the cos/sin table while the first copies fly.
         const int wt = threadIdx.x - kXf0;
-        const int j = (wt >> 5) & 3, hl = wt >> 7;
+        build_table(tab, p, wt, kNXf);
+        named_bar_sync(1, kNXf);
+        const int xw = wt >> 5;
+        const int j = xw & 3, head = xw >> 2;
         const int r = lane;
-        const int chunk = (((4 * hl + j) ^ (r & 7)) << 4) + r * 128;   // byte offset inside a box
+        // byte offset of the chunk in a stage: box head / 2, 64-byte half head % 2
+        const int chunk = (head >> 1) * kBox + r * 128 + (((4 * (head & 1) + j) ^ (r & 7)) << 4);
         const GroupRec g0 = group_rec(p, 2 * j), g1 = group_rec(p, 2 * j + 1);
-        Feat8 zs[2];
-#pragma unroll
-        for (int bx = 0; bx < 2; ++bx) zs[bx].e0 = zs[bx].o0 = zs[bx].e1 = zs[bx].o1 = make_float2(0.f, 0.f);
+        Feat8 zs;
+        zs.e0 = zs.o0 = zs.e1 = zs.o1 = make_float2(0.f, 0.f);
         UnitWalk w;
         w.start(S, x_begin);
         bool ok = true;
@@ -456,79 +512,58 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             w.to(S, x);
             const Seg sg = seg_of(w, x);
             const int nst = (sg.tok1 - sg.tok0 + 31) / 32;
+            Pos pq = token_pos(p, sg.n * p.L + sg.tok0 + r);   // this row's token in stage 0
             for (int st = 0; st < nst; ++st, ++i) {
                 const int s = i % kRRaw, o = i % kROp;
                 if (ok && !mbar_wait(&raw_full[s], (uint32_t)(i / kRRaw) & 1u, abort_word, &g_rope_wait_flag, 6))
                     ok = false;
-                if (ok && !mbar_wait(&op_empty[o], ((uint32_t)(i / kROp) & 1u) ^ 1u, abort_word, &g_rope_wait_flag, 7))
-                    ok = false;
                 const int tb = sg.tok0 + 32 * st + r;   // token of this row inside the block
                 const uint8_t *raw = smem + s * kRStage;
                 uint8_t *op = smem + kROpOff + o * kRStage;
+                uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;   // rows past the segment contribute nothing
                 if (ok && tb < sg.tok1) {
-                    const Pos pq = token_pos(p, sg.n * p.L + tb);
                     const float4 t0 = tab_rec(tab, g0, pq);
                     const float4 t1 = tab_rec(tab, g1, pq);
-#pragma unroll
-                    for (int bx = 0; bx < 2; ++bx) {
-                        const uint4 xv = *reinterpret_cast<const uint4 *>(raw + bx * kBox + chunk);
-                        uint4 hi, lo;
-                        Feat8 f;
-                        rope_chunk(xv, t0, t1, hi, lo, f);
-                        zs[bx].e0 = fadd2(zs[bx].e0, f.e0);
-                        zs[bx].o0 = fadd2(zs[bx].o0, f.o0);
-                        zs[bx].e1 = fadd2(zs[bx].e1, f.e1);
-                        zs[bx].o1 = fadd2(zs[bx].o1, f.o1);
-                        *reinterpret_cast<uint4 *>(op + bx * kBox + chunk) = hi;
-                        *reinterpret_cast<uint4 *>(op + 2 * kBox + bx * kBox + chunk) = lo;
-                    }
-                } else {
-                    // rows past the segment contribute nothing
-                    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-                    for (int bx = 0; bx < 2; ++bx) {
-                        *reinterpret_cast<uint4 *>(op + bx * kBox + chunk) = zero;
-                        *reinterpret_cast<uint4 *>(op + 2 * kBox + bx * kBox + chunk) = zero;
-                    }
+                    Feat8 f;
+                    rope_chunk(*reinterpret_cast<const uint4 *>(raw + chunk), t0, t1, hi, lo, f);
+                    zs.e0 = fadd2(zs.e0, f.e0);
+                    zs.o0 = fadd2(zs.o0, f.o0);
+                    zs.e1 = fadd2(zs.e1, f.e1);
+                    zs.o1 = fadd2(zs.o1, f.o1);
                 }
+                // the transformed stage is free once the MMAs of stage i - kROp are done
+                if (ok && !mbar_wait(&op_empty[o], ((uint32_t)(i / kROp) & 1u) ^ 1u, abort_word, &g_rope_wait_flag, 7))
+                    ok = false;
+                *reinterpret_cast<uint4 *>(op + chunk) = hi;
+                *reinterpret_cast<uint4 *>(op + 2 * kBox + chunk) = lo;
                 // the generic writes of this stage before the tensor cores read it
                 fence_proxy_async_smem();
-                mbar_arrive(&op_full[o]);
+                warp_arrive(&op_full[o]);
+                pos_step(p, pq, 32);
             }
-            // the segment's z: sum this thread's 16 features over the 32 rows
-            float zv[16];
+            // the segment's z: this thread's 8 features summed over the 32 rows
+            float zv[8] = {zs.e0.x, zs.o0.x, zs.e0.y, zs.o0.y, zs.e1.x, zs.o1.x, zs.e1.y, zs.o1.y};
+            zs.e0 = zs.o0 = zs.e1 = zs.o1 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int bx = 0; bx < 2; ++bx) {
-                const Feat8 &f = zs[bx];
-                float *t = zv + 8 * bx;
-                t[0] = f.e0.x; t[1] = f.o0.x; t[2] = f.e0.y; t[3] = f.o0.y;
-                t[4] = f.e1.x; t[5] = f.o1.x; t[6] = f.e1.y; t[7] = f.o1.y;
-                zs[bx].e0 = zs[bx].o0 = zs[bx].e1 = zs[bx].o1 = make_float2(0.f, 0.f);
-            }
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
+            for (int k = 0; k < 8; ++k)
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) zv[k] += __shfl_xor_sync(0xffffffffu, zv[k], off);
             const int a = sidx & 1;
             if (ok && !mbar_wait(&z_empty[a], ((uint32_t)(sidx >> 1) & 1u) ^ 1u, abort_word, &g_rope_wait_flag, 8))
                 ok = false;
             if (lane == 0) {
-#pragma unroll
-                for (int bx = 0; bx < 2; ++bx) {
-                    float4 *zz = reinterpret_cast<float4 *>(zbuf + a * 128 + (2 * bx + hl) * 32 + 8 * j);
-                    zz[0] = make_float4(zv[8 * bx], zv[8 * bx + 1], zv[8 * bx + 2], zv[8 * bx + 3]);
-                    zz[1] = make_float4(zv[8 * bx + 4], zv[8 * bx + 5], zv[8 * bx + 6], zv[8 * bx + 7]);
-                }
+                float4 *zz = reinterpret_cast<float4 *>(zbuf + a * 128 + head * 32 + 8 * j);
+                zz[0] = make_float4(zv[0], zv[1], zv[2], zv[3]);
+                zz[1] = make_float4(zv[4], zv[5], zv[6], zv[7]);
             }
-            __syncwarp();
-            mbar_arrive(&z_full[a]);
+            warp_arrive(&z_full[a]);
         }
     }
 
     // teardown: nothing may still write this CTA's shared memory or TMEM
-    if (warp == kWarpTma && lane == 0 && *abort_word) {
+    if ((warp == kWarpTma0 || warp == kWarpTma1) && lane == 0 && *abort_word) {
         for (int i = issued - kRRaw < 0 ? 0 : issued - kRRaw; i < issued; ++i)
-            final_wait(&raw_full[i % kRRaw], (uint32_t)(i / kRRaw) & 1u);
+            if ((i & 1) == ti) final_wait(&raw_full[i % kRRaw], (uint32_t)(i / kRRaw) & 1u);
     }
     tc_fence_before();
     __syncwarp();
@@ -578,17 +613,17 @@ rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (threadIdx.x == 0) {
         for (int s = 0; s < kARaw; ++s) {
             mbar_init(&raw_full[s], 1);
-            mbar_init(&raw_empty[s], kNXf);
+            mbar_init(&raw_empty[s], kXfWarps);
         }
         for (int o = 0; o < kAOp; ++o) {
-            mbar_init(&op_full[o], kNXf);
+            mbar_init(&op_full[o], kXfWarps);
             mbar_init(&op_empty[o], 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&acc_full[a], 1);
-            mbar_init(&acc_empty[a], kNEpi);
-            mbar_init(&den_full[a], kNXf);
-            mbar_init(&den_empty[a], kNEpi);
+            mbar_init(&acc_empty[a], kEpiWarps);
+            mbar_init(&den_full[a], kXfWarps);
+            mbar_init(&den_empty[a], kEpiWarps);
             mbar_init(&bop_full[a], 1);
             mbar_init(&bop_empty[a], 1);
         }
@@ -596,12 +631,11 @@ rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         *abort_word = 0;
         fence_barrier_init();
     }
-    build_table(tab, p, threadIdx.x, kThreads);
     if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, kATmemCols);
         tmem_relinquish();
     }
-    if (warp == kWarpTma && lane == 0) {
+    if ((warp == kWarpTma0 || warp == kWarpTma1) && lane == 0) {
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_out);
     }
@@ -609,9 +643,10 @@ rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    int issued = 0, bops_issued = 0;
+    int issued = 0, bops_issued = 0;   // by this TMA warp: the last q tile + 1, operands loaded
+    const int ti = warp == kWarpTma0 ? 0 : 1;
 
-    if (warp == kWarpTma) {
+    if (warp == kWarpTma0 || warp == kWarpTma1) {
         if (lane == 0) {
             auto load_q = [&](const UnitWalk &w, long long x, int i) {
                 const int s = i % kARaw;
@@ -638,23 +673,25 @@ rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 return true;
             };
             // q is an input of the call, complete before this call's reduce
-            // started: the first tiles are fetched while the combine still runs
+            // started: the first tiles are fetched while the combine still runs.
+            // This warp takes the q tiles i with i % 2 == ti; warp 0 also loads
+            // each unit's state operand once the combine is done.
             const int pre = ntiles < kARaw ? ntiles : kARaw;
             UnitWalk w;
             w.start(S, x_begin);
             for (int i = 0; i < pre; ++i) {
                 w.to(S, x_begin + i);
-                load_q(w, x_begin + i, i);
+                if ((i & 1) == ti) load_q(w, x_begin + i, i);
             }
-            pdl_wait();   // the packed operand and Z_eff are written by the combine
+            if (ti == 0) pdl_wait();   // the packed operand and Z_eff are written by the combine
             w.start(S, x_begin);
             int kb = 0;
             for (int i = 0; i < ntiles; ++i) {
                 const long long x = x_begin + i;
                 if (w.to(S, x) || i == 0) {
-                    if (!load_bop(w, kb++)) break;
+                    if (ti == 0 && !load_bop(w, kb++)) break;
                 }
-                if (i < pre) continue;
+                if (i < pre || (i & 1) != ti) continue;
                 const int s = i % kARaw;
                 if (!mbar_wait(&raw_empty[s], ((uint32_t)(i / kARaw) & 1u) ^ 1u, abort_word, &g_rope_wait_flag, 12))
                     break;
@@ -678,7 +715,7 @@ rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (!mbar_wait(&acc_empty[a], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_word, &g_rope_wait_flag, 14)) break;
                 if (!mbar_wait(&op_full[o], (uint32_t)(i / kAOp) & 1u, abort_word, &g_rope_wait_flag, 15)) break;
                 tc_fence_after();
-                const uint32_t qa = smem_u32(smem + kAOpOff + o * 2 * kATile);
+                const uint32_t qa = tmem + kATmemA + (uint32_t)(o * 64);
                 const uint32_t ba = smem_u32(bops + (kb & 1) * kABopBytes);
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
@@ -689,15 +726,13 @@ rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         const int apart = prod == 2 ? 1 : 0, bpart = prod == 1 ? 1 : 0;
 #pragma unroll
                         for (int kk = 0; kk < 2; ++kk) {
-                            // A: K-major, 128-byte swizzle; head hh is the 64-byte half of
-                            // each 128-byte row, 16 features = 32 bytes per step
-                            const uint64_t da =
-                                smem_desc(qa + apart * kATile + hh * 64 + kk * 32, 16, 1024, kLayoutSw128);
+                            // A in TMEM: token row = lane, 8 columns per 16 features
+                            const uint32_t ta = qa + (uint32_t)(hh * 32 + apart * 16 + kk * 8);
                             // B: K-major, no swizzle, core matrices 128 B apart along K,
                             // 8-row groups 512 B apart; 16 features = 256 bytes per step
                             const uint64_t db =
                                 smem_desc(ba + hh * 4096 + bpart * 2048 + kk * 256, 128, 512, kLayoutNone);
-                            mma_bf16(d, da, db, idesc, (prod | kk) ? 1u : 0u);
+                            mma_bf16_ta(d, ta, db, idesc, (prod | kk) ? 1u : 0u);
                         }
                     }
                 }
@@ -710,87 +745,106 @@ rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 final_wait(drain, 0);
             }
         }
-    } else if (warp >= 6) {
+    } else if (warp >= 7) {
         // ------------------------------------------------ transform: token row r of
-        // the tile, the 4 feature chunks of head hh
+        // the tile, feature chunks 2 jh and 2 jh + 1 of head hh.  A warp writes
+        // TMEM lanes 32 (warp % 4) .., so its rows are that quarter of the tile.
+        // The transform warps build the cos/sin table while the first q tiles fly.
         const int wt = threadIdx.x - kXf0;
-        const int hh = wt >> 7, r = wt & 127;
-        float2 ze[4][2], zo[4][2];   // Z_eff of head hh: chunk j, pairs (a, b) / (c, d), even / odd features
+        build_table(tab, p, wt, kNXf);
+        named_bar_sync(1, kNXf);
+        const int xw = (warp - 7) >> 2;   // 0..3: which of the 4 warps of a lane quarter
+        const int hh = xw >> 1, jh = xw & 1;
+        const int r = 32 * (warp & 3) + lane;
+        const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+        const GroupRec gr[2][2] = {{group_rec(p, 4 * jh), group_rec(p, 4 * jh + 1)},
+                                   {group_rec(p, 4 * jh + 2), group_rec(p, 4 * jh + 3)}};
+        float2 ze[2][2], zo[2][2];   // Z_eff of head hh: chunk, pairs (a, b) / (c, d), even / odd features
         UnitWalk w;
         w.start(S, x_begin);
         bool ok = true;
         int kb = -1;
+        Pos pq{};
         for (int i = 0; i < ntiles; ++i) {
             const long long x = x_begin + i;
-            if (w.to(S, x) || i == 0) {
+            w.to(S, x);
+            const int row0 = (int)(x - w.first) * 128;
+            if (i == 0 || x == w.first) {   // the first tile of a unit in this CTA
                 ++kb;
                 if (ok && !mbar_wait(&bop_full[kb & 1], (uint32_t)(kb >> 1) & 1u, abort_word, &g_rope_wait_flag, 16))
                     ok = false;
                 const float4 *zsrc = reinterpret_cast<const float4 *>(bops + (kb & 1) * kABopBytes + 8192 + hh * 128);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int c = 0; c < 2; ++c) {
+                    const int j = 2 * jh + c;
                     const float4 u0 = zsrc[2 * j], u1 = zsrc[2 * j + 1];   // features 8j .. 8j + 7
-                    ze[j][0] = make_float2(u0.x, u0.z);
-                    zo[j][0] = make_float2(u0.y, u0.w);
-                    ze[j][1] = make_float2(u1.x, u1.z);
-                    zo[j][1] = make_float2(u1.y, u1.w);
+                    ze[c][0] = make_float2(u0.x, u0.z);
+                    zo[c][0] = make_float2(u0.y, u0.w);
+                    ze[c][1] = make_float2(u1.x, u1.z);
+                    zo[c][1] = make_float2(u1.y, u1.w);
                 }
+                pq = token_pos(p, w.n * p.L + row0 + r);
+            } else {
+                pos_step(p, pq, 128);
             }
             const int s = i % kARaw, o = i % kAOp, a = i & 1;
             const int Ln = w.n < p.nb - 1 ? p.L : Llast;
-            const int row0 = (int)(x - w.first) * 128;
             const bool valid = r < Ln - row0;
             if (ok && !mbar_wait(&raw_full[s], (uint32_t)(i / kARaw) & 1u, abort_word, &g_rope_wait_flag, 17)) ok = false;
-            uint4 xq[4];
+            uint4 xq[2];
             const uint8_t *raw = smem + s * kATile + r * 128;
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                xq[j] = (ok && valid) ? *reinterpret_cast<const uint4 *>(raw + (((4 * hh + j) ^ (r & 7)) << 4))
+            for (int c = 0; c < 2; ++c)
+                xq[c] = (ok && valid) ? *reinterpret_cast<const uint4 *>(raw + (((4 * hh + 2 * jh + c) ^ (r & 7)) << 4))
                                       : make_uint4(0u, 0u, 0u, 0u);
             // the raw stage may be refilled as soon as every thread has read it:
             // order these generic reads before the async proxy's refill
             fence_proxy_async_smem();
-            mbar_arrive(&raw_empty[s]);
+            warp_arrive(&raw_empty[s]);
+            uint4 hi[2], lo[2];
+            float2 den = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                hi[c] = lo[c] = make_uint4(0u, 0u, 0u, 0u);
+                if (ok && valid) {
+                    Feat8 f;
+                    rope_chunk(xq[c], tab_rec(tab, gr[c][0], pq), tab_rec(tab, gr[c][1], pq), hi[c], lo[c], f);
+                    // the denominator takes the unrotated phi(q)
+                    den = ffma2(f.e0, ze[c][0], den);
+                    den = ffma2(f.o0, zo[c][0], den);
+                    den = ffma2(f.e1, ze[c][1], den);
+                    den = ffma2(f.o1, zo[c][1], den);
+                }
+            }
+            // the transformed tile is free once the MMAs of tile i - kAOp are done
             if (ok && !mbar_wait(&op_empty[o], ((uint32_t)(i / kAOp) & 1u) ^ 1u, abort_word, &g_rope_wait_flag, 18))
                 ok = false;
             if (ok && !mbar_wait(&den_empty[a], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_word, &g_rope_wait_flag, 19))
                 ok = false;
-            uint8_t *op = smem + kAOpOff + o * 2 * kATile + r * 128;
-            float2 den = make_float2(0.f, 0.f);
-            if (ok && valid) {
-                const Pos pq = token_pos(p, w.n * p.L + row0 + r);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float4 t0 = tab_rec(tab, group_rec(p, 2 * j), pq);
-                    const float4 t1 = tab_rec(tab, group_rec(p, 2 * j + 1), pq);
-                    uint4 hi, lo;
-                    Feat8 f;
-                    rope_chunk(xq[j], t0, t1, hi, lo, f);
-                    // the denominator takes the unrotated phi(q)
-                    den = ffma2(f.e0, ze[j][0], den);
-                    den = ffma2(f.o0, zo[j][0], den);
-                    den = ffma2(f.e1, ze[j][1], den);
-                    den = ffma2(f.o1, zo[j][1], den);
-                    const int pc = ((4 * hh + j) ^ (r & 7)) << 4;
-                    *reinterpret_cast<uint4 *>(op + pc) = hi;
-                    *reinterpret_cast<uint4 *>(op + kATile + pc) = lo;
-                }
-            } else {
-                const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int pc = ((4 * hh + j) ^ (r & 7)) << 4;
-                    *reinterpret_cast<uint4 *>(op + pc) = zero;
-                    *reinterpret_cast<uint4 *>(op + kATile + pc) = zero;
-                }
+            // the warp's lanes store together: a wait that gave up in one lane stops the warp
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+                tc_fence_after();
+                // features 16 jh .. 16 jh + 15 of head hh: TMEM columns 8 jh .. 8 jh + 7 of
+                // the head's hi and lo parts (two features per column)
+                const uint32_t ta = tmem + lane_off + kATmemA + (uint32_t)(o * 64 + hh * 32 + 8 * jh);
+                const uint32_t vh[8] = {hi[0].x, hi[0].y, hi[0].z, hi[0].w, hi[1].x, hi[1].y, hi[1].z, hi[1].w};
+                const uint32_t vl[8] = {lo[0].x, lo[0].y, lo[0].z, lo[0].w, lo[1].x, lo[1].y, lo[1].z, lo[1].w};
+                tmem_st8(ta, vh);
+                tmem_st8(ta + 16, vl);
+                tmem_wait_st();
             }
-            den_s[a * 256 + hh * 128 + r] = den.x + den.y;
-            fence_proxy_async_smem();
-            mbar_arrive(&op_full[o]);
-            mbar_arrive(&den_full[a]);
+            den_s[a * 512 + (2 * hh + jh) * 128 + r] = den.x + den.y;
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&op_full[o]);
+                mbar_arrive(&den_full[a]);
+            }
         }
     } else {
-        // ------------------------------------------------ epilogue warps 2..5
+        // ------------------------------------------------ epilogue warps 2..5, one
+        // head at a time
         const int q = warp & 3;
         const int r = 32 * q + lane;               // token row of this thread in a tile
         uint8_t *sb = smem + kAStgOff + q * kBox;  // this warp's staging box
@@ -806,82 +860,75 @@ rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                        mbar_wait(&den_full[a], aph, abort_word, &g_rope_wait_flag, 21);
             got = __all_sync(0xffffffffu, got);
             if (!got) ok = false;
-            float num0[32], num1[32], den0 = 0.f, den1 = 0.f;
-            if (got) {
-                tc_fence_after();
-                const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 64);
-                tmem_ld32(base, num0);
-                tmem_ld32(base + 32, num1);
-                tmem_wait_ld();
-                den0 = den_s[a * 256 + r];
-                den1 = den_s[a * 256 + 128 + r];
-            }
-            tc_fence_before();
-            mbar_arrive(&acc_empty[a]);
-            mbar_arrive(&den_empty[a]);
-            if (!got) continue;
-
             const int Ln = w.n < p.nb - 1 ? p.L : Llast;
             const int row0 = (int)(x - w.first) * 128;
             const int blk0 = w.n * p.L;                // first token of the block in the call
-            const int wrow0 = blk0 + row0 + 32 * q;    // first row of this warp
-            const float2 inv0 = make_float2(1.0f / (den0 + p.eps), 1.0f / (den0 + p.eps));
-            const float2 inv1 = make_float2(1.0f / (den1 + p.eps), 1.0f / (den1 + p.eps));
             // TMA store of the warp's 32 rows unless they run into the next block
             // (rows past the end of the tensor are clipped by TMA)
             const bool boxed = row0 + 32 * q + 32 <= Ln || blk0 + Ln == p.N;
-            if (boxed) {
-                if (lane == 0) bulk_wait_read<0>();   // the last store from this box has read it
-                __syncwarp();
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {          // logical 16-byte chunk c: head c / 4
-                    const float *v = c < 4 ? num0 : num1;
-                    const float2 inv = c < 4 ? inv0 : inv1;
-                    const int f0 = 8 * (c & 3);
-                    const float2 y0 = fmul2(make_float2(v[f0], v[f0 + 1]), inv);
-                    const float2 y1 = fmul2(make_float2(v[f0 + 2], v[f0 + 3]), inv);
-                    const float2 y2 = fmul2(make_float2(v[f0 + 4], v[f0 + 5]), inv);
-                    const float2 y3 = fmul2(make_float2(v[f0 + 6], v[f0 + 7]), inv);
-                    const int pc = c ^ (lane & 7);     // 128-byte swizzle (row % 8 == lane % 8)
-                    *reinterpret_cast<uint4 *>(sb + lane * 128 + pc * 16) =
-                        make_uint4(pack_bf2(y0.x, y0.y), pack_bf2(y1.x, y1.y), pack_bf2(y2.x, y2.y),
-                                   pack_bf2(y3.x, y3.y));
+            if (got) {
+                tc_fence_after();
+                if (boxed) {
+                    if (lane == 0) bulk_wait_read<0>();   // the last store from this box has read it
+                    __syncwarp();
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_3d(&tm_out, sb, w.u * 64, wrow0, w.b);
-                    bulk_commit();
-                }
-            } else if (row0 + r < Ln) {
-                // a short last tile of a block that is not the last of the tensor:
-                // the rows after the block belong to the next block
+                const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 64);
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    const float *v = hh ? num1 : num0;
-                    const float2 inv = hh ? inv1 : inv0;
-                    uint4 *dst = reinterpret_cast<uint4 *>(
-                        out + (((size_t)w.b * p.N + blk0 + row0 + r) * p.H + 2 * w.u + hh) * kD);
+                    float v[32];
+                    tmem_ld32(base + hh * 32, v);
+                    tmem_wait_ld();
+                    // the sum of the two halves of the denominator, in a fixed order
+                    const float den = den_s[a * 512 + (2 * hh) * 128 + r] + den_s[a * 512 + (2 * hh + 1) * 128 + r];
+                    const float iv = 1.0f / (den + p.eps);
+                    const float2 inv = make_float2(iv, iv);
+                    uint4 y[4];
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         const float2 y0 = fmul2(make_float2(v[8 * c], v[8 * c + 1]), inv);
                         const float2 y1 = fmul2(make_float2(v[8 * c + 2], v[8 * c + 3]), inv);
                         const float2 y2 = fmul2(make_float2(v[8 * c + 4], v[8 * c + 5]), inv);
                         const float2 y3 = fmul2(make_float2(v[8 * c + 6], v[8 * c + 7]), inv);
-                        dst[c] = make_uint4(pack_bf2(y0.x, y0.y), pack_bf2(y1.x, y1.y), pack_bf2(y2.x, y2.y),
-                                            pack_bf2(y3.x, y3.y));
+                        y[c] = make_uint4(pack_bf2(y0.x, y0.y), pack_bf2(y1.x, y1.y), pack_bf2(y2.x, y2.y),
+                                          pack_bf2(y3.x, y3.y));
                     }
+                    if (boxed) {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)   // logical chunk 4 hh + c, 128-byte swizzle (row % 8 == lane % 8)
+                            *reinterpret_cast<uint4 *>(sb + lane * 128 + (((4 * hh + c) ^ (lane & 7)) << 4)) = y[c];
+                    } else if (row0 + r < Ln) {
+                        // a short last tile of a block that is not the last of the
+                        // tensor: the rows after the block belong to the next block
+                        uint4 *dst = reinterpret_cast<uint4 *>(
+                            out + (((size_t)w.b * p.N + blk0 + row0 + r) * p.H + 2 * w.u + hh) * kD);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) dst[c] = y[c];
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&acc_empty[a]);
+                mbar_arrive(&den_empty[a]);
+            }
+            if (got && boxed) {
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(&tm_out, sb, w.u * 64, blk0 + row0 + 32 * q, w.b);
+                    bulk_commit();
                 }
             }
         }
         if (lane == 0) bulk_wait_all();
     }
 
-    if (warp == kWarpTma && lane == 0 && *abort_word) {
+    if ((warp == kWarpTma0 || warp == kWarpTma1) && lane == 0 && *abort_word) {
         for (int kb = bops_issued - 2 < 0 ? 0 : bops_issued - 2; kb < bops_issued; ++kb)
             final_wait(&bop_full[kb & 1], (uint32_t)(kb >> 1) & 1u);
         for (int i = issued - kARaw < 0 ? 0 : issued - kARaw; i < issued; ++i)
-            final_wait(&raw_full[i % kARaw], (uint32_t)(i / kARaw) & 1u);
+            if ((i & 1) == ti) final_wait(&raw_full[i % kARaw], (uint32_t)(i / kARaw) & 1u);
     }
     tc_fence_before();
     __syncwarp();
