@@ -430,7 +430,7 @@ def main():
     w = runner.w
     flush_w = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    flush_acc = torch.empty(1, dtype=torch.float32, device=dev)
+    flush_acc = torch.empty((), dtype=torch.float32, device=dev)
 
     class _Flush:
         @staticmethod
@@ -548,7 +548,7 @@ def main():
     wb_end = torch.cuda.Event(enable_timing=True, external=True)
     rd_start = torch.cuda.Event(enable_timing=True, external=True)
     rd_end = torch.cuda.Event(enable_timing=True, external=True)
-    evict = torch.empty(1, dtype=torch.float32, device=dev)
+    evict = torch.empty((), dtype=torch.float32, device=dev)
     graph_wb, graph_rd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph_wb):
         wb_start.record()

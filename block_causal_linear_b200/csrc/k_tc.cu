@@ -54,100 +54,6 @@ constexpr int kWarpTma = 0;
 constexpr int kWarpMma = 1;
 constexpr int kWork = 128;      // threads of warps 2..5
 
-// ---------------------------------------------------------------- RoPE table
-// (cos, sin) of every feature pair at every position a CTA can meet: pair p of
-// the frame axis at frames [f_lo, f_lo + nf) of the call, of the row axis at
-// rows [0, Hg), of the column axis at columns [0, Wg).  The segment of pair p
-// starts at rope_seg(p).  The host only takes this path when the table fits.
-constexpr int kTabMax = 1024;
-
-__device__ __forceinline__ int rope_len(const Plan &p, int pr, int nf) {
-    return p.axis[pr] == 0 ? nf : (p.axis[pr] == 1 ? p.Hg : p.Wg);
-}
-
-__device__ __forceinline__ int rope_seg(const Plan &p, int pr, int nf) {
-    int off = 0;
-    for (int q = 0; q < pr; ++q) off += rope_len(p, q, nf);
-    return off;
-}
-
-__device__ void build_rope_table(float2 *tab, const Plan &p, int f_lo, int nf, int tid, int nthreads) {
-    int off = 0;
-    for (int pr = 0; pr < kD / 2; ++pr) {
-        const int len = rope_len(p, pr, nf);
-        for (int pos = tid; pos < len; pos += nthreads) {
-            const int apos = p.axis[pr] == 0 ? p.t_offset + f_lo + pos : pos;
-            float s, c;
-            sincosf((float)apos * p.theta[pr], &s, &c);
-            tab[off + pos] = make_float2(c, s);
-        }
-        off += len;
-    }
-}
-
-// Per-thread view of the 4 feature pairs of one 16-byte chunk (features
-// 8*(L%4) .. +7 of a head): table segment and axis of each pair, as scalars
-// (so that they stay in registers).
-struct PairSet {
-    int seg0, seg1, seg2, seg3;
-    int ax0, ax1, ax2, ax3;
-};
-
-__device__ __forceinline__ PairSet pair_set(const Plan &p, int L, int nf) {
-    const int pr = (L & 3) * 4;
-    PairSet s;
-    s.seg0 = rope_seg(p, pr, nf);
-    s.seg1 = s.seg0 + rope_len(p, pr, nf);
-    s.seg2 = s.seg1 + rope_len(p, pr + 1, nf);
-    s.seg3 = s.seg2 + rope_len(p, pr + 2, nf);
-    s.ax0 = p.axis[pr];
-    s.ax1 = p.axis[pr + 1];
-    s.ax2 = p.axis[pr + 2];
-    s.ax3 = p.axis[pr + 3];
-    return s;
-}
-
-// (cos, sin) of the thread's 4 pairs at token t of the call: one position
-// (frame, row, column) per token, shared by every chunk of that token that
-// holds the same features (the same features of other heads).
-struct RowCS {
-    float2 c0, c1, c2, c3;
-};
-
-__device__ __forceinline__ RowCS row_cs(const float2 *tab, const PairSet &ps, const Plan &p, int ti, int f_lo) {
-    const int fq = fast_div(ti, p.hw_m, p.hw_s);
-    const int rem = ti - fq * p.Hg * p.Wg;
-    const int row = fast_div(rem, p.wg_m, p.wg_s);
-    const int col = rem - row * p.Wg;
-    const int fr = fq - f_lo;
-    RowCS r;
-    r.c0 = tab[ps.seg0 + (ps.ax0 == 0 ? fr : (ps.ax0 == 1 ? row : col))];
-    r.c1 = tab[ps.seg1 + (ps.ax1 == 0 ? fr : (ps.ax1 == 1 ? row : col))];
-    r.c2 = tab[ps.seg2 + (ps.ax2 == 0 ? fr : (ps.ax2 == 1 ? row : col))];
-    r.c3 = tab[ps.seg3 + (ps.ax3 == 0 ? fr : (ps.ax3 == 1 ? row : col))];
-    return r;
-}
-
-// ReLU one bf16 pair (one word), rotate it by cs, split into hi + lo bf16.
-__device__ __forceinline__ void rotate_pair(uint32_t x, float2 cs, float &x0, float &x1, uint32_t &h, uint32_t &l) {
-    const uint32_t w = relu2(x);
-    x0 = bf_lo(w);
-    x1 = bf_hi(w);
-    const float y0 = x0 * cs.x - x1 * cs.y;
-    const float y1 = x0 * cs.y + x1 * cs.x;
-    const __nv_bfloat162 yh = __floats2bfloat162_rn(y0, y1);
-    h = *reinterpret_cast<const uint32_t *>(&yh);
-    l = pack_bf2(y0 - __low2float(yh), y1 - __high2float(yh));
-}
-
-// ReLU one chunk of 8 bf16 and rotate its 4 pairs; f receives phi(x).
-__device__ __forceinline__ void relu_rotate_chunk(uint4 x, const RowCS &cs, uint4 &hi, uint4 &lo, float (&f)[8]) {
-    rotate_pair(x.x, cs.c0, f[0], f[1], hi.x, lo.x);
-    rotate_pair(x.y, cs.c1, f[2], f[3], hi.y, lo.y);
-    rotate_pair(x.z, cs.c2, f[4], f[5], hi.z, lo.z);
-    rotate_pair(x.w, cs.c3, f[6], f[7], hi.w, lo.w);
-}
-
 // ---------------------------------------------------------------- NVFP4
 // ReLU on 8 packed E2M1 codes: a code with its sign bit (bit 3 of the nibble)
 // set is negative or -0, and becomes +0.
@@ -199,14 +105,13 @@ static_assert(kRRows == 32, "the ReLU pass below maps 128 threads x 4 chunks ont
 // warps decode them into f16 boxes laid out as the bf16 path's tiles (a ring
 // of kDec decoded stages, shorter than the raw ring that covers the memory
 // latency), and the MMAs are kind::f16 on f16.
-template <bool ROPE, int IN = kInBf16>
+template <int IN = kInBf16>
 struct RCfg {
     static constexpr bool F8 = IN == kInE4m3, F4 = IN == kInNvfp4;
-    // 6 x 8 KiB with FP8 codes, 4 x 16 (24 with RoPE) KiB with bf16, 8 x 5 KiB raw with NVFP4
+    // 6 x 8 KiB with FP8 codes, 4 x 16 KiB with bf16, 8 x 5 KiB raw with NVFP4
     static constexpr int kStages = F8 ? 6 : (F4 ? 8 : 4);
-    // stage: k boxes (becoming R phi(k) hi with RoPE), [lo boxes], v boxes
-    static constexpr int kLoOff = 2 * kRBox;
-    static constexpr int kVOff = F8 ? kRRows * 128 : (ROPE ? 4 * kRBox : 2 * kRBox);
+    // stage: k boxes, then v boxes
+    static constexpr int kVOff = F8 ? kRRows * 128 : 2 * kRBox;
     static constexpr int kStageBytes = F8 ? 2 * kRRows * 128 : (F4 ? 5 * 1024 : kVOff + 2 * kRBox);
     // F4: decoded ring first (1024-byte aligned for the swizzled boxes), then the raw ring
     static constexpr int kDec = F4 ? 3 : 0;
@@ -215,17 +120,16 @@ struct RCfg {
     static constexpr int kCodeBytes = kRRows * 64;                  // F4: one tensor's codes in a raw stage
     static constexpr int kSfOff = 2 * kCodeBytes;                   // F4: k scales, then v scales (512 B each)
     static constexpr int kRawTx = 2 * kCodeBytes + 2 * kRRows * 16;
-    static constexpr int kAuxOff = kRawOff + kStages * kStageBytes; // ones (512 B) or RoPE table
-    static constexpr int kAuxBytes = ROPE ? kTabMax * 8 : 512;
+    static constexpr int kAuxOff = kRawOff + kStages * kStageBytes; // ones (512 B)
+    static constexpr int kAuxBytes = 512;
     static constexpr int kBarOff = kAuxOff + kAuxBytes;
     static constexpr int kNumBars = F4 ? 2 * kStages + 2 * kDec + 1 : 3 * kStages + 1;
     static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
-    static constexpr uint32_t kTmemCols = ROPE ? 128 : 256;
-    // threads that transform the k boxes (warps 2..): RoPE has 8 such warps,
-    // one token row per thread and stage, to hide the latency of its longer
-    // per-chunk work; NVFP4 8 warps, one 16-feature block of k and one of v per
-    // thread and stage; otherwise 4 warps, 4 chunks per thread
-    static constexpr int kXform = (ROPE || F4) ? 256 : 128;
+    static constexpr uint32_t kTmemCols = 256;
+    // threads that transform the k boxes (warps 2..): NVFP4 8 warps, one
+    // 16-feature block of k and one of v per thread and stage; otherwise 4
+    // warps, 4 chunks per thread
+    static constexpr int kXform = F4 ? 256 : 128;
     static constexpr int kThreadsR = 64 + kXform;
     static_assert(!F4 || kStageBytes >= kRawTx, "the raw stage holds codes and scales");
 };
@@ -289,17 +193,15 @@ __device__ void fused_combine(const Plan &p, const Fuse &fz, const float *part, 
 }
 
 // tm_ks, tm_vs: the NVFP4 block scales of k and v (unused otherwise).
-template <bool ROPE, int IN = kInBf16>
-__global__ void __launch_bounds__(RCfg<ROPE, IN>::kThreadsR, 2)
+template <int IN = kInBf16>
+__global__ void __launch_bounds__(RCfg<IN>::kThreadsR, 2)
 reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                  float *__restrict__ partials, const Plan p, const Fuse fz) {
     constexpr bool F8 = IN == kInE4m3, F4 = IN == kInNvfp4;
-    static_assert(!(ROPE && (F8 || F4)), "FP8 and NVFP4 inputs take no RoPE");
-    using C = RCfg<ROPE, IN>;
-    static_assert(C::kXform * 16 * 4 <= kFusePartOff &&
-                      kFusePartOff + 4 * kKVZ * 4 <= C::kStages * C::kStageBytes,
-                  "the fused split sums sit past the z scratch, inside the stages");
+    using C = RCfg<IN>;
+    static_assert(kFusePartOff + 4 * kKVZ * 4 <= C::kStages * C::kStageBytes,
+                  "the fused split sums fit inside the stages");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     uint8_t *aux = smem + C::kAuxOff;
@@ -349,10 +251,6 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         return;
     }
 
-    const long long hw = (long long)p.Hg * p.Wg;
-    const int f_lo = ROPE ? (int)(t0 / hw) : 0;
-    const int nf = ROPE ? (int)((t1 - 1) / hw) - f_lo + 1 : 0;
-
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) mbar_init(&full[s], 1);
         for (int s = 0; s < kRing; ++s) {
@@ -365,14 +263,10 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         *abort_word = 0;
         fence_barrier_init();
     }
-    if constexpr (ROPE) {
-        build_rope_table(reinterpret_cast<float2 *>(aux), p, f_lo, nf, threadIdx.x, C::kThreadsR);
-    } else {
-        // B operand of the z contraction: 16 x 16 ones (any layout reads 1.0)
-        // (1.0 is 0x3F80 in bf16, 0x38 in E4M3, 0x3C00 in f16)
-        for (int i = threadIdx.x; i < 128; i += C::kThreadsR)
-            reinterpret_cast<uint32_t *>(aux)[i] = F8 ? 0x38383838u : (F4 ? 0x3C003C00u : 0x3F803F80u);
-    }
+    // B operand of the z contraction: 16 x 16 ones (any layout reads 1.0)
+    // (1.0 is 0x3F80 in bf16, 0x38 in E4M3, 0x3C00 in f16)
+    for (int i = threadIdx.x; i < 128; i += C::kThreadsR)
+        reinterpret_cast<uint32_t *>(aux)[i] = F8 ? 0x38383838u : (F4 ? 0x3C003C00u : 0x3F803F80u);
     if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
@@ -455,12 +349,7 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     const uint64_t db = smem_desc(vaddr + kk * 2048, kRBox, 1024, kLayoutSw128);
                     const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
                     mma_bf16(tmem, da, db, id_kv, acc);
-                    if constexpr (ROPE) {
-                        const uint64_t dl = smem_desc(kaddr + C::kLoOff + kk * 2048, kRBox, 1024, kLayoutSw128);
-                        mma_bf16(tmem, dl, db, id_kv, 1u);
-                    } else {
-                        mma_bf16(tmem + 128, da, d_ones, id_z, acc);
-                    }
+                    mma_bf16(tmem + 128, da, d_ones, id_z, acc);
                 }
                 mma_commit(&empty[s]);
             }
@@ -468,17 +357,6 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
     } else {
         const int wt = threadIdx.x - 64;   // 0 .. C::kXform - 1
-        // with RoPE this thread always meets the same logical chunk L of a row
-        // (the swizzle phase (wt >> 3) & 7 is the same for all its chunks)
-        const int L = (wt & 7) ^ ((wt >> 3) & 7);
-        PairSet ps{};
-        if constexpr (ROPE) ps = pair_set(p, L, nf);
-        float zacc[2][8];
-#pragma unroll
-        for (int bx = 0; bx < 2; ++bx)
-#pragma unroll
-            for (int k = 0; k < 8; ++k) zacc[bx][k] = 0.f;
-        const float2 *tab = reinterpret_cast<const float2 *>(aux);
 
         for (int i = 0; i < nst; ++i) {
             const int s = i % C::kStages;
@@ -515,31 +393,6 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 decode_nvfp4_16(cv, sv, a, bq);
                 *reinterpret_cast<uint4 *>(drow + C::kVOff + p0) = a;
                 *reinterpret_cast<uint4 *>(drow + C::kVOff + p1) = bq;
-            } else if constexpr (ROPE) {
-                // the thread's chunks: token row r (and r + 16 with 4 warps), each
-                // in both boxes (heads 0-1 and 2-3), all with the same 8 features,
-                // so one position and one set of cos/sin per row
-#pragma unroll
-                for (int jr = 0; jr < 256 / C::kXform; ++jr) {
-                    const int r = (wt >> 3) + (C::kXform / 8) * jr;
-                    const bool valid = row0 + r < t1;   // rows past the split contribute nothing
-                    RowCS cs{};
-                    if (valid) cs = row_cs(tab, ps, p, (int)(row0 + r), f_lo);
-#pragma unroll
-                    for (int bx = 0; bx < 2; ++bx) {
-                        const int c = wt + C::kXform * jr + 256 * bx;   // 16-byte chunk of the two k boxes
-                        uint4 *ptr = reinterpret_cast<uint4 *>(kt + (size_t)c * 16);
-                        uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
-                        if (valid) {
-                            float f[8];
-                            relu_rotate_chunk(*ptr, cs, hi, lo, f);
-#pragma unroll
-                            for (int k = 0; k < 8; ++k) zacc[bx][k] += f[k];
-                        }
-                        *ptr = hi;
-                        *reinterpret_cast<uint4 *>(kt + C::kLoOff + (size_t)c * 16) = lo;
-                    }
-                }
             } else if constexpr (F8) {
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {             // the k box: 256 chunks of 16 codes, 2 per thread
@@ -586,30 +439,13 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         const int qd = warp & 3;
         const int h = g * 4 + qd;
         float z = 0.f;
-        if constexpr (ROPE) {
-            // z: the threads that met chunk L of a box each hold 8 sums; add
-            // them in thread order (stage 0 is free once every MMA is done)
-            float *zbuf = reinterpret_cast<float *>(smem);
-            static_assert(C::kXform * 16 * 4 <= C::kStageBytes, "z partials fit in stage 0");
-#pragma unroll
-            for (int bx = 0; bx < 2; ++bx)
-#pragma unroll
-                for (int k = 0; k < 8; ++k) zbuf[wt * 16 + bx * 8 + k] = zacc[bx][k];
-            named_bar_sync(1, C::kXform);
-            if (warp < 6) {
-                const int bx = qd >> 1;
-                const int Lz = ((qd & 1) << 2) | (lane >> 3);
-                for (int u = 0; u < C::kXform; ++u)
-                    if (((u & 7) ^ ((u >> 3) & 7)) == Lz) z += zbuf[u * 16 + bx * 8 + (lane & 7)];
-            }
-        }
         // warps 2..5 (one per TMEM lane quarter) write the split sums
         if (got && warp < 6) {
             tc_fence_after();
             const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
             float kv[32];
             tmem_ld32(tmem + lane_off + 32 * qd, kv);
-            if constexpr (!ROPE) z = tmem_ld1(tmem + lane_off + 128);
+            z = tmem_ld1(tmem + lane_off + 128);
             tmem_wait_ld();
             if constexpr (F8 || F4) {
                 // per-tensor scales: KV = sk sv sum phi(k^) v^T, z = sk sum phi(k^)
@@ -656,60 +492,51 @@ constexpr int kAThreads = 320;                 // 10 warps
 constexpr int kAXform0 = 192;                  // first thread of the transform warps 6..9
 constexpr int kAWarpStg = 32 * 128;            // one epilogue warp's staging box: [32 rows][64 bf16]
 
-template <bool ROPE, int IN = kInBf16>
+template <int IN = kInBf16>
 struct ACfg {
     static constexpr bool F8 = IN == kInE4m3, F4 = IN == kInNvfp4;
     // F8: a stage is the bf16 tile the MMA reads (16 KiB, 128-byte swizzle)
     // followed by the tile's E4M3 codes as TMA lands them (8 KiB, no swizzle).
     // F4: the bf16 tile, the tile's E2M1 codes (4 KiB: 32 bytes a row) and
     // the 16-byte box of E4M3 block scales of each row (2 KiB)
-    static constexpr int kStages = (F8 || F4) ? 3 : (ROPE ? 2 : 4);
+    static constexpr int kStages = (F8 || F4) ? 3 : 4;
     static constexpr int kCodeOff = kATile;
     static constexpr int kSfOff = kATile + kATile / 4;   // F4
     static constexpr int kQTx = F8 ? kATile / 2 : (F4 ? kATile / 4 + 128 * 16 : kATile);   // bytes TMA lands per tile
-    static constexpr int kStageBytes = F8 ? kATile + kATile / 2 : (F4 ? kSfOff + 128 * 16 : (ROPE ? 2 * kATile : kATile));
-    static constexpr int kStgBufs = (ROPE || F8) ? 1 : 2;             // staging boxes per epilogue warp
+    static constexpr int kStageBytes = F8 ? kATile + kATile / 2 : (F4 ? kSfOff + 128 * 16 : kATile);
+    static constexpr int kStgBufs = F8 ? 1 : 2;                        // staging boxes per epilogue warp
     static constexpr int kOutOff = kStages * kStageBytes;
     static constexpr int kBopOff = kOutOff + 4 * kStgBufs * kAWarpStg;
-    static constexpr int kDenOff = kBopOff + kABopBytes;             // RoPE: [2][128 rows][2 heads] fp32
-    static constexpr int kZOff = kDenOff + (ROPE ? 2 * 1024 : 0);     // RoPE: Z_eff of the 2 heads
-    static constexpr int kTabOff = kZOff + (ROPE ? 256 : 0);
-    static constexpr int kBarOff = kTabOff + (ROPE ? kTabMax * 8 : 0);
-    static constexpr int kNumBars = 3 * kStages + 2 + 2 + 2 + 2 + 3;  // + acc[2], acc_empty[2], den[2], den_free[2], bop, drain, dep
+    static constexpr int kBarOff = kBopOff + kABopBytes;
+    static constexpr int kNumBars = 3 * kStages + 2 + 2 + 3;          // + acc[2], acc_empty[2], bop, drain, dep
     static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
-    static constexpr int kAccCols = ROPE ? 64 : 96;                  // per TMEM buffer (2 heads)
-    static constexpr int kHeadCols = ROPE ? 32 : kOpRows;
-    static constexpr uint32_t kTmemCols = ROPE ? 128 : 256;
+    static constexpr int kAccCols = 96;                                // per TMEM buffer (2 heads)
+    static constexpr int kHeadCols = kOpRows;
+    static constexpr uint32_t kTmemCols = 256;
 };
 
 // Warp roles: 0 issues TMA, 1 owns TMEM and issues the MMAs, 2..5 run the
 // epilogue (warp w reads TMEM lanes 32*(w%4).. = token rows of the tile),
-// 6..9 apply phi (and RoPE) to the q tiles in shared memory.  The transform
+// 6..9 apply phi to the q tiles in shared memory.  The transform
 // of tile i+1 and the epilogue of tile i run at the same time.
 // tm_qs: the NVFP4 block scales of q (unused otherwise).
-template <bool ROPE, int IN = kInBf16>
+template <int IN = kInBf16>
 __global__ void __launch_bounds__(kAThreads, 2)
 apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qs,
                 const __grid_constant__ CUtensorMap tm_out, __nv_bfloat16 *__restrict__ out,
                 const uint8_t *__restrict__ bop, const float *__restrict__ seff, const Plan p) {
     constexpr bool F8 = IN == kInE4m3, F4 = IN == kInNvfp4;
-    static_assert(!(ROPE && (F8 || F4)), "FP8 and NVFP4 inputs take no RoPE");
-    using C = ACfg<ROPE, IN>;
+    using C = ACfg<IN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     uint8_t *stg = smem + C::kOutOff;
     uint8_t *bops = smem + C::kBopOff;
-    float *den_s = reinterpret_cast<float *>(smem + C::kDenOff);
-    float *zs = reinterpret_cast<float *>(smem + C::kZOff);
-    const float2 *tab = reinterpret_cast<const float2 *>(smem + C::kTabOff);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
     uint64_t *xform_done = full + C::kStages;
     uint64_t *empty = xform_done + C::kStages;
     uint64_t *acc_full = empty + C::kStages;   // [2]
     uint64_t *acc_empty = acc_full + 2;        // [2]
-    uint64_t *den_ready = acc_empty + 2;       // [2] RoPE: den_s[i & 1] written
-    uint64_t *den_free = den_ready + 2;        // [2] RoPE: den_s[i & 1] read
-    uint64_t *bop_full = den_free + 2;
+    uint64_t *bop_full = acc_empty + 2;
     uint64_t *drain = bop_full + 1;            // only used when a wait gave up
     uint64_t *dep_ready = drain + 1;           // the previous kernel (state combine) has completed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(dep_ready + 1);
@@ -731,9 +558,6 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (ta1 <= ta0) return;   // a split past the end of a short last block
     const int ntiles = (int)((ta1 - ta0 + 127) / 128);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long hw = (long long)p.Hg * p.Wg;
-    const int f_lo = ROPE ? (int)(ta0 / hw) : 0;
-    const int nf = ROPE ? (int)((ta1 - 1) / hw) - f_lo + 1 : 0;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -744,8 +568,6 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int a = 0; a < 2; ++a) {
             mbar_init(&acc_full[a], 1);
             mbar_init(&acc_empty[a], kWork);
-            mbar_init(&den_ready[a], kWork);
-            mbar_init(&den_free[a], kWork);
         }
         mbar_init(bop_full, 1);
         mbar_init(drain, 1);
@@ -753,8 +575,6 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         *abort_word = 0;
         fence_barrier_init();
     }
-    if constexpr (ROPE)
-        build_rope_table(reinterpret_cast<float2 *>(smem + C::kTabOff), p, f_lo, nf, threadIdx.x, kAThreads);
     if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
@@ -822,9 +642,9 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         const uint32_t d = tmem + ab * C::kAccCols + hh * C::kHeadCols;
-                        // (A part, B part) products: hi.hi, hi.lo and, with RoPE, lo.hi
+                        // (A part, B part) products: hi.hi, hi.lo
 #pragma unroll
-                        for (int prod = 0; prod < (ROPE ? 3 : 2); ++prod) {
+                        for (int prod = 0; prod < 2; ++prod) {
                             const int apart = prod == 2 ? 1 : 0;
                             const int bpart = prod == 1 ? 1 : 0;
 #pragma unroll
@@ -850,79 +670,13 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ------------------------------------------------ transform warps
         const int tt = threadIdx.x - kAXform0;   // 0..127
         bool ok = true;
-        if constexpr (ROPE) {
-            // Z_eff comes from the state combine (the previous kernel)
-            if (!mbar_wait(dep_ready, 0, abort_word, &g_wait_flag, 19)) ok = false;
-            if (tt < 2 * kD)
-                zs[tt] = __ldcg(seff + (((size_t)b * p.H + 2 * hp + (tt >> 5)) * p.nb + n) * kKVZ + kD * kD + (tt & 31));
-            named_bar_sync(2, kWork);
-        }
-        // RoPE: this thread handles chunk pairs (pc, pc ^ 4) of one row: the same
-        // 8 features of both heads, so positions and cos/sin are shared.  Its
-        // swizzle phase, and so its logical chunk L0 (head 0 or 1), is fixed.
-        const int L0 = (tt & 3) ^ ((tt >> 2) & 7);
-        PairSet ps{};
-        // Z_eff of this thread's 8 features of both heads (e = 0: logical chunk
-        // L0, e = 1: L0 ^ 4), for the unrotated denominator
-        float zf[2][8];
-#pragma unroll
-        for (int e = 0; e < 2; ++e)
-#pragma unroll
-            for (int k = 0; k < 8; ++k) zf[e][k] = 0.f;
-        if constexpr (ROPE) {
-            ps = pair_set(p, L0, nf);
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int L = L0 ^ (4 * e);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) zf[e][k] = zs[(L >> 2) * kD + (L & 3) * 8 + k];
-            }
-        }
         for (int i = 0; i < ntiles; ++i) {
             const int s = i % C::kStages;
             const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
             if (ok && !mbar_wait(&full[s], ph, abort_word, &g_wait_flag, 15)) ok = false;
             uint8_t *qt = smem + s * C::kStageBytes;
             const long long row0 = ta0 + 128LL * i;
-            if constexpr (ROPE) {
-                if (ok && !mbar_wait(&den_free[i & 1], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_word, &g_wait_flag, 17))
-                    ok = false;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int u = tt + 128 * j;       // chunk pair index
-                    const int rr = u >> 2;            // token row
-                    const int pc0 = u & 3;            // physical chunk of the first of the pair
-                    const bool valid = ok && row0 + rr < ta1;
-                    float dp[2] = {0.f, 0.f};
-                    RowCS cs{};
-                    if (valid) cs = row_cs(tab, ps, p, (int)(row0 + rr), f_lo);
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int pc = pc0 + 4 * e;   // logical chunk pc ^ (rr & 7): L0, then L0 ^ 4
-                        uint4 *ptr = reinterpret_cast<uint4 *>(qt + rr * 128 + pc * 16);
-                        uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
-                        if (valid) {
-                            float f[8];
-                            relu_rotate_chunk(*ptr, cs, hi, lo, f);
-#pragma unroll
-                            for (int k = 0; k < 8; ++k) dp[e] = fmaf(f[k], zf[e][k], dp[e]);
-                        }
-                        *ptr = hi;
-                        *reinterpret_cast<uint4 *>(qt + kATile + rr * 128 + pc * 16) = lo;
-                    }
-                    // the 4 chunk pairs of a row sit on 4 consecutive lanes
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        dp[e] += __shfl_xor_sync(0xffffffffu, dp[e], 1);
-                        dp[e] += __shfl_xor_sync(0xffffffffu, dp[e], 2);
-                    }
-                    if ((lane & 3) == 0) {
-                        const int h0 = L0 >> 2;
-                        den_s[(i & 1) * 256 + rr * 2 + h0] = dp[0];
-                        den_s[(i & 1) * 256 + rr * 2 + (h0 ^ 1)] = dp[1];
-                    }
-                }
-            } else if (F4 && ok) {
+            if (F4 && ok) {
                 // NVFP4 [128 rows][2 heads][32 codes] -> phi(q) in bf16, exact (<= 6
                 // significant bits), into the 128-byte swizzled tile the MMA reads:
                 // 4 blocks of 16 features per thread
@@ -970,7 +724,6 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             fence_proxy_async_smem();
             mbar_arrive(&xform_done[s]);
-            if constexpr (ROPE) mbar_arrive(&den_ready[i & 1]);
         }
     } else {
         // ------------------------------------------------ epilogue warps 2..5
@@ -983,7 +736,6 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int ab = i & 1;
             const uint32_t aph = (uint32_t)(i >> 1) & 1u;
             bool got = ok && mbar_wait(&acc_full[ab], aph, abort_word, &g_wait_flag, 16);
-            if constexpr (ROPE) got = got && mbar_wait(&den_ready[i & 1], aph, abort_word, &g_wait_flag, 18);
             got = __all_sync(0xffffffffu, got);
             if (!got) ok = false;
             float num0[32], num1[32], den0 = 0.f, den1 = 0.f;
@@ -992,19 +744,12 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const uint32_t base = tmem + lane_off + ab * C::kAccCols;
                 tmem_ld32(base, num0);
                 tmem_ld32(base + C::kHeadCols, num1);
-                if constexpr (!ROPE) {
-                    den0 = tmem_ld1(base + kD);
-                    den1 = tmem_ld1(base + C::kHeadCols + kD);
-                }
+                den0 = tmem_ld1(base + kD);
+                den1 = tmem_ld1(base + C::kHeadCols + kD);
                 tmem_wait_ld();
-                if constexpr (ROPE) {
-                    den0 = den_s[(i & 1) * 256 + r * 2];
-                    den1 = den_s[(i & 1) * 256 + r * 2 + 1];
-                }
             }
             tc_fence_before();
             mbar_arrive(&acc_empty[ab]);
-            if constexpr (ROPE) mbar_arrive(&den_free[i & 1]);
 
             const long long row0 = ta0 + 128LL * i;
             const long long wrow0 = row0 + 32 * qd;    // first row of this warp
@@ -1129,26 +874,14 @@ bool smem_ready() {
     static std::once_flag once;
     static bool ok = false;
     std::call_once(once, [] {
-        ok = set_smem((const void *)reduce_tc_kernel<false>, RCfg<false>::kSmem) &&
-             set_smem((const void *)reduce_tc_kernel<true>, RCfg<true>::kSmem) &&
-             set_smem((const void *)apply_tc_kernel<false>, ACfg<false>::kSmem) &&
-             set_smem((const void *)apply_tc_kernel<true>, ACfg<true>::kSmem) &&
-             set_smem((const void *)reduce_tc_kernel<false, kInE4m3>, RCfg<false, kInE4m3>::kSmem) &&
-             set_smem((const void *)apply_tc_kernel<false, kInE4m3>, ACfg<false, kInE4m3>::kSmem) &&
-             set_smem((const void *)reduce_tc_kernel<false, kInNvfp4>, RCfg<false, kInNvfp4>::kSmem) &&
-             set_smem((const void *)apply_tc_kernel<false, kInNvfp4>, ACfg<false, kInNvfp4>::kSmem);
+        ok = set_smem((const void *)reduce_tc_kernel<kInBf16>, RCfg<kInBf16>::kSmem) &&
+             set_smem((const void *)apply_tc_kernel<kInBf16>, ACfg<kInBf16>::kSmem) &&
+             set_smem((const void *)reduce_tc_kernel<kInE4m3>, RCfg<kInE4m3>::kSmem) &&
+             set_smem((const void *)apply_tc_kernel<kInE4m3>, ACfg<kInE4m3>::kSmem) &&
+             set_smem((const void *)reduce_tc_kernel<kInNvfp4>, RCfg<kInNvfp4>::kSmem) &&
+             set_smem((const void *)apply_tc_kernel<kInNvfp4>, ACfg<kInNvfp4>::kSmem);
     });
     return ok;
-}
-
-// Entries of the RoPE table of the widest CTA of a kernel whose CTAs cover
-// `span` consecutive tokens of a call.
-long long rope_table_entries(const Plan &p, long long span) {
-    const long long hw = (long long)p.Hg * p.Wg;
-    const long long nf = (span + hw - 1) / hw + 1;
-    long long e = 0;
-    for (int pr = 0; pr < kD / 2; ++pr) e += p.axis[pr] == 0 ? nf : (p.axis[pr] == 1 ? p.Hg : p.Wg);
-    return e;
 }
 
 }  // namespace
@@ -1177,7 +910,7 @@ bool make_bf16_map_nd(CUtensorMap *m, const void *base, int rank, const cuuint64
 
 
 int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &p, cudaStream_t s, const Fuse *fz) {
-    if (!smem_ready()) return -1;
+    if (p.rope || !smem_ready()) return -1;   // RoPE calls take the kernels of k_rope_tc.cu
     CUtensorMap mk, mv, mks{}, mvs{};
     const long long grid = (long long)p.B * (p.H / 4) * p.nb * p.P;
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
@@ -1196,24 +929,22 @@ int launch_reduce_tc(const void *k, const void *v, float *partials, const Plan &
             !make_map_bytes(&mks, p.sfk, p.B, p.N, (long long)p.H * kD / 16, 16, kRRows, false) ||
             !make_map_bytes(&mvs, p.sfv, p.B, p.N, (long long)p.H * kD / 16, 16, kRRows, false))
             return -1;
-        using C4 = RCfg<false, kInNvfp4>;
-        return go(reduce_tc_kernel<false, kInNvfp4>, C4::kThreadsR, C4::kSmem) ? 1 : -1;
+        using C4 = RCfg<kInNvfp4>;
+        return go(reduce_tc_kernel<kInNvfp4>, C4::kThreadsR, C4::kSmem) ? 1 : -1;
     }
     if (p.f8) {
         if (!make_map_bytes(&mk, k, p.B, p.N, (long long)p.H * kD, 128, kRRows, true) ||
             !make_map_bytes(&mv, v, p.B, p.N, (long long)p.H * kD, 128, kRRows, true))
             return -1;
-        using C8 = RCfg<false, kInE4m3>;
-        return go(reduce_tc_kernel<false, kInE4m3>, C8::kThreadsR, C8::kSmem) ? 1 : -1;
+        using C8 = RCfg<kInE4m3>;
+        return go(reduce_tc_kernel<kInE4m3>, C8::kThreadsR, C8::kSmem) ? 1 : -1;
     }
     if (!make_map(&mk, k, p.B, p.N, p.H, kRRows) || !make_map(&mv, v, p.B, p.N, p.H, kRRows)) return -1;
-    const bool ok = p.rope ? go(reduce_tc_kernel<true>, RCfg<true>::kThreadsR, RCfg<true>::kSmem)
-                           : go(reduce_tc_kernel<false>, RCfg<false>::kThreadsR, RCfg<false>::kSmem);
-    return ok ? 1 : -1;
+    return go(reduce_tc_kernel<kInBf16>, RCfg<kInBf16>::kThreadsR, RCfg<kInBf16>::kSmem) ? 1 : -1;
 }
 
 int launch_apply_tc(const void *q, void *out, const void *bop, const float *seff, const Plan &p, cudaStream_t s) {
-    if (!smem_ready()) return -1;
+    if (p.rope || !smem_ready()) return -1;   // RoPE calls take the kernels of k_rope_tc.cu
     CUtensorMap mq, mqs{}, mo;
     const long long grid = (long long)p.B * p.nb * p.Pa * (p.H / 2);
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
@@ -1225,7 +956,7 @@ int launch_apply_tc(const void *q, void *out, const void *bop, const float *seff
         if (p.H % 8 != 0 || !make_map_bytes(&mq, q, p.B, p.N, (long long)p.H * kD / 2, 32, 128, false) ||
             !make_map_bytes(&mqs, p.sfq, p.B, p.N, (long long)p.H * kD / 16, 16, 128, false))
             return -1;
-        return launch_pdl(apply_tc_kernel<false, kInNvfp4>, (unsigned)grid, kAThreads, ACfg<false, kInNvfp4>::kSmem,
+        return launch_pdl(apply_tc_kernel<kInNvfp4>, (unsigned)grid, kAThreads, ACfg<kInNvfp4>::kSmem,
                           s, mq, mqs, mo, o, bb, seff, p)
                    ? 1
                    : -1;
@@ -1233,17 +964,16 @@ int launch_apply_tc(const void *q, void *out, const void *bop, const float *seff
     if (p.f8) {
         // q codes: boxes of the 2 heads' 64 codes x 128 tokens, no swizzle; out bf16
         if (!make_map_bytes(&mq, q, p.B, p.N, (long long)p.H * kD, 64, 128, false)) return -1;
-        return launch_pdl(apply_tc_kernel<false, kInE4m3>, (unsigned)grid, kAThreads, ACfg<false, kInE4m3>::kSmem,
+        return launch_pdl(apply_tc_kernel<kInE4m3>, (unsigned)grid, kAThreads, ACfg<kInE4m3>::kSmem,
                           s, mq, mqs, mo, o, bb, seff, p)
                    ? 1
                    : -1;
     }
     if (!make_map(&mq, q, p.B, p.N, p.H, 128)) return -1;
-    const bool ok = p.rope ? launch_pdl(apply_tc_kernel<true>, (unsigned)grid, kAThreads, ACfg<true>::kSmem, s, mq,
-                                        mqs, mo, o, bb, seff, p)
-                           : launch_pdl(apply_tc_kernel<false>, (unsigned)grid, kAThreads, ACfg<false>::kSmem, s, mq,
-                                        mqs, mo, o, bb, seff, p);
-    return ok ? 1 : -1;
+    return launch_pdl(apply_tc_kernel<kInBf16>, (unsigned)grid, kAThreads, ACfg<kInBf16>::kSmem, s, mq, mqs, mo, o, bb,
+                      seff, p)
+               ? 1
+               : -1;
 }
 
 namespace {
