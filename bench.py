@@ -108,16 +108,17 @@ def measured_peaks():
 # the source files each timed kernel is built from (the shared headers too)
 KERNEL_SOURCES = {
     "reduce": ["k_tc.cu"], "apply": ["k_tc.cu"], "finish": ["k_finish.cu"],
+    "reduce_tc_rope": ["k_rope_tc.cu"], "apply_tc_rope": ["k_rope_tc.cu"],
     "bwd_q": ["k_bwd_q_tc.cu"], "bwd_k": ["k_bwd_tc.cu"], "dwconv": ["k_conv.cu"],
 }
 SHARED_SOURCES = ["la_internal.cuh", "la_sm100.cuh"]
 
 
 def kernel_sources_sha(kernel: str) -> str:
-    """Hash of the sources of `kernel` (by its name's first part), so that a
+    """Hash of the sources of `kernel` (by the longest known prefix of its name), so that a
     stored ncu figure is dropped when, and only when, that kernel changed."""
     csrc = os.path.join(ROOT, "block_causal_linear_b200", "csrc")
-    key = next((k for k in KERNEL_SOURCES if kernel.startswith(k)), None)
+    key = max((k for k in KERNEL_SOURCES if kernel.startswith(k)), key=len, default=None)
     files = sorted(os.listdir(csrc)) if key is None else KERNEL_SOURCES[key] + SHARED_SOURCES
     h = hashlib.sha256()
     for f in files:

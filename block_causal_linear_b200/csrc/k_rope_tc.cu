@@ -29,9 +29,10 @@
 // reproducible.
 //
 // Shared memory is laid out for depth: the TMA tiles land in a ring of raw
-// stages (176 KiB in the reduce, 144 KiB in the apply) separate from the
-// transformed operands the tensor cores read, so that a raw q stage is free
-// as soon as the transform has read it.  The cos/sin table holds records of
+// stages (160 KiB in the reduce, 176 KiB in the apply) separate from the
+// transformed operands the tensor cores read (shared memory in the reduce,
+// tensor memory in the apply), so that a raw stage is free as soon as the
+// transform has read it.  The cos/sin table holds records of
 // two feature pairs (cos a, cos b, sin a, sin b) per position of each axis;
 // a transform thread owns one token row, so the 8 lanes of a shared-memory
 // phase read 8 consecutive rows: distinct 16-byte chunks of the swizzled
@@ -97,10 +98,10 @@ constexpr int kRZOff = kRTabOff + kTabBytes;             // z sums [2][4 heads][
 constexpr int kRBarOff = kRZOff + 2 * 128 * 4;
 constexpr int kRNumBars = 2 * kRRaw + 2 * kROp + 2 * 4 + 1;
 constexpr int kRSmem = kRBarOff + kRNumBars * 8 + 16 + 1024;
-// Per 16 tokens one M=128 x N=256 MMA: A = V of the 4 heads (value features
-// as rows), B = [R phi(K) hi | R phi(K) lo] (key features as columns), so the
-// V tile is read once, not once per part; D = [V^T R phi(K)_hi | V^T R phi(K)_lo],
-// the 4 diagonal 32x32 blocks of each half used.  Two accumulators.
+// Per 16 tokens two M=128 x N=128 MMAs into one accumulator: A = R phi(K)
+// hi, then lo, of the 4 heads (key features as rows), B = V (value features
+// as columns); the 4 diagonal 32x32 blocks of D are used.  Two accumulators
+// of 128 columns.
 constexpr uint32_t kRTmemCols = 256;
 static_assert(kRSmem <= 232448, "reduce shared memory");
 
