@@ -77,9 +77,14 @@ def parse():
                          "(la_*_forward_nvfp4); bf16 out")
     ap.add_argument("--blocks", type=int, default=None,
                     help="streaming workloads: run only the first N blocks (small cases for profiling)")
-    ap.add_argument("--shard", default="problem", choices=["problem", "heads"],
+    ap.add_argument("--shard", default="problem", choices=["problem", "heads", "tokens"],
                     help="problem: an independent problem per rank (weak scaling); "
-                         "heads: one problem's heads split over the ranks (strong scaling)")
+                         "heads: one problem's heads split over the ranks (strong scaling); "
+                         "tokens: every block's tokens split over the ranks, la_block_reduce -> all-gather of "
+                         "the [S | Z] partials -> la_block_apply (strong scaling)")
+    ap.add_argument("--emulate-ranks", type=int, default=1,
+                    help="--shard tokens on one process: run this many ranks' slices one after another on "
+                         "the GPU (the gather is then a view of one buffer)")
     return ap.parse_args()
 
 
@@ -283,6 +288,200 @@ def run_reference(args, rank):
 DWCONV_C = 5120   # MLP channels: 2.5 x the 2048-wide attention (the pages give no width)
 
 
+def run_token_split(args, w, world, rank, dist, dev, la):
+    """--shard tokens: every call's block is split over the ranks by tokens
+    (whole frames with RoPE, so that positions continue across the slices).
+    Per call: la_block_reduce of each local rank's k, v slice, one all-gather
+    of the [S | Z] partials (NCCL, 4,224 bytes per (b, h) and rank), then
+    la_block_apply of each local rank's q slice, which adds the gathered
+    partials in rank order and commits the same state on every rank.  With one
+    process, --emulate-ranks R runs R ranks' slices one after another on the
+    GPU; the partials are then written straight into the gathered buffer.
+    Strong scaling: the job's work is the unsplit workload."""
+    if args.pass_ != "forward" or args.input != "native" or args.op != "attention":
+        raise SystemExit("--shard tokens times the native forward path")
+    if args.blocks is not None:
+        if w.mode != "stream" or not 1 <= args.blocks <= w.n_blocks:
+            raise SystemExit("--blocks needs a streaming workload and 1 <= N <= its block count")
+        w = w.shrink(n_blocks=args.blocks)
+    if w.mode == "full" and w.n_blocks != 1:
+        raise SystemExit("--shard tokens: a one-call workload must be one block")
+    R_local = args.emulate_ranks if world == 1 else 1
+    R = world * R_local
+    if R_local < 1 or R > 32:
+        raise SystemExit("--emulate-ranks: 1 .. 32 ranks in all")
+    N = w.n_blk if w.mode == "stream" else w.n_total
+    align = w.Hg * w.Wg if w.rope else 1
+    if (N + align - 1) // align < R:
+        raise SystemExit(f"--shard tokens: a block of {N} tokens has fewer "
+                         f"{'frames' if w.rope else 'tokens'} than the {R} ranks")
+    frames_blk = N // align if w.rope else 0
+    if w.mode == "stream":
+        calls = list(synth.stream(w, device=dev))
+    else:
+        calls = [(0, 0, *synth.full_sequence(w, device=dev))]
+    passes = w.passes if w.mode == "stream" else 1
+    local = [rank * R_local + j for j in range(R_local)]          # global rank of each local rank
+    slices = [ranks.token_slice(N, R, r, align) for r in local]
+    # each rank owns its slices (what a token-parallel producer leaves on its GPU)
+    ins = [[tuple(t[:, t0:t1].contiguous() for t in c[2:5]) for (t0, t1) in slices] for c in calls]
+    del calls
+    outs = [[torch.empty_like(x[0]) for x in c] for c in ins]
+    states = [la.State(w.B, w.H, w.d, device=dev) for _ in local]
+    ws = [la.alloc_workspace(w.B, t1 - t0, w.H, w.d, t1 - t0, device=dev) for (t0, t1) in slices]
+    part_shape = (w.B, w.H, w.d * w.d + w.d)
+    gathered = torch.empty((R,) + part_shape, dtype=torch.float32, device=dev)
+    mine = torch.empty(part_shape, dtype=torch.float32, device=dev)
+    exchange_bytes = gathered.numel() * 4                        # what every rank holds after one gather
+    launches = [0]
+
+    def rope_for(j, frames_before, reduce_side):
+        if not w.rope:
+            return None
+        first_frame = ranks.split_frame_offsets(frames_before, N, R, align)[local[j]][2]
+        T = 0 if reduce_side else frames_blk                      # apply: a commit advances by the block
+        return la.make_rope(Hg=w.Hg, Wg=w.Wg, T=T, t_offset=first_frame, dims=w.rope_dims, base=w.rope_base)
+
+    n_calls = len(ins)
+    # external: recorded inside a captured graph as event-record nodes
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(n_calls)]
+
+    def step(timed=False):
+        n = 0
+        for st in states:
+            rc = la.la_state_init(st.c, st.S.data_ptr(), st.Z.data_ptr(), w.B, w.H, w.d, la._stream_ptr(None))
+            if rc != la.LA_OK:
+                raise la.LAError(rc, "la_state_init")
+        for i, sl in enumerate(ins):
+            commit = i % passes == passes - 1
+            frames_before = states[0].t_next           # host counter, the same on every rank
+            e = ev[i]
+
+            def reduce_fn(j, k, v):
+                nonlocal n
+                dst = gathered[local[j]] if world == 1 else mine
+                la.block_reduce(k, v, rope=rope_for(j, frames_before, True), ws=ws[j], partial=dst)
+                n += la.la_last_launch_count()
+                return dst
+
+            def gather_fn(parts):
+                if timed:
+                    e[1].record()
+                if world > 1:
+                    dist.all_gather_into_tensor(gathered, parts[0])
+                if timed:
+                    e[2].record()
+                return gathered
+
+            def apply_fn(j, q, g):
+                nonlocal n
+                la.block_apply(q, g, states[j], commit=commit, rope=rope_for(j, frames_before, False), eps=w.eps,
+                               ws=ws[j], out=outs[i][j])
+                n += la.la_last_launch_count()
+
+            if timed:
+                e[0].record()
+            ranks.split_call([x[0] for x in sl], [(x[1], x[2]) for x in sl], reduce_fn, gather_fn, apply_fn)
+            if timed:
+                e[3].record()
+        launches[0] = n
+
+    flush_w = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    acc = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush(x):
+        flush_w.fill_(x)
+        torch.sum(flush_r, dim=0, out=acc)
+
+    for i in range(max(3, args.warmup)):                # eager warm-up (also brings up NCCL before capture)
+        step()
+    torch.cuda.synchronize()
+    la.device_status()
+    # One step as a CUDA graph (NCCL's all-gather is captured with it), timed
+    # between event nodes inside the graph; a second graph with events between
+    # the reduce, gather and apply of every call gives the stage times.
+    g0 = torch.cuda.Event(enable_timing=True, external=True)
+    g1 = torch.cuda.Event(enable_timing=True, external=True)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        g0.record()
+        step()
+        g1.record()
+    graph_st = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_st):
+        step(timed=True)
+    torch.cuda.synchronize()
+    for i in range(max(3, args.warmup)):
+        flush(float(i))
+        graph.replay()
+    torch.cuda.synchronize()
+    K = ranks.agree_steps(args.steps or 20, dist, dev)
+    sampler = ClockSampler()
+    if rank == 0:
+        sampler.start(dev)
+        time.sleep(0.3)
+    t = [0.0, 0.0, 0.0, 0.0]                          # total, reduce, gather, apply (ms)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for it in range(K):
+        flush(float(it))
+        graph.replay()
+        g1.synchronize()
+        t[0] += g0.elapsed_time(g1)
+    for it in range(K):
+        flush(float(it))
+        graph_st.replay()
+        torch.cuda.synchronize()
+        for e in ev:
+            t[1] += e[0].elapsed_time(e[1])
+            t[2] += e[1].elapsed_time(e[2])
+            t[3] += e[2].elapsed_time(e[3])
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clocks = sampler.stop(dev.index or 0) if rank == 0 else None
+    la.device_status()                                  # raises if a bounded device wait gave up
+    t = ranks.max_over_ranks(t, dist, dev)
+    units = w.token_heads                               # the unsplit workload, once per step
+    value = units * K / (t[0] / 1e3)
+    peak, peak_kind = measured_peaks()
+    step_gbs = w.alg_bytes / (t[0] / K / 1e3) / 1e9
+    bytes_per_side = units * 2 * w.d * w.elem_bytes     # reduce: k, v; apply: q, out
+    dom, dom_ms = ("reduce", t[1]) if t[1] >= t[3] else ("apply", t[3])
+    path = la.la_last_path()
+    kname = f"{dom}_{path}" + ("_rope" if w.rope and path == "tc" else "")
+    achieved = bytes_per_side / (dom_ms / K / 1e3) / 1e9
+    per_launch = w.B * (sum(t1 - t0 for t0, t1 in slices) // len(slices)) * w.H
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": max(3, args.warmup), "ms_per_step": t[0] / K, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": workload_config(w, {"pass": "forward", "input_dtype": w.dtype,
+                                          "parallelism": f"tokens of every block split over {R} ranks "
+                                                         f"({world} process{'es' if world > 1 else ''}"
+                                                         f"{', emulated one after another' if R_local > 1 else ''})",
+                                          "api": "la_block_reduce + all-gather + la_block_apply",
+                                          "l2": "flushed before every timed step (256 MiB write, then 256 MiB read)"}),
+            "achieved_hbm_gbs": step_gbs, "hbm_frac_of_" + peak_kind: step_gbs / peak,
+            "stage_ms_per_step": {"reduce": t[1] / K, "gather": t[2] / K, "apply": t[3] / K},
+            "exchange_bytes_per_call": exchange_bytes, "exchange_bytes_per_step": exchange_bytes * n_calls,
+            "roofline": {"bound": "hbm", "kernel": f"{kname} (stage: kernel and its combine)", "achieved": achieved,
+                         "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": ncu_traffic(kname, per_launch)},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": launches[0] * K, "path": path, "clocks": clocks,
+            "launch": "one CUDA graph per step (the all-gather captured with it); stage times from a second "
+                      "graph with events between the reduce, gather and apply of every call",
+        }
+        print(json.dumps(line), flush=True)
+    del graph, graph_st                                 # the graphs hold NCCL work: release them first
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def run_dwconv(args, w, world, rank, dist, dev, la):
     """One step = the two depthwise convolutions of the Spatial-Temporal
     Mix-FFN on one latent video: y1 = conv_1x3x3(x), y2 = conv_3x1x1(y1), bf16
@@ -408,6 +607,8 @@ def main():
     from block_causal_linear_b200.runner import BackwardRunner, Runner
 
     base = synth.WORKLOADS[args.config]
+    if args.shard == "tokens":
+        return run_token_split(args, base, world, rank, dist, torch.device("cuda", local_rank), la)
     if args.shard == "heads":
         h0, h1 = ranks.head_slice(base.H, world, rank)
         if h1 <= h0:

@@ -9,6 +9,12 @@ of the same shape (weak scaling: ``rank_workload``), or the heads of one
 problem are split across ranks (strong scaling: ``head_slice``), each rank
 owning its heads' tensors and state.  The only collectives are the host's:
 agreeing on a step count and taking the slowest rank's time.
+
+A block with too few (batch, head) pairs to fill the GPUs can instead be split
+by tokens (``token_slice``, ``split_call``): splitting along tokens leaves the
+block's KV a sum of the slices' KV (KV_{1-2} = KV_1 + KV_2 in the same
+section), so the ranks exchange one [S | Z] partial per (batch, head), an
+all-gather of 4,224 bytes each, and every rank commits the same state.
 """
 from __future__ import annotations
 
@@ -86,6 +92,29 @@ def token_split_block(q, k, v, reduce_fn, gather_fn, apply_fn):
     partial = reduce_fn(k, v)
     gathered = gather_fn(partial)
     return apply_fn(q, gathered)
+
+
+def split_call(q_slices, kv_slices, reduce_fn, gather_fn, apply_fn):
+    """One call of a block whose tokens are split over the ranks, for the ranks
+    this process holds (one, or several emulated ranks on one GPU): their
+    partial sums in local rank order (reduce_fn(j, k, v)), one exchange
+    (gather_fn: the local partials -> every rank's partials in global rank
+    order), then their outputs (apply_fn(j, q, gathered)).  Every rank adds the
+    same gathered partials to the same state, so all commit the same state."""
+    partials = [reduce_fn(j, k, v) for j, (k, v) in enumerate(kv_slices)]
+    gathered = gather_fn(partials)
+    return [apply_fn(j, q, gathered) for j, q in enumerate(q_slices)]
+
+
+def split_frame_offsets(frames_before: int, N: int, world: int, align: int) -> List[Tuple[int, int, int]]:
+    """(t0, t1, first frame) of every rank's slice of a block of N tokens that
+    follows `frames_before` frames of the stream, split in whole frames of
+    `align` tokens (RoPE positions continue across the ranks' slices)."""
+    out = []
+    for r in range(world):
+        t0, t1 = token_slice(N, world, r, align)
+        out.append((t0, t1, frames_before + t0 // align))
+    return out
 
 
 def nccl_gather(partial, dist):

@@ -220,3 +220,111 @@ def test_token_slice_partitions():
                 assert sl[0][0] == 0 and sl[-1][1] == N
                 assert all(a[1] == b[0] for a, b in zip(sl, sl[1:]))
                 assert all(a[0] % align == 0 for a in sl if a[0] < N)
+
+
+def _split_stream_worker(rank, world, port, errfile):
+    """The host logic of `bench.py --shard tokens`: a RoPE stream of 2 blocks x
+    2 passes whose blocks are split by frames over 4 ranks, 2 per process
+    (ranks.split_call, ranks.split_frame_offsets), with oracle steps and a
+    gloo all-gather; every call's outputs, concatenated in rank order, equal
+    the oracle's unsplit stream, and all 4 ranks commit the same state."""
+    try:
+        sys.path.insert(0, ROOT)
+        os.environ["MASTER_ADDR"] = "127.0.0.1"
+        os.environ["MASTER_PORT"] = str(port)
+        from datetime import timedelta
+
+        dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+        import oracle as orc
+        from block_causal_linear_b200 import ranks, synth
+
+        B, H, d, Hg, Wg, F = 1, 2, 32, 3, 5, 4           # 4 frames of 3 x 5 per block
+        N, align, R_local = F * Hg * Wg, Hg * Wg, 2
+        R = world * R_local
+        local = [rank * R_local + j for j in range(R_local)]
+        calls = [(blk, p, *synth.random_qkv(B, N, H, d, seed=40 + 2 * blk + p)) for blk in range(2) for p in range(2)]
+        states = [orc.State(B, H, d) for _ in local]
+        t_next = 0
+        mine = []
+        for i, (blk, p, q, k, v) in enumerate(calls):
+            commit = p == 1
+            offs = ranks.split_frame_offsets(t_next, N, R, align)
+            sl = [offs[r] for r in local]
+
+            def reduce_fn(j, kk, vv):
+                KV, z = orc.block_kv(kk, vv, rope=orc.make_rope(Hg, Wg, t_offset=sl[j][2]))
+                return torch.from_numpy(np.concatenate([KV.reshape(B, H, d * d), z], -1))
+
+            def gather_fn(parts):
+                stacked = torch.stack(parts)
+                every = [torch.empty_like(stacked) for _ in range(world)]
+                dist.all_gather(every, stacked)
+                return torch.cat(every)                  # global rank order
+
+            def apply_fn(j, qq, gathered):
+                st = states[j]
+                S, Z = st.S.copy(), st.Z.copy()
+                for r in range(R):
+                    S += gathered[r, :, :, : d * d].numpy().reshape(B, H, d, d)
+                    Z += gathered[r, :, :, d * d:].numpy()
+                if commit:
+                    st.S, st.Z = S, Z
+                return orc.apply(qq, S, Z, rope=orc.make_rope(Hg, Wg, t_offset=sl[j][2]))
+
+            outs = ranks.split_call([q[:, t0:t1].contiguous() for t0, t1, _ in sl],
+                                    [(k[:, t0:t1].contiguous(), v[:, t0:t1].contiguous()) for t0, t1, _ in sl],
+                                    reduce_fn, gather_fn, apply_fn)
+            mine += [(i, local[j], outs[j]) for j in range(R_local)]
+            if commit:
+                t_next += F
+        got = [None] * world
+        dist.all_gather_object(got, (mine, [(s.S, s.Z) for s in states]))
+        if rank == 0:
+            ref_st = orc.State(B, H, d)
+            every = [x for g in got for x in g[0]]
+            sts = [s for g in got for s in g[1]]
+            for i, (blk, p, q, k, v) in enumerate(calls):
+                ref = orc.block_forward(q, k, v, ref_st, commit=p == 1, rope=orc.make_rope(Hg, Wg, t_offset=F * blk))
+                parts = sorted((r, o) for c, r, o in every if c == i)
+                g = np.concatenate([o for _, o in parts], 1)
+                assert np.abs(g - ref).max() <= 1e-12 * np.abs(ref).max()
+            assert all(np.array_equal(s[0], sts[0][0]) and np.array_equal(s[1], sts[0][1]) for s in sts)
+            assert np.abs(sts[0][0] - ref_st.S).max() <= 1e-12 * np.abs(ref_st.S).max()
+            assert np.abs(sts[0][1] - ref_st.Z).max() <= 1e-12 * np.abs(ref_st.Z).max()
+        dist.barrier()
+        dist.destroy_process_group()
+    except BaseException as e:
+        import traceback
+
+        with open(errfile, "a") as f:
+            f.write(f"rank {rank}: {e!r}\n{traceback.format_exc()}\n")
+        raise
+
+
+def test_token_split_stream_four_ranks_on_two_gloo_processes(orc, tmp_path):
+    errfile = str(tmp_path / "errors.txt")
+    world = 2
+    ctx = mp.get_context("spawn")
+    port = _free_port()
+    procs = [ctx.Process(target=_split_stream_worker, args=(r, world, port, errfile)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    alive = [p for p in procs if p.is_alive()]
+    for p in alive:
+        p.kill()
+        p.join()
+    err = open(errfile).read() if os.path.exists(errfile) else ""
+    assert not alive, "a rank did not finish"
+    assert all(p.exitcode == 0 for p in procs), err
+
+
+def test_split_frame_offsets():
+    sys.path.insert(0, ROOT)
+    from block_causal_linear_b200 import ranks
+
+    offs = ranks.split_frame_offsets(7, 3 * 15, 3, 15)
+    assert offs == [(0, 15, 7), (15, 30, 8), (30, 45, 9)]
+    offs = ranks.split_frame_offsets(0, 100, 4, 1)
+    assert [o[:2] for o in offs] == [(0, 25), (25, 50), (50, 75), (75, 100)] and all(o[2] == o[0] for o in offs)
