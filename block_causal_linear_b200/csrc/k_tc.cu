@@ -386,13 +386,20 @@ reduce_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 } else {
                     ck = make_uint2(0u, 0u);   // rows past the split contribute nothing
                 }
+                // The 8 lanes of a shared-memory phase are one row: heads 0, 1
+                // write box 0 and heads 2, 3 box 1, 4 KiB apart, so the same
+                // chunk of both boxes falls on the same banks.  The box-1 lanes
+                // store their two chunks in the other order, so that every phase
+                // writes 8 distinct chunk positions (one wavefront, not two).
+                const bool swap = (hd >> 1) != 0;
+                const int pa = swap ? p1 : p0, pb = swap ? p0 : p1;
                 uint4 a, bq;
                 decode_nvfp4_16(ck, sk, a, bq);
-                *reinterpret_cast<uint4 *>(drow + p0) = a;
-                *reinterpret_cast<uint4 *>(drow + p1) = bq;
+                *reinterpret_cast<uint4 *>(drow + pa) = swap ? bq : a;
+                *reinterpret_cast<uint4 *>(drow + pb) = swap ? a : bq;
                 decode_nvfp4_16(cv, sv, a, bq);
-                *reinterpret_cast<uint4 *>(drow + C::kVOff + p0) = a;
-                *reinterpret_cast<uint4 *>(drow + C::kVOff + p1) = bq;
+                *reinterpret_cast<uint4 *>(drow + C::kVOff + pa) = swap ? bq : a;
+                *reinterpret_cast<uint4 *>(drow + C::kVOff + pb) = swap ? a : bq;
             } else if constexpr (F8) {
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {             // the k box: 256 chunks of 16 codes, 2 per thread
@@ -896,6 +903,22 @@ bool tc_available() {
 
 bool make_bf16_map(CUtensorMap *m, const void *base, int B, int N, int H, int box_rows) {
     return make_map(m, base, B, N, H, box_rows);
+}
+
+bool make_u8_map(CUtensorMap *m, const void *base, int B, int N, long long row_bytes, int box_inner, int box_rows,
+                 int swizzle_bytes) {
+    auto fn = encode_fn();
+    if (!fn || (swizzle_bytes != 0 && swizzle_bytes != 64 && swizzle_bytes != 128)) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)row_bytes, (cuuint64_t)N, (cuuint64_t)B};
+    cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)row_bytes * (cuuint64_t)N};
+    cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    const CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                        : CU_TENSOR_MAP_SWIZZLE_NONE;
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool make_bf16_map_nd(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims,
