@@ -114,6 +114,7 @@ def measured_peaks():
 KERNEL_SOURCES = {
     "reduce": ["k_tc.cu"], "apply": ["k_tc.cu"], "finish": ["k_finish.cu"],
     "reduce_tc_rope": ["k_rope_tc.cu"], "apply_tc_rope": ["k_rope_tc.cu"],
+    "reduce_tc_e4m3_rope": ["k_rope_tc.cu"], "apply_tc_e4m3_rope": ["k_rope_tc.cu"],
     "bwd_q": ["k_bwd_q_tc.cu"], "bwd_k": ["k_bwd_tc.cu"], "dwconv": ["k_conv.cu"],
 }
 SHARED_SOURCES = ["la_internal.cuh", "la_sm100.cuh"]
@@ -805,7 +806,7 @@ def main():
         # dominant kernel: the larger of reduce (reads k, v) and apply (reads q, writes out)
         dom, dom_ms = ("reduce", red_ms) if red_ms >= app_ms else ("apply", app_ms)
         ntens = 2
-        kname = f"{dom}_{path}" + ("_rope" if w.rope and path == "tc" else "")
+        kname = f"{dom}_{path}" + ("_rope" if w.rope and path.startswith("tc") else "")
     if f8:   # reduce: k, v codes; apply: q codes and bf16 out
         kern_bytes = per_call_th * w.d * (2 if dom == "reduce" else 3)
     elif f4:   # reduce: k, v codes and block scales; apply: q codes and scales, bf16 out

@@ -47,6 +47,8 @@
 // its TMEM and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -87,47 +89,65 @@ __device__ __forceinline__ void warp_arrive(uint64_t *bar) {
 }
 
 // ---------------------------------------------------------------- reduce layout
-// The raw ring is as deep as shared memory allows: under load a copy takes
-// ~4 us from issue to arrival, and only the stages in flight move data.
-constexpr int kRRaw = 10;                // raw stages: k (2 boxes) and v (2 boxes) of 32 tokens x 4 heads
-constexpr int kROp = 3;                  // transformed stages: R phi(k) hi (2 boxes), lo (2 boxes)
-constexpr int kRStage = 4 * kBox;        // 16 KiB, raw and transformed alike
-constexpr int kROpOff = kRRaw * kRStage;
-constexpr int kRTabOff = kROpOff + kROp * kRStage;
-constexpr int kRZOff = kRTabOff + kTabBytes;             // z sums [2][4 heads][32] fp32
-constexpr int kRBarOff = kRZOff + 2 * 128 * 4;
-constexpr int kRNumBars = 2 * kRRaw + 2 * kROp + 2 * 4 + 1;
-constexpr int kRSmem = kRBarOff + kRNumBars * 8 + 16 + 1024;
+// F8 false: bf16 k, v.  A raw stage holds k and v of 32 tokens x 4 heads (two
+// 64-feature boxes each, 16 KiB); the transformed stage R phi(k) hi and lo
+// (bf16, two boxes each); the MMAs read v from the raw stage.
+// F8 true: E4M3 codes.  A raw stage holds one 128-code box of k and one of v
+// (4 KiB each, 128-byte swizzle); the transformed stage R phi(k) hi and lo and
+// the decoded v, all f16 in the bf16 path's box layout (24 KiB), so the raw
+// stage is free once the transform has read it.
+template <bool F8>
+struct RR {
+    // The raw ring is as deep as shared memory allows: under load a copy takes
+    // ~4 us from issue to arrival, and only the stages in flight move data.
+    static constexpr int kRaw = F8 ? 16 : 10;
+    static constexpr int kRawStage = F8 ? 8192 : 4 * kBox;
+    static constexpr int kVRaw = F8 ? 4096 : 2 * kBox;      // v in a raw stage
+    static constexpr int kOp = 3;                          // transformed stages
+    static constexpr int kOpStage = F8 ? 6 * kBox : 4 * kBox;
+    static constexpr int kOpOff = kRaw * kRawStage;
+    static constexpr int kTabOff = kOpOff + kOp * kOpStage;
+    static constexpr int kZOff = kTabOff + kTabBytes;      // z sums [2][4 heads][32] fp32
+    static constexpr int kBarOff = kZOff + 2 * 128 * 4;
+    static constexpr int kNumBars = 2 * kRaw + 2 * kOp + 2 * 4 + 1;
+    static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
+    static_assert(kSmem <= 232448, "reduce shared memory");
+};
 // Per 16 tokens two M=128 x N=128 MMAs into one accumulator: A = R phi(K)
 // hi, then lo, of the 4 heads (key features as rows), B = V (value features
 // as columns); the 4 diagonal 32x32 blocks of D are used.  Two accumulators
 // of 128 columns.
 constexpr uint32_t kRTmemCols = 256;
-static_assert(kRSmem <= 232448, "reduce shared memory");
 
 // ---------------------------------------------------------------- apply layout
-constexpr int kATile = 128 * 128;        // 128 tokens x 64 bf16 features (2 heads): 16 KiB
 // The apply is bound by shared-memory bandwidth, so the rotated phi(q) (hi and
 // lo parts) goes to the tensor cores through tensor memory, not shared
 // memory: the transform stores it with tcgen05.st and the MMA reads A from
-// TMEM.  That leaves shared memory to the raw ring.
-constexpr int kARaw = 11;                // raw q stages
+// TMEM.  That leaves shared memory to the raw ring of q tiles (128 tokens x 2
+// heads): bf16, 16 KiB each (one box of 64 features, 128-byte swizzle); E4M3
+// codes, 8 KiB each (one box of 64 codes, 64-byte
+// swizzle), twice as many.
 constexpr int kAOp = 4;                  // transformed tiles in TMEM (hi, lo of 2 heads: 64 columns each)
-constexpr int kAStgOff = kARaw * kATile; // one [32 rows][64 bf16] staging box per epilogue warp
 constexpr int kABopBytes = 4 * 2048 + 256;              // S rows hi, lo of 2 heads, then Z_eff of 2 heads
-constexpr int kABopOff = kAStgOff + 4 * kBox;
-constexpr int kADenOff = kABopOff + 2 * kABopBytes;     // denominator halves [2][2 heads][2][128 rows] fp32
-constexpr int kATabOff = kADenOff + 2 * 512 * 4;
-constexpr int kABarOff = kATabOff + kTabBytes;
-constexpr int kANumBars = 2 * kARaw + 2 * kAOp + 2 * 2 + 2 * 2 + 2 * 2 + 1;
-constexpr int kASmem = kABarOff + kANumBars * 8 + 16 + 1024;
+template <bool F8>
+struct AA {
+    static constexpr int kTile = F8 ? 128 * 64 : 128 * 128;
+    static constexpr int kRaw = F8 ? 22 : 11;                     // raw q stages
+    static constexpr int kStgOff = kRaw * kTile;                 // one [32 rows][64 bf16] staging box per epilogue warp
+    static constexpr int kBopOff = kStgOff + 4 * kBox;
+    static constexpr int kDenOff = kBopOff + 2 * kABopBytes;     // denominator halves [2][2 heads][2][128 rows] fp32
+    static constexpr int kTabOff = kDenOff + 2 * 512 * 4;
+    static constexpr int kBarOff = kTabOff + kTabBytes;
+    static constexpr int kNumBars = 2 * kRaw + 2 * kAOp + 2 * 2 + 2 * 2 + 2 * 2 + 1;
+    static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
+    static_assert(kSmem <= 232448, "apply shared memory");
+    static_assert(kABopBytes % 16 == 0 && kBopOff % 16 == 0, "bulk copies need 16-byte alignment");
+};
 // TMEM: two accumulators of 2 heads x 32 columns (columns 0..127), then the
 // transformed tiles (columns 128..255): head hh at + 32 hh, hi at + 0, lo at
 // + 16, the 16-feature K step kk at + 8 kk
 constexpr uint32_t kATmemCols = 512;
 constexpr uint32_t kATmemA = 128;
-static_assert(kASmem <= 232448, "apply shared memory");
-static_assert(kABopBytes % 16 == 0 && kABopOff % 16 == 0, "bulk copies need 16-byte alignment");
 
 // ---------------------------------------------------------------- small helpers
 
@@ -168,29 +188,88 @@ struct Feat8 {
     float2 e1, o1;   // pairs c, d
 };
 
-// ReLU one chunk of 8 bf16 (4 feature pairs), rotate pair (x0, x1) by its
-// (cos, sin) to (x0 cos - x1 sin, x0 sin + x1 cos), and split the rotated
-// values into bf16 hi = RN(y) and lo = RN(y - hi).  t0 = (cos a, cos b,
-// sin a, sin b), t1 the same for pairs c, d.  f receives phi(x).
-__device__ __forceinline__ void rope_chunk(uint4 x, float4 t0, float4 t1, uint4 &hi, uint4 &lo, Feat8 &f) {
+// ReLU of one chunk of 8 bf16 (4 feature pairs) as fp32.
+__device__ __forceinline__ Feat8 relu_unpack_bf16(uint4 x) {
     const uint32_t wa = relu2(x.x), wb = relu2(x.y), wc = relu2(x.z), wd = relu2(x.w);
+    Feat8 f;
     f.e0 = make_float2(bf_lo(wa), bf_lo(wb));
     f.o0 = make_float2(bf_hi(wa), bf_hi(wb));
     f.e1 = make_float2(bf_lo(wc), bf_lo(wd));
     f.o1 = make_float2(bf_hi(wc), bf_hi(wd));
+    return f;
+}
+
+// Two FP8 E4M3 codes (the low 16 bits of c, the low byte first) as f16x2
+// (first code in the low half), exactly: every E4M3 value is an f16 value.
+__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t c) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(c & 0xFFFFu), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+__device__ __forceinline__ float2 f16x2_f32(uint32_t h) {
+    return __half22float2(*reinterpret_cast<const __half2 *>(&h));
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
+    const __half2 t = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&t);
+}
+
+// ReLU of one chunk of 8 E4M3 codes (features in byte order), decoded to fp32
+// without the tensor's scale.  As signed bytes every negative code (sign bit
+// set, -0 included) is below 0, so a signed max with 0 is ReLU on the codes.
+__device__ __forceinline__ Feat8 relu_decode_e4m3(uint2 c) {
+    const uint32_t w0 = __vmaxs4(c.x, 0u), w1 = __vmaxs4(c.y, 0u);
+    const float2 a = f16x2_f32(e4m3x2_f16x2(w0)), b = f16x2_f32(e4m3x2_f16x2(w0 >> 16));
+    const float2 cc = f16x2_f32(e4m3x2_f16x2(w1)), d = f16x2_f32(e4m3x2_f16x2(w1 >> 16));
+    Feat8 f;
+    f.e0 = make_float2(a.x, b.x);
+    f.o0 = make_float2(a.y, b.y);
+    f.e1 = make_float2(cc.x, d.x);
+    f.o1 = make_float2(cc.y, d.y);
+    return f;
+}
+
+// Rotate the 4 feature pairs (x0, x1) of a chunk by their (cos, sin) to
+// (x0 cos - x1 sin, x0 sin + x1 cos) and split the rotated values into a hi
+// part RN(y) and a lo part RN(y - hi), bf16 (H16 false) or f16 (H16 true).
+// t0 = (cos a, cos b, sin a, sin b), t1 the same for pairs c, d.
+template <bool H16>
+__device__ __forceinline__ void rotate_split(const Feat8 &f, float4 t0, float4 t1, uint4 &hi, uint4 &lo) {
     const float2 c0 = make_float2(t0.x, t0.y), s0 = make_float2(t0.z, t0.w);
     const float2 c1 = make_float2(t1.x, t1.y), s1 = make_float2(t1.z, t1.w);
     const float2 ye0 = ffma2(f.o0, make_float2(-s0.x, -s0.y), fmul2(f.e0, c0));
     const float2 yo0 = ffma2(f.o0, c0, fmul2(f.e0, s0));
     const float2 ye1 = ffma2(f.o1, make_float2(-s1.x, -s1.y), fmul2(f.e1, c1));
     const float2 yo1 = ffma2(f.o1, c1, fmul2(f.e1, s1));
-    hi = make_uint4(pack_bf2(ye0.x, yo0.x), pack_bf2(ye0.y, yo0.y), pack_bf2(ye1.x, yo1.x), pack_bf2(ye1.y, yo1.y));
-    // y - hi is exact in fp32
-    const float2 re0 = fsub2(ye0, make_float2(bf_lo(hi.x), bf_lo(hi.y)));
-    const float2 ro0 = fsub2(yo0, make_float2(bf_hi(hi.x), bf_hi(hi.y)));
-    const float2 re1 = fsub2(ye1, make_float2(bf_lo(hi.z), bf_lo(hi.w)));
-    const float2 ro1 = fsub2(yo1, make_float2(bf_hi(hi.z), bf_hi(hi.w)));
-    lo = make_uint4(pack_bf2(re0.x, ro0.x), pack_bf2(re0.y, ro0.y), pack_bf2(re1.x, ro1.x), pack_bf2(re1.y, ro1.y));
+    if constexpr (!H16) {
+        hi = make_uint4(pack_bf2(ye0.x, yo0.x), pack_bf2(ye0.y, yo0.y), pack_bf2(ye1.x, yo1.x),
+                        pack_bf2(ye1.y, yo1.y));
+        // y - hi is exact in fp32
+        const float2 re0 = fsub2(ye0, make_float2(bf_lo(hi.x), bf_lo(hi.y)));
+        const float2 ro0 = fsub2(yo0, make_float2(bf_hi(hi.x), bf_hi(hi.y)));
+        const float2 re1 = fsub2(ye1, make_float2(bf_lo(hi.z), bf_lo(hi.w)));
+        const float2 ro1 = fsub2(yo1, make_float2(bf_hi(hi.z), bf_hi(hi.w)));
+        lo = make_uint4(pack_bf2(re0.x, ro0.x), pack_bf2(re0.y, ro0.y), pack_bf2(re1.x, ro1.x),
+                        pack_bf2(re1.y, ro1.y));
+    } else {
+        hi = make_uint4(pack_f16x2(ye0.x, yo0.x), pack_f16x2(ye0.y, yo0.y), pack_f16x2(ye1.x, yo1.x),
+                        pack_f16x2(ye1.y, yo1.y));
+        const float2 h0 = f16x2_f32(hi.x), h1 = f16x2_f32(hi.y), h2 = f16x2_f32(hi.z), h3 = f16x2_f32(hi.w);
+        const float2 re0 = fsub2(ye0, make_float2(h0.x, h1.x));
+        const float2 ro0 = fsub2(yo0, make_float2(h0.y, h1.y));
+        const float2 re1 = fsub2(ye1, make_float2(h2.x, h3.x));
+        const float2 ro1 = fsub2(yo1, make_float2(h2.y, h3.y));
+        lo = make_uint4(pack_f16x2(re0.x, ro0.x), pack_f16x2(re0.y, ro0.y), pack_f16x2(re1.x, ro1.x),
+                        pack_f16x2(re1.y, ro1.y));
+    }
+}
+
+// ReLU one chunk of 8 bf16, rotate and split into bf16 hi and lo parts; f
+// receives phi(x).
+__device__ __forceinline__ void rope_chunk(uint4 x, float4 t0, float4 t1, uint4 &hi, uint4 &lo, Feat8 &f) {
+    f = relu_unpack_bf16(x);
+    rotate_split<false>(f, t0, t1, hi, lo);
 }
 
 // The (cos, sin) records of every position of the call: for each of the 8
@@ -294,14 +373,17 @@ struct UnitWalk {
 
 // ================================================================ reduce
 
+template <bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
 rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    float *__restrict__ partials, const Plan p) {
+    using C = RR<F8>;
+    constexpr int kRRaw = C::kRaw, kROp = C::kOp;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
-    uint8_t *tab = smem + kRTabOff;
-    float *zbuf = reinterpret_cast<float *>(smem + kRZOff);
-    uint64_t *raw_full = reinterpret_cast<uint64_t *>(smem + kRBarOff);
+    uint8_t *tab = smem + C::kTabOff;
+    float *zbuf = reinterpret_cast<float *>(smem + C::kZOff);
+    uint64_t *raw_full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
     uint64_t *raw_empty = raw_full + kRRaw;
     uint64_t *op_full = raw_empty + kRRaw;
     uint64_t *op_empty = op_full + kROp;
@@ -328,7 +410,8 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     if (threadIdx.x == 0) {
         for (int s = 0; s < kRRaw; ++s) {
             mbar_init(&raw_full[s], 1);
-            mbar_init(&raw_empty[s], 1);
+            // bf16: the MMAs free a raw stage (they read v there); E4M3: the transform
+            mbar_init(&raw_empty[s], F8 ? kXfWarps : 1);
         }
         for (int o = 0; o < kROp; ++o) {
             mbar_init(&op_full[o], kXfWarps);
@@ -396,21 +479,26 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                         ok = false;
                         break;
                     }
-                    uint8_t *stg = smem + s * kRStage;
+                    uint8_t *stg = smem + s * C::kRawStage;
                     const int row = sg.n * p.L + sg.tok0 + 32 * st;
-                    const int c0 = sg.g * 128;
-                    mbar_arrive_expect_tx(&raw_full[s], kRStage);
-                    tma_load_3d(stg, &tm_k, &raw_full[s], c0, row, sg.b);
-                    tma_load_3d(stg + kBox, &tm_k, &raw_full[s], c0 + 64, row, sg.b);
-                    tma_load_3d(stg + 2 * kBox, &tm_v, &raw_full[s], c0, row, sg.b);
-                    tma_load_3d(stg + 3 * kBox, &tm_v, &raw_full[s], c0 + 64, row, sg.b);
+                    const int c0 = sg.g * 128;   // features, = bytes for E4M3 codes
+                    mbar_arrive_expect_tx(&raw_full[s], C::kRawStage);
+                    if constexpr (F8) {
+                        tma_load_3d(stg, &tm_k, &raw_full[s], c0, row, sg.b);
+                        tma_load_3d(stg + C::kVRaw, &tm_v, &raw_full[s], c0, row, sg.b);
+                    } else {
+                        tma_load_3d(stg, &tm_k, &raw_full[s], c0, row, sg.b);
+                        tma_load_3d(stg + kBox, &tm_k, &raw_full[s], c0 + 64, row, sg.b);
+                        tma_load_3d(stg + C::kVRaw, &tm_v, &raw_full[s], c0, row, sg.b);
+                        tma_load_3d(stg + C::kVRaw + kBox, &tm_v, &raw_full[s], c0 + 64, row, sg.b);
+                    }
                     issued = i + 1;
                 }
             }
         }
     } else if (warp == kWarpMma) {
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(128, 128, 1, 1);
+            const uint32_t idesc = F8 ? idesc_f16(128, 128, 1, 1) : idesc_bf16(128, 128, 1, 1);
             UnitWalk w;
             w.start(S, x_begin);
             bool ok = true;
@@ -433,8 +521,9 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t hi = smem_u32(smem + kROpOff + o * kRStage);
-                    const uint32_t va = smem_u32(smem + s * kRStage + 2 * kBox);
+                    const uint32_t hi = smem_u32(smem + C::kOpOff + o * C::kOpStage);
+                    // v: the raw stage (bf16), or the decoded box after lo (E4M3)
+                    const uint32_t va = F8 ? hi + 4 * kBox : smem_u32(smem + s * C::kRawStage + C::kVRaw);
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk) {
                         // MN-major, 128-byte swizzle: the 64-feature boxes are the MN
@@ -447,7 +536,7 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                         mma_bf16(d, dl, dv, idesc, 1u);
                     }
                     mma_commit(&op_empty[o]);
-                    mma_commit(&raw_empty[s]);   // v is read from the raw stage
+                    if constexpr (!F8) mma_commit(&raw_empty[s]);   // v is read from the raw stage
                 }
                 if (!ok) break;
                 mma_commit(&acc_full[a]);
@@ -479,7 +568,15 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             float kv[32];
             tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 128 + 32 * q), kv);
             tmem_wait_ld();
-            const float z = zbuf[a * 128 + q * 32 + lane];
+            float z = zbuf[a * 128 + q * 32 + lane];
+            if constexpr (F8) {
+                // the sums are over the codes: KV = sk sv sum R phi(k^) v^, z = sk sum phi(k^)
+                // (ReLU commutes with the positive scale, the rotation is linear)
+                const float skv = p.sk * p.sv;
+#pragma unroll
+                for (int k = 0; k < 32; ++k) kv[k] *= skv;
+                z *= p.sk;
+            }
             tc_fence_before();
             warp_arrive(&acc_empty[a]);
             warp_arrive(&z_empty[a]);
@@ -502,6 +599,8 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         const int r = lane;
         // byte offset of the chunk in a stage: box head / 2, 64-byte half head % 2
         const int chunk = (head >> 1) * kBox + r * 128 + (((4 * (head & 1) + j) ^ (r & 7)) << 4);
+        // E4M3: the same 8 features in the 128-code row of the raw box
+        const int chunk8 = r * 128 + (((2 * head + (j >> 1)) ^ (r & 7)) << 4) + ((j & 1) << 3);
         const GroupRec g0 = group_rec(p, 2 * j), g1 = group_rec(p, 2 * j + 1);
         Feat8 zs;
         zs.e0 = zs.o0 = zs.e1 = zs.o1 = make_float2(0.f, 0.f);
@@ -519,10 +618,29 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 if (ok && !mbar_wait(&raw_full[s], (uint32_t)(i / kRRaw) & 1u, abort_word, &g_rope_wait_flag, 6))
                     ok = false;
                 const int tb = sg.tok0 + 32 * st + r;   // token of this row inside the block
-                const uint8_t *raw = smem + s * kRStage;
-                uint8_t *op = smem + kROpOff + o * kRStage;
-                uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;   // rows past the segment contribute nothing
-                if (ok && tb < sg.tok1) {
+                const uint8_t *raw = smem + s * C::kRawStage;
+                uint8_t *op = smem + C::kOpOff + o * C::kOpStage;
+                uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi, vd = hi;   // rows past the segment contribute nothing
+                if constexpr (F8) {
+                    uint2 ck = make_uint2(0u, 0u), cv = ck;
+                    if (ok) {
+                        ck = *reinterpret_cast<const uint2 *>(raw + chunk8);
+                        cv = *reinterpret_cast<const uint2 *>(raw + C::kVRaw + chunk8);
+                    }
+                    // the raw stage may be refilled once every thread has read it
+                    fence_proxy_async_smem();
+                    warp_arrive(&raw_empty[s]);
+                    if (ok && tb < sg.tok1) {
+                        const Feat8 f = relu_decode_e4m3(ck);
+                        rotate_split<true>(f, tab_rec(tab, g0, pq), tab_rec(tab, g1, pq), hi, lo);
+                        zs.e0 = fadd2(zs.e0, f.e0);
+                        zs.o0 = fadd2(zs.o0, f.o0);
+                        zs.e1 = fadd2(zs.e1, f.e1);
+                        zs.o1 = fadd2(zs.o1, f.o1);
+                        vd = make_uint4(e4m3x2_f16x2(cv.x), e4m3x2_f16x2(cv.x >> 16), e4m3x2_f16x2(cv.y),
+                                        e4m3x2_f16x2(cv.y >> 16));
+                    }
+                } else if (ok && tb < sg.tok1) {
                     const float4 t0 = tab_rec(tab, g0, pq);
                     const float4 t1 = tab_rec(tab, g1, pq);
                     Feat8 f;
@@ -537,6 +655,7 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                     ok = false;
                 *reinterpret_cast<uint4 *>(op + chunk) = hi;
                 *reinterpret_cast<uint4 *>(op + 2 * kBox + chunk) = lo;
+                if constexpr (F8) *reinterpret_cast<uint4 *>(op + 4 * kBox + chunk) = vd;
                 // the generic writes of this stage before the tensor cores read it
                 fence_proxy_async_smem();
                 warp_arrive(&op_full[o]);
@@ -577,16 +696,19 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 
 // ================================================================ apply
 
+template <bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
 rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_out,
                   __nv_bfloat16 *__restrict__ out, const uint8_t *__restrict__ bop, const float *__restrict__ seff,
                   const Plan p) {
+    using C = AA<F8>;
+    constexpr int kARaw = C::kRaw, kATile = C::kTile;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
-    uint8_t *tab = smem + kATabOff;
-    uint8_t *bops = smem + kABopOff;
-    float *den_s = reinterpret_cast<float *>(smem + kADenOff);
-    uint64_t *raw_full = reinterpret_cast<uint64_t *>(smem + kABarOff);
+    uint8_t *tab = smem + C::kTabOff;
+    uint8_t *bops = smem + C::kBopOff;
+    float *den_s = reinterpret_cast<float *>(smem + C::kDenOff);
+    uint64_t *raw_full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
     uint64_t *raw_empty = raw_full + kARaw;
     uint64_t *op_full = raw_empty + kARaw;
     uint64_t *op_empty = op_full + kAOp;
@@ -793,11 +915,23 @@ rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const bool valid = r < Ln - row0;
             if (ok && !mbar_wait(&raw_full[s], (uint32_t)(i / kARaw) & 1u, abort_word, &g_rope_wait_flag, 17)) ok = false;
             uint4 xq[2];
-            const uint8_t *raw = smem + s * kATile + r * 128;
+            if constexpr (F8) {
+                // 16 codes (features 16 jh ..) of the 64-code row, 64-byte swizzle:
+                // 16-byte chunk c of row r at c ^ ((r / 2) % 4)
+                const uint8_t *raw = smem + s * kATile + r * 64;
+                const uint4 x8 = (ok && valid)
+                                     ? *reinterpret_cast<const uint4 *>(raw + (((2 * hh + jh) ^ ((r >> 1) & 3)) << 4))
+                                     : make_uint4(0u, 0u, 0u, 0u);
+                xq[0] = make_uint4(x8.x, x8.y, 0u, 0u);
+                xq[1] = make_uint4(x8.z, x8.w, 0u, 0u);
+            } else {
+                const uint8_t *raw = smem + s * kATile + r * 128;
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
-                xq[c] = (ok && valid) ? *reinterpret_cast<const uint4 *>(raw + (((4 * hh + 2 * jh + c) ^ (r & 7)) << 4))
-                                      : make_uint4(0u, 0u, 0u, 0u);
+                for (int c = 0; c < 2; ++c)
+                    xq[c] = (ok && valid)
+                                ? *reinterpret_cast<const uint4 *>(raw + (((4 * hh + 2 * jh + c) ^ (r & 7)) << 4))
+                                : make_uint4(0u, 0u, 0u, 0u);
+            }
             // the raw stage may be refilled as soon as every thread has read it:
             // order these generic reads before the async proxy's refill
             fence_proxy_async_smem();
@@ -809,7 +943,13 @@ rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 hi[c] = lo[c] = make_uint4(0u, 0u, 0u, 0u);
                 if (ok && valid) {
                     Feat8 f;
-                    rope_chunk(xq[c], tab_rec(tab, gr[c][0], pq), tab_rec(tab, gr[c][1], pq), hi[c], lo[c], f);
+                    if constexpr (F8) {
+                        // the codes without the tensor's scale (the epilogue applies it)
+                        f = relu_decode_e4m3(make_uint2(xq[c].x, xq[c].y));
+                        rotate_split<false>(f, tab_rec(tab, gr[c][0], pq), tab_rec(tab, gr[c][1], pq), hi[c], lo[c]);
+                    } else {
+                        rope_chunk(xq[c], tab_rec(tab, gr[c][0], pq), tab_rec(tab, gr[c][1], pq), hi[c], lo[c], f);
+                    }
                     // the denominator takes the unrotated phi(q)
                     den = ffma2(f.e0, ze[c][0], den);
                     den = ffma2(f.o0, zo[c][0], den);
@@ -848,7 +988,7 @@ rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         // head at a time
         const int q = warp & 3;
         const int r = 32 * q + lane;               // token row of this thread in a tile
-        uint8_t *sb = smem + kAStgOff + q * kBox;  // this warp's staging box
+        uint8_t *sb = smem + C::kStgOff + q * kBox;  // this warp's staging box
         UnitWalk w;
         w.start(S, x_begin);
         bool ok = true;
@@ -881,7 +1021,8 @@ rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     tmem_wait_ld();
                     // the sum of the two halves of the denominator, in a fixed order
                     const float den = den_s[a * 512 + (2 * hh) * 128 + r] + den_s[a * 512 + (2 * hh + 1) * 128 + r];
-                    const float iv = 1.0f / (den + p.eps);
+                    // E4M3: out = sq num^ / (sq den^ + eps), num^ and den^ from the codes
+                    const float iv = F8 ? p.sq / (p.sq * den + p.eps) : 1.0f / (den + p.eps);
                     const float2 inv = make_float2(iv, iv);
                     uint4 y[4];
 #pragma unroll
@@ -944,7 +1085,10 @@ bool smem_ready() {
     static std::once_flag once;
     static bool ok = false;
     std::call_once(once, [] {
-        ok = set_smem((const void *)rope_reduce_kernel, kRSmem) && set_smem((const void *)rope_apply_kernel, kASmem);
+        ok = set_smem((const void *)rope_reduce_kernel<false>, RR<false>::kSmem) &&
+             set_smem((const void *)rope_apply_kernel<false>, AA<false>::kSmem) &&
+             set_smem((const void *)rope_reduce_kernel<true>, RR<true>::kSmem) &&
+             set_smem((const void *)rope_apply_kernel<true>, AA<true>::kSmem);
     });
     return ok;
 }
@@ -1018,16 +1162,38 @@ bool tc_rope_fits(const Plan &p) { return p.rope && p.tab_bytes > 0 && p.H % 4 =
 int launch_reduce_rope_tc(const void *k, const void *v, float *partials, const Plan &p, cudaStream_t s) {
     if (!smem_ready() || !tc_rope_fits(p) || !p.sk_layout) return -1;
     CUtensorMap mk, mv;
+    if (p.f8) {
+        // E4M3 codes: boxes of the 4 heads' 128 codes x 32 tokens, 128-byte swizzle
+        const long long row = (long long)p.H * kD;
+        if (!make_u8_map(&mk, k, p.B, p.N, row, 128, 32, 128) || !make_u8_map(&mv, v, p.B, p.N, row, 128, 32, 128))
+            return -1;
+        return launch_pdl(rope_reduce_kernel<true>, (unsigned)p.skr.C, kThreads, RR<true>::kSmem, s, mk, mv, partials,
+                          p)
+                   ? 1
+                   : -1;
+    }
     if (!make_bf16_map(&mk, k, p.B, p.N, p.H, 32) || !make_bf16_map(&mv, v, p.B, p.N, p.H, 32)) return -1;
-    return launch_pdl(rope_reduce_kernel, (unsigned)p.skr.C, kThreads, kRSmem, s, mk, mv, partials, p) ? 1 : -1;
+    return launch_pdl(rope_reduce_kernel<false>, (unsigned)p.skr.C, kThreads, RR<false>::kSmem, s, mk, mv, partials,
+                      p)
+               ? 1
+               : -1;
 }
 
 int launch_apply_rope_tc(const void *q, void *out, const void *bop, const float *seff, const Plan &p,
                          cudaStream_t s) {
     if (!smem_ready() || !tc_rope_fits(p)) return -1;
     CUtensorMap mq, mo;
-    if (!make_bf16_map(&mq, q, p.B, p.N, p.H, 128) || !make_bf16_map(&mo, out, p.B, p.N, p.H, 32)) return -1;
-    return launch_pdl(rope_apply_kernel, (unsigned)p.ska.C, kThreads, kASmem, s, mq, mo,
+    if (!make_bf16_map(&mo, out, p.B, p.N, p.H, 32)) return -1;
+    if (p.f8) {
+        // E4M3 codes: boxes of a head pair's 64 codes x 128 tokens, 64-byte swizzle
+        if (!make_u8_map(&mq, q, p.B, p.N, (long long)p.H * kD, 64, 128, 64)) return -1;
+        return launch_pdl(rope_apply_kernel<true>, (unsigned)p.ska.C, kThreads, AA<true>::kSmem, s, mq, mo,
+                          static_cast<__nv_bfloat16 *>(out), static_cast<const uint8_t *>(bop), seff, p)
+                   ? 1
+                   : -1;
+    }
+    if (!make_bf16_map(&mq, q, p.B, p.N, p.H, 128)) return -1;
+    return launch_pdl(rope_apply_kernel<false>, (unsigned)p.ska.C, kThreads, AA<false>::kSmem, s, mq, mo,
                       static_cast<__nv_bfloat16 *>(out), static_cast<const uint8_t *>(bop), seff, p)
                ? 1
                : -1;

@@ -119,13 +119,14 @@ la_status common_checks(const void *q, const void *k, const void *v, void *out, 
 // reduce groups, 2-head apply tiles) and, with RoPE, a cos/sin table that fits
 // their shared memory; the rest runs on the CUDA cores.
 bool use_tc(la_dtype dt, const la::Plan &p) {
-    if (p.f8) return (p.H % 4) == 0 && !p.rope && la::tc_available();
+    if (p.f8) return (p.H % 4) == 0 && (!p.rope || la::tc_rope_fits(p)) && la::tc_available();
     if (p.f4) return (p.H % 8) == 0 && !p.rope && la::tc_available();
     return dt == LA_BF16 && (p.H % 4) == 0 && (!p.rope || la::tc_rope_fits(p)) && la::tc_available();
 }
 
 // FP8 E4M3 calls: q, k, v codes with per-tensor scales, bf16 out; tensor cores
-// only (H a multiple of 4), no RoPE.
+// only (H a multiple of 4; with RoPE, a grid whose cos/sin table fits the RoPE
+// kernels' shared memory).
 la_status e4m3_checks(const void *q, const void *k, const void *v, void *out, int B, int N, int H, int d,
                       float eps, float sq, float sk, float sv) {
     la_status e = common_checks(q, k, v, out, LA_BF16, B, N, H, d, eps);
@@ -177,7 +178,7 @@ la_status run(const void *q, const void *k, const void *v, void *out, la_dtype d
         if (r < 0 || !mark(3, s)) return LA_ECUDA;
         n += r;
         g_last_launches = n;
-        g_last_path = "tc";
+        g_last_path = p.f8 ? "tc_e4m3" : "tc";
         return LA_OK;
     }
     if (tc && fuse_plan(p)) {
@@ -393,10 +394,11 @@ la_status la_full_backward(const void *q, const void *k, const void *v, const vo
 
 la_status la_full_forward_e4m3(const void *q, const void *k, const void *v, float scale_q, float scale_k,
                                float scale_v, void *out, int B, int N, int H, int d, int tokens_per_block,
-                               float eps, void *ws, size_t ws_bytes, void *stream) {
+                               const la_rope *rope, float eps, void *ws, size_t ws_bytes, void *stream) {
     la_status e = e4m3_checks(q, k, v, out, B, N, H, d, eps, scale_q, scale_k, scale_v);
     if (e != LA_OK) return e;
     if (tokens_per_block < 0) return LA_EINVAL;
+    if ((e = check_rope(rope, d, false)) != LA_OK) return e;
     const size_t need = la_workspace_size(B, N, H, d, tokens_per_block);
     if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return LA_EWORKSPACE;
     la::Plan p{};
@@ -407,17 +409,19 @@ la_status la_full_forward_e4m3(const void *q, const void *k, const void *v, floa
     p.f8 = 1;
     p.sq = scale_q; p.sk = scale_k; p.sv = scale_v;
     make_splits(p);
-    fill_rope(p, nullptr, 0);
+    fill_rope(p, rope, rope ? rope->t_offset : 0);
+    if (!use_tc(LA_BF16, p)) return LA_EUNSUPPORTED;   // E4M3 runs on the tensor cores only
     return run(q, k, v, out, LA_BF16, p, nullptr, nullptr, ws, static_cast<cudaStream_t>(stream));
 }
 
 la_status la_block_forward_e4m3(const void *q, const void *k, const void *v, float scale_q, float scale_k,
                                 float scale_v, void *out, int B, int N_blk, int H, int d, la_state *st, int commit,
-                                float eps, void *ws, size_t ws_bytes, void *stream) {
+                                const la_rope *rope, float eps, void *ws, size_t ws_bytes, void *stream) {
     la_status e = e4m3_checks(q, k, v, out, B, N_blk, H, d, eps, scale_q, scale_k, scale_v);
     if (e != LA_OK) return e;
     if (!st || !st->S || !st->Z) return LA_EINVAL;
     if (st->B != B || st->H != H || st->d != d) return LA_EINVAL;
+    if ((e = check_rope(rope, d, true)) != LA_OK) return e;
     const size_t need = la_workspace_size(B, N_blk, H, d, N_blk);
     if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return LA_EWORKSPACE;
     la::Plan p{};
@@ -428,10 +432,14 @@ la_status la_block_forward_e4m3(const void *q, const void *k, const void *v, flo
     p.f8 = 1;
     p.sq = scale_q; p.sk = scale_k; p.sv = scale_v;
     make_splits(p);
-    fill_rope(p, nullptr, 0);
+    fill_rope(p, rope, rope ? (rope->t_offset < 0 ? st->t_next : rope->t_offset) : 0);
+    if (!use_tc(LA_BF16, p)) return LA_EUNSUPPORTED;   // E4M3 runs on the tensor cores only
     e = run(q, k, v, out, LA_BF16, p, st->S, st->Z, ws, static_cast<cudaStream_t>(stream));
     if (e != LA_OK) return e;
-    if (commit) st->blocks_committed += 1;
+    if (commit) {
+        st->blocks_committed += 1;
+        if (rope) st->t_next += rope->T;
+    }
     return LA_OK;
 }
 

@@ -302,6 +302,10 @@ inline bool set_smem(const void *kernel, int bytes) {
 // 3D TMA map of a [B][N][H*32] bf16 tensor: boxes of 64 features x box_rows
 // tokens, 128-byte swizzle.
 bool make_bf16_map(CUtensorMap *m, const void *base, int B, int N, int H, int box_rows);
+// 3D view of a [B][N][row_bytes] byte tensor (E4M3 codes): boxes of box_inner
+// bytes x box_rows tokens, swizzle of 0, 64 or 128 bytes.
+bool make_u8_map(CUtensorMap *m, const void *base, int B, int N, long long row_bytes, int box_inner, int box_rows,
+                 int swizzle_bytes);
 
 // A rank-dimensional TMA map of a bf16 tensor (dims innermost first, byte
 // strides of dims 1.., box extents), no swizzle, zero fill out of range.

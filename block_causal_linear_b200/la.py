@@ -76,10 +76,11 @@ def lib() -> ctypes.CDLL:
         L.la_full_forward_static_ws.argtypes = [vp, vp, vp, vp, ip, ip, ip, ip, ip, ip,
                                                 ctypes.POINTER(la_rope), fp, vp]
         L.la_full_forward_static_ws.restype = ip
-        L.la_full_forward_e4m3.argtypes = [vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ip, fp, vp, sz, vp]
+        L.la_full_forward_e4m3.argtypes = [vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ip, ctypes.POINTER(la_rope),
+                                           fp, vp, sz, vp]
         L.la_full_forward_e4m3.restype = ip
         L.la_block_forward_e4m3.argtypes = [vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ctypes.POINTER(la_state), ip,
-                                            fp, vp, sz, vp]
+                                            ctypes.POINTER(la_rope), fp, vp, sz, vp]
         L.la_block_forward_e4m3.restype = ip
         L.la_full_forward_nvfp4.argtypes = [vp, vp, vp, vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ip, fp, vp, sz, vp]
         L.la_full_forward_nvfp4.restype = ip
@@ -161,14 +162,18 @@ def la_full_forward_static_ws(q, k, v, out, dt, B, N, H, d, tokens_per_block, ro
 LA_STATIC_WS_BYTES = 16 << 20
 
 
-def la_full_forward_e4m3(q, k, v, sq, sk, sv, out, B, N, H, d, tokens_per_block, eps, ws, ws_bytes, stream) -> int:
-    return int(lib().la_full_forward_e4m3(q, k, v, sq, sk, sv, out, B, N, H, d, tokens_per_block, eps, ws, ws_bytes,
+def la_full_forward_e4m3(q, k, v, sq, sk, sv, out, B, N, H, d, tokens_per_block, rope, eps, ws, ws_bytes,
+                         stream) -> int:
+    return int(lib().la_full_forward_e4m3(q, k, v, sq, sk, sv, out, B, N, H, d, tokens_per_block,
+                                          ctypes.byref(rope) if rope is not None else None, eps, ws, ws_bytes,
                                           stream))
 
 
-def la_block_forward_e4m3(q, k, v, sq, sk, sv, out, B, N_blk, H, d, st, commit, eps, ws, ws_bytes, stream) -> int:
-    return int(lib().la_block_forward_e4m3(q, k, v, sq, sk, sv, out, B, N_blk, H, d, ctypes.byref(st), commit, eps,
-                                           ws, ws_bytes, stream))
+def la_block_forward_e4m3(q, k, v, sq, sk, sv, out, B, N_blk, H, d, st, commit, rope, eps, ws, ws_bytes,
+                          stream) -> int:
+    return int(lib().la_block_forward_e4m3(q, k, v, sq, sk, sv, out, B, N_blk, H, d, ctypes.byref(st), commit,
+                                           ctypes.byref(rope) if rope is not None else None, eps, ws, ws_bytes,
+                                           stream))
 
 
 def la_dwconv3d(x, y, dt, B, T, Hg, Wg, C, kt, kh, kw, weight, bias, stream) -> int:
@@ -404,9 +409,9 @@ def _check_codes(q, k, v):
 
 
 def full_forward_e4m3(q, k, v, scales, tokens_per_block=0, eps=1e-6, ws: Optional[torch.Tensor] = None,
-                      out: Optional[torch.Tensor] = None, stream=None):
+                      out: Optional[torch.Tensor] = None, stream=None, rope=None):
     """la_full_forward on FP8 E4M3 codes (uint8 tensors) with per-tensor
-    scales (sq, sk, sv); out is bf16."""
+    scales (sq, sk, sv), optional 3D RoPE; out is bf16."""
     _check_codes(q, k, v)
     B, N, H, d = q.shape
     if ws is None:
@@ -415,7 +420,7 @@ def full_forward_e4m3(q, k, v, scales, tokens_per_block=0, eps=1e-6, ws: Optiona
         out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
     sq, sk, sv = (float(x) for x in scales)
     rc = la_full_forward_e4m3(q.data_ptr(), k.data_ptr(), v.data_ptr(), sq, sk, sv, out.data_ptr(), B, N, H, d,
-                              int(tokens_per_block), float(eps), ws.data_ptr(), ws.numel() * ws.element_size(),
+                              int(tokens_per_block), rope, float(eps), ws.data_ptr(), ws.numel() * ws.element_size(),
                               _stream_ptr(stream))
     if rc != LA_OK:
         raise LAError(rc, "la_full_forward_e4m3")
@@ -423,7 +428,7 @@ def full_forward_e4m3(q, k, v, scales, tokens_per_block=0, eps=1e-6, ws: Optiona
 
 
 def block_forward_e4m3(q, k, v, scales, state: "State", commit=True, eps=1e-6, ws: Optional[torch.Tensor] = None,
-                       out: Optional[torch.Tensor] = None, stream=None):
+                       out: Optional[torch.Tensor] = None, stream=None, rope=None):
     _check_codes(q, k, v)
     B, N, H, d = q.shape
     if ws is None:
@@ -432,8 +437,8 @@ def block_forward_e4m3(q, k, v, scales, state: "State", commit=True, eps=1e-6, w
         out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
     sq, sk, sv = (float(x) for x in scales)
     rc = la_block_forward_e4m3(q.data_ptr(), k.data_ptr(), v.data_ptr(), sq, sk, sv, out.data_ptr(), B, N, H, d,
-                               state.c, int(bool(commit)), float(eps), ws.data_ptr(), ws.numel() * ws.element_size(),
-                               _stream_ptr(stream))
+                               state.c, int(bool(commit)), rope, float(eps), ws.data_ptr(),
+                               ws.numel() * ws.element_size(), _stream_ptr(stream))
     if rc != LA_OK:
         raise LAError(rc, "la_block_forward_e4m3")
     return out

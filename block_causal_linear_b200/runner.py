@@ -41,8 +41,6 @@ class Runner:
         self.scales = None
         if e4m3:
             # FP8 inputs: each call's q, k, v as E4M3 codes with per-tensor scales
-            if w.rope:
-                raise ValueError("the E4M3 path takes no RoPE")
             self.scales = []
             for i, c in enumerate(self.calls):
                 qk = [synth.to_e4m3(t) for t in c[2:5]]
@@ -83,7 +81,7 @@ class Runner:
                                       out=self.outs[0], stream=stream)
             elif self.e4m3:
                 la.full_forward_e4m3(q, k, v, self.scales[0], self.tokens_per_block, eps=w.eps, ws=self.ws,
-                                     out=self.outs[0], stream=stream)
+                                     out=self.outs[0], stream=stream, rope=self.rope)
             else:
                 la.full_forward(q, k, v, self.tokens_per_block, rope=self.rope, eps=w.eps, ws=self.ws,
                                 out=self.outs[0], stream=stream)
@@ -102,7 +100,7 @@ class Runner:
                                            ws=self.ws, out=self.outs[i], stream=stream)
                 elif self.e4m3:
                     la.block_forward_e4m3(q, k, v, self.scales[i], st, commit=(p == w.passes - 1), eps=w.eps,
-                                          ws=self.ws, out=self.outs[i], stream=stream)
+                                          ws=self.ws, out=self.outs[i], stream=stream, rope=self.rope)
                 else:
                     la.block_forward(q, k, v, st, commit=(p == w.passes - 1), rope=self.rope, eps=w.eps,
                                      ws=self.ws, out=self.outs[i], stream=stream)

@@ -251,18 +251,24 @@ LA_API la_status la_full_backward(const void *q, const void *k, const void *v, c
  * başlattı", section "Etkin eğitim ve çıkarım stratejileri": SVDQuant); FP8
  * q, k, v here shrink the bytes this path moves (160 instead of 256 per token
  * and head).
+ * With rope, the rotation acts on phi(q^), phi(k^) as in the bf16 calls (a
+ * rotation is linear, so the scales still factor out), and rope follows the
+ * bf16 calls' rules (la_block_forward_e4m3: t_offset < 0 takes the state's
+ * t_next, a commit advances it by rope->T).
  * Scales must be finite and > 0 (LA_EINVAL); H must be a multiple of 4 and
- * the GPU must take the tensor-core path (else LA_EUNSUPPORTED); no RoPE.
- * Workspace and every other argument as in the bf16 calls.
+ * the GPU must take the tensor-core path, which with rope also needs the
+ * call's cos/sin records (8 groups of 4 features, each group on one axis,
+ * over the call's frames, rows and columns) to fit 8 KiB (else
+ * LA_EUNSUPPORTED).  Workspace and every other argument as in the bf16 calls.
  */
 LA_API la_status la_full_forward_e4m3(const void *q, const void *k, const void *v, float scale_q,
                                       float scale_k, float scale_v, void *out, int B, int N, int H,
-                                      int d, int tokens_per_block, float eps, void *ws,
-                                      size_t ws_bytes, void *stream);
+                                      int d, int tokens_per_block, const la_rope *rope, float eps,
+                                      void *ws, size_t ws_bytes, void *stream);
 LA_API la_status la_block_forward_e4m3(const void *q, const void *k, const void *v, float scale_q,
                                        float scale_k, float scale_v, void *out, int B, int N_blk,
-                                       int H, int d, la_state *st, int commit, float eps, void *ws,
-                                       size_t ws_bytes, void *stream);
+                                       int H, int d, la_state *st, int commit, const la_rope *rope,
+                                       float eps, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * NVFP4 inputs, the format the pages deploy the model in ("Nvidia, MIT ve

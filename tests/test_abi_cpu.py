@@ -149,10 +149,11 @@ def test_backward_workspace_size(la):
 def test_e4m3_validation(la):
     def full(**kw):
         a = dict(q=FAKE, k=FAKE, v=FAKE, sq=0.01, sk=0.01, sv=0.01, out=FAKE, B=1, N=256, H=4, d=32, tpb=0,
-                 eps=1e-6, ws=FAKE, ws_bytes=1 << 30, stream=None)
+                 rope=None, eps=1e-6, ws=FAKE, ws_bytes=1 << 30, stream=None)
         a.update(kw)
         return la.la_full_forward_e4m3(a["q"], a["k"], a["v"], a["sq"], a["sk"], a["sv"], a["out"], a["B"], a["N"],
-                                       a["H"], a["d"], a["tpb"], a["eps"], a["ws"], a["ws_bytes"], a["stream"])
+                                       a["H"], a["d"], a["tpb"], a["rope"], a["eps"], a["ws"], a["ws_bytes"],
+                                       a["stream"])
     assert full(q=None) == la.LA_EINVAL
     assert full(out=FAKE + 4) == la.LA_EINVAL
     assert full(sq=0.0) == la.LA_EINVAL
@@ -160,8 +161,11 @@ def test_e4m3_validation(la):
     assert full(sv=float("nan")) == la.LA_EINVAL
     assert full(d=16) == la.LA_EUNSUPPORTED
     assert full(H=6) == la.LA_EUNSUPPORTED             # the E4M3 path takes 4-head groups
+    # RoPE is checked like the bf16 calls': dims must add up to d, even and >= 0
+    assert full(rope=la.make_rope(Hg=3, Wg=5, dims=(8, 12, 10))) in (la.LA_EINVAL, la.LA_EUNSUPPORTED)
+    assert full(rope=la.make_rope(Hg=3, Wg=5, t_offset=-1)) in (la.LA_EINVAL, la.LA_EUNSUPPORTED)
     st = la.la_state()
-    assert la.la_block_forward_e4m3(FAKE, FAKE, FAKE, 1.0, 1.0, 1.0, FAKE, 1, 64, 4, 32, st, 1, 1e-6, FAKE,
+    assert la.la_block_forward_e4m3(FAKE, FAKE, FAKE, 1.0, 1.0, 1.0, FAKE, 1, 64, 4, 32, st, 1, None, 1e-6, FAKE,
                                     1 << 30, None) in (la.LA_EINVAL, la.LA_EUNSUPPORTED)
     assert st.blocks_committed == 0
 

@@ -3,7 +3,10 @@
 fp32 path:  max_i |g_i - o_i| / max(|o_i|, 1e-2 * RMS(o)) <= 1e-4
             (relative error per element; the floor keeps outputs near zero
             from dividing by almost nothing)
-bf16 path:  max_i |g_i - o_i| / RMS(o) <= 2e-2
+bf16 path:  max_i |g_i - o_i| / RMS(o) <= 2e-2, or, for an output whose
+            correctly rounded bf16 form already misses that bound (rounding
+            costs up to 2^-8 |o_i|, so outputs with max |o| / RMS(o) above ~5
+            can), within 5% of that rounding's own error (tol_bf16_for)
 state:      max |S_gpu - S_oracle| / max |S_oracle| <= 1e-5
 bf16 gradients (backward pass; no tolerance is stated for it, this one is
             derived from the arithmetic): max_i |g_i - o_i| / max(|o_i|, RMS(o))
@@ -42,6 +45,15 @@ def err_bf16(g, o):
     if rms == 0.0:
         return float(np.max(np.abs(g - o))) if o.size else 0.0
     return float(np.max(np.abs(g - o)) / rms)
+
+
+def tol_bf16_for(o):
+    """The bf16 bound for the oracle output o: TOL_BF16, unless rounding o to
+    bf16 (the best any bf16 result can do) already exceeds it; then 5% above
+    that rounding's error."""
+    o = as_np(o)
+    r = torch.from_numpy(o).to(torch.bfloat16)
+    return max(TOL_BF16, 1.05 * err_bf16(r, o))
 
 
 def err_out(g, o, dtype):
