@@ -115,6 +115,7 @@ KERNEL_SOURCES = {
     "reduce": ["k_tc.cu"], "apply": ["k_tc.cu"], "finish": ["k_finish.cu"],
     "reduce_tc_rope": ["k_rope_tc.cu"], "apply_tc_rope": ["k_rope_tc.cu"],
     "reduce_tc_e4m3_rope": ["k_rope_tc.cu"], "apply_tc_e4m3_rope": ["k_rope_tc.cu"],
+    "reduce_tc_nvfp4_rope": ["k_rope_tc.cu"], "apply_tc_nvfp4_rope": ["k_rope_tc.cu"],
     "bwd_q": ["k_bwd_q_tc.cu"], "bwd_k": ["k_bwd_tc.cu"], "dwconv": ["k_conv.cu"],
 }
 SHARED_SOURCES = ["la_internal.cuh", "la_sm100.cuh"]

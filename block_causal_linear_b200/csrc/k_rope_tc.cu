@@ -48,6 +48,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
@@ -89,22 +90,26 @@ __device__ __forceinline__ void warp_arrive(uint64_t *bar) {
 }
 
 // ---------------------------------------------------------------- reduce layout
-// F8 false: bf16 k, v.  A raw stage holds k and v of 32 tokens x 4 heads (two
+// bf16 k, v: a raw stage holds k and v of 32 tokens x 4 heads (two
 // 64-feature boxes each, 16 KiB); the transformed stage R phi(k) hi and lo
 // (bf16, two boxes each); the MMAs read v from the raw stage.
-// F8 true: E4M3 codes.  A raw stage holds one 128-code box of k and one of v
-// (4 KiB each, 128-byte swizzle); the transformed stage R phi(k) hi and lo and
-// the decoded v, all f16 in the bf16 path's box layout (24 KiB), so the raw
-// stage is free once the transform has read it.
-template <bool F8>
+// E4M3 codes: a raw stage holds one 128-code box of k and one of v (4 KiB
+// each, 128-byte swizzle).  NVFP4: the 4 heads' E2M1 codes of k and of v (a
+// 64-byte box row each: 2 KiB), then the 16-byte boxes holding their E4M3
+// block scales (512 bytes each).  For both, the transformed stage holds R
+// phi(k) hi and lo and the decoded v, all f16 in the bf16 path's box layout
+// (24 KiB), so the raw stage is free once the transform has read it.
+template <int IN>
 struct RR {
+    static constexpr bool Q = IN != kInBf16;               // quantised codes
     // The raw ring is as deep as shared memory allows: under load a copy takes
     // ~4 us from issue to arrival, and only the stages in flight move data.
-    static constexpr int kRaw = F8 ? 16 : 10;
-    static constexpr int kRawStage = F8 ? 8192 : 4 * kBox;
-    static constexpr int kVRaw = F8 ? 4096 : 2 * kBox;      // v in a raw stage
+    static constexpr int kRaw = IN == kInE4m3 ? 16 : (IN == kInNvfp4 ? 24 : 10);
+    static constexpr int kRawStage = IN == kInE4m3 ? 8192 : (IN == kInNvfp4 ? 5120 : 4 * kBox);
+    static constexpr int kVRaw = IN == kInE4m3 ? 4096 : (IN == kInNvfp4 ? 2048 : 2 * kBox);   // v in a raw stage
+    static constexpr int kKsRaw = 4096, kVsRaw = 4608;     // NVFP4: the block-scale boxes of k, v
     static constexpr int kOp = 3;                          // transformed stages
-    static constexpr int kOpStage = F8 ? 6 * kBox : 4 * kBox;
+    static constexpr int kOpStage = Q ? 6 * kBox : 4 * kBox;
     static constexpr int kOpOff = kRaw * kRawStage;
     static constexpr int kTabOff = kOpOff + kOp * kOpStage;
     static constexpr int kZOff = kTabOff + kTabBytes;      // z sums [2][4 heads][32] fp32
@@ -129,10 +134,13 @@ constexpr uint32_t kRTmemCols = 256;
 // swizzle), twice as many.
 constexpr int kAOp = 4;                  // transformed tiles in TMEM (hi, lo of 2 heads: 64 columns each)
 constexpr int kABopBytes = 4 * 2048 + 256;              // S rows hi, lo of 2 heads, then Z_eff of 2 heads
-template <bool F8>
+// NVFP4 q tiles: the pair's E2M1 codes (a 32-byte box row: 4 KiB), then the
+// 16-byte box holding its E4M3 block scales (2 KiB).
+template <int IN>
 struct AA {
-    static constexpr int kTile = F8 ? 128 * 64 : 128 * 128;
-    static constexpr int kRaw = F8 ? 22 : 11;                     // raw q stages
+    static constexpr int kTile = IN == kInE4m3 ? 128 * 64 : (IN == kInNvfp4 ? 6144 : 128 * 128);
+    static constexpr int kQsOff = 4096;                          // NVFP4: the scale box in a tile
+    static constexpr int kRaw = IN == kInE4m3 ? 22 : (IN == kInNvfp4 ? 29 : 11);   // raw q stages
     static constexpr int kStgOff = kRaw * kTile;                 // one [32 rows][64 bf16] staging box per epilogue warp
     static constexpr int kBopOff = kStgOff + 4 * kBox;
     static constexpr int kDenOff = kBopOff + 2 * kABopBytes;     // denominator halves [2][2 heads][2][128 rows] fp32
@@ -227,6 +235,40 @@ __device__ __forceinline__ Feat8 relu_decode_e4m3(uint2 c) {
     f.o0 = make_float2(a.y, b.y);
     f.e1 = make_float2(cc.x, d.x);
     f.o1 = make_float2(cc.y, d.y);
+    return f;
+}
+
+// ReLU on 8 packed E2M1 codes (a nibble each): a code with its sign bit (bit
+// 3) set is negative or -0 and becomes +0.
+__device__ __forceinline__ uint32_t relu_e2m1x8(uint32_t w) {
+    const uint32_t neg = (w >> 3) & 0x11111111u;
+    return w & ~(neg * 15u);
+}
+
+// 8 E2M1 codes (element 2i in the low nibble of byte i) times their E4M3
+// block scale as 8 f16 in feature order, exactly: a code value has 2
+// significant bits and a scale 4, so every product (0 or 2^-10 .. 2688) is an
+// f16.
+__device__ __forceinline__ uint4 decode_nvfp4_8(uint32_t c, uint8_t sf) {
+    const __half2 s2 = __half2half2(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)sf, __NV_E4M3)));
+    uint32_t o[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const __nv_fp4x2_storage_t pair = (__nv_fp4x2_storage_t)((c >> (8 * m)) & 0xFFu);
+        const __half2 h = __hmul2(__half2(__nv_cvt_fp4x2_to_halfraw2(pair, __NV_E2M1)), s2);
+        o[m] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// 8 f16 in feature order (4 pairs) as fp32 features.
+__device__ __forceinline__ Feat8 feat_from_f16(uint4 h) {
+    const float2 a = f16x2_f32(h.x), b = f16x2_f32(h.y), c = f16x2_f32(h.z), d = f16x2_f32(h.w);
+    Feat8 f;
+    f.e0 = make_float2(a.x, b.x);
+    f.o0 = make_float2(a.y, b.y);
+    f.e1 = make_float2(c.x, d.x);
+    f.o1 = make_float2(c.y, d.y);
     return f;
 }
 
@@ -373,11 +415,13 @@ struct UnitWalk {
 
 // ================================================================ reduce
 
-template <bool F8>
+template <int IN>
 __global__ void __launch_bounds__(kThreads, 1)
 rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                    float *__restrict__ partials, const Plan p) {
-    using C = RR<F8>;
+    using C = RR<IN>;
+    constexpr bool F8 = IN == kInE4m3, F4 = IN == kInNvfp4, Q = C::Q;
     constexpr int kRRaw = C::kRaw, kROp = C::kOp;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
@@ -411,7 +455,7 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         for (int s = 0; s < kRRaw; ++s) {
             mbar_init(&raw_full[s], 1);
             // bf16: the MMAs free a raw stage (they read v there); E4M3: the transform
-            mbar_init(&raw_empty[s], F8 ? kXfWarps : 1);
+            mbar_init(&raw_empty[s], Q ? kXfWarps : 1);
         }
         for (int o = 0; o < kROp; ++o) {
             mbar_init(&op_full[o], kXfWarps);
@@ -486,6 +530,12 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                     if constexpr (F8) {
                         tma_load_3d(stg, &tm_k, &raw_full[s], c0, row, sg.b);
                         tma_load_3d(stg + C::kVRaw, &tm_v, &raw_full[s], c0, row, sg.b);
+                    } else if constexpr (F4) {
+                        // the group's 64 code bytes; the 16-byte box holding its 8 scale bytes
+                        tma_load_3d(stg, &tm_k, &raw_full[s], sg.g * 64, row, sg.b);
+                        tma_load_3d(stg + C::kVRaw, &tm_v, &raw_full[s], sg.g * 64, row, sg.b);
+                        tma_load_3d(stg + C::kKsRaw, &tm_ks, &raw_full[s], (sg.g >> 1) * 16, row, sg.b);
+                        tma_load_3d(stg + C::kVsRaw, &tm_vs, &raw_full[s], (sg.g >> 1) * 16, row, sg.b);
                     } else {
                         tma_load_3d(stg, &tm_k, &raw_full[s], c0, row, sg.b);
                         tma_load_3d(stg + kBox, &tm_k, &raw_full[s], c0 + 64, row, sg.b);
@@ -498,7 +548,7 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         }
     } else if (warp == kWarpMma) {
         if (lane == 0) {
-            const uint32_t idesc = F8 ? idesc_f16(128, 128, 1, 1) : idesc_bf16(128, 128, 1, 1);
+            const uint32_t idesc = Q ? idesc_f16(128, 128, 1, 1) : idesc_bf16(128, 128, 1, 1);
             UnitWalk w;
             w.start(S, x_begin);
             bool ok = true;
@@ -523,7 +573,7 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                     tc_fence_after();
                     const uint32_t hi = smem_u32(smem + C::kOpOff + o * C::kOpStage);
                     // v: the raw stage (bf16), or the decoded box after lo (E4M3)
-                    const uint32_t va = F8 ? hi + 4 * kBox : smem_u32(smem + s * C::kRawStage + C::kVRaw);
+                    const uint32_t va = Q ? hi + 4 * kBox : smem_u32(smem + s * C::kRawStage + C::kVRaw);
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk) {
                         // MN-major, 128-byte swizzle: the 64-feature boxes are the MN
@@ -536,7 +586,7 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                         mma_bf16(d, dl, dv, idesc, 1u);
                     }
                     mma_commit(&op_empty[o]);
-                    if constexpr (!F8) mma_commit(&raw_empty[s]);   // v is read from the raw stage
+                    if constexpr (!Q) mma_commit(&raw_empty[s]);   // v is read from the raw stage
                 }
                 if (!ok) break;
                 mma_commit(&acc_full[a]);
@@ -569,8 +619,9 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 128 + 32 * q), kv);
             tmem_wait_ld();
             float z = zbuf[a * 128 + q * 32 + lane];
-            if constexpr (F8) {
-                // the sums are over the codes: KV = sk sv sum R phi(k^) v^, z = sk sum phi(k^)
+            if constexpr (Q) {
+                // the sums are over the decoded values without the per-tensor
+                // scales: KV = sk sv sum R phi(k^) v^, z = sk sum phi(k^)
                 // (ReLU commutes with the positive scale, the rotation is linear)
                 const float skv = p.sk * p.sv;
 #pragma unroll
@@ -599,8 +650,10 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         const int r = lane;
         // byte offset of the chunk in a stage: box head / 2, 64-byte half head % 2
         const int chunk = (head >> 1) * kBox + r * 128 + (((4 * (head & 1) + j) ^ (r & 7)) << 4);
-        // E4M3: the same 8 features in the 128-code row of the raw box
+        // E4M3: the same 8 features in the 128-code row of the raw box;
+        // NVFP4: their 4 code bytes in the 64-byte row
         const int chunk8 = r * 128 + (((2 * head + (j >> 1)) ^ (r & 7)) << 4) + ((j & 1) << 3);
+        const int chunk4 = r * 64 + head * 16 + j * 4;
         const GroupRec g0 = group_rec(p, 2 * j), g1 = group_rec(p, 2 * j + 1);
         Feat8 zs;
         zs.e0 = zs.o0 = zs.e1 = zs.o1 = make_float2(0.f, 0.f);
@@ -621,7 +674,29 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 const uint8_t *raw = smem + s * C::kRawStage;
                 uint8_t *op = smem + C::kOpOff + o * C::kOpStage;
                 uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi, vd = hi;   // rows past the segment contribute nothing
-                if constexpr (F8) {
+                if constexpr (F4) {
+                    uint32_t ck = 0u, cv = 0u;
+                    uint8_t sk = 0, sv = 0;
+                    if (ok) {
+                        // the scale byte of this 16-feature block in the group's half of the box row
+                        const int sb = r * 16 + (sg.g & 1) * 8 + head * 2 + (j >> 1);
+                        ck = *reinterpret_cast<const uint32_t *>(raw + chunk4);
+                        cv = *reinterpret_cast<const uint32_t *>(raw + C::kVRaw + chunk4);
+                        sk = raw[C::kKsRaw + sb];
+                        sv = raw[C::kVsRaw + sb];
+                    }
+                    fence_proxy_async_smem();
+                    warp_arrive(&raw_empty[s]);
+                    if (ok && tb < sg.tok1) {
+                        const Feat8 f = feat_from_f16(decode_nvfp4_8(relu_e2m1x8(ck), sk));
+                        rotate_split<true>(f, tab_rec(tab, g0, pq), tab_rec(tab, g1, pq), hi, lo);
+                        zs.e0 = fadd2(zs.e0, f.e0);
+                        zs.o0 = fadd2(zs.o0, f.o0);
+                        zs.e1 = fadd2(zs.e1, f.e1);
+                        zs.o1 = fadd2(zs.o1, f.o1);
+                        vd = decode_nvfp4_8(cv, sv);
+                    }
+                } else if constexpr (F8) {
                     uint2 ck = make_uint2(0u, 0u), cv = ck;
                     if (ok) {
                         ck = *reinterpret_cast<const uint2 *>(raw + chunk8);
@@ -655,7 +730,7 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                     ok = false;
                 *reinterpret_cast<uint4 *>(op + chunk) = hi;
                 *reinterpret_cast<uint4 *>(op + 2 * kBox + chunk) = lo;
-                if constexpr (F8) *reinterpret_cast<uint4 *>(op + 4 * kBox + chunk) = vd;
+                if constexpr (Q) *reinterpret_cast<uint4 *>(op + 4 * kBox + chunk) = vd;
                 // the generic writes of this stage before the tensor cores read it
                 fence_proxy_async_smem();
                 warp_arrive(&op_full[o]);
@@ -696,12 +771,13 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 
 // ================================================================ apply
 
-template <bool F8>
+template <int IN>
 __global__ void __launch_bounds__(kThreads, 1)
-rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_out,
-                  __nv_bfloat16 *__restrict__ out, const uint8_t *__restrict__ bop, const float *__restrict__ seff,
-                  const Plan p) {
-    using C = AA<F8>;
+rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qs,
+                  const __grid_constant__ CUtensorMap tm_out, __nv_bfloat16 *__restrict__ out,
+                  const uint8_t *__restrict__ bop, const float *__restrict__ seff, const Plan p) {
+    using C = AA<IN>;
+    constexpr bool F8 = IN == kInE4m3, F4 = IN == kInNvfp4, Q = IN != kInBf16;
     constexpr int kARaw = C::kRaw, kATile = C::kTile;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
@@ -775,7 +851,13 @@ rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int s = i % kARaw;
                 const int row = w.n * p.L + (int)(x - w.first) * 128;
                 mbar_arrive_expect_tx(&raw_full[s], kATile);
-                tma_load_3d(smem + s * kATile, &tm_q, &raw_full[s], w.u * 64, row, w.b);
+                if constexpr (F4) {
+                    // the pair's 32 code bytes; the 16-byte box holding its 4 scale bytes
+                    tma_load_3d(smem + s * kATile, &tm_q, &raw_full[s], w.u * 32, row, w.b);
+                    tma_load_3d(smem + s * kATile + C::kQsOff, &tm_qs, &raw_full[s], (w.u >> 2) * 16, row, w.b);
+                } else {
+                    tma_load_3d(smem + s * kATile, &tm_q, &raw_full[s], w.u * 64, row, w.b);
+                }
                 issued = i + 1;
             };
             // the packed operand rows of S_eff (hi, lo) and Z_eff of the unit's 2 heads
@@ -915,7 +997,19 @@ rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const bool valid = r < Ln - row0;
             if (ok && !mbar_wait(&raw_full[s], (uint32_t)(i / kARaw) & 1u, abort_word, &g_rope_wait_flag, 17)) ok = false;
             uint4 xq[2];
-            if constexpr (F8) {
+            if constexpr (F4) {
+                // the 16 codes of block jh of head hh (8 bytes of the 32-byte row) and
+                // their scale byte; ReLU on the codes, then f16 values
+                const uint8_t *raw = smem + s * kATile;
+                uint2 c = make_uint2(0u, 0u);
+                uint8_t sf = 0;
+                if (ok && valid) {
+                    c = *reinterpret_cast<const uint2 *>(raw + r * 32 + hh * 16 + jh * 8);
+                    sf = raw[C::kQsOff + r * 16 + (w.u & 3) * 4 + hh * 2 + jh];
+                }
+                xq[0] = decode_nvfp4_8(relu_e2m1x8(c.x), sf);
+                xq[1] = decode_nvfp4_8(relu_e2m1x8(c.y), sf);
+            } else if constexpr (F8) {
                 // 16 codes (features 16 jh ..) of the 64-code row, 64-byte swizzle:
                 // 16-byte chunk c of row r at c ^ ((r / 2) % 4)
                 const uint8_t *raw = smem + s * kATile + r * 64;
@@ -943,7 +1037,10 @@ rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 hi[c] = lo[c] = make_uint4(0u, 0u, 0u, 0u);
                 if (ok && valid) {
                     Feat8 f;
-                    if constexpr (F8) {
+                    if constexpr (F4) {
+                        f = feat_from_f16(xq[c]);   // without the tensor's scale (the epilogue applies it)
+                        rotate_split<false>(f, tab_rec(tab, gr[c][0], pq), tab_rec(tab, gr[c][1], pq), hi[c], lo[c]);
+                    } else if constexpr (F8) {
                         // the codes without the tensor's scale (the epilogue applies it)
                         f = relu_decode_e4m3(make_uint2(xq[c].x, xq[c].y));
                         rotate_split<false>(f, tab_rec(tab, gr[c][0], pq), tab_rec(tab, gr[c][1], pq), hi[c], lo[c]);
@@ -1021,8 +1118,8 @@ rope_apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     tmem_wait_ld();
                     // the sum of the two halves of the denominator, in a fixed order
                     const float den = den_s[a * 512 + (2 * hh) * 128 + r] + den_s[a * 512 + (2 * hh + 1) * 128 + r];
-                    // E4M3: out = sq num^ / (sq den^ + eps), num^ and den^ from the codes
-                    const float iv = F8 ? p.sq / (p.sq * den + p.eps) : 1.0f / (den + p.eps);
+                    // E4M3, NVFP4: out = sq num^ / (sq den^ + eps), num^ and den^ without sq
+                    const float iv = Q ? p.sq / (p.sq * den + p.eps) : 1.0f / (den + p.eps);
                     const float2 inv = make_float2(iv, iv);
                     uint4 y[4];
 #pragma unroll
@@ -1085,10 +1182,12 @@ bool smem_ready() {
     static std::once_flag once;
     static bool ok = false;
     std::call_once(once, [] {
-        ok = set_smem((const void *)rope_reduce_kernel<false>, RR<false>::kSmem) &&
-             set_smem((const void *)rope_apply_kernel<false>, AA<false>::kSmem) &&
-             set_smem((const void *)rope_reduce_kernel<true>, RR<true>::kSmem) &&
-             set_smem((const void *)rope_apply_kernel<true>, AA<true>::kSmem);
+        ok = set_smem((const void *)rope_reduce_kernel<kInBf16>, RR<kInBf16>::kSmem) &&
+             set_smem((const void *)rope_apply_kernel<kInBf16>, AA<kInBf16>::kSmem) &&
+             set_smem((const void *)rope_reduce_kernel<kInE4m3>, RR<kInE4m3>::kSmem) &&
+             set_smem((const void *)rope_apply_kernel<kInE4m3>, AA<kInE4m3>::kSmem) &&
+             set_smem((const void *)rope_reduce_kernel<kInNvfp4>, RR<kInNvfp4>::kSmem) &&
+             set_smem((const void *)rope_apply_kernel<kInNvfp4>, AA<kInNvfp4>::kSmem);
     });
     return ok;
 }
@@ -1161,19 +1260,32 @@ bool tc_rope_fits(const Plan &p) { return p.rope && p.tab_bytes > 0 && p.H % 4 =
 
 int launch_reduce_rope_tc(const void *k, const void *v, float *partials, const Plan &p, cudaStream_t s) {
     if (!smem_ready() || !tc_rope_fits(p) || !p.sk_layout) return -1;
-    CUtensorMap mk, mv;
+    CUtensorMap mk, mv, mks, mvs;
+    const unsigned grid = (unsigned)p.skr.C;
+    const long long row = (long long)p.H * kD;   // features (bf16), codes (E4M3)
+    if (p.f4) {
+        // NVFP4: 64-byte boxes of the group's codes, 16-byte boxes of scales
+        if (p.H % 8 != 0 || !make_u8_map(&mk, k, p.B, p.N, row / 2, 64, 32, 0) ||
+            !make_u8_map(&mv, v, p.B, p.N, row / 2, 64, 32, 0) ||
+            !make_u8_map(&mks, p.sfk, p.B, p.N, row / 16, 16, 32, 0) ||
+            !make_u8_map(&mvs, p.sfv, p.B, p.N, row / 16, 16, 32, 0))
+            return -1;
+        return launch_pdl(rope_reduce_kernel<kInNvfp4>, grid, kThreads, RR<kInNvfp4>::kSmem, s, mk, mv, mks, mvs,
+                          partials, p)
+                   ? 1
+                   : -1;
+    }
     if (p.f8) {
         // E4M3 codes: boxes of the 4 heads' 128 codes x 32 tokens, 128-byte swizzle
-        const long long row = (long long)p.H * kD;
         if (!make_u8_map(&mk, k, p.B, p.N, row, 128, 32, 128) || !make_u8_map(&mv, v, p.B, p.N, row, 128, 32, 128))
             return -1;
-        return launch_pdl(rope_reduce_kernel<true>, (unsigned)p.skr.C, kThreads, RR<true>::kSmem, s, mk, mv, partials,
-                          p)
+        return launch_pdl(rope_reduce_kernel<kInE4m3>, grid, kThreads, RR<kInE4m3>::kSmem, s, mk, mv, mk, mv,
+                          partials, p)
                    ? 1
                    : -1;
     }
     if (!make_bf16_map(&mk, k, p.B, p.N, p.H, 32) || !make_bf16_map(&mv, v, p.B, p.N, p.H, 32)) return -1;
-    return launch_pdl(rope_reduce_kernel<false>, (unsigned)p.skr.C, kThreads, RR<false>::kSmem, s, mk, mv, partials,
+    return launch_pdl(rope_reduce_kernel<kInBf16>, grid, kThreads, RR<kInBf16>::kSmem, s, mk, mv, mk, mv, partials,
                       p)
                ? 1
                : -1;
@@ -1182,19 +1294,32 @@ int launch_reduce_rope_tc(const void *k, const void *v, float *partials, const P
 int launch_apply_rope_tc(const void *q, void *out, const void *bop, const float *seff, const Plan &p,
                          cudaStream_t s) {
     if (!smem_ready() || !tc_rope_fits(p)) return -1;
-    CUtensorMap mq, mo;
+    CUtensorMap mq, mqs, mo;
+    const unsigned grid = (unsigned)p.ska.C;
+    const long long row = (long long)p.H * kD;
     if (!make_bf16_map(&mo, out, p.B, p.N, p.H, 32)) return -1;
+    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
+    const uint8_t *b = static_cast<const uint8_t *>(bop);
+    if (p.f4) {
+        // NVFP4: 32-byte boxes of a head pair's codes x 128 tokens, 16-byte boxes of scales
+        if (p.H % 8 != 0 || !make_u8_map(&mq, q, p.B, p.N, row / 2, 32, 128, 0) ||
+            !make_u8_map(&mqs, p.sfq, p.B, p.N, row / 16, 16, 128, 0))
+            return -1;
+        return launch_pdl(rope_apply_kernel<kInNvfp4>, grid, kThreads, AA<kInNvfp4>::kSmem, s, mq, mqs, mo, o, b,
+                          seff, p)
+                   ? 1
+                   : -1;
+    }
     if (p.f8) {
         // E4M3 codes: boxes of a head pair's 64 codes x 128 tokens, 64-byte swizzle
-        if (!make_u8_map(&mq, q, p.B, p.N, (long long)p.H * kD, 64, 128, 64)) return -1;
-        return launch_pdl(rope_apply_kernel<true>, (unsigned)p.ska.C, kThreads, AA<true>::kSmem, s, mq, mo,
-                          static_cast<__nv_bfloat16 *>(out), static_cast<const uint8_t *>(bop), seff, p)
+        if (!make_u8_map(&mq, q, p.B, p.N, row, 64, 128, 64)) return -1;
+        return launch_pdl(rope_apply_kernel<kInE4m3>, grid, kThreads, AA<kInE4m3>::kSmem, s, mq, mq, mo, o, b, seff,
+                          p)
                    ? 1
                    : -1;
     }
     if (!make_bf16_map(&mq, q, p.B, p.N, p.H, 128)) return -1;
-    return launch_pdl(rope_apply_kernel<false>, (unsigned)p.ska.C, kThreads, AA<false>::kSmem, s, mq, mo,
-                      static_cast<__nv_bfloat16 *>(out), static_cast<const uint8_t *>(bop), seff, p)
+    return launch_pdl(rope_apply_kernel<kInBf16>, grid, kThreads, AA<kInBf16>::kSmem, s, mq, mq, mo, o, b, seff, p)
                ? 1
                : -1;
 }

@@ -120,7 +120,7 @@ la_status common_checks(const void *q, const void *k, const void *v, void *out, 
 // their shared memory; the rest runs on the CUDA cores.
 bool use_tc(la_dtype dt, const la::Plan &p) {
     if (p.f8) return (p.H % 4) == 0 && (!p.rope || la::tc_rope_fits(p)) && la::tc_available();
-    if (p.f4) return (p.H % 8) == 0 && !p.rope && la::tc_available();
+    if (p.f4) return (p.H % 8) == 0 && (!p.rope || la::tc_rope_fits(p)) && la::tc_available();
     return dt == LA_BF16 && (p.H % 4) == 0 && (!p.rope || la::tc_rope_fits(p)) && la::tc_available();
 }
 
@@ -139,7 +139,8 @@ la_status e4m3_checks(const void *q, const void *k, const void *v, void *out, in
 
 // NVFP4 calls: q, k, v E2M1 codes [B][N][H][16] bytes, E4M3 block scales
 // [B][N][H][2] bytes, per-tensor scales; bf16 out; tensor cores only (H a
-// multiple of 8: the scale rows are then whole 16-byte units), no RoPE.
+// multiple of 8: the scale rows are then whole 16-byte units; with RoPE, a
+// grid whose cos/sin table fits the RoPE kernels' shared memory).
 la_status nvfp4_checks(const void *q, const void *k, const void *v, const void *sq_blk, const void *sk_blk,
                        const void *sv_blk, void *out, int B, int N, int H, int d, float eps, float sq, float sk,
                        float sv) {
@@ -178,7 +179,7 @@ la_status run(const void *q, const void *k, const void *v, void *out, la_dtype d
         if (r < 0 || !mark(3, s)) return LA_ECUDA;
         n += r;
         g_last_launches = n;
-        g_last_path = p.f8 ? "tc_e4m3" : "tc";
+        g_last_path = p.f8 ? "tc_e4m3" : (p.f4 ? "tc_nvfp4" : "tc");
         return LA_OK;
     }
     if (tc && fuse_plan(p)) {
@@ -446,11 +447,12 @@ la_status la_block_forward_e4m3(const void *q, const void *k, const void *v, flo
 la_status la_full_forward_nvfp4(const void *q, const void *k, const void *v, const void *q_blk_scale,
                                 const void *k_blk_scale, const void *v_blk_scale, float scale_q, float scale_k,
                                 float scale_v, void *out, int B, int N, int H, int d, int tokens_per_block,
-                                float eps, void *ws, size_t ws_bytes, void *stream) {
+                                const la_rope *rope, float eps, void *ws, size_t ws_bytes, void *stream) {
     la_status e = nvfp4_checks(q, k, v, q_blk_scale, k_blk_scale, v_blk_scale, out, B, N, H, d, eps, scale_q,
                                scale_k, scale_v);
     if (e != LA_OK) return e;
     if (tokens_per_block < 0) return LA_EINVAL;
+    if ((e = check_rope(rope, d, false)) != LA_OK) return e;
     const size_t need = la_workspace_size(B, N, H, d, tokens_per_block);
     if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return LA_EWORKSPACE;
     la::Plan p{};
@@ -462,19 +464,21 @@ la_status la_full_forward_nvfp4(const void *q, const void *k, const void *v, con
     p.sq = scale_q; p.sk = scale_k; p.sv = scale_v;
     p.sfq = q_blk_scale; p.sfk = k_blk_scale; p.sfv = v_blk_scale;
     make_splits(p);
-    fill_rope(p, nullptr, 0);
+    fill_rope(p, rope, rope ? rope->t_offset : 0);
+    if (!use_tc(LA_BF16, p)) return LA_EUNSUPPORTED;   // NVFP4 runs on the tensor cores only
     return run(q, k, v, out, LA_BF16, p, nullptr, nullptr, ws, static_cast<cudaStream_t>(stream));
 }
 
 la_status la_block_forward_nvfp4(const void *q, const void *k, const void *v, const void *q_blk_scale,
                                  const void *k_blk_scale, const void *v_blk_scale, float scale_q, float scale_k,
                                  float scale_v, void *out, int B, int N_blk, int H, int d, la_state *st, int commit,
-                                 float eps, void *ws, size_t ws_bytes, void *stream) {
+                                 const la_rope *rope, float eps, void *ws, size_t ws_bytes, void *stream) {
     la_status e = nvfp4_checks(q, k, v, q_blk_scale, k_blk_scale, v_blk_scale, out, B, N_blk, H, d, eps, scale_q,
                                scale_k, scale_v);
     if (e != LA_OK) return e;
     if (!st || !st->S || !st->Z) return LA_EINVAL;
     if (st->B != B || st->H != H || st->d != d) return LA_EINVAL;
+    if ((e = check_rope(rope, d, true)) != LA_OK) return e;
     const size_t need = la_workspace_size(B, N_blk, H, d, N_blk);
     if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return LA_EWORKSPACE;
     la::Plan p{};
@@ -486,10 +490,14 @@ la_status la_block_forward_nvfp4(const void *q, const void *k, const void *v, co
     p.sq = scale_q; p.sk = scale_k; p.sv = scale_v;
     p.sfq = q_blk_scale; p.sfk = k_blk_scale; p.sfv = v_blk_scale;
     make_splits(p);
-    fill_rope(p, nullptr, 0);
+    fill_rope(p, rope, rope ? (rope->t_offset < 0 ? st->t_next : rope->t_offset) : 0);
+    if (!use_tc(LA_BF16, p)) return LA_EUNSUPPORTED;   // NVFP4 runs on the tensor cores only
     e = run(q, k, v, out, LA_BF16, p, st->S, st->Z, ws, static_cast<cudaStream_t>(stream));
     if (e != LA_OK) return e;
-    if (commit) st->blocks_committed += 1;
+    if (commit) {
+        st->blocks_committed += 1;
+        if (rope) st->t_next += rope->T;
+    }
     return LA_OK;
 }
 

@@ -82,10 +82,11 @@ def lib() -> ctypes.CDLL:
         L.la_block_forward_e4m3.argtypes = [vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ctypes.POINTER(la_state), ip,
                                             ctypes.POINTER(la_rope), fp, vp, sz, vp]
         L.la_block_forward_e4m3.restype = ip
-        L.la_full_forward_nvfp4.argtypes = [vp, vp, vp, vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ip, fp, vp, sz, vp]
+        L.la_full_forward_nvfp4.argtypes = [vp, vp, vp, vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ip,
+                                            ctypes.POINTER(la_rope), fp, vp, sz, vp]
         L.la_full_forward_nvfp4.restype = ip
         L.la_block_forward_nvfp4.argtypes = [vp, vp, vp, vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip,
-                                             ctypes.POINTER(la_state), ip, fp, vp, sz, vp]
+                                             ctypes.POINTER(la_state), ip, ctypes.POINTER(la_rope), fp, vp, sz, vp]
         L.la_block_forward_nvfp4.restype = ip
         L.la_dwconv3d.argtypes = [vp, vp, ip, ip, ip, ip, ip, ip, ip, ip, ip, vp, vp, vp]
         L.la_dwconv3d.restype = ip
@@ -444,16 +445,19 @@ def block_forward_e4m3(q, k, v, scales, state: "State", commit=True, eps=1e-6, w
     return out
 
 
-def la_full_forward_nvfp4(q, k, v, q_sf, k_sf, v_sf, sq, sk, sv, out, B, N, H, d, tokens_per_block, eps, ws, ws_bytes,
-                          stream) -> int:
+def la_full_forward_nvfp4(q, k, v, q_sf, k_sf, v_sf, sq, sk, sv, out, B, N, H, d, tokens_per_block, rope, eps, ws,
+                          ws_bytes, stream) -> int:
     return int(lib().la_full_forward_nvfp4(q, k, v, q_sf, k_sf, v_sf, sq, sk, sv, out, B, N, H, d, tokens_per_block,
-                                           eps, ws, ws_bytes, stream))
+                                           ctypes.byref(rope) if rope is not None else None, eps, ws, ws_bytes,
+                                           stream))
 
 
-def la_block_forward_nvfp4(q, k, v, q_sf, k_sf, v_sf, sq, sk, sv, out, B, N_blk, H, d, st, commit, eps, ws, ws_bytes,
-                           stream) -> int:
+def la_block_forward_nvfp4(q, k, v, q_sf, k_sf, v_sf, sq, sk, sv, out, B, N_blk, H, d, st, commit, rope, eps, ws,
+                           ws_bytes, stream) -> int:
     return int(lib().la_block_forward_nvfp4(q, k, v, q_sf, k_sf, v_sf, sq, sk, sv, out, B, N_blk, H, d,
-                                            ctypes.byref(st), commit, eps, ws, ws_bytes, stream))
+                                            ctypes.byref(st), commit,
+                                            ctypes.byref(rope) if rope is not None else None, eps, ws, ws_bytes,
+                                            stream))
 
 
 def _check_nvfp4(x):
@@ -469,9 +473,10 @@ def _check_nvfp4(x):
 
 
 def full_forward_nvfp4(q, k, v, tokens_per_block=0, eps=1e-6, ws: Optional[torch.Tensor] = None,
-                       out: Optional[torch.Tensor] = None, stream=None):
+                       out: Optional[torch.Tensor] = None, stream=None, rope=None):
     """la_full_forward on NVFP4 inputs: q, k, v each (codes, block scales,
-    per-tensor scale) as synth.to_nvfp4 returns them; out is bf16."""
+    per-tensor scale) as synth.to_nvfp4 returns them, optional 3D RoPE; out
+    is bf16."""
     shapes = {_check_nvfp4(x) for x in (q, k, v)}
     if len(shapes) != 1:
         raise ValueError("q, k, v must agree in shape")
@@ -482,15 +487,15 @@ def full_forward_nvfp4(q, k, v, tokens_per_block=0, eps=1e-6, ws: Optional[torch
         out = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=q[0].device)
     rc = la_full_forward_nvfp4(q[0].data_ptr(), k[0].data_ptr(), v[0].data_ptr(), q[1].data_ptr(), k[1].data_ptr(),
                                v[1].data_ptr(), float(q[2]), float(k[2]), float(v[2]), out.data_ptr(), B, N, H, d,
-                               int(tokens_per_block), float(eps), ws.data_ptr(), ws.numel() * ws.element_size(),
-                               _stream_ptr(stream))
+                               int(tokens_per_block), rope, float(eps), ws.data_ptr(),
+                               ws.numel() * ws.element_size(), _stream_ptr(stream))
     if rc != LA_OK:
         raise LAError(rc, "la_full_forward_nvfp4")
     return out
 
 
 def block_forward_nvfp4(q, k, v, state: "State", commit=True, eps=1e-6, ws: Optional[torch.Tensor] = None,
-                        out: Optional[torch.Tensor] = None, stream=None):
+                        out: Optional[torch.Tensor] = None, stream=None, rope=None):
     shapes = {_check_nvfp4(x) for x in (q, k, v)}
     if len(shapes) != 1:
         raise ValueError("q, k, v must agree in shape")
@@ -501,8 +506,8 @@ def block_forward_nvfp4(q, k, v, state: "State", commit=True, eps=1e-6, ws: Opti
         out = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=q[0].device)
     rc = la_block_forward_nvfp4(q[0].data_ptr(), k[0].data_ptr(), v[0].data_ptr(), q[1].data_ptr(), k[1].data_ptr(),
                                 v[1].data_ptr(), float(q[2]), float(k[2]), float(v[2]), out.data_ptr(), B, N, H, d,
-                                state.c, int(bool(commit)), float(eps), ws.data_ptr(), ws.numel() * ws.element_size(),
-                                _stream_ptr(stream))
+                                state.c, int(bool(commit)), rope, float(eps), ws.data_ptr(),
+                                ws.numel() * ws.element_size(), _stream_ptr(stream))
     if rc != LA_OK:
         raise LAError(rc, "la_block_forward_nvfp4")
     return out

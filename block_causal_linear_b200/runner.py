@@ -49,8 +49,6 @@ class Runner:
         self.fp4 = None
         if nvfp4:
             # NVFP4 inputs: each call's q, k, v as (E2M1 codes, E4M3 block scales, per-tensor scale)
-            if w.rope:
-                raise ValueError("the NVFP4 path takes no RoPE")
             self.fp4 = []
             for i, c in enumerate(self.calls):
                 self.fp4.append([synth.to_nvfp4(t) for t in c[2:5]])
@@ -78,7 +76,7 @@ class Runner:
             _, _, q, k, v = self.calls[0]
             if self.nvfp4:
                 la.full_forward_nvfp4(*self.fp4[0], self.tokens_per_block, eps=w.eps, ws=self.ws,
-                                      out=self.outs[0], stream=stream)
+                                      out=self.outs[0], stream=stream, rope=self.rope)
             elif self.e4m3:
                 la.full_forward_e4m3(q, k, v, self.scales[0], self.tokens_per_block, eps=w.eps, ws=self.ws,
                                      out=self.outs[0], stream=stream, rope=self.rope)
@@ -97,7 +95,7 @@ class Runner:
             for i, (blk, p, q, k, v) in enumerate(self.calls):
                 if self.nvfp4:
                     la.block_forward_nvfp4(*self.fp4[i], st, commit=(p == w.passes - 1), eps=w.eps,
-                                           ws=self.ws, out=self.outs[i], stream=stream)
+                                           ws=self.ws, out=self.outs[i], stream=stream, rope=self.rope)
                 elif self.e4m3:
                     la.block_forward_e4m3(q, k, v, self.scales[i], st, commit=(p == w.passes - 1), eps=w.eps,
                                           ws=self.ws, out=self.outs[i], stream=stream, rope=self.rope)

@@ -287,24 +287,26 @@ LA_API la_status la_block_forward_e4m3(const void *q, const void *k, const void 
  * (scale_q phi(q^) . Z_eff + eps), KV and z carry scale_k scale_v and
  * scale_k), out in bf16, the state fp32 in real units.  q, k, v move 18
  * bytes per token and head each instead of 64.
+ * With rope, the rotation acts on the decoded phi(q^), phi(k^) and rope
+ * follows the bf16 calls' rules, as for the E4M3 calls.
  * Errors: null or not 16-byte aligned pointers, or a scale_x not finite and
- * > 0, LA_EINVAL; H not a multiple of 8 or no tensor-core path,
- * LA_EUNSUPPORTED; no RoPE.  A block scale with the sign bit set or NaN gives
- * unspecified values (no fault).  Workspace and every other argument as in
- * the bf16 calls.
+ * > 0, LA_EINVAL; H not a multiple of 8, no tensor-core path, or a RoPE grid
+ * whose cos/sin records do not fit 8 KiB, LA_EUNSUPPORTED.  A block scale
+ * with the sign bit set or NaN gives unspecified values (no fault).
+ * Workspace and every other argument as in the bf16 calls.
  */
 LA_API la_status la_full_forward_nvfp4(const void *q, const void *k, const void *v,
                                        const void *q_blk_scale, const void *k_blk_scale,
                                        const void *v_blk_scale, float scale_q, float scale_k,
                                        float scale_v, void *out, int B, int N, int H, int d,
-                                       int tokens_per_block, float eps, void *ws, size_t ws_bytes,
-                                       void *stream);
+                                       int tokens_per_block, const la_rope *rope, float eps, void *ws,
+                                       size_t ws_bytes, void *stream);
 LA_API la_status la_block_forward_nvfp4(const void *q, const void *k, const void *v,
                                         const void *q_blk_scale, const void *k_blk_scale,
                                         const void *v_blk_scale, float scale_q, float scale_k,
                                         float scale_v, void *out, int B, int N_blk, int H, int d,
-                                        la_state *st, int commit, float eps, void *ws,
-                                        size_t ws_bytes, void *stream);
+                                        la_state *st, int commit, const la_rope *rope, float eps,
+                                        void *ws, size_t ws_bytes, void *stream);
 
 /*
  * Depthwise 3D convolution of the Spatial-Temporal Mix-FFN, the step after

@@ -173,11 +173,11 @@ def test_e4m3_validation(la):
 def test_nvfp4_validation(la):
     def full(**kw):
         a = dict(q=FAKE, k=FAKE, v=FAKE, qs=FAKE, ks=FAKE, vs=FAKE, sq=0.01, sk=0.01, sv=0.01, out=FAKE, B=1, N=256,
-                 H=8, d=32, tpb=0, eps=1e-6, ws=FAKE, ws_bytes=1 << 30, stream=None)
+                 H=8, d=32, tpb=0, rope=None, eps=1e-6, ws=FAKE, ws_bytes=1 << 30, stream=None)
         a.update(kw)
         return la.la_full_forward_nvfp4(a["q"], a["k"], a["v"], a["qs"], a["ks"], a["vs"], a["sq"], a["sk"], a["sv"],
-                                        a["out"], a["B"], a["N"], a["H"], a["d"], a["tpb"], a["eps"], a["ws"],
-                                        a["ws_bytes"], a["stream"])
+                                        a["out"], a["B"], a["N"], a["H"], a["d"], a["tpb"], a["rope"], a["eps"],
+                                        a["ws"], a["ws_bytes"], a["stream"])
     assert full(k=None) == la.LA_EINVAL
     assert full(vs=None) == la.LA_EINVAL                # a missing block-scale tensor
     assert full(qs=FAKE + 8) == la.LA_EINVAL            # block scales must be 16-byte aligned
@@ -185,9 +185,10 @@ def test_nvfp4_validation(la):
     assert full(sv=float("inf")) == la.LA_EINVAL
     assert full(d=64) == la.LA_EUNSUPPORTED
     assert full(H=4) == la.LA_EUNSUPPORTED              # rows of block scales must be whole 16-byte units
+    assert full(rope=la.make_rope(Hg=3, Wg=5, dims=(8, 12, 10))) in (la.LA_EINVAL, la.LA_EUNSUPPORTED)
     st = la.la_state()
     assert la.la_block_forward_nvfp4(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1.0, 1.0, 1.0, FAKE, 1, 64, 8, 32, st, 1,
-                                     1e-6, FAKE, 1 << 30, None) in (la.LA_EINVAL, la.LA_EUNSUPPORTED)
+                                     None, 1e-6, FAKE, 1 << 30, None) in (la.LA_EINVAL, la.LA_EUNSUPPORTED)
     assert st.blocks_committed == 0
 
 

@@ -8,7 +8,7 @@ import pytest
 import torch
 
 from block_causal_linear_b200 import synth
-from tolerances import TOL_STATE, err_bf16, err_state, TOL_BF16
+from tolerances import TOL_STATE, err_bf16, err_state, tol_bf16_for, TOL_BF16
 
 pytestmark = pytest.mark.gpu
 EPS = 1e-6
@@ -114,3 +114,56 @@ def test_nvfp4_argument_errors(la):
         la.full_forward_nvfp4(*bad, 0, eps=EPS)
     assert e.value.status == la.LA_EINVAL
     la.device_status()
+
+
+def orc_rope(orc, r):
+    return orc.make_rope(Hg=r.Hg, Wg=r.Wg, t_offset=r.t_offset, dims=(r.dt, r.dh, r.dw), base=r.base)
+
+
+# RoPE on the NVFP4 path (the stream-K RoPE kernels decoding codes and block
+# scales): ragged tails, multi-block scans, two batches, 2..8 head groups (H 24:
+# the last group's scales at the end of a 48-byte row)
+@pytest.mark.parametrize("B,N,H,L,grid", [(1, 517, 8, 0, (3, 5)), (2, 300, 8, 128, (3, 5)),
+                                          (1, 1000, 24, 250, (4, 10)), (1, 4099, 64, 0, (7, 9)),
+                                          (2, 2700, 16, 900, (9, 20))])
+def test_full_forward_nvfp4_rope_matches_oracle(la, orc, B, N, H, L, grid):
+    qkv = fp4_inputs(B, N, H, seed=260 + N + H)
+    rope = la.make_rope(Hg=grid[0], Wg=grid[1], t_offset=2)
+    g = la.full_forward_nvfp4(*on_gpu(qkv), L, eps=EPS, rope=rope)
+    torch.cuda.synchronize()
+    la.device_status()
+    assert la.la_last_path() == "tc_nvfp4"
+    ref = orc.full_forward(*decoded(orc, qkv), L, rope=orc_rope(orc, rope), eps=EPS)
+    assert err_bf16(g, ref) <= tol_bf16_for(ref)
+
+
+def test_block_forward_nvfp4_rope_streaming(la, orc):
+    """Streamed blocks with RoPE positions from the state (t_offset < 0), a
+    read-only pass in the middle; outputs and committed state against the
+    oracle, t_next advanced by the committed blocks' frames; repeated calls
+    give the same bits."""
+    B, H, Hg, Wg, F, nb = 2, 8, 3, 50, 3, 3
+    Nb = F * Hg * Wg
+    st = la.State(B, H)
+    ost = orc.State(B, H, 32)
+    rope = la.make_rope(Hg=Hg, Wg=Wg, T=F, t_offset=-1)
+    frames = 0
+    for i in range(nb):
+        qkv = fp4_inputs(B, Nb, H, seed=280 + i, scale=0.7, bias=0.05)
+        commit = i != 1
+        g = la.block_forward_nvfp4(*on_gpu(qkv), st, commit=commit, eps=EPS, rope=rope)
+        ref = orc.block_forward(*decoded(orc, qkv), ost, commit=commit, rope=orc.make_rope(Hg=Hg, Wg=Wg, t_offset=frames),
+                                eps=EPS)
+        torch.cuda.synchronize()
+        la.device_status()
+        assert err_bf16(g, ref) <= tol_bf16_for(ref)
+        assert err_state(st.S, ost.S) <= TOL_STATE and err_state(st.Z, ost.Z) <= TOL_STATE
+        if commit:
+            frames += F
+    assert st.blocks_committed == 2 and st.t_next == 2 * F
+    qkv = on_gpu(fp4_inputs(1, 3000, 8, seed=299))
+    r2 = la.make_rope(Hg=6, Wg=10, t_offset=0)
+    a = la.full_forward_nvfp4(*qkv, 700, eps=EPS, rope=r2).clone()
+    b = la.full_forward_nvfp4(*qkv, 700, eps=EPS, rope=r2)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
