@@ -118,7 +118,7 @@ KERNEL_SOURCES = {
     "reduce_tc_nvfp4_rope": ["k_rope_tc.cu"], "apply_tc_nvfp4_rope": ["k_rope_tc.cu"],
     "bwd_q": ["k_bwd_q_tc.cu"], "bwd_k": ["k_bwd_tc.cu"], "dwconv": ["k_conv.cu"],
 }
-SHARED_SOURCES = ["la_internal.cuh", "la_sm100.cuh"]
+SHARED_SOURCES = ["la_internal.cuh", "la_sm100.cuh", "la_rope.cuh"]
 
 
 def kernel_sources_sha(kernel: str) -> str:

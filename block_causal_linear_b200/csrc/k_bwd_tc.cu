@@ -11,10 +11,19 @@
 // pages give ("Nvidia, MIT ve diğerleri video yapay zeka devrimini başlattı",
 // section "Sabit Bellekli KV önbelleğe alma mekanizması"), for training.
 //
+// With RoPE (R the numerator rotation of each token, sd114.wiki SANA-Video
+// summary, section "两大核心技术突破", item 1):
+//   dv_t = G_m^T R phi(k_t),  dk_t = 1[k_t > 0] (R^T (G_m v_t) + Gz_m).
+// The transform warps rotate phi(k) and split it into a bf16 hi part (in
+// place of the k tile) and a lo part (a second tile), so dv takes three
+// products (hi G_hi, hi G_lo, lo G_hi); the dk epilogue applies R^T to each
+// head's 32 values of G_m v_t before adding Gz and the ReLU mask.
+//
 // Warp roles: 0 TMA (k and v tiles, prefetched before the dependency wait,
-// then the packed operands), 1 TMEM + MMAs, 6..9 ReLU on the k tile in shared
-// memory and its sign bits, 2..5 epilogue (TMEM -> dk, dv, TMA stores).  Every
-// wait is bounded; a wait that gives up raises the device flag.
+// then the packed operands), 1 TMEM + MMAs, 6..9 ReLU (and RoPE) on the k tile
+// in shared memory and its sign bits, 2..5 epilogue (TMEM -> dk, dv, TMA
+// stores).  Every wait is bounded; a wait that gives up raises the device
+// flag.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -22,6 +31,7 @@
 #include <mutex>
 
 #include "la_internal.cuh"
+#include "la_rope.cuh"
 #include "la_sm100.cuh"
 
 namespace la {
@@ -40,29 +50,41 @@ constexpr int kKTTile = 128 * 128;             // [128 rows][64 bf16]: 2 heads o
 constexpr int kKTStages = 2;
 constexpr int kKTStage = 2 * kKTTile;          // k tile, v tile
 constexpr int kKTWarpStg = 32 * 128;           // one epilogue warp's staging box
-constexpr int kKTStgOff = kKTStages * kKTStage;
-constexpr int kKTOpsOff = kKTStgOff + 4 * kKTWarpStg;
 constexpr int kKTOpsBytes = 2 * 4 * kGopBytes;  // 2 heads x (G hi, G lo, G^T hi, G^T lo)
-constexpr int kKTMaskOff = kKTOpsOff + kKTOpsBytes;
 constexpr int kKTMaskBytes = 2 * 128 * 8;       // [acc buffer][row][logical chunk] sign bytes
-constexpr int kKTGzOff = kKTMaskOff + kKTMaskBytes;
-constexpr int kKTBarOff = kKTGzOff + 2 * kD * 4;
 constexpr int kKTNumBars = 3 * kKTStages + 2 + 2 + 2 + 3;   // ring, acc_full, acc_empty, mask_ready, ops, dep, drain
-constexpr int kKTSmem = kKTBarOff + kKTNumBars * 8 + 16 + 1024;
+constexpr int kKTTabBytes = 8192;              // RoPE: the call's cos/sin table
+// Shared memory; with RoPE the lo parts of the rotated k tiles and the table
+// are added (one CTA per SM then, two without).
+template <bool ROPE>
+struct KT {
+    static constexpr int kLoOff = kKTStages * kKTStage;
+    static constexpr int kStgOff = kLoOff + (ROPE ? kKTStages * kKTTile : 0);
+    static constexpr int kOpsOff = kStgOff + 4 * kKTWarpStg;
+    static constexpr int kMaskOff = kOpsOff + kKTOpsBytes;
+    static constexpr int kGzOff = kMaskOff + kKTMaskBytes;
+    static constexpr int kTabOff = kGzOff + 2 * kD * 4;
+    static constexpr int kBarOff = kTabOff + (ROPE ? kKTTabBytes : 0);
+    static constexpr int kSmem = kBarOff + kKTNumBars * 8 + 16 + 1024;
+    static_assert(kSmem <= (ROPE ? 232448 : 232448 / 2), "key-side shared memory");
+};
 constexpr uint32_t kKTTmemCols = 256;           // 2 buffers x [dv h0 | dv h1 | dpk h0 | dpk h1]
 
-__global__ void __launch_bounds__(kKTThreads, 2)
+template <bool ROPE>
+__global__ void __launch_bounds__(kKTThreads, ROPE ? 1 : 2)
 bwd_k_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                 __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv, const float *__restrict__ G,
                 const uint8_t *__restrict__ gop, const Plan p) {
+    using C = KT<ROPE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
-    uint8_t *stg = smem + kKTStgOff;
-    uint8_t *ops = smem + kKTOpsOff;
-    uint8_t *mask8 = smem + kKTMaskOff;
-    float *gz = reinterpret_cast<float *>(smem + kKTGzOff);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kKTBarOff);
+    uint8_t *stg = smem + C::kStgOff;
+    uint8_t *ops = smem + C::kOpsOff;
+    uint8_t *mask8 = smem + C::kMaskOff;
+    uint8_t *tab = smem + C::kTabOff;
+    float *gz = reinterpret_cast<float *>(smem + C::kGzOff);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
     uint64_t *xform_done = full + kKTStages;
     uint64_t *empty = xform_done + kKTStages;
     uint64_t *acc_full = empty + kKTStages;     // [2]
@@ -116,6 +138,7 @@ bwd_k_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         prefetch_tmap(&tm_dk);
         prefetch_tmap(&tm_dv);
     }
+    if constexpr (ROPE) build_table(tab, p, threadIdx.x, kKTThreads);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -166,14 +189,20 @@ bwd_k_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     if (!mbar_wait(&acc_empty[ab], aph ^ 1u, abort_word, &g_wait_flag, 54)) break;
                     tc_fence_after();
                     const uint32_t kaddr = smem_u32(smem + s * kKTStage), vaddr = kaddr + kKTTile;
+                    const uint32_t loaddr = smem_u32(smem + C::kLoOff + s * kKTTile);   // RoPE: R phi(K) lo
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
                         for (int which = 0; which < 2; ++which) {   // 0: dv from phi(K) and G; 1: dpk from V and G^T
                             const uint32_t d = tmem + ab * 128 + which * 64 + hh * kD;
-                            const uint32_t abase = (which ? vaddr : kaddr) + hh * 64;
+                            // products (A part, B part): (hi, hi), (hi, lo), and with RoPE for dv
+                            // (lo, hi): A = R phi(K) is then a hi and a lo tile
+                            const int nprod = (ROPE && which == 0) ? 3 : 2;
 #pragma unroll
-                            for (int part = 0; part < 2; ++part) {
+                            for (int prod = 0; prod < 3; ++prod) {
+                                if (prod >= nprod) break;
+                                const int apart = prod == 2 ? 1 : 0, part = prod == 1 ? 1 : 0;
+                                const uint32_t abase = (which ? vaddr : (apart ? loaddr : kaddr)) + hh * 64;
 #pragma unroll
                                 for (int kk = 0; kk < 2; ++kk) {
                                     // A: K-major, 128-byte swizzle, head hh = 64-byte half of a row;
@@ -181,7 +210,7 @@ bwd_k_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                                     const uint64_t da = smem_desc(abase + kk * 32, 16, 1024, kLayoutSw128);
                                     const uint64_t db = smem_desc(oaddr + (hh * 4 + which * 2 + part) * kGopBytes + kk * 256,
                                                                   128, 512, kLayoutNone);
-                                    mma_bf16(d, da, db, idesc, (part | kk) ? 1u : 0u);
+                                    mma_bf16(d, da, db, idesc, (prod | kk) ? 1u : 0u);
                                 }
                             }
                         }
@@ -194,6 +223,10 @@ bwd_k_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     } else if (warp >= 6) {
         // ------------------------------------------------ ReLU on the k tile, sign bytes
         const int tt = threadIdx.x - kKTXform0;
+        // RoPE: this thread's chunks are all logical chunk L (the same 8 features of
+        // one head) of rows tt / 8 + 16 j, so two table groups serve all of them
+        const int Lc = (tt & 7) ^ ((tt >> 3) & 7);
+        const GroupRec gr0 = group_rec(p, 2 * (Lc & 3)), gr1 = group_rec(p, 2 * (Lc & 3) + 1);
         bool ok = true;
         for (int i = 0; i < ntiles; ++i) {
             const int s = i % kKTStages;
@@ -204,6 +237,9 @@ bwd_k_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             // the sign bytes of buffer ab are free once the epilogue of tile i-2 read them
             if (ok && !mbar_wait(&acc_empty[ab], aph ^ 1u, abort_word, &g_wait_flag, 56)) ok = false;
             uint8_t *kt = smem + s * kKTStage;
+            uint8_t *lot = smem + C::kLoOff + s * kKTTile;
+            Pos pq{};
+            if constexpr (ROPE) pq = token_pos(p, (int)(ta0 + 128LL * i + (tt >> 3)));
             if (ok) {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
@@ -220,7 +256,20 @@ bwd_k_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         bits |= (((w[m] & 0x80000000u) == 0u && (w[m] & 0x7FFF0000u) != 0u) ? 1u : 0u) << (2 * m + 1);
                     }
                     mask8[ab * 1024 + row * 8 + L] = (uint8_t)bits;
-                    *ptr = make_uint4(relu2(x.x), relu2(x.y), relu2(x.z), relu2(x.w));
+                    if constexpr (ROPE) {
+                        // rows past the tensor (TMA's zero fill) get zero hi and lo, and
+                        // no table lookup at a position past the call's frames
+                        uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
+                        if (ta0 + 128LL * i + row < p.N) {
+                            Feat8 f;
+                            rope_chunk(x, tab_rec(tab, gr0, pq), tab_rec(tab, gr1, pq), hi, lo, f);
+                        }
+                        *ptr = hi;
+                        *reinterpret_cast<uint4 *>(lot + (size_t)u * 16) = lo;
+                        pos_step(p, pq, 16);
+                    } else {
+                        *ptr = make_uint4(relu2(x.x), relu2(x.y), relu2(x.z), relu2(x.w));
+                    }
                 }
             }
             fence_proxy_async_smem();
@@ -252,6 +301,10 @@ bwd_k_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const uint32_t m0 = mk.x, m1 = mk.y;
             const long long row0 = ta0 + 128LL * i;
             const long long wrow0 = row0 + 32 * qd;
+            // RoPE: this row's position (rows past the tensor take the last token's;
+            // their results are not stored)
+            Pos pr{};
+            if constexpr (ROPE) pr = token_pos(p, (int)(row0 + r < p.N ? row0 + r : p.N - 1));
             const bool boxed = wrow0 + 32 <= ta1 || ta1 == p.N;
             const uint32_t base = tmem + lane_off + ab * 128;
             for (int which = 0; which < 2; ++which) {   // 0: dk (TMEM columns 64..127), 1: dv (0..63)
@@ -267,6 +320,19 @@ bwd_k_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         tmem_wait_ld();
                         if (!which) {
                             const uint32_t m = hh ? m1 : m0;
+                            if constexpr (ROPE) {
+                                // d phi(k) = R^T d psi(k): pair (x0, x1) by its (cos, sin) to
+                                // (x0 cos + x1 sin, x1 cos - x0 sin); group g holds features 4g .. 4g + 3
+#pragma unroll
+                                for (int g = 0; g < 8; ++g) {
+                                    const float4 t = tab_rec(tab, group_rec(p, g), pr);
+                                    const float a0 = h[4 * g], a1 = h[4 * g + 1], b0 = h[4 * g + 2], b1 = h[4 * g + 3];
+                                    h[4 * g] = fmaf(a1, t.z, a0 * t.x);
+                                    h[4 * g + 1] = fmaf(-a0, t.z, a1 * t.x);
+                                    h[4 * g + 2] = fmaf(b1, t.w, b0 * t.y);
+                                    h[4 * g + 3] = fmaf(-b0, t.w, b1 * t.y);
+                                }
+                            }
 #pragma unroll
                             for (int a = 0; a < 32; ++a) h[a] = (m >> a) & 1u ? h[a] + gz[hh * kD + a] : 0.f;
                         }
@@ -329,25 +395,33 @@ bwd_k_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
 }  // namespace
 
-bool bwd_k_tc_available(const Plan &p) { return tc_available() && p.H % 4 == 0 && !p.rope && !p.f8; }
+bool bwd_k_tc_available(const Plan &p) {
+    return tc_available() && p.H % 4 == 0 && !p.f8 && (!p.rope || (p.tab_bytes > 0 && p.tab_bytes <= kKTTabBytes));
+}
 
 int launch_bwd_k_tc(const void *k, const void *v, const float *G, const void *gop, void *dk, void *dv,
                     const Plan &p, cudaStream_t s) {
     static std::once_flag once;
     static bool attr_ok = false;
-    std::call_once(once, [] { attr_ok = set_smem((const void *)bwd_k_tc_kernel, kKTSmem); });
+    std::call_once(once, [] {
+        attr_ok = set_smem((const void *)bwd_k_tc_kernel<false>, KT<false>::kSmem) &&
+                  set_smem((const void *)bwd_k_tc_kernel<true>, KT<true>::kSmem);
+    });
     if (!attr_ok) return -1;
+    if (p.rope && !bwd_k_tc_available(p)) return -1;
     CUtensorMap mk, mv, mdk, mdv;
     if (!make_bf16_map(&mk, k, p.B, p.N, p.H, 128) || !make_bf16_map(&mv, v, p.B, p.N, p.H, 128) ||
         !make_bf16_map(&mdk, dk, p.B, p.N, p.H, 32) || !make_bf16_map(&mdv, dv, p.B, p.N, p.H, 32))
         return -1;
     const long long grid = (long long)p.B * p.nb * p.Pa * (p.H / 2);
     if (grid <= 0 || grid > 0x7fffffffLL) return -1;
-    return launch_pdl(bwd_k_tc_kernel, (unsigned)grid, kKTThreads, kKTSmem, s, mk, mv, mdk, mdv,
-                      static_cast<__nv_bfloat16 *>(dk), static_cast<__nv_bfloat16 *>(dv), G,
-                      static_cast<const uint8_t *>(gop), p)
-               ? 1
-               : -1;
+    __nv_bfloat16 *dk16 = static_cast<__nv_bfloat16 *>(dk), *dv16 = static_cast<__nv_bfloat16 *>(dv);
+    const uint8_t *g8 = static_cast<const uint8_t *>(gop);
+    const bool ok = p.rope ? launch_pdl(bwd_k_tc_kernel<true>, (unsigned)grid, kKTThreads, KT<true>::kSmem, s, mk, mv,
+                                        mdk, mdv, dk16, dv16, G, g8, p)
+                           : launch_pdl(bwd_k_tc_kernel<false>, (unsigned)grid, kKTThreads, KT<false>::kSmem, s, mk,
+                                        mv, mdk, mdv, dk16, dv16, G, g8, p);
+    return ok ? 1 : -1;
 }
 
 int read_and_clear_bwd_k_flag(unsigned *flag_out) {

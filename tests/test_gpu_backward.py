@@ -46,6 +46,9 @@ CASES = [  # dtype, B, N, H, tokens_per_block, rope
     (torch.bfloat16, 2, 250, 6, 100, False),      # CUDA-core path (H % 4 != 0)
     (torch.bfloat16, 1, 240, 4, 60, True),
     (torch.float32, 1, 180, 2, 45, True),
+    (torch.bfloat16, 1, 1000, 8, 250, True),     # RoPE: key side on the tensor cores, ragged tiles
+    (torch.bfloat16, 2, 777, 4, 300, True),      # RoPE: two batches, a short last block
+    (torch.bfloat16, 1, 2100, 16, 0, True),      # RoPE: one block, many tiles per split
 ]
 
 
@@ -58,6 +61,8 @@ def test_backward_matches_oracle(la, orc, case):
     got = la.full_backward(q.cuda(), k.cuda(), v.cuda(), dout.cuda(), L, rope=rope, eps=EPS)
     torch.cuda.synchronize()
     la.device_status()
+    if use_rope and dtype == torch.bfloat16 and H % 4 == 0:
+        assert la.la_last_path() == "bwd(tc state, tc keys)"   # key side on the tensor cores
     want = orc.full_backward(q, k, v, dout, L, rope=orope, eps=EPS)
     for name, g, w in zip(("dq", "dk", "dv"), got, want):
         e = err_grad(g, w, dtype)
@@ -92,6 +97,29 @@ def test_backward_fullsize_sampled_heads(la, orc):
     idx = torch.tensor(heads, device="cuda")
     sub = [t.index_select(2, idx).contiguous().cpu() for t in (q, k, v, dout)]
     want = orc.full_backward(*sub, w.n_blk, eps=EPS)
+    for name, g, wt in zip(("dq", "dk", "dv"), got, want):
+        e = err_grad(g.index_select(2, idx).cpu(), wt, torch.bfloat16)
+        assert e <= tol_grad(torch.bfloat16), (name, e)
+
+
+def test_backward_rope_deterministic_and_fullsize_sampled(la, orc):
+    """RoPE backward on two 720p B4 blocks (2 x 10,800 tokens, 3 x 45 x 80
+    latent frames each, 64 heads): repeated calls give the same bits, and a
+    sample of heads matches the oracle (heads are independent)."""
+    w = synth.WORKLOADS[5]
+    B, N = 1, 2 * w.n_blk
+    q, k, v, dout = (t.cuda() for t in inputs(B, N, 64, torch.bfloat16, seed=13))
+    rope = la.make_rope(Hg=w.Hg, Wg=w.Wg, t_offset=0)
+    got = [t.clone() for t in la.full_backward(q, k, v, dout, w.n_blk, rope=rope, eps=EPS)]
+    again = la.full_backward(q, k, v, dout, w.n_blk, rope=rope, eps=EPS)
+    torch.cuda.synchronize()
+    la.device_status()
+    for x, y in zip(got, again):
+        assert torch.equal(x.view(torch.int16), y.view(torch.int16))
+    heads = [0, 29, 63]
+    idx = torch.tensor(heads, device="cuda")
+    sub = [t.index_select(2, idx).contiguous().cpu() for t in (q, k, v, dout)]
+    want = orc.full_backward(*sub, w.n_blk, rope=orc.make_rope(Hg=w.Hg, Wg=w.Wg, t_offset=0), eps=EPS)
     for name, g, wt in zip(("dq", "dk", "dv"), got, want):
         e = err_grad(g.index_select(2, idx).cpu(), wt, torch.bfloat16)
         assert e <= tol_grad(torch.bfloat16), (name, e)
