@@ -19,20 +19,10 @@
 #include <cuda_runtime.h>
 
 #include "la_internal.cuh"
+#include "la_rope.cuh"
 
 namespace la {
 namespace {
-
-// Angle of feature pair pr of token j of the call (numerator RoPE).
-__device__ __forceinline__ float pair_angle(const Plan &p, long long j, int pr) {
-    const long long per_frame = (long long)p.Hg * p.Wg;
-    const int ax = p.axis[pr];
-    long long pos;
-    if (ax == 0) pos = p.t_offset + j / per_frame;
-    else if (ax == 1) pos = (j % per_frame) / p.Wg;
-    else pos = (j % per_frame) % p.Wg;
-    return (float)pos * p.theta[pr];
-}
 
 constexpr int kBThreads = 256;   // bwd_finish_kernel
 
@@ -73,10 +63,33 @@ __device__ __forceinline__ void store_row(__nv_bfloat16 *p, const float (&x)[kD]
                                                      bf2(x[8 * i + 4], x[8 * i + 5]), bf2(x[8 * i + 6], x[8 * i + 7]));
 }
 
-// cos, sin of the 16 feature pairs of token t (numerator RoPE).
+// cos, sin of the 16 feature pairs of token t of the call (numerator RoPE):
+// the token's frame t_offset + t / (Hg Wg), row and column once (32-bit
+// division by multiply-shift), then each pair's angle pos * theta along the
+// pair's axis.
 __device__ __forceinline__ void token_cs(const Plan &p, long long t, float (&c)[kD / 2], float (&s)[kD / 2]) {
+    const Pos q = token_pos(p, (int)t);
+    const int f = p.t_offset + q.f;
 #pragma unroll
-    for (int pr = 0; pr < kD / 2; ++pr) sincosf(pair_angle(p, t, pr), &s[pr], &c[pr]);
+    for (int pr = 0; pr < kD / 2; ++pr) {
+        const int ax = p.axis[pr];
+        const int pos = ax == 0 ? f : (ax == 1 ? q.h : q.w);
+        sincosf((float)pos * p.theta[pr], &s[pr], &c[pr]);
+    }
+}
+// The same values read from the call's cos/sin table (built with the same
+// sincosf of the same products): 8 records, one per group of 4 features.
+__device__ __forceinline__ void token_cs_tab(const Plan &p, const uint8_t *tab, long long t, float (&c)[kD / 2],
+                                             float (&s)[kD / 2]) {
+    const Pos q = token_pos(p, (int)t);
+#pragma unroll
+    for (int m = 0; m < kD / 4; ++m) {
+        const float4 r = tab_rec(tab, group_rec(p, m), q);
+        c[2 * m] = r.x;
+        c[2 * m + 1] = r.y;
+        s[2 * m] = r.z;
+        s[2 * m + 1] = r.w;
+    }
 }
 // x <- R x (sgn = +1) or R^T x (sgn = -1), pair by pair.
 __device__ __forceinline__ void rotate_row(float (&x)[kD], const float (&c)[kD / 2], const float (&s)[kD / 2],
@@ -92,7 +105,8 @@ __device__ __forceinline__ void rotate_row(float (&x)[kD], const float (&c)[kD /
 constexpr int kQThreads = 128;
 constexpr int kQRows = 128;              // token rows per round: one per thread
 constexpr int kQStride = kD + 4;         // 36 floats: rows 16-byte aligned, 4 banks apart
-constexpr int kQSmem = (kKVZ + 3 * kQRows * kQStride + kQRows) * 4;
+constexpr int kQTab = 8192;              // the call's cos/sin table, when it fits
+constexpr int kQSmem = (kKVZ + 3 * kQRows * kQStride + kQRows) * 4 + kQTab;
 
 // One CTA per (b, h, block n, split sp): dq of the split's tokens and the
 // split's [dS | dZ] sums.  seff: [B][H][nb][1056] inclusive prefix state.
@@ -124,6 +138,9 @@ bwd_q_kernel(const T *__restrict__ q, const T *__restrict__ dout, const float *_
     const size_t bh = (size_t)b * p.H + h;
     const float *src = seff + (bh * p.nb + n) * kKVZ;
     for (int e = tid; e < kKVZ; e += kQThreads) Ss[e] = src[e];
+    uint8_t *tab = reinterpret_cast<uint8_t *>(cc + kQRows);
+    const bool use_tab = p.rope && p.tab_bytes > 0 && p.tab_bytes <= kQTab;
+    if (use_tab) build_table(tab, p, tid, kQThreads);
 
     const int gi = tid >> 6, j = tid & 63;            // accumulation: row half, 4 x 4 block
     const int a0 = 4 * (j >> 3), c0 = 4 * (j & 7);
@@ -152,7 +169,8 @@ bwd_q_kernel(const T *__restrict__ q, const T *__restrict__ dout, const float *_
         }
         float cs_c[kD / 2], cs_s[kD / 2];
         if (p.rope && valid) {
-            token_cs(p, t, cs_c, cs_s);
+            if (use_tab) token_cs_tab(p, tab, t, cs_c, cs_s);
+            else token_cs(p, t, cs_c, cs_s);
             rotate_row(ps, cs_c, cs_s, 1.f);
         }
 #pragma unroll
