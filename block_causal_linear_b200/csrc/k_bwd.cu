@@ -115,7 +115,7 @@ constexpr int kQSmem = (kKVZ + 3 * kQRows * kQStride + kQRows) * 4 + kQTab;
 // a 4 x 4 block of dS for half of the rows (the two halves are added in a
 // fixed order at the end).
 template <typename T>
-__global__ void __launch_bounds__(kQThreads)
+__global__ void __launch_bounds__(kQThreads, 3)   // at most 168 registers: 3 CTAs per SM (4: slower, spills)
 bwd_q_kernel(const T *__restrict__ q, const T *__restrict__ dout, const float *__restrict__ seff,
              T *__restrict__ dq, float *__restrict__ bpart, Plan p) {
     extern __shared__ __align__(16) float qsm[];
