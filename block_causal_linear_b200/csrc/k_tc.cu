@@ -8,23 +8,18 @@
 //   heads (M = 4 x 32 key features, stored MN-major as TMA lands it), B = V of
 //   the same 4 heads (N = 4 x 32 value features).  Only the 4 diagonal 32x32
 //   blocks of D are used.  fp32 accumulation in TMEM across the whole split.
-//   Without RoPE, z comes from a second MMA against a 16-column matrix of
-//   ones.  With RoPE (sd114.wiki, "两大核心技术突破" item 1), the rotated
-//   features R phi(k) go to the MMA as a hi and a lo bf16 part (R phi(k) =
-//   hi + lo to ~16 bits), and z = sum phi(k) is summed on the CUDA cores while
-//   phi is applied.
-// apply: out_t = psi(q_t) S_eff / (phi(q_t) . Z_eff + eps) for 128-token tiles
-//   of 2 heads.  Without RoPE: per head one M=128 x N=48 x K=32 contraction of
-//   phi(Q) against the packed [S | Z | 0] operand, as a hi and a lo bf16 part
-//   accumulated in the same TMEM columns.  With RoPE: the numerator is
-//   (R phi(q))_hi.S_hi + (R phi(q))_hi.S_lo + (R phi(q))_lo.S_hi (N = 32) and the
-//   unrotated denominator phi(q).Z_eff is summed in fp32 on the CUDA cores.
-//   The epilogue divides, rounds to bf16 and stores with TMA.
+//   z comes from a second MMA against a 16-column matrix of ones.
+// apply: out_t = phi(q_t) S_eff / (phi(q_t) . Z_eff + eps) for 128-token tiles
+//   of 2 heads: per head one M=128 x N=48 x K=32 contraction of phi(Q) against
+//   the packed [S | Z | 0] operand, as a hi and a lo bf16 part accumulated in
+//   the same TMEM columns.  The epilogue divides, rounds to bf16 and stores
+//   with TMA.
+// Calls with RoPE run the kernels of k_rope_tc.cu instead.
 //
 // Warp roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs.  In the
-// reduce, warps 2..5 apply phi = ReLU (and RoPE) in shared memory and run the
-// epilogue; in the apply, warps 6..9 transform the q tiles while warps 2..5 run
-// the epilogue of the previous tile.  Every wait is bounded (la_sm100.cuh); a
+// reduce, warps 2..5 apply phi = ReLU in shared memory and run the epilogue; in
+// the apply, warps 6..9 transform the q tiles while warps 2..5 run the epilogue
+// of the previous tile.  Every wait is bounded (la_sm100.cuh); a
 // wait that gives up raises the device flag read by la_device_status and the
 // CTA drains and returns.
 #include <cuda.h>
@@ -135,7 +130,8 @@ struct RCfg {
 };
 
 // Fused state combine: the split sums of the CTA's 4 heads ([4][kKVZ] fp32)
-// in shared memory, past the z scratch of the RoPE epilogue.
+// in shared memory, inside the stage ring (no copy or MMA touches the ring
+// once the split's last MMA has completed).
 constexpr int kFusePartOff = 16384;
 constexpr int kZeroRowsOp = kOpRows - kD - 1;   // zero rows 33..47 of the packed operand
 

@@ -219,8 +219,8 @@ int read_and_clear_rope_flag(unsigned *flag_out);
 int launch_bwd_q(int is_bf16, const void *q, const void *dout, const float *seff, void *dq, float *bpart,
                  const Plan &p, cudaStream_t s);
 int launch_bwd_finish(const float *bpart, float *G, void *gop, const Plan &p, cudaStream_t s);
-// Key side on the tensor cores (bf16, H % 4 == 0, no RoPE): dk, dv from k, v
-// and the packed G operands; Gz from G.
+// Key side on the tensor cores (bf16, H % 4 == 0; with RoPE when the call's
+// cos/sin table fits): dk, dv from k, v and the packed G operands; Gz from G.
 bool bwd_k_tc_available(const Plan &p);
 int launch_bwd_k_tc(const void *k, const void *v, const float *G, const void *gop, void *dk, void *dv,
                     const Plan &p, cudaStream_t s);
