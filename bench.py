@@ -117,6 +117,7 @@ KERNEL_SOURCES = {
     "reduce_tc_e4m3_rope": ["k_rope_tc.cu"], "apply_tc_e4m3_rope": ["k_rope_tc.cu"],
     "reduce_tc_nvfp4_rope": ["k_rope_tc.cu"], "apply_tc_nvfp4_rope": ["k_rope_tc.cu"],
     "bwd_q": ["k_bwd_q_tc.cu"], "bwd_k": ["k_bwd_tc.cu"], "dwconv": ["k_conv.cu"],
+    "bwd_q_rope": ["k_bwd.cu"], "bwd_k_rope": ["k_bwd_tc.cu"],
 }
 SHARED_SOURCES = ["la_internal.cuh", "la_sm100.cuh", "la_rope.cuh"]
 
@@ -802,7 +803,7 @@ def main():
         # (reads k, v, writes dk, dv); the dominant one of the two sides
         side = [("bwd_q", fin_ms, 3), ("bwd_k", app_ms, 4)]
         dom, dom_ms, ntens = max(side, key=lambda x: x[1])
-        kname = dom
+        kname = dom + ("_rope" if w.rope else "")   # with RoPE: the CUDA-core query side, the RoPE key side
     else:
         # dominant kernel: the larger of reduce (reads k, v) and apply (reads q, writes out)
         dom, dom_ms = ("reduce", red_ms) if red_ms >= app_ms else ("apply", app_ms)
