@@ -217,3 +217,28 @@ def test_one_workspace_serves_calls_of_different_shapes(la, orc):
         la.device_status()
         ref = orc.full_forward(q, k, v, L, eps=EPS)
         assert err_out(g, ref, torch.bfloat16) <= tol_out(torch.bfloat16)
+
+
+def test_rope_grid_beyond_the_table(la, orc):
+    """A RoPE grid whose cos/sin records do not fit the tensor-core kernels'
+    8 KiB table (3 x 200 per frame: 200 column positions x 48 bytes alone)
+    takes the CUDA-core kernels, which compute the angles per element, and
+    matches the oracle; the E4M3 and NVFP4 calls, which have no CUDA-core
+    path, refuse it with LA_EUNSUPPORTED before enqueueing anything."""
+    B, N, H = 1, 1200, 8
+    q, k, v = synth.random_qkv(B, N, H, 32, seed=77)
+    rope = la.make_rope(Hg=3, Wg=200, t_offset=1)
+    g = la.full_forward(q.cuda(), k.cuda(), v.cuda(), 0, rope=rope, eps=EPS)
+    torch.cuda.synchronize()
+    la.device_status()
+    assert la.la_last_path() == "ffma"
+    ref = orc.full_forward(q, k, v, 0, rope=orc_rope(orc, rope), eps=EPS)
+    assert err_out(g, ref, torch.bfloat16) <= tol_out(torch.bfloat16)
+    codes = [synth.to_e4m3(t) for t in (q, k, v)]
+    with pytest.raises(la.LAError) as e:
+        la.full_forward_e4m3(*[c.cuda() for c, _ in codes], [s_ for _, s_ in codes], 0, eps=EPS, rope=rope)
+    assert e.value.status == la.LA_EUNSUPPORTED
+    fp4 = [synth.to_nvfp4(t) for t in (q, k, v)]
+    with pytest.raises(la.LAError) as e:
+        la.full_forward_nvfp4(*[(c.cuda(), sf.cuda(), s_) for c, sf, s_ in fp4], 0, eps=EPS, rope=rope)
+    assert e.value.status == la.LA_EUNSUPPORTED
