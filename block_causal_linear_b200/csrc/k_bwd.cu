@@ -47,6 +47,26 @@ __device__ __forceinline__ void load_row(const __nv_bfloat16 *p, float (&x)[kD])
         }
     }
 }
+// Half a token row (16 features) between global memory and registers.
+__device__ __forceinline__ void load_half(const float *p, float (&x)[kD / 2]) {
+#pragma unroll
+    for (int i = 0; i < kD / 8; ++i) {
+        const float4 v = reinterpret_cast<const float4 *>(p)[i];
+        x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
+    }
+}
+__device__ __forceinline__ void load_half(const __nv_bfloat16 *p, float (&x)[kD / 2]) {
+#pragma unroll
+    for (int i = 0; i < kD / 16; ++i) {
+        const uint4 v = reinterpret_cast<const uint4 *>(p)[i];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            x[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+            x[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+    }
+}
 __device__ __forceinline__ void store_row(float *p, const float (&x)[kD]) {
 #pragma unroll
     for (int i = 0; i < kD / 4; ++i)
@@ -59,6 +79,17 @@ __device__ __forceinline__ uint32_t bf2(float a, float b) {
 __device__ __forceinline__ void store_row(__nv_bfloat16 *p, const float (&x)[kD]) {
 #pragma unroll
     for (int i = 0; i < kD / 8; ++i)
+        reinterpret_cast<uint4 *>(p)[i] = make_uint4(bf2(x[8 * i], x[8 * i + 1]), bf2(x[8 * i + 2], x[8 * i + 3]),
+                                                     bf2(x[8 * i + 4], x[8 * i + 5]), bf2(x[8 * i + 6], x[8 * i + 7]));
+}
+__device__ __forceinline__ void store_half(float *p, const float (&x)[kD / 2]) {
+#pragma unroll
+    for (int i = 0; i < kD / 8; ++i)
+        reinterpret_cast<float4 *>(p)[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+}
+__device__ __forceinline__ void store_half(__nv_bfloat16 *p, const float (&x)[kD / 2]) {
+#pragma unroll
+    for (int i = 0; i < kD / 16; ++i)
         reinterpret_cast<uint4 *>(p)[i] = make_uint4(bf2(x[8 * i], x[8 * i + 1]), bf2(x[8 * i + 2], x[8 * i + 3]),
                                                      bf2(x[8 * i + 4], x[8 * i + 5]), bf2(x[8 * i + 6], x[8 * i + 7]));
 }
@@ -103,19 +134,19 @@ __device__ __forceinline__ void rotate_row(float (&x)[kD], const float (&c)[kD /
 }
 
 constexpr int kQThreads = 128;
-constexpr int kQRows = 128;              // token rows per round: one per thread
+constexpr int kQRows = 64;               // token rows per round: two threads each
 constexpr int kQStride = kD + 4;         // 36 floats: rows 16-byte aligned, 4 banks apart
 constexpr int kQTab = 8192;              // the call's cos/sin table, when it fits
 constexpr int kQSmem = (kKVZ + 3 * kQRows * kQStride + kQRows) * 4 + kQTab;
 
 // One CTA per (b, h, block n, split sp): dq of the split's tokens and the
 // split's [dS | dZ] sums.  seff: [B][H][nb][1056] inclusive prefix state.
-// Per round of 128 tokens: each thread takes one token (num, den, g, c, dq);
-// then [dS | dZ] += [psi(q) g^T | c phi(q)] over the round's rows, each thread
-// a 4 x 4 block of dS for half of the rows (the two halves are added in a
-// fixed order at the end).
+// Per round of 64 tokens: two threads take each token (num, den, g, c, dq,
+// half of the features each); then [dS | dZ] += [psi(q) g^T | c phi(q)] over
+// the round's rows, each thread a 4 x 4 block of dS for half of the rows (the
+// two halves are added in a fixed order at the end).
 template <typename T>
-__global__ void __launch_bounds__(kQThreads, 3)   // at most 168 registers: 3 CTAs per SM (4: slower, spills)
+__global__ void __launch_bounds__(kQThreads, 4)   // at most 128 registers: 4 CTAs per SM (measured best)
 bwd_q_kernel(const T *__restrict__ q, const T *__restrict__ dout, const float *__restrict__ seff,
              T *__restrict__ dq, float *__restrict__ bpart, Plan p) {
     extern __shared__ __align__(16) float qsm[];
@@ -153,11 +184,16 @@ bwd_q_kernel(const T *__restrict__ q, const T *__restrict__ dout, const float *_
     }
     __syncthreads();
 
+    // Two threads per token (lanes 2i, 2i + 1 of a warp): each produces half
+    // of num, g and dq (value columns, and key features, 16 hf ..), and the
+    // halves of the two dot products are added in a fixed order (half 0, then
+    // half 1) by both threads.
+    const int tr = tid >> 1, hf = tid & 1;
     for (long long r0 = t0; r0 < t1; r0 += kQRows) {
-        const long long t = r0 + tid;
+        const long long t = r0 + tr;
         const bool valid = t < t1;
         const size_t off = (((size_t)b * p.N + (valid ? t : t0)) * p.H + h) * kD;
-        float x[kD], ps[kD];
+        float x[kD];
         uint32_t pos = 0;                              // bit a: q_a > 0
         if (valid) load_row(q + off, x);
 #pragma unroll
@@ -165,76 +201,98 @@ bwd_q_kernel(const T *__restrict__ q, const T *__restrict__ dout, const float *_
             const float v = valid ? x[a] : 0.f;
             pos |= (v > 0.f ? 1u : 0u) << a;
             x[a] = fmaxf(v, 0.f);                      // phi(q)
-            ps[a] = x[a];
         }
+        // register arrays are indexed by constants only (a runtime half index
+        // would put them in local memory): this thread's half by a select
+        auto xh = [&](int a) { return hf ? x[16 + a] : x[a]; };
+        float dh = 0.f;                                // phi(q) . Z over this thread's half
+#pragma unroll
+        for (int a = 0; a < kD / 2; ++a) dh = fmaf(xh(a), Ss[kD * kD + 16 * hf + a], dh);
+        const float dx = __shfl_xor_sync(0xffffffffu, dh, 1);
+        const float den = (hf ? dx + dh : dh + dx) + p.eps;
+#pragma unroll
+        for (int a = 0; a < kD / 2; a += 4)
+            *reinterpret_cast<float4 *>(fq + tr * kQStride + 16 * hf + a) = make_float4(xh(a), xh(a + 1), xh(a + 2), xh(a + 3));
         float cs_c[kD / 2], cs_s[kD / 2];
         if (p.rope && valid) {
             if (use_tab) token_cs_tab(p, tab, t, cs_c, cs_s);
             else token_cs(p, t, cs_c, cs_s);
-            rotate_row(ps, cs_c, cs_s, 1.f);
+            rotate_row(x, cs_c, cs_s, 1.f);            // x is psi(q) from here on
         }
 #pragma unroll
-        for (int a = 0; a < kD; a += 4) {
-            *reinterpret_cast<float4 *>(pq + tid * kQStride + a) = make_float4(ps[a], ps[a + 1], ps[a + 2], ps[a + 3]);
-            *reinterpret_cast<float4 *>(fq + tid * kQStride + a) = make_float4(x[a], x[a + 1], x[a + 2], x[a + 3]);
-        }
-        float den = 0.f;
+        for (int a = 0; a < kD / 2; a += 4)
+            *reinterpret_cast<float4 *>(pq + tr * kQStride + 16 * hf + a) = make_float4(xh(a), xh(a + 1), xh(a + 2), xh(a + 3));
+        // num = psi(q) S_n over this thread's 16 value columns
+        float num[kD / 2];
 #pragma unroll
-        for (int a = 0; a < kD; ++a) den = fmaf(x[a], Ss[kD * kD + a], den);
-        den += p.eps;
-        // num = psi(q) S_n: one S row (8 broadcast 16-byte loads) per feature
-        float num[kD];
+        for (int c = 0; c < kD / 2; ++c) num[c] = 0.f;
 #pragma unroll
-        for (int c = 0; c < kD; ++c) num[c] = 0.f;
-#pragma unroll 4
         for (int a = 0; a < kD; ++a) {
-            const float4 *row = reinterpret_cast<const float4 *>(Ss + a * kD);
+            const float4 *row = reinterpret_cast<const float4 *>(Ss + a * kD + 16 * hf);
 #pragma unroll
-            for (int c4 = 0; c4 < kD / 4; ++c4) {
+            for (int c4 = 0; c4 < kD / 8; ++c4) {
                 const float4 sv = row[c4];
-                num[4 * c4] = fmaf(ps[a], sv.x, num[4 * c4]);
-                num[4 * c4 + 1] = fmaf(ps[a], sv.y, num[4 * c4 + 1]);
-                num[4 * c4 + 2] = fmaf(ps[a], sv.z, num[4 * c4 + 2]);
-                num[4 * c4 + 3] = fmaf(ps[a], sv.w, num[4 * c4 + 3]);
+                num[4 * c4] = fmaf(x[a], sv.x, num[4 * c4]);
+                num[4 * c4 + 1] = fmaf(x[a], sv.y, num[4 * c4 + 1]);
+                num[4 * c4 + 2] = fmaf(x[a], sv.z, num[4 * c4 + 2]);
+                num[4 * c4 + 3] = fmaf(x[a], sv.w, num[4 * c4 + 3]);
             }
         }
-        float o[kD];
-        if (valid) load_row(dout + off, o);
-        float dn = 0.f;
+        float o[kD / 2];
+        if (valid) load_half(dout + off + 16 * hf, o);
+        float nh = 0.f;
 #pragma unroll
-        for (int c = 0; c < kD; ++c) {
+        for (int c = 0; c < kD / 2; ++c) {
             if (!valid) o[c] = 0.f;
-            dn = fmaf(o[c], num[c], dn);
+            nh = fmaf(o[c], num[c], nh);
         }
+        const float nx = __shfl_xor_sync(0xffffffffu, nh, 1);
+        const float dn = hf ? nx + nh : nh + nx;
         const float inv = 1.0f / den;
         const float cr = valid ? -dn * inv * inv : 0.f;
 #pragma unroll
-        for (int c = 0; c < kD; ++c) o[c] *= inv;      // g
+        for (int c = 0; c < kD / 2; ++c) o[c] *= inv;  // g, this thread's half
 #pragma unroll
-        for (int c = 0; c < kD; c += 4)
-            *reinterpret_cast<float4 *>(gg + tid * kQStride + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
-        cc[tid] = cr;
+        for (int c = 0; c < kD / 2; c += 4)
+            *reinterpret_cast<float4 *>(gg + tr * kQStride + 16 * hf + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+        if (hf == 0) cc[tr] = cr;
+        __syncwarp();                                  // the partner's half of g is in gg
         if (valid) {
-            // dq = mask (R^T (S g) + c Z)
-            float dp[kD];
-#pragma unroll 4
-            for (int a = 0; a < kD; ++a) {
-                const float4 *row = reinterpret_cast<const float4 *>(Ss + a * kD);
-                float s = 0.f;
+            // dq = mask (R^T (S g) + c Z) over this thread's 16 key features
+            float gv[kD];
+#pragma unroll
+            for (int c = 0; c < kD; c += 4) {
+                const float4 gq = *reinterpret_cast<const float4 *>(gg + tr * kQStride + c);
+                gv[c] = gq.x; gv[c + 1] = gq.y; gv[c + 2] = gq.z; gv[c + 3] = gq.w;
+            }
+            float dp[kD / 2];
+#pragma unroll
+            for (int a = 0; a < kD / 2; ++a) {
+                const float4 *row = reinterpret_cast<const float4 *>(Ss + (16 * hf + a) * kD);
+                float sacc = 0.f;
 #pragma unroll
                 for (int c4 = 0; c4 < kD / 4; ++c4) {
                     const float4 sv = row[c4];
-                    s = fmaf(sv.x, o[4 * c4], s);
-                    s = fmaf(sv.y, o[4 * c4 + 1], s);
-                    s = fmaf(sv.z, o[4 * c4 + 2], s);
-                    s = fmaf(sv.w, o[4 * c4 + 3], s);
+                    sacc = fmaf(sv.x, gv[4 * c4], sacc);
+                    sacc = fmaf(sv.y, gv[4 * c4 + 1], sacc);
+                    sacc = fmaf(sv.z, gv[4 * c4 + 2], sacc);
+                    sacc = fmaf(sv.w, gv[4 * c4 + 3], sacc);
                 }
-                dp[a] = s;
+                dp[a] = sacc;
             }
-            if (p.rope) rotate_row(dp, cs_c, cs_s, -1.f);
+            if (p.rope) {
 #pragma unroll
-            for (int a = 0; a < kD; ++a) dp[a] = (pos >> a) & 1u ? fmaf(cr, Ss[kD * kD + a], dp[a]) : 0.f;
-            store_row(dq + off, dp);
+                for (int pr = 0; pr < kD / 4; ++pr) {   // this half's pairs 8 hf + pr, by R^T
+                    const float c = hf ? cs_c[8 + pr] : cs_c[pr], sn = hf ? cs_s[8 + pr] : cs_s[pr];
+                    const float u = dp[2 * pr], w = dp[2 * pr + 1];
+                    dp[2 * pr] = u * c + w * sn;
+                    dp[2 * pr + 1] = -u * sn + w * c;
+                }
+            }
+#pragma unroll
+            for (int a = 0; a < kD / 2; ++a)
+                dp[a] = (pos >> (16 * hf + a)) & 1u ? fmaf(cr, Ss[kD * kD + 16 * hf + a], dp[a]) : 0.f;
+            store_half(dq + off + 16 * hf, dp);
         }
         __syncthreads();
         // [dS | dZ] over this thread's half of the round's rows, row order
