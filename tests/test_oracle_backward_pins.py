@@ -118,7 +118,7 @@ def test_backward_matches_autograd_of_brute_definition(orc, case):
     out = brute_torch(*xs, L, ang)
     # the forward restatement agrees with the oracle's forward first
     assert np.abs(out.detach().numpy() - orc.full_forward(q, k, v, L, rope=rope, eps=EPS)).max() <= 1e-12 * max(
-        1.0, float(out.abs().max()))
+        1.0, float(out.detach().abs().max()))
     (out * dout).sum().backward()
     got = orc.full_backward(q, k, v, dout, L, rope=rope, eps=EPS)
     for g, x in zip(got, xs):
