@@ -432,8 +432,9 @@ rope_reduce_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         }
     } else if (warp < 6) {
         // ------------------------------------------------ epilogue: warp quarter q
-        // reads TMEM lanes 32q.. = value features of head 4g + q; its key
-        // features are columns 32q.. of the hi half and 128 + 32q.. of the lo half
+        // reads TMEM lanes 32q.. (the key features of head 4g + q) in columns
+        // 32q.. of the accumulator (its value features); the hi and the lo MMA
+        // of a stage add into the same columns
         const int q = warp & 3;
         UnitWalk w;
         w.start(S, x_begin);
