@@ -1,6 +1,8 @@
 """The C ABI without a GPU: the library loads, exports every entry point that
-include/la.h declares, sizes its workspace on the host, and rejects bad
-arguments before enqueuing anything (so no call here reaches a kernel)."""
+include/la.h declares, the Python binding's ctypes signatures and structures
+match the header's declarations and C layouts, the library sizes its workspace
+on the host, and it rejects bad arguments before enqueuing anything (so no
+call here reaches a kernel)."""
 import ctypes
 import os
 import re
@@ -41,6 +43,75 @@ def test_library_exports_every_declared_symbol(la):
     for n in declared_symbols():
         assert hasattr(lib, n), n
         assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
+
+
+def _c_kind(decl):
+    """The ABI kind of one C parameter or return type of include/la.h."""
+    t = " ".join(decl.replace("const", " ").split())
+    if "*" in t:
+        return "char*" if t.startswith("char") and t.count("*") == 1 and t.split("*")[0].strip() == "char" \
+            else "ptr"
+    base = t.split()[0] if t else "void"
+    return {"size_t": "size_t", "float": "float", "void": "void", "long": "int64"}.get(base, "int")
+
+
+def _ctypes_kind(t):
+    if t is None:
+        return "void"
+    if t is ctypes.c_char_p:
+        return "char*"
+    if t is ctypes.c_void_p or isinstance(t, type(ctypes.POINTER(ctypes.c_int))):
+        return "ptr"
+    return {ctypes.c_size_t: "size_t", ctypes.c_float: "float", ctypes.c_int: "int",
+            ctypes.c_longlong: "int64"}.get(t, repr(t))
+
+
+def test_binding_signatures_match_the_header(la):
+    """Every entry point's ctypes argtypes and restype in la.py agree with its
+    C declaration: same count, and pointer / int / float / size_t in the same
+    places (a drifted signature would pass garbage across the boundary)."""
+    text = re.sub(r"/\*.*?\*/", "", "".join(open(os.path.join(ROOT, "include", h)).read()
+                                            for h in os.listdir(os.path.join(ROOT, "include")) if h.endswith(".h")),
+                  flags=re.S)
+    decls = re.findall(r"LA_API\s+([\w\s\*]+?)\b(la_\w+)\s*\(([^)]*)\)\s*;", text)
+    assert len(decls) == len(declared_symbols())
+    lib = la.lib()
+    for ret, name, params in decls:
+        params = " ".join(params.split())
+        want = [] if params in ("", "void") else [
+            _c_kind(re.sub(r"\b\w+$", "", p.strip()) if not p.strip().endswith("*") else p) for p in params.split(",")]
+        fn = getattr(lib, name)
+        got = [_ctypes_kind(a) for a in (fn.argtypes or [])]
+        assert got == want, f"{name}: la.py {got} vs la.h {want}"
+        assert _ctypes_kind(fn.restype) == _c_kind(ret), f"{name}: restype"
+
+
+def test_binding_structs_match_the_header(la, tmp_path):
+    """la_rope, la_state and la_state_counters have the same size and field
+    offsets in la.py's ctypes structures as the C compiler gives them."""
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    structs = {"la_rope": la.la_rope, "la_state": la.la_state, "la_state_counters": la.la_state_counters}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "la.h"', "int main(void) {"]
+    for s, py in structs.items():
+        lines.append(f'printf("{s} size %zu\\n", sizeof({s}));')
+        for f, _ in py._fields_:
+            lines.append(f'printf("{s} {f} %zu\\n", offsetof({s}, {f}));')
+    lines += ["return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    out = subprocess.check_output([str(exe)], text=True).split("\n")
+    got = {tuple(x.split()[:2]): int(x.split()[2]) for x in out if x.strip()}
+    for s, py in structs.items():
+        assert got[(s, "size")] == ctypes.sizeof(py), s
+        for f, _ in py._fields_:
+            assert got[(s, f)] == getattr(py, f).offset, f"{s}.{f}"
 
 
 def test_status_strings(la):
