@@ -282,3 +282,22 @@ def test_rejects_bad_arguments(orc):
         orc.brute(q, k, v, rope=bad)
     with pytest.raises(ValueError):
         orc.block_kv(k, v, 3, 2)
+
+
+def test_recurrence_cost_is_linear_in_tokens(orc):
+    # The method's cost is O(N) in tokens (a fixed-size state per head): four
+    # times the tokens must cost about four times the time, far from the 16x
+    # of the quadratic brute form.  Median of three runs each.
+    import time
+
+    def t(N):
+        q, k, v = synth.random_qkv(1, N, 2, 32, seed=24, dtype=torch.float32)
+        ts = []
+        for _ in range(3):
+            t0 = time.perf_counter()
+            orc.full_forward(q, k, v, 0, eps=EPS)
+            ts.append(time.perf_counter() - t0)
+        return sorted(ts)[1]
+
+    ratio = t(32768) / t(8192)
+    assert 1.5 < ratio < 8.0, ratio
